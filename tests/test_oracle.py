@@ -1,0 +1,361 @@
+"""Pins for the fp64 oracle (CPU only).
+
+Each test checks the oracle against something other than itself: a closed
+form, a brute-force restatement, a hand-worked example or a limiting case the
+pages state. Together they fail on a dropped term, a wrong sign, a transposed
+operand, a misplaced decay or a read-before-write.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from brute import states_by_kron, states_by_product, transitions
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_examples_d2.json")
+MODES = ("none", "scalar", "channel")
+
+
+def _rand_problem(rng, B, T, H, dk, dv, mode, unit_keys=True, g_scale=0.3):
+    q = rng.standard_normal((B, T, H, dk))
+    k = rng.standard_normal((B, T, H, dk))
+    if unit_keys:
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+        q /= np.linalg.norm(q, axis=-1, keepdims=True)
+    v = rng.standard_normal((B, T, H, dv))
+    beta = rng.uniform(0.0, 1.0, (B, T, H))
+    if mode == "scalar":
+        g = -g_scale * rng.uniform(0, 1, (B, T, H))
+    elif mode == "channel":
+        g = -g_scale * rng.uniform(0, 1, (B, T, H, dk))
+    else:
+        g = None
+    return q, k, v, g, beta
+
+
+def _run(q, k, v, g, beta, mode, S0=None, **kw):
+    return oracle.recurrent(q, k, v, g, beta, mode, S0=S0, f64_inputs=True, **kw)
+
+
+# ---------------------------------------------------------------- golden ---
+def test_hand_worked_examples():
+    """Hand-worked tiny examples of the update rule (tests/golden)."""
+    spec = json.load(open(GOLDEN))
+    for case in spec["cases"]:
+        k = np.array(case["k"], float)[None, :, None, :]
+        v = np.array(case["v"], float)[None, :, None, :]
+        q = np.array(case["q"], float)[None, :, None, :]
+        beta = np.array(case["beta"], float)[None, :, None]
+        g = np.log(np.array(case["alpha"], float))
+        g = g[None, :, None] if case["mode"] == "scalar" else g[None, :, None, :]
+        S0 = None if case["S0"] is None else np.array(case["S0"], float)[None, None]
+        T = k.shape[1]
+        for t in range(1, T + 1):  # every prefix: intermediate states too
+            o, S = _run(q[:, :t], k[:, :t], v[:, :t], g[:, :t], beta[:, :t], case["mode"], S0,
+                        scale=case["scale"])
+            np.testing.assert_allclose(o[0, :, 0], np.array(case["o"], float)[:t], atol=1e-12)
+            np.testing.assert_allclose(S[0, 0], np.array(case["S"], float)[t - 1], atol=1e-12)
+
+
+# ----------------------------------------------------------- brute force ---
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("generalised", [False, True])
+def test_matches_transition_products(mode, generalised):
+    """Per-token states and outputs equal the explicit product of affine
+    transitions and the d_v*d_k Kronecker form on tiny T (T<=8, d<=6)."""
+    rng = np.random.default_rng(11 + MODES.index(mode) + 7 * generalised)
+    B, T, H, dk, dv = 2, 7, 2, 5, 4
+    q, k, v, g, beta = _rand_problem(rng, B, T, H, dk, dv, mode, unit_keys=not generalised, g_scale=0.7)
+    S0 = rng.standard_normal((B, H, dv, dk))
+    erase = rng.uniform(0, 1.2, (B, T, H)) if generalised else beta
+    write = rng.uniform(-1, 1, (B, T, H)) if generalised else beta
+    scale = 0.37
+    o, S_T = _run(q, k, v, g, beta, mode, S0, erase=erase, write=write, scale=scale)
+    for b in range(B):
+        for h in range(H):
+            gg = None if g is None else g[b, :, h]
+            As, Bs = transitions(k[b, :, h], v[b, :, h], gg, mode, erase[b, :, h], write[b, :, h])
+            Sp = states_by_product(S0[b, h], As, Bs)
+            Sk = states_by_kron(S0[b, h], As, Bs)
+            for t in range(T):
+                np.testing.assert_allclose(Sp[t], Sk[t], atol=1e-12)
+                np.testing.assert_allclose(o[b, t, h], scale * Sp[t] @ q[b, t, h], atol=1e-12)
+            np.testing.assert_allclose(S_T[b, h], Sp[-1], atol=1e-12)
+
+
+# ---------------------------------------------------------- closed forms ---
+@pytest.mark.parametrize("mode", MODES)
+def test_erase_free_is_decayed_linear_attention(mode):
+    """Erase-free mode (e=0, w=1) is (decayed) linear attention, whose output has
+    the closed form scale * (Q K^T (.) D) V with D_ti = exp(Gamma_t - Gamma_i) for
+    i <= t (D = causal mask incl. the diagonal when alpha = 1): "linear attention
+    and its gated descendants", Chunkwise Parallel Form, and "Linear Attention &
+    DeltaNet", item 1."""
+    rng = np.random.default_rng(3 + MODES.index(mode))
+    B, T, H, dk, dv = 1, 41, 2, 8, 6
+    q, k, v, g, beta = _rand_problem(rng, B, T, H, dk, dv, mode, unit_keys=False)
+    zeros, ones = np.zeros((B, T, H)), np.ones((B, T, H))
+    o, S_T = _run(q, k, v, g, beta, mode, erase=zeros, write=ones, scale=1.0)
+    for h in range(H):
+        Q, K, V = q[0, :, h], k[0, :, h], v[0, :, h]
+        if mode == "channel":
+            Gam = np.cumsum(g[0, :, h], axis=0)  # [T, dk]
+            ref = np.zeros((T, dv))
+            for t in range(T):
+                for i in range(t + 1):
+                    ref[t] += V[i] * np.dot(K[i] * np.exp(Gam[t] - Gam[i]), Q[t])
+            Sref = sum(np.outer(V[i], K[i] * np.exp(Gam[-1] - Gam[i])) for i in range(T))
+        else:
+            Gam = np.zeros(T) if mode == "none" else np.cumsum(g[0, :, h])
+            D = np.tril(np.exp(Gam[:, None] - Gam[None, :]))
+            ref = ((Q @ K.T) * D) @ V
+            Sref = (V * np.exp(Gam[-1] - Gam)[:, None]).T @ K
+        np.testing.assert_allclose(o[0, :, h], ref, atol=1e-11)
+        np.testing.assert_allclose(S_T[0, h], Sref, atol=1e-11)
+
+
+def test_plain_linear_attention_mask_includes_diagonal():
+    """With alpha = 1, e = 0, w = 1: o = (Q K^T (.) M) V, M lower-triangular with the
+    diagonal (token t reads its own write). A strictly-lower mask must fail."""
+    rng = np.random.default_rng(5)
+    T, d = 16, 4
+    q, k, v, _, beta = _rand_problem(rng, 1, T, 1, d, d, "none", unit_keys=False)
+    o, _ = _run(q, k, v, None, beta, "none", erase=np.zeros_like(beta), write=np.ones_like(beta), scale=1.0)
+    Q, K, V = q[0, :, 0], k[0, :, 0], v[0, :, 0]
+    np.testing.assert_allclose(o[0, :, 0], np.tril(Q @ K.T) @ V, atol=1e-12)
+    assert np.abs(o[0, :, 0] - np.tril(Q @ K.T, -1) @ V).max() > 1e-3
+
+
+# --------------------------------------------------- delta-rule semantics ---
+def test_exact_recall_orthonormal_keys():
+    """alpha=1, beta=1 and orthonormal keys: the memory stores and recalls each
+    value exactly, S_T k_i = v_i; a query equal to k_i reads v_i / sqrt(d_k)
+    ("linear attention and its gated descendants", DeltaNet: orthogonal keys
+    isolate v_j; "Linear Attention & DeltaNet", item 3)."""
+    rng = np.random.default_rng(7)
+    dk, dv, T = 16, 9, 12
+    Qm, _ = np.linalg.qr(rng.standard_normal((dk, dk)))
+    keys = Qm[:, :T].T  # T orthonormal rows
+    k = keys[None, :, None, :]
+    v = rng.standard_normal((1, T, 1, dv))
+    q = keys[rng.permutation(T)][None, :, None, :]  # query some earlier or later key
+    beta = np.ones((1, T, 1))
+    o, S_T = _run(q, k, v, None, beta, "none")
+    for i in range(T):
+        np.testing.assert_allclose(S_T[0, 0] @ keys[i], v[0, i, 0], atol=1e-12)
+    qidx = [int(np.argmax(np.abs(keys @ q[0, t, 0]))) for t in range(T)]
+    for t in range(T):
+        want = v[0, qidx[t], 0] / np.sqrt(dk) if qidx[t] <= t else np.zeros(dv)
+        np.testing.assert_allclose(o[0, t, 0], want, atol=1e-12)
+
+
+def test_overwrite_same_key_recalls_latest():
+    rng = np.random.default_rng(8)
+    dk, dv = 8, 5
+    kk = rng.standard_normal(dk); kk /= np.linalg.norm(kk)
+    k = np.stack([kk, kk])[None, :, None, :]
+    v = rng.standard_normal((1, 2, 1, dv))
+    _, S_T = _run(k, k, v, None, np.ones((1, 2, 1)), "none")
+    np.testing.assert_allclose(S_T[0, 0] @ kk, v[0, 1, 0], atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_beta_blend_at_current_key(mode):
+    """For a unit key: S_t k_t = (1 - beta) Sbar k_t + beta v_t (beta = 1 replaces,
+    beta = 0 keeps, 0 < beta < 1 blends -- the DeltaNet section)."""
+    rng = np.random.default_rng(9 + MODES.index(mode))
+    B, T, H, dk, dv = 1, 6, 1, 7, 3
+    q, k, v, g, beta = _rand_problem(rng, B, T, H, dk, dv, mode)
+    S0 = rng.standard_normal((B, H, dv, dk))
+    S = S0[0, 0].copy()
+    for t in range(T):
+        _, St = _run(q[:, t:t + 1], k[:, t:t + 1], v[:, t:t + 1], None if g is None else g[:, t:t + 1],
+                     beta[:, t:t + 1], mode, S[None, None])
+        if mode == "none":
+            a = np.ones(dk)
+        elif mode == "scalar":
+            a = np.full(dk, np.exp(g[0, t, 0]))
+        else:
+            a = np.exp(g[0, t, 0])
+        kt = k[0, t, 0]
+        Sbar = S * a[None, :]
+        want = (1 - beta[0, t, 0]) * (Sbar @ kt) + beta[0, t, 0] * v[0, t, 0]
+        np.testing.assert_allclose(St[0, 0] @ kt, want, atol=1e-12)
+        S = St[0, 0]
+
+
+@pytest.mark.parametrize("mode", ("scalar", "channel"))
+def test_beta_zero_only_decays(mode):
+    """beta = 0 writes nothing: S_T = S0 Diag(prod alpha), o_t = scale S0 Diag(prod_{s<=t} alpha) q_t."""
+    rng = np.random.default_rng(12)
+    B, T, H, dk, dv = 1, 9, 2, 6, 5
+    q, k, v, g, _ = _rand_problem(rng, B, T, H, dk, dv, mode)
+    S0 = rng.standard_normal((B, H, dv, dk))
+    o, S_T = _run(q, k, v, g, np.zeros((B, T, H)), mode, S0)
+    for h in range(H):
+        Gam = np.cumsum(g[0, :, h], axis=0)
+        Gam = Gam[:, None] * np.ones(dk) if mode == "scalar" else Gam
+        for t in range(T):
+            np.testing.assert_allclose(o[0, t, h], (S0[0, h] * np.exp(Gam[t])[None, :]) @ q[0, t, h] / np.sqrt(dk),
+                                       atol=1e-12)
+        np.testing.assert_allclose(S_T[0, h], S0[0, h] * np.exp(Gam[-1])[None, :], atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", ("scalar", "channel"))
+def test_alpha_zero_resets_every_token(mode):
+    """alpha = 0 (g = -1e4, exp underflows to exactly 0): S_t = beta_t v_t k_t^T and
+    o_t = scale beta_t (k_t . q_t) v_t, whatever came before."""
+    rng = np.random.default_rng(13)
+    B, T, H, dk, dv = 2, 8, 2, 6, 4
+    q, k, v, g, beta = _rand_problem(rng, B, T, H, dk, dv, mode)
+    g = np.full_like(g, -1e4)
+    S0 = rng.standard_normal((B, H, dv, dk))
+    o, S_T = _run(q, k, v, g, beta, mode, S0)
+    want_o = (beta * np.einsum("bthd,bthd->bth", k, q))[..., None] * v / np.sqrt(dk)
+    np.testing.assert_allclose(o, want_o, atol=1e-12)
+    want_S = beta[:, -1, :, None, None] * np.einsum("bhv,bhk->bhvk", v[:, -1], k[:, -1])
+    np.testing.assert_allclose(S_T, want_S, atol=1e-12)
+
+
+# ------------------------------------------------------------- reductions ---
+def test_channel_with_constant_channels_is_scalar():
+    """KDA whose per-channel gate is constant across channels is Gated DeltaNet."""
+    rng = np.random.default_rng(14)
+    B, T, H, dk, dv = 2, 30, 2, 8, 8
+    q, k, v, g, beta = _rand_problem(rng, B, T, H, dk, dv, "scalar")
+    S0 = rng.standard_normal((B, H, dv, dk))
+    o1, s1 = _run(q, k, v, g, beta, "scalar", S0)
+    o2, s2 = _run(q, k, v, np.repeat(g[..., None], dk, axis=-1), beta, "channel", S0)
+    np.testing.assert_allclose(o1, o2, atol=1e-13)
+    np.testing.assert_allclose(s1, s2, atol=1e-13)
+
+
+def test_scalar_with_zero_log_decay_is_deltanet():
+    rng = np.random.default_rng(15)
+    B, T, H, dk, dv = 1, 25, 3, 8, 4
+    q, k, v, _, beta = _rand_problem(rng, B, T, H, dk, dv, "none")
+    S0 = rng.standard_normal((B, H, dv, dk))
+    o1, s1 = _run(q, k, v, None, beta, "none", S0)
+    o2, s2 = _run(q, k, v, np.zeros((B, T, H)), beta, "scalar", S0)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(s1, s2)
+
+
+def test_first_order_small_beta_limit():
+    """beta = eps, alpha = 1, S0 = 0: o / eps -> scale (Q K^T (.) M) V with error O(eps)."""
+    rng = np.random.default_rng(16)
+    T, dk, dv = 20, 8, 5
+    q, k, v, _, _ = _rand_problem(rng, 1, T, 1, dk, dv, "none")
+    eps = 1e-6
+    o, _ = _run(q, k, v, None, np.full((1, T, 1), eps), "none")
+    Q, K, V = q[0, :, 0], k[0, :, 0], v[0, :, 0]
+    ref = np.tril(Q @ K.T) @ V / np.sqrt(dk)
+    err = np.abs(o[0, :, 0] / eps - ref).max()
+    assert err < 50 * eps * T, err
+
+
+# ---------------------------------------------------------- structure ------
+@pytest.mark.parametrize("mode", MODES)
+def test_state_carry_split(mode):
+    """Running T1 then T2 from the carried state equals running T1+T2 at once
+    (state additivity over splits, the Chunk-Boundary State step)."""
+    rng = np.random.default_rng(17)
+    B, T, H, dk, dv = 2, 37, 2, 8, 6
+    q, k, v, g, beta = _rand_problem(rng, B, T, H, dk, dv, mode)
+    S0 = rng.standard_normal((B, H, dv, dk))
+    o, S_T = _run(q, k, v, g, beta, mode, S0)
+    t1 = 15
+    sl1, sl2 = slice(0, t1), slice(t1, T)
+    gs = (lambda s: None) if g is None else (lambda s: g[:, s])
+    o1, s1 = _run(q[:, sl1], k[:, sl1], v[:, sl1], gs(sl1), beta[:, sl1], mode, S0)
+    o2, s2 = _run(q[:, sl2], k[:, sl2], v[:, sl2], gs(sl2), beta[:, sl2], mode, s1)
+    np.testing.assert_allclose(np.concatenate([o1, o2], axis=1), o, atol=1e-12)
+    np.testing.assert_allclose(s2, S_T, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_linear_in_values_and_initial_state(mode):
+    rng = np.random.default_rng(18)
+    B, T, H, dk, dv = 1, 19, 2, 6, 5
+    q, k, v1, g, beta = _rand_problem(rng, B, T, H, dk, dv, mode)
+    v2 = rng.standard_normal(v1.shape)
+    s01, s02 = rng.standard_normal((2, B, H, dv, dk))
+    a, b = 0.7, -1.3
+    o1, S1 = _run(q, k, v1, g, beta, mode, s01)
+    o2, S2 = _run(q, k, v2, g, beta, mode, s02)
+    o3, S3 = _run(q, k, a * v1 + b * v2, g, beta, mode, a * s01 + b * s02)
+    np.testing.assert_allclose(o3, a * o1 + b * o2, atol=1e-12)
+    np.testing.assert_allclose(S3, a * S1 + b * S2, atol=1e-12)
+
+
+def test_value_rows_are_independent():
+    """Permuting the value channels (rows of S) permutes the outputs the same way."""
+    rng = np.random.default_rng(19)
+    B, T, H, dk, dv = 1, 21, 1, 6, 7
+    q, k, v, g, beta = _rand_problem(rng, B, T, H, dk, dv, "channel")
+    S0 = rng.standard_normal((B, H, dv, dk))
+    perm = rng.permutation(dv)
+    o, S = _run(q, k, v, g, beta, "channel", S0)
+    op, Sp = _run(q, k, v[..., perm], g, beta, "channel", S0[:, :, perm])
+    np.testing.assert_allclose(op, o[..., perm], atol=1e-13)
+    np.testing.assert_allclose(Sp, S[:, :, perm], atol=1e-13)
+
+
+def test_state_norm_bound():
+    """For unit keys, beta in [0,1], alpha <= 1 the erase factor is a contraction:
+    ||S_t||_2 <= ||S_{t-1}||_2 + beta_t ||v_t||."""
+    rng = np.random.default_rng(20)
+    dk, dv, T = 8, 8, 40
+    q, k, v, g, beta = _rand_problem(rng, 1, T, 1, dk, dv, "channel")
+    S = rng.standard_normal((1, 1, dv, dk))
+    for t in range(T):
+        _, Sn = _run(q[:, t:t + 1], k[:, t:t + 1], v[:, t:t + 1], g[:, t:t + 1], beta[:, t:t + 1], "channel", S)
+        assert np.linalg.norm(Sn[0, 0], 2) <= np.linalg.norm(S[0, 0], 2) + beta[0, t, 0] * np.linalg.norm(v[0, t, 0]) + 1e-12
+        S = Sn
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_decode_steps_equal_forward(mode):
+    """The recurrent decode step applied T times equals the forward over T tokens."""
+    rng = np.random.default_rng(21)
+    B, T, H, dk, dv = 2, 5, 3, 6, 4
+    q, k, v, g, beta = _rand_problem(rng, B, T, H, dk, dv, mode)
+    S0 = rng.standard_normal((B, H, dv, dk))
+    o, S_T = _run(q, k, v, g, beta, mode, S0)
+    S = S0
+    for t in range(T):
+        od, S = oracle.decode_step(q[:, t], k[:, t], v[:, t], None if g is None else g[:, t], beta[:, t], S,
+                                   mode, f64_inputs=True)
+        np.testing.assert_allclose(od, o[:, t], atol=1e-13)
+    np.testing.assert_allclose(S, S_T, atol=1e-13)
+
+
+def test_float32_inputs_read_exactly():
+    """bf16/fp32 inputs are read as their exact values (float32 path == float64 path)."""
+    rng = np.random.default_rng(22)
+    q, k, v, g, beta = _rand_problem(rng, 1, 13, 2, 8, 8, "scalar")
+    f = lambda x: x.astype(np.float32)
+    o32, s32 = oracle.recurrent(f(q), f(k), f(v), f(g), f(beta), "scalar")
+    o64, s64 = oracle.recurrent(*(f(x).astype(np.float64) for x in (q, k, v, g, beta)), "scalar", f64_inputs=True)
+    np.testing.assert_array_equal(o32, o64)
+    np.testing.assert_array_equal(s32, s64)
+
+
+def test_threads_do_not_change_results():
+    rng = np.random.default_rng(23)
+    q, k, v, g, beta = _rand_problem(rng, 2, 30, 3, 8, 40, "channel")
+    o1, s1 = _run(q, k, v, g, beta, "channel", threads=1)
+    o2, s2 = _run(q, k, v, g, beta, "channel", threads=4)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(s1, s2)
+
+
+def test_bad_arguments_raise():
+    rng = np.random.default_rng(24)
+    q, k, v, g, beta = _rand_problem(rng, 1, 4, 1, 4, 4, "scalar")
+    with pytest.raises(ValueError):
+        _run(q, k, v, g[..., None].repeat(4, -1), beta, "scalar")
+    with pytest.raises(ValueError):
+        _run(q, k, v, g, beta, "bogus")
