@@ -1,0 +1,395 @@
+"""Benchmark: gated delta-rule chunked forward (Gated DeltaNet, B=8 H=8 T=4096 d=128,
+chunk 64, bf16 in / fp32 state) on B200, plus the decode step (B=256 H=16).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on rank 0. A step is one chunked forward over the whole batch
+(o and S_T). Timing: W untimed steps, then K steps between CUDA events on the
+launching stream, bracketed by a barrier and a device synchronize; the time is
+the max over ranks. Two input sets (each 270 MB, larger than the 126 MB L2) are
+alternated so no step reads the previous step's inputs from L2.
+Multi-GPU: every rank runs its own batch (weak scaling, no data-path collective).
+``--impl reference`` times the fp64 CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from gated_delta_rule_143_b200.inputs import (CHUNK_WORKLOADS, DECODE_WORKLOADS, WORKLOAD_SEEDS,  # noqa: E402
+                                              make_decode_state, make_decode_step, workload_inputs)
+
+WORKLOAD = "gdn_bf16_b8_h8_t4096_d128"
+DECODE = "gdn_decode_bf16_b256_h16_d128"
+METRIC = "gated-delta-rule fwd tokens/s on 1 B200; % of roofline (TC FLOP/s or HBM GB/s)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------- counts --
+def chunk_flops_per_token_head(C, dk, dv):
+    """Dense chunk-tile flops of the chunk form per token-head: A, W, QK^T (C*dk each),
+    U and P.Delta (C*dv each), W S^T, Delta^T K and Q S^T (dk*dv each)."""
+    return 2 * (C * (3 * dk + 2 * dv) + 3 * dk * dv)
+
+
+OUT_BYTES = 4  # o is written in fp32 (the accumulation precision)
+
+
+def chunk_bytes(w):
+    """Algorithmic HBM bytes of one forward: q, k, v (input dtype) read once, o (fp32)
+    written once, beta and g read once, S_T written once (S0 is null for these workloads)."""
+    eb = 2 if w.dtype == "bf16" else 4
+    th = w.B * w.T * w.H
+    g = 0 if w.mode == "none" else (4 if w.mode == "scalar" else 4 * w.dk)
+    per_th = eb * (2 * w.dk + w.dv) + OUT_BYTES * w.dv + 4 + g
+    return th * per_th + w.B * w.H * w.dv * w.dk * 4
+
+
+def decode_bytes(w):
+    """S read and written once (fp32), q, k, v read, o (fp32) written, beta and g read."""
+    eb = 2 if w.dtype == "bf16" else 4
+    nh = w.B * w.H
+    g = 0 if w.mode == "none" else (4 if w.mode == "scalar" else 4 * w.dk)
+    return nh * (2 * 4 * w.dk * w.dv + eb * (2 * w.dk + w.dv) + OUT_BYTES * w.dv + 4 + g)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.out.flush()
+        rows = []
+        try:
+            with open(self.out.name) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        finally:
+            os.unlink(self.out.name)
+        return self._summary(rows)
+
+    @staticmethod
+    def _summary(rows):
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def smi_id(dev, local):
+    """nvidia-smi --id for this process's device: its UUID when torch exposes it, else the
+    physical index from CUDA_VISIBLE_DEVICES, else the local ordinal."""
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        if u:
+            return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        pass
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local < len(ids):
+            return ids[local]
+    return str(local)
+
+
+# ------------------------------------------------------------- distributed --
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif n_gpus > 1:
+        raise SystemExit("--gpus N > 1 must be launched with torch.distributed.run (one process per GPU)")
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------- ours --
+def time_device(fn, steps, warmup, world, stream):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return e0.elapsed_time(e1)  # ms over `steps`
+
+
+def run_ours(args):
+    import gated_delta_rule_143_b200 as gdr
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    w = CHUNK_WORKLOADS[WORKLOAD]
+    stream = torch.cuda.current_stream(dev)
+
+    # two resident input sets, each larger than L2; one seed per rank (weak scaling)
+    sets = []
+    for s in range(2):
+        x = workload_inputs(w, seed=WORKLOAD_SEEDS[WORKLOAD] + 1000 * rank + s)
+        sets.append({k: (None if t is None else t.to(dev)) for k, t in x.items()})
+    o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=dev)
+    st = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
+    ws_n = gdr.workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.chunk, w.mode, torch.bfloat16, torch.float32)
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev) if ws_n else None
+
+    def step(i=0):
+        x = sets[i & 1]
+        gdr.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], mode=w.mode, chunk=w.chunk,
+                      out=o, state_out=st, workspace=ws)
+
+    clocks = ClockSampler(smi_id(dev, local))
+    for _ in range(args.warmup):
+        step()
+    clocks.start()
+    ms = time_device(step, args.steps, 0, world, stream)
+    clk = clocks.stop()
+    gdr.sync_status()
+    ms = max_over_ranks(ms, world)
+    ms_step = ms / args.steps
+    tokens = w.B * w.T
+    value = world * tokens / (ms_step * 1e-3)
+
+    nbytes = chunk_bytes(w)
+    flops = chunk_flops_per_token_head(w.chunk, w.dk, w.dv) * w.B * w.T * w.H
+    kernels_per_step = gdr_kernels_per_step(w)
+    achieved_gbs = nbytes / (ms_step * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved_gbs / peaks["hbm_gbs"], 4), "traffic": traffic_from_profile(),
+                "peak_source": peak_src, "algorithmic_bytes_per_launch": nbytes,
+                "tensor_view": {"flops_per_launch": flops,
+                                "achieved_tflops": round(flops / (ms_step * 1e-3) / 1e12, 1),
+                                "peak_tflops": peaks["bf16_tflops"],
+                                "frac": round(flops / (ms_step * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)},
+                "roofline_us": round(max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)) * 1e6, 2)}
+
+    # end to end: pinned host inputs -> device -> kernels -> host outputs, every step
+    hx = {k: (None if t is None else t.cpu().pin_memory()) for k, t in sets[0].items()}
+    h_o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, pin_memory=True)
+    h_s = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, pin_memory=True)
+
+    def e2e_step(i=0):
+        gdr.chunk_fwd(hx["q"], hx["k"], hx["v"], hx["g"], hx["beta"], None, mode=w.mode, chunk=w.chunk,
+                      out=h_o, state_out=h_s)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    e2e_ms = max_over_ranks(time_device(e2e_step, e2e_steps, max(1, min(args.warmup, 3)), world, stream), world)
+    h2d = sum(t.numel() * t.element_size() for t in hx.values() if t is not None)
+    d2h = h_o.numel() * h_o.element_size() + h_s.numel() * h_s.element_size()
+
+    dec = bench_decode(args, dev, peaks, world)
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": w.B, "T": w.T, "H": w.H, "d_k": w.dk, "d_v": w.dv, "chunk": w.chunk,
+                   "decay": w.mode, "inputs": "bf16 q/k/v, fp32 g/beta, fp32 state; S0 = 0; returns o (fp32) and S_T",
+                   "l2": "two resident input sets alternated, each 270 MB > 126 MB L2 (no flush)",
+                   "parallelism": f"replicas x{world} (independent batches per GPU)"},
+        "e2e": {"value": round(world * tokens / (e2e_ms / e2e_steps * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": kernels_per_step * args.steps,
+        "roofline": roofline,
+        "clocks": clk,
+        "decode": dec,
+    }
+    if rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def gdr_kernels_per_step(w):
+    import gated_delta_rule_143_b200 as gdr
+    return gdr.launches_per_chunk_fwd(w.B, w.T, w.H, w.dk, w.dv, w.chunk, w.mode, torch.bfloat16, torch.float32)
+
+
+def traffic_from_profile():
+    """DRAM bytes per launch from the committed ncu summary of the current kernel, if recorded."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d.get(WORKLOAD)
+    return None
+
+
+def bench_decode(args, dev, peaks, world):
+    import gated_delta_rule_143_b200 as gdr
+    w = DECODE_WORKLOADS[DECODE]
+    S = make_decode_state(w, WORKLOAD_SEEDS[DECODE]).to(dev)
+    toks = []
+    for s in range(2):
+        x = make_decode_step(w, WORKLOAD_SEEDS[DECODE], s)
+        toks.append({k: (None if t is None else t.to(dev)) for k, t in x.items()})
+    o = torch.empty((w.B, w.H, w.dv), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i=0):
+        x = toks[i & 1]
+        gdr.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], S, mode=w.mode, out=o)
+
+    n = max(20, min(args.steps, 200))
+    ms = max_over_ranks(time_device(step, n, max(3, args.warmup), world, stream), world) / n
+    nbytes = decode_bytes(w)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": DECODE, "ms_per_step": round(ms, 5), "tokens_per_s": round(world * w.B / (ms * 1e-3), 1),
+            "steps": n, "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                                     "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                     "algorithmic_bytes_per_launch": nbytes},
+            "l2": "state 537 MB > L2, streamed once per step"}
+
+
+# ------------------------------------------------------------------- oracle --
+def _oracle_sample(w, b_count=1):
+    """A bounded sample of the workload for the CPU oracle: the first b_count sequences
+    (all heads, all tokens)."""
+    x = workload_inputs(w)
+    return {k: (None if t is None else t[:b_count].contiguous()) for k, t in x.items()}
+
+
+def cpu_baseline(w):
+    import oracle
+    x = _oracle_sample(w, b_count=w.B)
+    t0 = time.perf_counter()
+    oracle.recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], w.mode, S0=x["S0"])
+    dt = time.perf_counter() - t0
+    return {"value": round(w.B * w.T / dt, 1), "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"full workload once ({w.B}x{w.T} tokens x {w.H} heads), fp64 token-by-token recurrence",
+            "seconds": round(dt, 3)}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    w = CHUNK_WORKLOADS[WORKLOAD]
+    x = _oracle_sample(w, b_count=1)
+    sample_tokens = x["q"].shape[0] * w.T
+
+    def once():
+        oracle.recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], w.mode, S0=x["S0"])
+
+    for _ in range(args.warmup):
+        once()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        once()
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    value = round(sample_tokens / dt, 1)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": w.B, "T": w.T, "H": w.H, "d_k": w.dk, "d_v": w.dv, "chunk": w.chunk,
+                   "decay": w.mode},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+                         "sample": f"1 of {w.B} sequences per step ({w.T} tokens x {w.H} heads)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

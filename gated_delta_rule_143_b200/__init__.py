@@ -1,0 +1,152 @@
+"""Gated delta-rule mixer for NVIDIA B200 (sm_100a): Python binding of libgdr.so.
+
+Argument marshalling only: every step of the computation runs in the library's
+CUDA kernels; PyTorch provides device memory and streams. The two operations:
+
+* ``chunk_fwd``   -- chunkwise-parallel forward over whole sequences (prefill /
+  training form) for DeltaNet (mode "none"), Gated DeltaNet ("scalar") and
+  Kimi Delta Attention ("channel");
+* ``decode_step`` -- one recurrent token step on a batch of fp32 states, in place.
+
+Both take device tensors. ``chunk_fwd`` also accepts host (CPU) tensors: it
+then copies them to the current device on the current stream, runs, and copies
+the outputs back (the end-to-end path a host-resident caller uses).
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from ._lib import DECAY_MODES, DTYPE_BF16, DTYPE_F32, GdrError, check, lib
+
+__all__ = ["chunk_fwd", "decode_step", "sync_status", "workspace_bytes", "launches_per_chunk_fwd", "GdrError", "DECAY_MODES"]
+
+
+def _mode(mode) -> int:
+    if isinstance(mode, str):
+        if mode not in DECAY_MODES:
+            raise ValueError(f"unknown decay mode {mode!r}")
+        return DECAY_MODES[mode]
+    return int(mode)
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return DTYPE_BF16
+    if dt == torch.float32:
+        return DTYPE_F32
+    raise TypeError(f"tensors must be bfloat16 or float32, got {dt}")
+
+
+def _dtype(t: torch.Tensor) -> int:
+    return _dtype_code(t.dtype)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def workspace_bytes(B: int, T: int, H: int, dk: int, dv: int, chunk: int, mode, dtype: torch.dtype,
+                    out_dtype: torch.dtype = torch.float32) -> int:
+    """Device scratch ``chunk_fwd`` needs for this problem (bytes)."""
+    return int(lib().gdr_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, _mode(mode), _dtype_code(dtype),
+                                                   _dtype_code(out_dtype)))
+
+
+def launches_per_chunk_fwd(B: int, T: int, H: int, dk: int, dv: int, chunk: int, mode, dtype: torch.dtype,
+                           out_dtype: torch.dtype = torch.float32) -> int:
+    """Kernel launches one ``chunk_fwd`` makes for this problem (as the library reports)."""
+    return int(lib().gdr_chunk_fwd_launches(B, T, H, dk, dv, chunk, _mode(mode), _dtype_code(dtype),
+                                            _dtype_code(out_dtype)))
+
+
+_ws_cache = {}
+
+
+def _workspace(nbytes: int, device: torch.device) -> Optional[torch.Tensor]:
+    if nbytes == 0:
+        return None
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _ws_cache[key] = buf
+    return buf
+
+
+def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optional[torch.Tensor],
+              beta: torch.Tensor, S0: Optional[torch.Tensor] = None, *, mode="scalar", chunk: int = 64,
+              return_state: bool = True, out: Optional[torch.Tensor] = None,
+              out_dtype: torch.dtype = torch.float32,
+              state_out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked forward. q, k [B,T,H,dk]; v [B,T,H,dv] (bf16 or fp32, same dtype);
+    g fp32 [B,T,H] ("scalar") / [B,T,H,dk] ("channel") / None ("none"); beta fp32
+    [B,T,H]; S0 fp32 [B,H,dv,dk] or None. Returns (o [B,T,H,dv], S_T or None).
+    o is fp32 by default (``out_dtype``, or the dtype of ``out``; bf16 allowed for bf16
+    inputs). ``state_out`` may be ``S0`` itself (in-place carry)."""
+    if q.device.type == "cpu":
+        return _chunk_fwd_host(q, k, v, g, beta, S0, mode=mode, chunk=chunk, return_state=return_state,
+                               out=out, out_dtype=out_dtype, state_out=state_out, stream=stream)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype(q)
+    m = _mode(mode)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=out_dtype, device=q.device)
+    odt = _dtype(out)
+    if return_state and state_out is None:
+        state_out = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = _workspace(lib().gdr_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, m, dt, odt), q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().gdr_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(out),
+                             _ptr(state_out) if return_state else None, B, T, H, dk, dv, chunk, m, dt, odt,
+                             _ptr(workspace), ws_bytes, _stream_handle(stream))
+    check(rc)
+    return out, (state_out if return_state else None)
+
+
+def _chunk_fwd_host(q, k, v, g, beta, S0, *, mode, chunk, return_state, out, out_dtype, state_out, stream):
+    """Host-resident inputs: H2D copies, the device call and D2H copies, all on one stream."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    with torch.cuda.stream(s):
+        d = [None if t is None else t.to(dev, non_blocking=True) for t in (q, k, v, g, beta, S0)]
+        o_d, s_d = chunk_fwd(*d, mode=mode, chunk=chunk, return_state=return_state,
+                             out_dtype=out.dtype if out is not None else out_dtype, stream=s)
+        if out is None:
+            out = torch.empty(o_d.shape, dtype=o_d.dtype, pin_memory=True)
+        out.copy_(o_d, non_blocking=True)
+        if return_state:
+            if state_out is None:
+                state_out = torch.empty(s_d.shape, dtype=s_d.dtype, pin_memory=True)
+            state_out.copy_(s_d, non_blocking=True)
+    return out, (state_out if return_state else None)
+
+
+def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optional[torch.Tensor],
+                beta: torch.Tensor, S: torch.Tensor, *, mode="scalar", out: Optional[torch.Tensor] = None,
+                out_dtype: torch.dtype = torch.float32,
+                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """One recurrent step: q, k [B,H,dk], v [B,H,dv], g [B,H] / [B,H,dk] / None,
+    beta [B,H], S fp32 [B,H,dv,dk] updated in place. Returns o [B,H,dv] (fp32 by default)."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=out_dtype, device=q.device)
+    rc = lib().gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(out), B, H, dk, dv,
+                               _mode(mode), _dtype(q), _dtype(out), _stream_handle(stream))
+    check(rc)
+    return out
+
+
+def sync_status(stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Wait for the stream and raise if a kernel recorded a device-side error."""
+    check(lib().gdr_sync_status(_stream_handle(stream)))

@@ -1,0 +1,228 @@
+// gdr_api.cu -- the library's C ABI (declared in include/gdr.h): argument validation, the
+// per-device status word and dispatch to the kernels. No entry point allocates device memory.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "gdr_internal.cuh"
+
+namespace gdr {
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int ok() {
+    g_last_error[0] = '\0';
+    return GDR_OK;
+}
+
+// Device status word: kernels record the first device-side error here (a bounded wait that
+// expired). A statically sized __device__ variable, so it needs no allocation; each device
+// that loads the library has its own copy. Host code reaches it through its address.
+__device__ int g_status_word = 0;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mutex;
+int* g_status_ptr[kMaxDevices] = {};
+int g_dev_major[kMaxDevices] = {};
+
+// Resolves (once per device) the status word's device address and the compute capability.
+int device_setup(int** status, int* major) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
+    if (dev < 0 || dev >= kMaxDevices) return fail(GDR_ERR_DEVICE, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (g_status_ptr[dev] == nullptr) {
+        int maj = 0;
+        err = cudaDeviceGetAttribute(&maj, cudaDevAttrComputeCapabilityMajor, dev);
+        if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(err));
+        void* p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_status_word);
+        if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "cudaGetSymbolAddress(status): %s", cudaGetErrorString(err));
+        g_dev_major[dev] = maj;
+        g_status_ptr[dev] = static_cast<int*>(p);
+    }
+    *status = g_status_ptr[dev];
+    *major = g_dev_major[dev];
+    return GDR_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+    if (a == nullptr || b == nullptr || na == 0 || nb == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+size_t elem_bytes(int dtype) { return dtype == GDR_BF16 ? 2 : 4; }
+
+int check_enums(int mode, int dtype, int o_dtype) {
+    if (mode != GDR_DECAY_NONE && mode != GDR_DECAY_SCALAR && mode != GDR_DECAY_CHANNEL)
+        return fail(GDR_ERR_INVALID_ARG, "unknown decay mode %d", mode);
+    if (dtype != GDR_F32 && dtype != GDR_BF16) return fail(GDR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+    if (o_dtype != GDR_F32 && o_dtype != GDR_BF16) return fail(GDR_ERR_INVALID_ARG, "unknown o_dtype %d", o_dtype);
+    if (dtype == GDR_F32 && o_dtype == GDR_BF16)
+        return fail(GDR_ERR_UNSUPPORTED, "fp32 inputs with a bf16 output are not supported");
+    return GDR_OK;
+}
+
+int chunk_shape_check(int B, int T, int H, int dk, int dv, int chunk, int mode, int dtype, int o_dtype) {
+    if (int rc = check_enums(mode, dtype, o_dtype)) return rc;
+    if (B <= 0 || T <= 0 || H <= 0 || dk <= 0 || dv <= 0 || chunk <= 0)
+        return fail(GDR_ERR_INVALID_ARG, "sizes must be positive (B=%d T=%d H=%d d_k=%d d_v=%d chunk=%d)", B, T, H,
+                    dk, dv, chunk);
+    if (H > 65535 || B > 65535) return fail(GDR_ERR_UNSUPPORTED, "B and H must be <= 65535");
+    if (!chunk_tc_supported(dk, dv, chunk, dtype, o_dtype) && !chunk_simt_supported(dk, dv, chunk))
+        return fail(GDR_ERR_UNSUPPORTED,
+                    "unsupported shape d_k=%d d_v=%d chunk=%d (supported: chunk 64 with d_k, d_v in {32, 64, 128})",
+                    dk, dv, chunk);
+    return GDR_OK;
+}
+
+}  // namespace
+}  // namespace gdr
+
+using namespace gdr;
+
+extern "C" {
+
+int gdr_version(void) { return 100; }
+
+const char* gdr_last_error(void) { return g_last_error; }
+
+size_t gdr_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int mode, int dtype,
+                                     int o_dtype) {
+    char saved[sizeof(g_last_error)];
+    memcpy(saved, g_last_error, sizeof(saved));
+    const int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype);
+    memcpy(g_last_error, saved, sizeof(saved));
+    if (rc != GDR_OK) return 0;
+    if (chunk_tc_supported(dk, dv, chunk, dtype, o_dtype)) return chunk_tc_workspace_bytes(B, T, H, dk, dv, chunk, mode);
+    return 0;
+}
+
+int gdr_chunk_fwd_launches(int B, int T, int H, int dk, int dv, int chunk, int mode, int dtype, int o_dtype) {
+    char saved[sizeof(g_last_error)];
+    memcpy(saved, g_last_error, sizeof(saved));
+    const int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype);
+    memcpy(g_last_error, saved, sizeof(saved));
+    if (rc != GDR_OK) return 0;
+    return chunk_tc_supported(dk, dv, chunk, dtype, o_dtype) ? chunk_tc_launches(B, T, H, dk, dv, chunk, mode) : 1;
+}
+
+int gdr_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                  const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk,
+                  int mode, int dtype, int o_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    if (int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype)) return rc;
+    if (!q || !k || !v || !beta || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, beta and o must be non-null");
+    if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
+    const void* ptrs[] = {q, k, v, g, beta, S0, o, S_T, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return fail(GDR_ERR_MISALIGNED, "pointer %p is not 16-byte aligned", p);
+    const size_t ntok = (size_t)B * T * H;
+    const size_t eb = elem_bytes(dtype);
+    const size_t bq = ntok * dk * eb, bv = ntok * dv * eb, bb = ntok * sizeof(float);
+    const size_t bo = ntok * dv * elem_bytes(o_dtype);
+    const size_t bg = mode == GDR_DECAY_NONE ? 0 : (mode == GDR_DECAY_SCALAR ? bb : ntok * dk * sizeof(float));
+    const size_t bs = (size_t)B * H * dv * dk * sizeof(float);
+    struct Span { const void* p; size_t n; const char* name; };
+    const Span ins[] = {{q, bq, "q"}, {k, bq, "k"}, {v, bv, "v"}, {mode == GDR_DECAY_NONE ? nullptr : g, bg, "g"},
+                        {beta, bb, "beta"}, {S0, bs, "S0"}};
+    for (const Span& s : ins) {
+        if (overlap(o, bo, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "o overlaps input %s", s.name);
+        if (S_T != S0 && overlap(S_T, bs, s.p, s.n))
+            return fail(GDR_ERR_INVALID_ARG, "S_T overlaps input %s (only S_T == S0 is allowed)", s.name);
+    }
+    if (overlap(o, bo, S_T, bs)) return fail(GDR_ERR_INVALID_ARG, "o overlaps S_T");
+    const bool use_tc = chunk_tc_supported(dk, dv, chunk, dtype, o_dtype);
+    const size_t need = use_tc ? chunk_tc_workspace_bytes(B, T, H, dk, dv, chunk, mode) : 0;
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+        return fail(GDR_ERR_WORKSPACE, "workspace of %zu bytes required (got %zu at %p)", need, workspace_bytes,
+                    workspace);
+    if (need > 0) {
+        for (const Span& s : ins)
+            if (overlap(workspace, need, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "workspace overlaps %s", s.name);
+        if (overlap(workspace, need, o, bo) || overlap(workspace, need, S_T, bs))
+            return fail(GDR_ERR_INVALID_ARG, "workspace overlaps an output");
+    }
+    int* status = nullptr;
+    int major = 0;
+    if (int rc = device_setup(&status, &major)) return rc;
+    if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
+
+    ChunkProblem p{q, k, v, mode == GDR_DECAY_NONE ? nullptr : g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode,
+                   dtype, o_dtype, workspace, workspace_bytes, status, (float)(1.0 / sqrt((double)dk))};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t err = use_tc ? launch_chunk_tc(p, s) : launch_chunk_simt(p, s);
+    if (err != cudaSuccess)
+        return fail(GDR_ERR_CUDA, "%s chunk launch: %s", use_tc ? "tensor-core" : "fp32", cudaGetErrorString(err));
+    return ok();
+}
+
+int gdr_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta, float* S,
+                    void* o, int B, int H, int dk, int dv, int mode, int dtype, int o_dtype, void* stream) {
+    if (int rc = check_enums(mode, dtype, o_dtype)) return rc;
+    if (B <= 0 || H <= 0 || dk <= 0 || dv <= 0)
+        return fail(GDR_ERR_INVALID_ARG, "sizes must be positive (B=%d H=%d d_k=%d d_v=%d)", B, H, dk, dv);
+    if ((size_t)B * H > 0x7fffffffu) return fail(GDR_ERR_UNSUPPORTED, "B*H too large");
+    if (!decode_supported(dk, dv))
+        return fail(GDR_ERR_UNSUPPORTED, "unsupported d_k=%d (supported: 32, 64, 128, 256)", dk);
+    if (!q || !k || !v || !beta || !S || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, beta, S and o must be non-null");
+    if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
+    const void* ptrs[] = {q, k, v, g, beta, S, o};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return fail(GDR_ERR_MISALIGNED, "pointer %p is not 16-byte aligned", p);
+    const size_t nh = (size_t)B * H, eb = elem_bytes(dtype);
+    const size_t bs = nh * dv * dk * sizeof(float), bo = nh * dv * elem_bytes(o_dtype);
+    struct Span { const void* p; size_t n; const char* name; };
+    const Span ins[] = {{q, nh * dk * eb, "q"}, {k, nh * dk * eb, "k"}, {v, nh * dv * eb, "v"},
+                        {mode == GDR_DECAY_NONE ? nullptr : g,
+                         mode == GDR_DECAY_CHANNEL ? nh * dk * sizeof(float) : nh * sizeof(float), "g"},
+                        {beta, nh * sizeof(float), "beta"}};
+    for (const Span& s : ins) {
+        if (overlap(S, bs, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "S overlaps input %s", s.name);
+        if (overlap(o, bo, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "o overlaps input %s", s.name);
+    }
+    if (overlap(o, bo, S, bs)) return fail(GDR_ERR_INVALID_ARG, "o overlaps S");
+    int* status = nullptr;
+    int major = 0;
+    if (int rc = device_setup(&status, &major)) return rc;
+    if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
+    DecodeProblem p{q, k, v, mode == GDR_DECAY_NONE ? nullptr : g, beta, S, o, B, H, dk, dv, mode, dtype, o_dtype,
+                    status, (float)(1.0 / sqrt((double)dk))};
+    const cudaError_t err = launch_decode(p, static_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
+    return ok();
+}
+
+int gdr_sync_status(void* stream) {
+    int* status = nullptr;
+    int major = 0;
+    if (int rc = device_setup(&status, &major)) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t err = cudaStreamSynchronize(s);
+    if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "stream error: %s", cudaGetErrorString(err));
+    int h = 0;
+    err = cudaMemcpyAsync(&h, status, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (err == cudaSuccess) err = cudaMemsetAsync(status, 0, sizeof(int), s);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+    if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "reading the status word: %s", cudaGetErrorString(err));
+    if (h == GDR_ERR_TIMEOUT) return fail(GDR_ERR_TIMEOUT, "a kernel's bounded wait expired; its outputs are invalid");
+    if (h != 0) return fail(h, "device reported status %d", h);
+    return ok();
+}
+
+}  // extern "C"

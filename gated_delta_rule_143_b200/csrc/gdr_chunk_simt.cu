@@ -1,0 +1,277 @@
+// gdr_chunk_simt.cu -- chunked gated delta-rule forward on the CUDA cores in fp32.
+//
+// This is the exact-precision path (fp32 inputs, fp32 arithmetic, no TF32) and the path for
+// shapes the tensor-core kernel does not take. One CTA owns a slice of DVS rows of one head's
+// state S (rows of S evolve independently given k, beta and alpha) and walks the chunks of
+// that head in order. Per chunk of n <= C tokens (Gamma = inclusive cumulative log-decay,
+// gamma = exp(Gamma)):
+//
+//   A_ri  = beta_r sum_c k_rc k_ic exp(Gamma_rc - Gamma_ic)   (i < r)   strictly lower
+//   P_ri  =        sum_c q_rc k_ic exp(Gamma_rc - Gamma_ic)   (i <= r)  causal incl. diagonal
+//   R     = diag(beta) (V - (K*gamma) S^T)                    right-hand side
+//   Delta = (I + A)^-1 R                                      forward substitution
+//   O     = scale [ (Q*gamma) S^T + P Delta ]
+//   S    <- S Diag(gamma_n) + Delta^T (K * gamma_n / gamma)
+//
+// which is the chunk form of "linear attention and its gated descendants" (Chunkwise
+// Parallel Form) with the WY/UT compact form of a chunk of delta-rule updates ("Linear
+// Attention & DeltaNet", item 3): (I + A)^-1 applied to R gives U - W S^T directly.
+// Pairwise decays exp(Gamma_r - Gamma_i) with i <= r never exceed 1, so any g <= 0 is safe.
+#include "gdr_internal.cuh"
+
+namespace gdr {
+namespace {
+
+constexpr int kC = 64;        // chunk length
+constexpr int kDVS = 32;      // state rows per CTA
+constexpr int kThreads = 256;
+
+template <int DK>
+struct SimtSmem {
+    static constexpr int kLd = DK + 1;        // padded row stride of K, Q, Gamma, S
+    static constexpr int kLdC = kC + 1;       // padded stride of A, P
+    static constexpr int kLdV = kDVS + 1;     // padded stride of the value slice
+    static constexpr size_t floats =
+        2 * kC * kLd          // K, Q
+        + kC * kLd            // Gamma (per channel; scalar mode uses column 0)
+        + kDVS * kLd          // S slice
+        + 2 * kC * kLdV       // R/Delta, O_inter
+        + 2 * kC * kLdC       // A, P
+        + 2 * kC;             // beta, tail decay (scalar)
+    static constexpr size_t bytes = floats * sizeof(float);
+};
+
+template <typename Tin, typename Tout, int MODE, int DK>
+__global__ void __launch_bounds__(kThreads)
+chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+                  const float* __restrict__ g, const float* __restrict__ beta, const float* S0,
+                  Tout* __restrict__ o, float* S_T, int T, int H, int dv, float scale) {
+    using L = SimtSmem<DK>;
+    extern __shared__ float smem[];
+    float* sK = smem;
+    float* sQ = sK + kC * L::kLd;
+    float* sG = sQ + kC * L::kLd;
+    float* sS = sG + kC * L::kLd;
+    float* sR = sS + kDVS * L::kLd;
+    float* sOi = sR + kC * L::kLdV;
+    float* sA = sOi + kC * L::kLdV;
+    float* sP = sA + kC * L::kLdC;
+    float* sBeta = sP + kC * L::kLdC;
+    float* sTail = sBeta + kC;
+
+    const int tid = threadIdx.x;
+    const int j0 = blockIdx.x * kDVS;           // first state row of this CTA
+    const int h = blockIdx.y;
+    const int b = blockIdx.z;
+    const int nrows = min(kDVS, dv - j0);
+    const size_t bh = (size_t)b * H + h;
+
+    // initial state slice
+    for (int idx = tid; idx < kDVS * DK; idx += kThreads) {
+        const int j = idx / DK, c = idx % DK;
+        float s = 0.f;
+        if (S0 != nullptr && j < nrows) s = S0[(bh * dv + j0 + j) * DK + c];
+        sS[j * L::kLd + c] = s;
+    }
+
+    for (int c0 = 0; c0 < T; c0 += kC) {
+        const int n = min(kC, T - c0);
+        __syncthreads();
+        // ---- stage the chunk: K, Q, value slice, beta, cumulative log-decay
+        for (int idx = tid; idx < n * DK; idx += kThreads) {
+            const int r = idx / DK, c = idx % DK;
+            const size_t tok = ((size_t)b * T + c0 + r) * H + h;
+            sK[r * L::kLd + c] = load_f32(k + tok * DK + c);
+            sQ[r * L::kLd + c] = load_f32(q + tok * DK + c);
+        }
+        for (int idx = tid; idx < n * kDVS; idx += kThreads) {
+            const int r = idx / kDVS, j = idx % kDVS;
+            const size_t tok = ((size_t)b * T + c0 + r) * H + h;
+            sR[r * L::kLdV + j] = (j < nrows) ? load_f32(v + tok * dv + j0 + j) : 0.f;
+        }
+        for (int r = tid; r < n; r += kThreads) sBeta[r] = beta[((size_t)b * T + c0 + r) * H + h];
+        if (MODE == GDR_DECAY_SCALAR) {
+            if (tid == 0) {
+                float acc = 0.f;
+                for (int r = 0; r < n; ++r) {
+                    acc += g[((size_t)b * T + c0 + r) * H + h];
+                    sG[r * L::kLd] = acc;
+                }
+            }
+        } else if (MODE == GDR_DECAY_CHANNEL) {
+            for (int c = tid; c < DK; c += kThreads) {
+                float acc = 0.f;
+                for (int r = 0; r < n; ++r) {
+                    acc += g[(((size_t)b * T + c0 + r) * H + h) * DK + c];
+                    sG[r * L::kLd + c] = acc;
+                }
+            }
+        }
+        __syncthreads();
+        if (MODE == GDR_DECAY_SCALAR) {
+            for (int i = tid; i < n; i += kThreads) sTail[i] = expf(sG[(n - 1) * L::kLd] - sG[i * L::kLd]);
+        }
+
+        // ---- A (strictly lower, beta_r folded in) and P (causal incl. diagonal)
+        for (int idx = tid; idx < kC * kC; idx += kThreads) {
+            const int r = idx / kC, i = idx % kC;
+            float a = 0.f, p = 0.f;
+            if (r < n && i <= r) {
+                const float* kr = sK + r * L::kLd;
+                const float* ki = sK + i * L::kLd;
+                const float* qr = sQ + r * L::kLd;
+                if (MODE == GDR_DECAY_CHANNEL) {
+                    const float* Gr = sG + r * L::kLd;
+                    const float* Gi = sG + i * L::kLd;
+                    for (int c = 0; c < DK; ++c) {
+                        const float kid = ki[c] * expf(Gr[c] - Gi[c]);
+                        a = fmaf(kr[c], kid, a);
+                        p = fmaf(qr[c], kid, p);
+                    }
+                } else {
+                    for (int c = 0; c < DK; ++c) {
+                        a = fmaf(kr[c], ki[c], a);
+                        p = fmaf(qr[c], ki[c], p);
+                    }
+                    if (MODE == GDR_DECAY_SCALAR) {
+                        const float d = expf(sG[r * L::kLd] - sG[i * L::kLd]);
+                        a *= d;
+                        p *= d;
+                    }
+                }
+                a = (i < r) ? sBeta[r] * a : 0.f;
+            }
+            sA[r * L::kLdC + i] = a;
+            sP[r * L::kLdC + i] = p;
+        }
+
+        // ---- R = diag(beta)(V - (K*gamma) S^T) and O_inter = (Q*gamma) S^T
+        for (int idx = tid; idx < n * kDVS; idx += kThreads) {
+            const int r = idx / kDVS, j = idx % kDVS;
+            const float* kr = sK + r * L::kLd;
+            const float* qr = sQ + r * L::kLd;
+            const float* sj = sS + j * L::kLd;
+            float x = 0.f, y = 0.f;
+            if (MODE == GDR_DECAY_CHANNEL) {
+                const float* Gr = sG + r * L::kLd;
+                for (int c = 0; c < DK; ++c) {
+                    const float sg = sj[c] * expf(Gr[c]);
+                    x = fmaf(kr[c], sg, x);
+                    y = fmaf(qr[c], sg, y);
+                }
+            } else {
+                for (int c = 0; c < DK; ++c) {
+                    x = fmaf(kr[c], sj[c], x);
+                    y = fmaf(qr[c], sj[c], y);
+                }
+                if (MODE == GDR_DECAY_SCALAR) {
+                    const float gr = expf(sG[r * L::kLd]);
+                    x *= gr;
+                    y *= gr;
+                }
+            }
+            sR[r * L::kLdV + j] = sBeta[r] * (sR[r * L::kLdV + j] - x);
+            sOi[r * L::kLdV + j] = y;
+        }
+        __syncthreads();
+
+        // ---- forward substitution Delta = (I + A)^-1 R; 8 lanes cooperate on one column
+        {
+            const int j = tid >> 3;        // column 0..31
+            const int sub = tid & 7;
+            for (int r = 1; r < n; ++r) {
+                float part = 0.f;
+                for (int i = sub; i < r; i += 8) part = fmaf(sA[r * L::kLdC + i], sR[i * L::kLdV + j], part);
+                part += __shfl_xor_sync(0xffffffffu, part, 1);
+                part += __shfl_xor_sync(0xffffffffu, part, 2);
+                part += __shfl_xor_sync(0xffffffffu, part, 4);
+                if (sub == 0) sR[r * L::kLdV + j] -= part;
+                __syncwarp();
+            }
+        }
+        __syncthreads();
+
+        // ---- output O = scale [O_inter + P Delta]
+        for (int idx = tid; idx < n * kDVS; idx += kThreads) {
+            const int r = idx / kDVS, j = idx % kDVS;
+            if (j >= nrows) continue;
+            float acc = sOi[r * L::kLdV + j];
+            for (int i = 0; i <= r; ++i) acc = fmaf(sP[r * L::kLdC + i], sR[i * L::kLdV + j], acc);
+            const size_t tok = ((size_t)b * T + c0 + r) * H + h;
+            store_f32(o + tok * dv + j0 + j, scale * acc);
+        }
+
+        // ---- state S <- S Diag(gamma_n) + Delta^T (K * gamma_n / gamma)
+        for (int idx = tid; idx < kDVS * DK; idx += kThreads) {
+            const int j = idx / DK, c = idx % DK;
+            float s = sS[j * L::kLd + c];
+            if (MODE == GDR_DECAY_CHANNEL) {
+                const float Gn = sG[(n - 1) * L::kLd + c];
+                s *= expf(Gn);
+                for (int i = 0; i < n; ++i)
+                    s = fmaf(sR[i * L::kLdV + j], sK[i * L::kLd + c] * expf(Gn - sG[i * L::kLd + c]), s);
+            } else if (MODE == GDR_DECAY_SCALAR) {
+                s *= expf(sG[(n - 1) * L::kLd]);
+                for (int i = 0; i < n; ++i) s = fmaf(sR[i * L::kLdV + j] * sTail[i], sK[i * L::kLd + c], s);
+            } else {
+                for (int i = 0; i < n; ++i) s = fmaf(sR[i * L::kLdV + j], sK[i * L::kLd + c], s);
+            }
+            sS[j * L::kLd + c] = s;
+        }
+    }
+    __syncthreads();
+    if (S_T != nullptr) {
+        for (int idx = tid; idx < nrows * DK; idx += kThreads) {
+            const int j = idx / DK, c = idx % DK;
+            S_T[(bh * dv + j0 + j) * DK + c] = sS[j * L::kLd + c];
+        }
+    }
+}
+
+template <typename Tin, typename Tout, int MODE, int DK>
+cudaError_t launch_typed(const ChunkProblem& p, cudaStream_t stream) {
+    auto kern = chunk_simt_kernel<Tin, Tout, MODE, DK>;
+    const size_t smem = SimtSmem<DK>::bytes;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    dim3 grid((p.dv + kDVS - 1) / kDVS, p.H, p.B);
+    kern<<<grid, kThreads, smem, stream>>>(
+        static_cast<const Tin*>(p.q), static_cast<const Tin*>(p.k), static_cast<const Tin*>(p.v), p.g, p.beta,
+        p.S0, static_cast<Tout*>(p.o), p.S_T, p.T, p.H, p.dv, p.scale);
+    return cudaGetLastError();
+}
+
+template <typename Tin, typename Tout, int MODE>
+cudaError_t launch_mode(const ChunkProblem& p, cudaStream_t stream) {
+    switch (p.dk) {
+        case 32: return launch_typed<Tin, Tout, MODE, 32>(p, stream);
+        case 64: return launch_typed<Tin, Tout, MODE, 64>(p, stream);
+        case 128: return launch_typed<Tin, Tout, MODE, 128>(p, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename Tin, typename Tout>
+cudaError_t launch_dtype(const ChunkProblem& p, cudaStream_t stream) {
+    switch (p.mode) {
+        case GDR_DECAY_NONE: return launch_mode<Tin, Tout, GDR_DECAY_NONE>(p, stream);
+        case GDR_DECAY_SCALAR: return launch_mode<Tin, Tout, GDR_DECAY_SCALAR>(p, stream);
+        case GDR_DECAY_CHANNEL: return launch_mode<Tin, Tout, GDR_DECAY_CHANNEL>(p, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+bool chunk_simt_supported(int dk, int dv, int chunk) {
+    return (dk == 32 || dk == 64 || dk == 128) && (dv == 32 || dv == 64 || dv == 128) && chunk == kC;
+}
+
+cudaError_t launch_chunk_simt(const ChunkProblem& p, cudaStream_t stream) {
+    if (p.dtype == GDR_BF16 && p.o_dtype == GDR_BF16) return launch_dtype<__nv_bfloat16, __nv_bfloat16>(p, stream);
+    if (p.dtype == GDR_BF16 && p.o_dtype == GDR_F32) return launch_dtype<__nv_bfloat16, float>(p, stream);
+    if (p.dtype == GDR_F32 && p.o_dtype == GDR_F32) return launch_dtype<float, float>(p, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace gdr

@@ -1,0 +1,83 @@
+// gdr_internal.cuh -- declarations shared by the library's CUDA translation units.
+// Not installed; the public interface is include/gdr.h.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "gdr.h"
+
+namespace gdr {
+
+// Everything one chunked-forward launch needs. Pointers are device pointers.
+struct ChunkProblem {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* g;
+    const float* beta;
+    const float* S0;
+    void* o;
+    float* S_T;
+    int B, T, H, dk, dv, chunk, mode, dtype, o_dtype;
+    void* workspace;
+    size_t workspace_bytes;
+    int* status;  // device status word (first error wins)
+    float scale;
+};
+
+struct DecodeProblem {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* g;
+    const float* beta;
+    float* S;
+    void* o;
+    int B, H, dk, dv, mode, dtype, o_dtype;
+    int* status;
+    float scale;
+};
+
+// Device status codes written by kernels (mirror gdr_status).
+constexpr int kStatusTimeout = GDR_ERR_TIMEOUT;
+
+__device__ __forceinline__ void report_status(int* status, int code) {
+    if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+template <typename T>
+__device__ __forceinline__ float load_f32(const T* p);
+template <>
+__device__ __forceinline__ float load_f32<float>(const float* p) { return *p; }
+template <>
+__device__ __forceinline__ float load_f32<__nv_bfloat16>(const __nv_bfloat16* p) {
+    return __bfloat162float(*p);
+}
+
+template <typename T>
+__device__ __forceinline__ void store_f32(T* p, float x);
+template <>
+__device__ __forceinline__ void store_f32<float>(float* p, float x) { *p = x; }
+template <>
+__device__ __forceinline__ void store_f32<__nv_bfloat16>(__nv_bfloat16* p, float x) {
+    *p = __float2bfloat16_rn(x);
+}
+
+// CUDA-core fp32 chunked forward (any supported shape, fp32 or bf16 inputs).
+bool chunk_simt_supported(int dk, int dv, int chunk);
+cudaError_t launch_chunk_simt(const ChunkProblem& p, cudaStream_t stream);
+
+// Tensor-core (tcgen05) chunked forward: bf16, d_k = d_v = 128, chunk = 64.
+bool chunk_tc_supported(int dk, int dv, int chunk, int dtype, int o_dtype);
+size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int mode);
+cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream);
+int chunk_tc_launches(int B, int T, int H, int dk, int dv, int chunk, int mode);
+
+// Bandwidth-bound decode step.
+bool decode_supported(int dk, int dv);
+cudaError_t launch_decode(const DecodeProblem& p, cudaStream_t stream);
+
+}  // namespace gdr

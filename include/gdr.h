@@ -1,0 +1,151 @@
+/*
+ * gdr.h -- C ABI of the gated delta-rule mixer library (libgdr.so, NVIDIA B200 / sm_100a).
+ *
+ * The operation. Per head, with state S in R^{d_v x d_k} (value-by-key, read as o = S q):
+ *
+ *     S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = S_t q_t / sqrt(d_k)                     (read after the token's write)
+ *
+ * alpha_t = exp(g_t): 1 for DeltaNet, a per-head scalar for Gated DeltaNet, a per-key-channel
+ * vector for Kimi Delta Attention. Sources: "linear attention and its gated descendants",
+ * sections DeltaNet, Gated DeltaNet and Kimi Delta Attention (update rules and the
+ * key-dimension decay); "Linear Attention Architectures: Mechanisms, Trade-offs, and
+ * Cross-Layer Routing", Sec. 3 (the diagonal decay multiplies the memory on the right, along
+ * the key-feature dimension); "Linear Attention & DeltaNet", How it works, items 3-4. The
+ * 1/sqrt(d_k) read scale is fixed by this library (the pages read o = S q unscaled).
+ *
+ * Conventions shared by every entry point:
+ *  - All pointers are DEVICE pointers unless stated, owned by the caller, contiguous
+ *    row-major, and 16-byte aligned. The library keeps no pointer after a call returns.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream) and
+ *    the call returns without waiting. Calls on one stream run in order.
+ *  - Return value: GDR_OK (0) or a negative gdr_status. Argument errors are detected on the
+ *    host before anything is enqueued; the message is available from gdr_last_error() on
+ *    the calling thread. Errors found on the device (a bounded wait that expired) are
+ *    recorded in a per-device status word and reported by gdr_sync_status(). Nothing in
+ *    the library traps, aborts or exits.
+ *  - No entry point allocates device memory on the call path: scratch space is the
+ *    caller's `workspace`. The status word is a statically sized device variable.
+ */
+#ifndef GDR_H_
+#define GDR_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDR_OK = 0,
+    GDR_ERR_INVALID_ARG = -1,  /* null pointer, non-positive size, bad enum, S_T overlaps an input */
+    GDR_ERR_UNSUPPORTED = -2,  /* shape outside what the kernels implement (see each entry point) */
+    GDR_ERR_MISALIGNED = -3,   /* a pointer not 16-byte aligned */
+    GDR_ERR_WORKSPACE = -4,    /* workspace missing or smaller than *_workspace_bytes() */
+    GDR_ERR_CUDA = -5,         /* a CUDA runtime call or launch failed (message has the CUDA error) */
+    GDR_ERR_TIMEOUT = -6,      /* a device-side bounded wait expired (reported by gdr_sync_status) */
+    GDR_ERR_DEVICE = -7        /* the current device is not an sm_100 part */
+} gdr_status;
+
+typedef enum {
+    GDR_DECAY_NONE = 0,     /* DeltaNet: alpha = 1, g unused (may be NULL) */
+    GDR_DECAY_SCALAR = 1,   /* Gated DeltaNet: g is [.., H] (one log-decay per head and token) */
+    GDR_DECAY_CHANNEL = 2   /* Kimi Delta Attention: g is [.., H, d_k] (per key channel) */
+} gdr_decay_mode;
+
+typedef enum {
+    GDR_F32 = 0,   /* float32 */
+    GDR_BF16 = 1   /* bfloat16 */
+} gdr_dtype;
+
+/* Element types: `dtype` is the type of q, k, v; `o_dtype` the type of the output o. Supported
+ * pairs: (F32, F32), (BF16, F32) and (BF16, BF16). Arithmetic is fp32 (fp32 accumulation, fp32
+ * state) in every case. A bf16 output adds its own rounding (up to 2^-8 relative per element)
+ * on top of the computation's error. */
+
+/*
+ * gdr_chunk_fwd -- chunkwise-parallel forward over a whole sequence (training / prefill form).
+ *
+ * Defined by: "linear attention and its gated descendants", Chunkwise Parallel Form (state
+ * carried across chunk boundaries, a masked intra-chunk part, chunk size C) generalised to the
+ * delta rule through the compact WY/UT form of a chunk of updates ("Linear Attention &
+ * DeltaNet", item 3): per chunk, T = (I + strictly_lower(diag(beta) (K*gamma)(K/gamma)^T))^-1,
+ * W = T diag(beta)(K*gamma), U = T diag(beta) V, Delta = U - W S^T,
+ * O = [(Q*gamma) S^T + (M * (Q*gamma)(K/gamma)^T) Delta] / sqrt(d_k) with M causal including
+ * the diagonal, and S <- S Diag(gamma_C) + Delta^T (K * gamma_C/gamma), where gamma_r is the
+ * exponential of the inclusive cumulative log-decay inside the chunk. The result equals the
+ * token-by-token recurrence above up to rounding.
+ *
+ *   q, k      [B, T, H, d_k]   dtype            queries and keys (the caller applies any
+ *                                               feature map / normalisation)
+ *   v         [B, T, H, d_v]   dtype            values
+ *   g         fp32 log-decay (<= 0 for a decay): [B, T, H] for SCALAR, [B, T, H, d_k] for
+ *             CHANNEL, ignored (may be NULL) for NONE. alpha = exp(g).
+ *   beta      [B, T, H]        fp32             write strength, normally in [0, 1]
+ *   S0        [B, H, d_v, d_k] fp32, or NULL for a zero initial state
+ *   o         [B, T, H, d_v]   o_dtype          output (written)
+ *   S_T       [B, H, d_v, d_k] fp32, or NULL; the state after the last token. It may be the
+ *             same pointer as S0 (in-place carry); any other overlap with an input is an error.
+ *   B, T, H   batch, tokens, heads (T may be any value >= 1; a ragged last chunk is masked)
+ *   dtype, o_dtype  element types of q/k/v and of o (see gdr_dtype).
+ *   d_k, d_v  head dims. Supported: bf16 with d_k = d_v = 128 and chunk = 64 runs on the
+ *             tensor cores (tcgen05); otherwise d_k, d_v in {32, 64, 128} run on an fp32
+ *             CUDA-core path (fp32 accumulation, no TF32). Anything else: GDR_ERR_UNSUPPORTED.
+ *   chunk     chunk size C; 64 is the supported value.
+ *   workspace device scratch of at least gdr_chunk_fwd_workspace_bytes(...) bytes (may be
+ *             NULL when that is 0). Contents on entry do not matter; the library does not
+ *             keep it after the enqueued work completes. Two calls in flight at the same time
+ *             must not share one workspace.
+ */
+int gdr_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                  const float* S0, void* o, float* S_T, int B, int T, int H, int d_k, int d_v,
+                  int chunk, int mode, int dtype, int o_dtype, void* workspace,
+                  size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace gdr_chunk_fwd needs for this problem (0 if none). Returns 0 for
+ * arguments gdr_chunk_fwd would reject. Host-only; enqueues nothing. */
+size_t gdr_chunk_fwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, int mode,
+                                     int dtype, int o_dtype);
+
+/*
+ * gdr_decode_step -- one recurrent step for a batch of states (the decoding view).
+ *
+ * Defined by: "linear attention and its gated descendants", Recurrent Linear Attention for
+ * Inference (constant-size state, fixed cost per token) and the update rules above; "Linear
+ * Attention & DeltaNet", minimal pseudocode (one update then one read per token).
+ * Per (b, h) and per row j of S:  s_bar = s_j * alpha;  p = s_bar . k;  a = s_bar . q;
+ * delta = beta (v_j - p);  o_j = (a + delta (k . q)) / sqrt(d_k);  s_j <- s_bar + delta k.
+ * S is read once and written once.
+ *
+ *   q, k   [B, H, d_k] dtype;  v [B, H, d_v] dtype;  beta [B, H] fp32
+ *   g      [B, H] (SCALAR) or [B, H, d_k] (CHANNEL) fp32, ignored for NONE
+ *   S      [B, H, d_v, d_k] fp32, updated in place
+ *   o      [B, H, d_v] o_dtype (written); dtype / o_dtype pairs as for gdr_chunk_fwd
+ *   d_k in {32, 64, 128, 256}, d_v >= 1.
+ */
+int gdr_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                    float* S, void* o, int B, int H, int d_k, int d_v, int mode, int dtype,
+                    int o_dtype, void* stream);
+
+/* Number of kernel launches one gdr_chunk_fwd call makes for this problem (0 if it would be
+ * rejected). Host-only. */
+int gdr_chunk_fwd_launches(int B, int T, int H, int d_k, int d_v, int chunk, int mode, int dtype,
+                           int o_dtype);
+
+/* Waits for `stream`, then reads and clears the calling device's status word. Returns
+ * GDR_OK, GDR_ERR_TIMEOUT (a kernel's bounded wait expired; its outputs are invalid) or
+ * GDR_ERR_CUDA (the stream reported a CUDA error). */
+int gdr_sync_status(void* stream);
+
+/* Message for the last non-zero return on the calling thread ("" if none). The pointer stays
+ * valid until the next gdr_* call on the same thread. */
+const char* gdr_last_error(void);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int gdr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H_ */

@@ -1,0 +1,95 @@
+"""Host-side checks of the C ABI (CPU only: nothing here launches a kernel).
+
+The library must load, export every function include/gdr.h declares, and turn
+bad arguments into error codes before touching the device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_143_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdr.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(gdr_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    for want in ("gdr_chunk_fwd", "gdr_chunk_fwd_workspace_bytes", "gdr_decode_step", "gdr_sync_status",
+                 "gdr_last_error", "gdr_version"):
+        assert want in names
+    assert set(names) == set(_lib.SIGNATURES), "binding signatures and header disagree"
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = _lib.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.gdr_version() >= 100
+
+
+def test_library_links_no_oracle_code():
+    """The product library and the oracle share nothing: no oracle symbol in libgdr.so."""
+    data = open(_lib.LIB_PATH, "rb").read()
+    assert b"gdr_oracle" not in data
+
+
+def _chunk(**kw):
+    """Calls gdr_chunk_fwd with fake addresses. Only ever used with an argument error."""
+    M = 1 << 24  # fake, widely spaced addresses: every case below fails validation on the host
+    a = dict(q=1 * M, k=2 * M, v=3 * M, g=4 * M, beta=5 * M, S0=None, o=6 * M, S_T=None, B=1, T=64, H=1, dk=128, dv=128,
+             chunk=64, mode=1, dtype=1, odt=0, ws=None, wsb=0, stream=None)
+    a.update(kw)
+    lib = _lib.lib()
+    return lib.gdr_chunk_fwd(a["q"], a["k"], a["v"], a["g"], a["beta"], a["S0"], a["o"], a["S_T"], a["B"], a["T"],
+                             a["H"], a["dk"], a["dv"], a["chunk"], a["mode"], a["dtype"], a["odt"], a["ws"],
+                             a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), -1), (dict(T=0), -1), (dict(H=-1), -1), (dict(dk=0), -1),
+    (dict(mode=7), -1), (dict(dtype=3), -1), (dict(odt=5), -1), (dict(dtype=0, odt=1), -2),
+    (dict(dk=96), -2), (dict(dv=256), -2), (dict(chunk=32), -2),
+    (dict(q=None), -1), (dict(beta=None), -1), (dict(o=None), -1), (dict(g=None), -1),
+    (dict(q=(1 << 24) + 2), -3), (dict(o=(6 << 24) + 4), -3),
+])
+def test_chunk_fwd_rejects_bad_arguments_on_host(kw, code):
+    assert _chunk(**kw) == code
+    assert len(_lib.lib().gdr_last_error()) > 0
+
+
+def test_chunk_fwd_rejects_output_aliasing_an_input():
+    # o overlapping q is an error (addresses are never dereferenced: it fails on the host)
+    assert _chunk(o=1 << 24) == -1
+    assert b"overlaps" in _lib.lib().gdr_last_error()
+
+
+def test_workspace_query_is_host_only():
+    lib = _lib.lib()
+    assert lib.gdr_chunk_fwd_workspace_bytes(0, 64, 1, 128, 128, 64, 1, 1, 0) == 0  # invalid -> 0
+    n = lib.gdr_chunk_fwd_workspace_bytes(8, 4096, 8, 128, 128, 64, 1, 1, 0)
+    assert n >= 0 and n < (1 << 34)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), -1), (dict(dk=48), -2), (dict(mode=5), -1), (dict(S=None), -1), (dict(S=20), -3),
+])
+def test_decode_rejects_bad_arguments_on_host(kw, code):
+    a = dict(q=16, k=32, v=48, g=64, beta=80, S=1 << 20, o=1 << 21, B=2, H=2, dk=128, dv=128, mode=1, dtype=1, odt=0)
+    a.update(kw)
+    rc = _lib.lib().gdr_decode_step(a["q"], a["k"], a["v"], a["g"], a["beta"], a["S"], a["o"], a["B"], a["H"],
+                                    a["dk"], a["dv"], a["mode"], a["dtype"], a["odt"], None)
+    assert rc == code
+
+
+def test_error_object_carries_status_name():
+    e = _lib.GdrError(-3, "x")
+    assert e.status == "GDR_ERR_MISALIGNED" and "x" in str(e)

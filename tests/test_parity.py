@@ -1,0 +1,210 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs, element by element, at small ragged sizes and at the full
+workload sizes the bench times.
+
+Bar: max |GPU - oracle| <= 1e-4 * rms(oracle) for fp32 inputs and
+<= 2e-2 * rms(oracle) for bf16 inputs, for o and for the final state S_T.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_143_b200 as gdr
+import oracle
+from gated_delta_rule_143_b200.inputs import (CHUNK_WORKLOADS, DECODE_WORKLOADS, WORKLOAD_SEEDS,
+                                              make_chunk_inputs, make_decode_state, make_decode_step,
+                                              workload_inputs)
+from gpu_util import BF16_HALF_ULP, TOL, guard_ok, guarded_empty, rel_err, run_chunk, to_dev
+
+pytestmark = pytest.mark.gpu
+
+MODES = ("none", "scalar", "channel")
+
+
+def check_chunk(x, mode, dtype, S0=None, label=""):
+    o, st = run_chunk(x, mode, S0=S0)
+    s0 = x["S0"] if S0 is None else S0
+    o_ref, s_ref = oracle.recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], mode, S0=s0)
+    assert not np.isnan(o).any(), f"{label}: unwritten or NaN output"
+    eo, _ = rel_err(o, o_ref)
+    es, _ = rel_err(st, s_ref)
+    assert eo <= TOL[dtype], f"{label}: o max err {eo:.3e} * rms > {TOL[dtype]}"
+    assert es <= TOL[dtype], f"{label}: S_T max err {es:.3e} * rms > {TOL[dtype]}"
+    return eo, es
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("dtype,d", [("f32", 64), ("f32", 128), ("f32", 32), ("bf16", 64), ("bf16", 128)])
+@pytest.mark.parametrize("T", [1, 63, 200])
+@pytest.mark.parametrize("with_s0", [False, True])
+def test_chunk_small(mode, dtype, d, T, with_s0):
+    """Several chunks plus a ragged tail; T = 1 and T = C - 1 edge cases."""
+    seed = 1000 + 100 * MODES.index(mode) + d + T + (7 if with_s0 else 0) + (3 if dtype == "bf16" else 0)
+    x = make_chunk_inputs(2, T, 3, d, d, mode, dtype, seed, s0_std=0.1 if with_s0 else None)
+    check_chunk(x, mode, dtype, label=f"{mode}/{dtype}/d{d}/T{T}")
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_chunk_unequal_head_dims(mode):
+    x = make_chunk_inputs(1, 130, 2, 128, 64, mode, "bf16", 77, s0_std=0.05)
+    check_chunk(x, mode, "bf16")
+    x = make_chunk_inputs(1, 130, 2, 64, 128, mode, "f32", 78, s0_std=0.05)
+    check_chunk(x, mode, "f32")
+
+
+@pytest.mark.parametrize("name", list(CHUNK_WORKLOADS))
+def test_chunk_full_workload(name):
+    """Every named workload at full size, whole output against the oracle."""
+    w = CHUNK_WORKLOADS[name]
+    x = workload_inputs(w)
+    eo, es = check_chunk(x, w.mode, w.dtype, label=name)
+    print(f"{name}: max|do|/rms(o) = {eo:.3e}, max|dS|/rms(S) = {es:.3e}")
+
+
+def test_state_carry_split_and_inplace():
+    """fwd(T1) then fwd(T2, S0 = S_T(T1)) equals fwd(T1+T2); S_T may alias S0."""
+    x = make_chunk_inputs(2, 300, 2, 128, 128, "scalar", "bf16", 91, s0_std=0.05)
+    o_all, s_all = run_chunk(x, "scalar")
+    d = to_dev(x)
+    S = d["S0"].clone()
+    outs = []
+    for sl in (slice(0, 100), slice(100, 300)):
+        part = {k: (None if v is None else v[:, sl].contiguous()) for k, v in d.items() if k != "S0"}
+        o, _ = gdr.chunk_fwd(part["q"], part["k"], part["v"], part["g"], part["beta"], S, mode="scalar",
+                             state_out=S)  # in place
+        outs.append(o)
+    gdr.sync_status()
+    o_split = torch.cat(outs, dim=1).double().cpu().numpy()
+    e1, _ = rel_err(o_split, o_all)
+    e2, _ = rel_err(S.double().cpu().numpy(), s_all)
+    assert e1 <= TOL["bf16"] and e2 <= TOL["bf16"], (e1, e2)
+
+
+def test_alpha_zero_resets():
+    """g = -1e4 (alpha underflows to 0): o_t = scale beta_t (k_t.q_t) v_t."""
+    x = make_chunk_inputs(1, 150, 2, 128, 128, "scalar", "bf16", 92, s0_std=0.1)
+    x["g"] = torch.full_like(x["g"], -1e4)
+    check_chunk(x, "scalar", "bf16")
+
+
+def test_channel_constant_equals_scalar():
+    x = make_chunk_inputs(2, 192, 2, 128, 128, "scalar", "bf16", 93)
+    o1, s1 = run_chunk(x, "scalar")
+    xc = dict(x)
+    xc["g"] = x["g"][..., None].expand(-1, -1, -1, 128).contiguous()
+    o2, s2 = run_chunk(xc, "channel")
+    assert rel_err(o2, o1)[0] <= TOL["bf16"]
+    assert rel_err(s2, s1)[0] <= TOL["bf16"]
+
+
+def test_zero_beta_output_is_decayed_initial_state():
+    x = make_chunk_inputs(1, 128, 2, 128, 128, "channel", "bf16", 94, s0_std=0.1)
+    x["beta"] = torch.zeros_like(x["beta"])
+    check_chunk(x, "channel", "bf16")
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_bf16_output(mode):
+    """bf16 output: each element within the computation bound plus its own bf16 rounding,
+    |o - o_ref| <= 2e-2 rms(o_ref) + 2^-8 |o_ref|."""
+    x = make_chunk_inputs(2, 333, 3, 128, 128, mode, "bf16", 99 + MODES.index(mode), s0_std=0.05)
+    o, st = run_chunk(x, mode, out_dtype=torch.bfloat16)
+    o_ref, s_ref = oracle.recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], mode, S0=x["S0"])
+    rms = np.sqrt(np.mean(o_ref ** 2))
+    excess = np.abs(o - o_ref) - (TOL["bf16"] * rms + BF16_HALF_ULP * np.abs(o_ref))
+    assert excess.max() <= 0, excess.max()
+    assert rel_err(st, s_ref)[0] <= TOL["bf16"]
+
+
+def test_no_state_output():
+    x = make_chunk_inputs(1, 70, 1, 128, 128, "none", "bf16", 95)
+    o, st = run_chunk(x, "none", want_state=False)
+    o_ref, _ = oracle.recurrent(x["q"], x["k"], x["v"], None, x["beta"], "none")
+    assert rel_err(o, o_ref)[0] <= TOL["bf16"]
+
+
+def test_host_tensors_roundtrip():
+    """chunk_fwd on host tensors stages through the device and returns host tensors."""
+    x = make_chunk_inputs(1, 100, 2, 128, 128, "scalar", "bf16", 96)
+    o, st = gdr.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, mode="scalar")
+    torch.cuda.synchronize()
+    assert o.device.type == "cpu" and st.device.type == "cpu"
+    o_ref, s_ref = oracle.recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], "scalar")
+    assert rel_err(o.double().numpy(), o_ref)[0] <= TOL["bf16"]
+    assert rel_err(st.double().numpy(), s_ref)[0] <= TOL["bf16"]
+
+
+# ------------------------------------------------------------- decode -----
+def run_decode_steps(w_B, w_H, dk, dv, mode, dtype, steps, seed, s_std=0.02, out_dtype=torch.float32):
+    from gated_delta_rule_143_b200.inputs import DecodeWorkload
+    w = DecodeWorkload("t", mode, dtype, w_B, w_H, dk, dv, steps, s_std)
+    S0 = make_decode_state(w, seed)
+    S_dev = S0.cuda()
+    S_ref = S0.double().numpy()
+    worst = 0.0
+    for st in range(steps):
+        x = make_decode_step(w, seed, st)
+        d = to_dev(x)
+        o, obuf = guarded_empty((w_B, w_H, dv), out_dtype, "cuda")
+        gdr.decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], S_dev, mode=mode, out=o)
+        gdr.sync_status()
+        assert guard_ok(obuf, o.numel())
+        o_ref, S_ref = oracle.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], S_ref, mode)
+        og = o.double().cpu().numpy()
+        e, rms = rel_err(og, o_ref)
+        worst = max(worst, e)
+        if out_dtype == torch.bfloat16:
+            assert (np.abs(og - o_ref) - TOL[dtype] * rms - BF16_HALF_ULP * np.abs(o_ref)).max() <= 0
+        else:
+            assert e <= TOL[dtype], f"step {st}: o err {e:.3e}"
+    es, _ = rel_err(S_dev.double().cpu().numpy(), S_ref)
+    assert es <= TOL[dtype], f"final state err {es:.3e}"
+    return worst, es
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (32, 40), (256, 96)])
+def test_decode_small(mode, dtype, dk, dv):
+    run_decode_steps(3, 5, dk, dv, mode, dtype, 6, 300 + dk + dv)
+
+
+def test_decode_bf16_output():
+    run_decode_steps(4, 8, 128, 128, "scalar", "bf16", 4, 555, out_dtype=torch.bfloat16)
+
+
+def test_decode_full_workload():
+    """The full decode workload: 256 steps at B=256, H=16 from random fp32 states; o checked at
+    every step and the final states at the end."""
+    w = DECODE_WORKLOADS["gdn_decode_bf16_b256_h16_d128"]
+    worst, es = run_decode_steps(w.B, w.H, w.dk, w.dv, w.mode, w.dtype, w.steps, WORKLOAD_SEEDS[w.name], w.s_std)
+    print(f"decode: worst per-step max|do|/rms = {worst:.3e}, final state {es:.3e}")
+
+
+def test_decode_steps_equal_chunked_forward():
+    """T decode steps from S0 reproduce the chunked forward over the same T tokens."""
+    x = make_chunk_inputs(2, 40, 2, 128, 128, "channel", "bf16", 97, s0_std=0.05)
+    o_fwd, s_fwd = run_chunk(x, "channel")
+    d = to_dev(x)
+    S = d["S0"].clone()
+    outs = []
+    for t in range(40):
+        outs.append(gdr.decode_step(d["q"][:, t].contiguous(), d["k"][:, t].contiguous(), d["v"][:, t].contiguous(),
+                                    d["g"][:, t].contiguous(), d["beta"][:, t].contiguous(), S, mode="channel"))
+    gdr.sync_status()
+    o_dec = torch.stack(outs, dim=1).double().cpu().numpy()
+    assert rel_err(o_dec, o_fwd)[0] <= TOL["bf16"]
+    assert rel_err(S.double().cpu().numpy(), s_fwd)[0] <= TOL["bf16"]
+
+
+# ------------------------------------------------------------- errors -----
+def test_device_errors_are_codes_not_faults():
+    x = to_dev(make_chunk_inputs(1, 64, 1, 128, 128, "scalar", "bf16", 98))
+    with pytest.raises(gdr.GdrError) as e:  # misaligned view of a real buffer
+        q2 = torch.empty(x["q"].numel() + 8, dtype=torch.bfloat16, device="cuda")[1:1 + x["q"].numel()]
+        gdr.chunk_fwd(q2.view_as(x["q"]), x["k"], x["v"], x["g"], x["beta"], None, mode="scalar")
+    assert e.value.code == -3
+    with pytest.raises(gdr.GdrError) as e:
+        gdr.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, mode="scalar", chunk=48)
+    assert e.value.code == -2
+    gdr.sync_status()
