@@ -17,6 +17,7 @@ GDR_OK = 0
 STATUS_NAMES = {
     0: "GDR_OK", -1: "GDR_ERR_INVALID_ARG", -2: "GDR_ERR_UNSUPPORTED", -3: "GDR_ERR_MISALIGNED",
     -4: "GDR_ERR_WORKSPACE", -5: "GDR_ERR_CUDA", -6: "GDR_ERR_TIMEOUT", -7: "GDR_ERR_DEVICE",
+    -8: "GDR_ERR_RANGE",
 }
 DECAY_MODES = {"none": 0, "scalar": 1, "channel": 2}
 DTYPE_F32, DTYPE_BF16 = 0, 1

@@ -221,6 +221,8 @@ int gdr_sync_status(void* stream) {
     if (err == cudaSuccess) err = cudaStreamSynchronize(s);
     if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "reading the status word: %s", cudaGetErrorString(err));
     if (h == GDR_ERR_TIMEOUT) return fail(GDR_ERR_TIMEOUT, "a kernel's bounded wait expired; its outputs are invalid");
+    if (h == GDR_ERR_RANGE)
+        return fail(GDR_ERR_RANGE, "a decay factor left the fp16 operand range (channel gate spread within a chunk)");
     if (h != 0) return fail(h, "device reported status %d", h);
     return ok();
 }

@@ -1,0 +1,186 @@
+// gdr_sm100.cuh -- thin wrappers over the sm_100a instructions the tensor-core kernels use:
+// mbarriers with bounded waits, tcgen05 TMEM allocation / MMA / commit / load, shared-memory
+// matrix descriptors, and TMA tensor loads. Encodings follow the public PTX ISA for sm_100a
+// (tcgen05 instruction descriptor for kind::f16 and the shared-memory matrix descriptor).
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+#include "gdr_internal.cuh"
+
+namespace gdr {
+namespace sm100 {
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ------------------------------------------------------------------ mbarrier --
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wall-clock bound on every wait: a wait that has not completed after this long records
+// GDR_ERR_TIMEOUT in the status word and gives up instead of hanging the GPU.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+// Waits for the phase with the given parity to complete. Returns false (and records a
+// timeout) if it does not complete within kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            report_status(status, kStatusTimeout);
+            return false;
+        }
+    }
+}
+
+// --------------------------------------------------------------------- fences --
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// ----------------------------------------------------------------------- TMEM --
+// Allocation is warp-wide; the allocated base address is written to shared memory.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread t of the warp gets lane (base lane + t).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// ------------------------------------------------------------ MMA descriptors --
+// Shared-memory matrix descriptor (64-bit): start address >> 4 in bits [0,14), leading byte
+// offset >> 4 in [16,30), stride byte offset >> 4 in [32,46), version 1 in [46,48), base offset
+// 0, layout type in [61,64) (2 = 128-byte swizzle).
+constexpr uint64_t kLayoutSw128 = 2;
+
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (kLayoutSw128 << 61);
+}
+
+// Instruction descriptor for kind::f16 with an fp32 accumulator: c_format F32 (bit 4), a_format
+// and b_format in bits 7-9 and 10-12 (0 = f16, 1 = bf16; A and B always share one type), negate A
+// (bit 13), negate B (bit 14), A major (bit 15, 1 = MN-major), B major (bit 16), N >> 3 in bits
+// [17,23), M >> 4 in bits [24,29).
+__host__ __device__ constexpr uint32_t idesc_kind_f16(int M, int N, bool a_mn_major, bool b_mn_major, uint32_t fmt,
+                                                      bool neg_a = false) {
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((neg_a ? 1u : 0u) << 13) | ((a_mn_major ? 1u : 0u) << 15) |
+           ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major,
+                                                  bool neg_a = false) {
+    return idesc_kind_f16(M, N, a_mn_major, b_mn_major, 1u, neg_a);
+}
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn_major, bool b_mn_major,
+                                                 bool neg_a = false) {
+    return idesc_kind_f16(M, N, a_mn_major, b_mn_major, 0u, neg_a);
+}
+
+// D[tmem] (+)= A[smem] * B[smem] (kind::f16: f16 or bf16 operands per the instruction
+// descriptor); issued by one thread.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+        : "memory");
+}
+
+// Arrives on the mbarrier once all previously issued MMAs of this thread have completed.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// ------------------------------------------------------- swizzled tile layouts --
+// (Offsets in bytes for 2-byte elements, f16 or bf16.)
+// 128-byte-swizzled, K-major operand tile of R rows (the M or N index) by 64 elements along K:
+// row r occupies 128 bytes at (r / 8) * 1024 + (r % 8) * 128; its 16-byte chunk c sits at
+// chunk (c ^ (r % 8)). Descriptor: SBO = 1024 (8-row groups), LBO unused (16); a K step of
+// 16 elements advances the start address by 32 bytes. Tiles wider than 64 along K are stored
+// as consecutive 64-wide blocks of R * 128 bytes.
+__host__ __device__ constexpr uint32_t kmajor_off(int r, int k, int R) {
+    return (uint32_t)((k >> 6) * R * 128 + (r >> 3) * 1024 + (r & 7) * 128 + ((((k & 63) >> 3) ^ (r & 7)) << 4) +
+                      ((k & 7) << 1));
+}
+
+// 128-byte-swizzled, MN-major operand tile: K rows by MN elements (MN contiguous). Blocks of
+// 8 K-rows x 64 MN-elements (1 KiB); K-row k of a block at (k % 8) * 128 with its 16-byte
+// chunk c at chunk (c ^ (k % 8)). Blocks along K are SBO = 1024 bytes apart and blocks along MN
+// are LBO = (Krows / 8) * 1024 bytes apart. A K step of 16 rows advances the start by 2048 bytes.
+__host__ __device__ constexpr uint32_t mnmajor_off(int k, int n, int Krows) {
+    return (uint32_t)((n >> 6) * (Krows >> 3) * 1024 + (k >> 3) * 1024 + (k & 7) * 128 +
+                      ((((n & 63) >> 3) ^ (k & 7)) << 4) + ((n & 7) << 1));
+}
+
+}  // namespace sm100
+}  // namespace gdr

@@ -44,7 +44,9 @@ typedef enum {
     GDR_ERR_WORKSPACE = -4,    /* workspace missing or smaller than *_workspace_bytes() */
     GDR_ERR_CUDA = -5,         /* a CUDA runtime call or launch failed (message has the CUDA error) */
     GDR_ERR_TIMEOUT = -6,      /* a device-side bounded wait expired (reported by gdr_sync_status) */
-    GDR_ERR_DEVICE = -7        /* the current device is not an sm_100 part */
+    GDR_ERR_DEVICE = -7,       /* the current device is not an sm_100 part */
+    GDR_ERR_RANGE = -8         /* device-side: a value left the range the kernel supports (the
+                                  channel gate's within-chunk log-decay spread; see gdr_chunk_fwd) */
 } gdr_status;
 
 typedef enum {
@@ -92,6 +94,10 @@ typedef enum {
  *             tensor cores (tcgen05); otherwise d_k, d_v in {32, 64, 128} run on an fp32
  *             CUDA-core path (fp32 accumulation, no TF32). Anything else: GDR_ERR_UNSUPPORTED.
  *   chunk     chunk size C; 64 is the supported value.
+ *   Range: on the tensor-core path the channel gate's decay factors are applied to fp16 operands
+ *             around a mid-chunk reference, so per key channel the cumulative log-decay may vary by
+ *             at most about 22 within one chunk (e.g. g >= -0.35 per token on average); beyond that
+ *             the call reports GDR_ERR_RANGE through gdr_sync_status and its outputs are invalid.
  *   workspace device scratch of at least gdr_chunk_fwd_workspace_bytes(...) bytes (may be
  *             NULL when that is 0). Contents on entry do not matter; the library does not
  *             keep it after the enqueued work completes. Two calls in flight at the same time
@@ -133,8 +139,8 @@ int gdr_chunk_fwd_launches(int B, int T, int H, int d_k, int d_v, int chunk, int
                            int o_dtype);
 
 /* Waits for `stream`, then reads and clears the calling device's status word. Returns
- * GDR_OK, GDR_ERR_TIMEOUT (a kernel's bounded wait expired; its outputs are invalid) or
- * GDR_ERR_CUDA (the stream reported a CUDA error). */
+ * GDR_OK, GDR_ERR_TIMEOUT (a kernel's bounded wait expired; its outputs are invalid),
+ * GDR_ERR_RANGE (see gdr_chunk_fwd) or GDR_ERR_CUDA (the stream reported a CUDA error). */
 int gdr_sync_status(void* stream);
 
 /* Message for the last non-zero return on the calling thread ("" if none). The pointer stays
