@@ -14,6 +14,7 @@ Multi-GPU: every rank runs its own batch (weak scaling, no data-path collective)
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -88,13 +89,21 @@ class ClockSampler:
         self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
 
     def start(self):
+        """Starts sampling every 20 ms and returns once the first sample has arrived (so the
+        samples cover the timed region that follows), or after 5 s."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=self.out, stderr=subprocess.DEVNULL)
+                 "-lms", "20"], stdout=self.out, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
-        self.t0 = time.time()
+        t0 = time.time()
+        while self.proc is not None and time.time() - t0 < 5.0:
+            self.out.flush()
+            if os.path.getsize(self.out.name) > 0:
+                break
+            time.sleep(0.01)
+        self.size0 = os.path.getsize(self.out.name)
 
     def stop(self):
         if self.proc is not None:
@@ -107,6 +116,7 @@ class ClockSampler:
         rows = []
         try:
             with open(self.out.name) as f:
+                f.seek(self.size0)  # only samples taken after start() returned
                 for line in f:
                     parts = [p.strip() for p in line.split(",")]
                     if len(parts) >= 9:
@@ -201,6 +211,8 @@ def run_ours(args):
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
     w = CHUNK_WORKLOADS[WORKLOAD]
+    if args.batch:
+        w = dataclasses.replace(w, B=args.batch)
     stream = torch.cuda.current_stream(dev)
 
     # two resident input sets, each larger than L2; one seed per rank (weak scaling)
@@ -221,6 +233,7 @@ def run_ours(args):
     clocks = ClockSampler(smi_id(dev, local))
     for _ in range(args.warmup):
         step()
+    torch.cuda.synchronize()
     clocks.start()
     ms = time_device(step, args.steps, 0, world, stream)
     clk = clocks.stop()
@@ -242,6 +255,13 @@ def run_ours(args):
                                 "peak_tflops": peaks["bf16_tflops"],
                                 "frac": round(flops / (ms_step * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)},
                 "roofline_us": round(max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)) * 1e6, 2)}
+
+    if args.only == "fwd":
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
+                              "ms_per_step": round(ms_step, 5), "config": {"workload": WORKLOAD, "B": w.B},
+                              "roofline_frac": round(nbytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}))
+        return
 
     # end to end: pinned host inputs -> device -> kernels -> host outputs, every step
     hx = {k: (None if t is None else t.cpu().pin_memory()) for k, t in sets[0].items()}
@@ -382,6 +402,9 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--only", choices=("all", "fwd"), default="all",
+                    help="fwd: time the forward only (no e2e, decode or CPU baseline), for profiling runs")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
