@@ -228,3 +228,57 @@ int gdr_sync_status(void* stream) {
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------- allocation-free variant --
+// gdr_chunk_fwd_noalloc: the tensor-core chunked forward for callers that cannot allocate device
+// memory (see include/gdr.h for who they are). Its scratch is this fixed area, part of the
+// library's device image: every GPU that loads the library holds it until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GDR_NOALLOC_SCRATCH_BYTES];
+
+namespace gdr {
+namespace {
+
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch area on the current device. In host code the array's name is
+// only a host-side stand-in, so the address is looked up once per device, with it current.
+int noalloc_scratch(void** ptr) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
+    if (dev < 0 || dev >= kMaxDevices) return fail(GDR_ERR_DEVICE, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (err != cudaSuccess)
+            return fail(GDR_ERR_CUDA, "cudaGetSymbolAddress(scratch area): %s", cudaGetErrorString(err));
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return GDR_OK;
+}
+
+}  // namespace
+}  // namespace gdr
+
+extern "C" int gdr_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                                     const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv,
+                                     int chunk, int mode, int dtype, int o_dtype, void* stream) {
+    if (int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype)) return rc;
+    if (!chunk_tc_supported(dk, dv, chunk, dtype, o_dtype))
+        return fail(GDR_ERR_UNSUPPORTED,
+                    "gdr_chunk_fwd_noalloc covers the shapes that need scratch (bf16 q/k/v, d_k = d_v = 128, "
+                    "chunk 64); this shape needs none: call gdr_chunk_fwd with a null workspace");
+    const size_t need = chunk_tc_workspace_bytes(B, T, H, dk, dv, chunk, mode);
+    if (need > (size_t)GDR_NOALLOC_SCRATCH_BYTES)
+        return fail(GDR_ERR_UNSUPPORTED,
+                    "this problem needs %zu bytes of scratch but the built-in area holds %zu "
+                    "(B * H * ceil(T / 64) must be <= %zu); use gdr_chunk_fwd with a workspace",
+                    need, (size_t)GDR_NOALLOC_SCRATCH_BYTES,
+                    (size_t)GDR_NOALLOC_SCRATCH_BYTES / (need / ((size_t)B * H * ((T + 63) / 64))));
+    void* ws = nullptr;
+    if (int rc = noalloc_scratch(&ws)) return rc;
+    return gdr_chunk_fwd(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, ws,
+                         (size_t)GDR_NOALLOC_SCRATCH_BYTES, stream);
+}

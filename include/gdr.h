@@ -138,6 +138,39 @@ int gdr_decode_step(const void* q, const void* k, const void* v, const float* g,
 int gdr_chunk_fwd_launches(int B, int T, int H, int d_k, int d_v, int chunk, int mode, int dtype,
                            int o_dtype);
 
+/* Size of the scratch area built into the library for gdr_chunk_fwd_noalloc: 32 MiB of device
+ * memory on every GPU that loads the library, held until the process exits. */
+#define GDR_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * gdr_chunk_fwd_noalloc -- gdr_chunk_fwd for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart; this is a convenience of this library. Some callers cannot
+ * call cudaMalloc for a workspace: a plugin inside a host program that owns all device memory
+ * and hands the plugin only its inputs and outputs; code running in a loop where an allocation
+ * (which may synchronise the device) is not allowed; a program that must not grow its device
+ * footprint after start-up. This entry point takes the same arguments as gdr_chunk_fwd minus the
+ * workspace and uses a fixed scratch area compiled into the library instead
+ * (GDR_NOALLOC_SCRATCH_BYTES, enough for B * H * ceil(T / 64) <= 448 chunks). It allocates
+ * nothing on any call.
+ *
+ *  - Shapes: only those that need scratch (bf16 q/k/v, d_k = d_v = 128, chunk = 64); other
+ *    shapes need none and are rejected with GDR_ERR_UNSUPPORTED (call gdr_chunk_fwd with a null
+ *    workspace for them). A problem needing more scratch than the area holds is rejected with
+ *    GDR_ERR_UNSUPPORTED and a message giving both sizes; nothing is enqueued.
+ *  - Set-up: the first call on each device looks up the area's device address (once per device,
+ *    with that device current). Make that first call before any stream capture.
+ *  - Sharing: every call on a device uses the same area, which keeps the last call's contents.
+ *    Nothing in it needs to start at zero: every byte a call reads there is written earlier by
+ *    the same call, in stream order. Calls whose execution overlaps on the GPU (for example on two
+ *    streams) race on the area and produce wrong results; serialise them.
+ * Errors and everything else: as gdr_chunk_fwd.
+ */
+int gdr_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* S0, void* o, float* S_T, int B, int T,
+                          int H, int d_k, int d_v, int chunk, int mode, int dtype, int o_dtype,
+                          void* stream);
+
 /* Waits for `stream`, then reads and clears the calling device's status word. Returns
  * GDR_OK, GDR_ERR_TIMEOUT (a kernel's bounded wait expired; its outputs are invalid),
  * GDR_ERR_RANGE (see gdr_chunk_fwd) or GDR_ERR_CUDA (the stream reported a CUDA error). */
