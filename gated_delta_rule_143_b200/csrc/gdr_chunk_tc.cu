@@ -1,10 +1,10 @@
 // gdr_chunk_tc.cu -- chunked gated delta-rule forward on the 5th-generation tensor cores.
 //
 // bf16 q/k/v, d_k = d_v = 128, chunk C = 64; fp16 MMA operands, fp32 accumulation (TMEM) and fp32
-// state (registers).
-// The chunk form ("linear attention and its gated descendants", Chunkwise Parallel Form, with the
-// WY/UT compact form of a chunk of delta-rule updates from "Linear Attention & DeltaNet", item 3),
-// with Gamma the inclusive cumulative log-decay inside the chunk and gamma = exp(Gamma):
+// state (registers). The chunk form ("linear attention and its gated descendants", Chunkwise
+// Parallel Form, with the WY/UT compact form of a chunk of delta-rule updates from "Linear
+// Attention & DeltaNet", item 3), with Gamma the inclusive cumulative log-decay inside the chunk
+// and gamma = exp(Gamma):
 //
 //   A  = strictly_lower(diag(beta) (K*gamma)(K/gamma)^T),  T = (I + A)^-1      (UT transform)
 //   W  = T diag(beta) (K*gamma),  U = T diag(beta) V                           (WY factors)
@@ -13,19 +13,28 @@
 //   O  = scale [ (Q*gamma) S^T + P Delta ]
 //   S <- S Diag(gamma_C) + Delta^T (K * gamma_C / gamma)
 //
-// Two kernels. The prep kernel runs one CTA per chunk, all chunks in parallel: it computes the
-// S-independent factors (two tcgen05 GEMM groups around a CUDA-core triangular solve) and writes
-// them to the workspace as ready-to-use, 128-byte-swizzled shared-memory operand images. The state
-// kernel runs one CTA per (b, h) and walks the chunks in order: it bulk-copies each chunk's images
-// into a double-buffered stage and runs the three S-dependent tcgen05 GEMM groups; the fp32 state
-// lives in registers and enters the MMAs as an fp16 copy in shared memory.
+// Work split. A prep pass (one 128-thread pipeline per chunk, all chunks independent) computes the
+// S-independent factors and writes them as ready-to-use, 128-byte-swizzled fp16 operand images
+// (the "hand-off block"); a state pass (one 512-thread CTA per (b, h)) walks the chunks in order,
+// copies each block into shared memory with bulk copies and runs the S-dependent MMAs; the fp32
+// state lives in registers and enters the MMAs as an fp16 copy.
 //
-// Decay handling: for the scalar gate the Gram products use raw K, Q and are scaled elementwise by
-// exp(Gamma_r - Gamma_i) <= 1 afterwards (safe for any g <= 0). For the channel gate the factors
-// are folded into the operands around a mid-chunk reference Gamma_ref:
-// (K e^{Gamma - Gamma_ref})(K e^{Gamma_ref - Gamma})^T. A factor above the fp16 range (a
-// within-chunk spread of the cumulative log-decay beyond about 22 on one channel) is detected and
+// Prep, per chunk: TMA loads of the bf16 K, Q, V tiles straight into the swizzled K-major layout;
+// Gram products [K; Q] K^T on tcgen05 (bf16 operands for the scalar gate and DeltaNet, exact with
+// fp32 accumulation; fp16 decay-factored operands for the channel gate); A and P from TMEM with the
+// pairwise decays; T = (I + A)^-1 by forward substitution on 16x16 diagonal blocks and two levels
+// of block merges on warp MMAs (tf32); then W = [T diag(beta); 0] (K*gamma) (M = 128, N = d_k) and
+// U^T = V^T (T diag(beta))^T (M = d_v) on tcgen05.
+//
+// Decay handling: the scalar gate's Gram products are scaled elementwise by exp(Gamma_r - Gamma_i)
+// <= 1 (safe for any g <= 0). The channel gate's factors are folded into the operands around a
+// mid-chunk reference: (K e^{Gamma - Gamma_ref})(K e^{Gamma_ref - Gamma})^T; a factor beyond the
+// fp16 range (a within-chunk spread of the cumulative log-decay above about 22 on one channel) is
 // reported as GDR_ERR_RANGE through the status word.
+//
+// Operands are fp16, not bf16: with bf16 operands the rounding of the intermediate factors alone
+// exceeded the 2e-2 * rms(o) parity bar; fp16 holds the bf16 inputs exactly at these ranges and
+// runs at the same tensor-core rate.
 #include <cuda_fp16.h>
 
 #include "gdr_sm100.cuh"
@@ -37,58 +46,67 @@ using namespace sm100;
 
 constexpr int kC = 64;    // chunk length
 constexpr int kD = 128;   // d_k = d_v
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kF16Max = 65504.f;
 
-// Per-chunk hand-off block in the workspace (byte offsets). Every image is laid out exactly as
-// the state kernel's MMAs read it from shared memory.
-constexpr uint32_t kOffWT = 0;            // W^T:          MN-major, K = d_k (128 rows) x N = C (64)
-constexpr uint32_t kOffQG = 16384;        // Q*gamma:      K-major,  N = C (64 rows)  x K = d_k (128)
-constexpr uint32_t kOffKT = 32768;        // K*gamma_C/gamma: MN-major, K = C (64 rows) x N = d_k (128)
-constexpr uint32_t kOffUT = 49152;        // U^T:          plain row-major fp16 [d_v][C]
-constexpr uint32_t kOffP = 65536;         // P:            K-major,  N = C (r, 64 rows) x K = C (i, 64)
-constexpr uint32_t kOffGam = 73728;       // gamma_C:      128 fp32 (per key channel)
-constexpr uint32_t kHandoffBytes = 74240;   // bytes copied per chunk (multiple of 16)
-constexpr uint32_t kHandoffStride = 74752;  // per-chunk stride (multiple of 1024)
+// ------------------------------------------------------------------ hand-off block --
+// Per-chunk block in the workspace (byte offsets). Images are laid out exactly as the state
+// pass's MMAs read them. Part A (double-buffered in the state pass) is [0, kPartA); U^T follows.
+constexpr uint32_t kOffWQ = 0;          // [W; Q*gamma]  fp16 K-major, 128 rows (r | 64 + r) x 128 (d_k)
+constexpr uint32_t kOffP = 32768;       // P             fp16 K-major, 64 rows (r) x 64 (i)
+constexpr uint32_t kOffKT = 40960;      // K*gamma_C/gamma fp16 MN-major, 64 rows (i) x 128 (d_k)
+constexpr uint32_t kOffGam = 57344;     // gamma_C       fp32 [128]
+constexpr uint32_t kPartA = 57856;      // bytes of part A (multiple of 16)
+constexpr uint32_t kOffUT = 58368;      // U^T           fp16 K-major, 128 rows (d_v) x 64 (r)
+constexpr uint32_t kHandoffStride = 74752;  // multiple of 1024
 
+// ------------------------------------------------------------------ prep pipeline --
 constexpr int kPrepThreads = 128;
-constexpr int kStateThreads = 256;
+// shared memory of one prep pipeline (offsets from a 1024-aligned base)
+constexpr uint32_t kPKQ = 0;          // [K; Q] bf16 (TMA) K-major 128 x 128; K rows become K*gamma (fp16)
+constexpr uint32_t kPV = 32768;       // V bf16 (TMA) K-major 64 x 128, converted in place to fp16
+constexpr uint32_t kPTBZ = 49152;     // [Z | T diag(beta) | Z] fp16 K-major 64-row blocks (3 x 8 KiB)
+constexpr uint32_t kPA = 73728;       // A^T fp32 [64][kLdA]
+constexpr int kLdA = 68;
+constexpr uint32_t kPT = kPA + 64 * kLdA * 4;   // T fp32 [64][kLdT]
+constexpr int kLdT = 68;
+constexpr uint32_t kPX = kPT + 64 * kLdT * 4;   // merge scratch fp32 [32][kLdX]
+constexpr int kLdX = 36;
+constexpr uint32_t kPBeta = kPX + 32 * kLdX * 4;     // beta [64]
+constexpr uint32_t kPGam = kPBeta + 256;             // Gamma * log2(e): [64] or [64][128] (channel)
+constexpr uint32_t kPKB = (kPGam + 32768 + 1023) & ~1023u;  // channel: K'' fp16 K-major 64 x 128
+constexpr uint32_t kPrepBytesScalar = kPGam + 256;
+constexpr uint32_t kPrepBytesChannel = kPKB + 16384;
 
-// prep kernel shared memory (offsets from a 1024-aligned base)
-constexpr uint32_t kPrepAG = 0;           // [K'; Q'] K-major 128 rows x 128      32 KiB
-constexpr uint32_t kPrepBG = 32768;       // K'' K-major 64 rows x 128            16 KiB
-constexpr uint32_t kPrepKG = 49152;       // K*gamma K-major 64 x 128             16 KiB
-constexpr uint32_t kPrepV = 65536;        // V K-major 64 x 128                   16 KiB
-constexpr uint32_t kPrepTB = 81920;       // T diag(beta) K-major 64 x 64          8 KiB
-constexpr uint32_t kPrepGam = 90112;      // Gamma fp32 [64][128] (channel) or [64] 32 KiB
-constexpr uint32_t kPrepBeta = 122880;    // beta fp32 [64]
-constexpr uint32_t kPrepSmem = 123136 + 1024;
-// solve scratch, aliasing the Gram operands once the Gram MMA has completed
-constexpr uint32_t kPrepA = 0;            // A fp32 [64][65]
-constexpr uint32_t kPrepT = 17408;        // T fp32 [64][65]
-constexpr uint32_t kPrepX = 34816;        // block products fp32 [3][16][17]
-constexpr int kLd = 65;
+// TMEM columns of one prep pipeline
+constexpr uint32_t kTG = 0, kTW = 64, kTU = 192, kPrepTmemCols = 256;
 
-// state kernel shared memory
-constexpr uint32_t kStS = 2 * kHandoffStride;    // S fp16 K-major 128 x 128   32 KiB
-constexpr uint32_t kStDT = kStS + 32768;         // Delta^T fp16 K-major 128 x 64 16 KiB
-constexpr uint32_t kStateSmem = kStDT + 16384 + 1024;
+struct PrepArgs {
+    const float* g;
+    const float* beta;
+    int T, H, NC;
+    int* status;
+};
+
+struct PrepSmem {
+    uint8_t* base;
+    uint64_t* bars;  // [3]: TMA, Gram, W/U
+    uint32_t tmem;
+    int bar_id;      // named barrier of this pipeline's 128 threads
+};
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// MMA operands are fp16 (10-bit mantissa): bf16 inputs convert to it exactly, and with bf16
-// operands the rounding of the intermediate factors alone exceeded the 2e-2 * rms(o) parity bar.
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
+__device__ __forceinline__ uint32_t pack2h(float a, float b) {
     __half2 t = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&t);
 }
-
-__device__ __forceinline__ uint4 pack8(const float* f) {
-    return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+__device__ __forceinline__ uint4 pack8h(const float* f) {
+    return make_uint4(pack2h(f[0], f[1]), pack2h(f[2], f[3]), pack2h(f[4], f[5]), pack2h(f[6], f[7]));
 }
-
-// 8 bf16 (inputs) to fp32
-__device__ __forceinline__ void unpack8(uint4 u, float* f) {
+__device__ __forceinline__ void unpack8bf(uint4 u, float* f) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -97,8 +115,6 @@ __device__ __forceinline__ void unpack8(uint4 u, float* f) {
         f[2 * i + 1] = __high2float(t);
     }
 }
-
-// 8 fp16 (operand images) to fp32
 __device__ __forceinline__ void unpack8h(uint4 u, float* f) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -108,106 +124,147 @@ __device__ __forceinline__ void unpack8h(uint4 u, float* f) {
         f[2 * i + 1] = __high2float(t);
     }
 }
-
-constexpr float kF16Max = 65504.f;
-
 __device__ __forceinline__ void st16(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
+__device__ __forceinline__ uint4 ld16(const void* p) { return *reinterpret_cast<const uint4*>(p); }
 
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// T = (I + A)^-1 for a 64 x 64 strictly-lower A (fp32, stride kLd). Diagonal 16 x 16 blocks by
-// forward substitution, then block rows top-down: T_IJ = -T_II sum_{J<=K<I} A_IK T_KJ.
-__device__ void unit_lower_inverse64(const float* __restrict__ A, float* __restrict__ Tm, float* __restrict__ X,
-                                     int tid) {
-    if (tid < 64) {
-        const int base = (tid >> 4) * 16, j = tid & 15;
-        float t[16];
+// 16 x 16 output tile of C = A (16 x K) * B (K x 16) on warp MMAs (tf32, fp32 accumulate).
+// A(row, k) and B(k, col) are read through the accessors; the result stays in fragments
+// (c[nt][0..3] for the two 8-column halves).
+template <typename FA, typename FB>
+__device__ __forceinline__ void warp_gemm16(float (&c)[2][4], FA A, FB B, int K, int lane) {
+    const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc = (r == j) ? 1.f : 0.f;
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int i = 0; i < r; ++i) acc = fmaf(-A[(base + r) * kLd + base + i], t[i], acc);
-            t[r] = (r < j) ? 0.f : acc;
-        }
+        for (int e = 0; e < 4; ++e) c[nt][e] = 0.f;
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a[4] = {to_tf32(A(g, k0 + t)), to_tf32(A(g + 8, k0 + t)), to_tf32(A(g, k0 + t + 4)),
+                               to_tf32(A(g + 8, k0 + t + 4))};
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Tm[(base + r) * kLd + base + j] = t[r];
-    } else {
-        // zero the strictly-upper 16 x 16 blocks (6 blocks)
-        for (int e = tid - 64; e < 6 * 256; e += 64) {
-            const int blk = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-            const int I = (blk < 3) ? 0 : (blk < 5 ? 1 : 2);
-            const int J = (blk < 3) ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-            Tm[(16 * I + rr) * kLd + 16 * J + cc] = 0.f;
+        for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t bb[2] = {to_tf32(B(k0 + t, nt * 8 + g)), to_tf32(B(k0 + t + 4, nt * 8 + g))};
+            mma_tf32_16x8x8(c[nt], a, bb);
         }
-    }
-    __syncthreads();
-    for (int I = 1; I < 4; ++I) {
-        for (int e = tid; e < I * 256; e += kPrepThreads) {
-            const int J = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-            float acc = 0.f;
-            for (int K = J; K < I; ++K)
-#pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    acc = fmaf(A[(16 * I + rr) * kLd + 16 * K + m], Tm[(16 * K + m) * kLd + 16 * J + cc], acc);
-            X[J * 272 + rr * 17 + cc] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < I * 256; e += kPrepThreads) {
-            const int J = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-            float acc = 0.f;
-            for (int m = 0; m <= rr; ++m) acc = fmaf(Tm[(16 * I + rr) * kLd + 16 * I + m], X[J * 272 + m * 17 + cc], acc);
-            Tm[(16 * I + rr) * kLd + 16 * J + cc] = -acc;
-        }
-        __syncthreads();
     }
 }
 
-// ------------------------------------------------------------------------ prep --
+// Stores a 16 x 16 fragment tile (times `sign`) through the accessor dst(row, col) = value.
+template <typename FD>
+__device__ __forceinline__ void warp_store16(const float (&c)[2][4], FD D, float sign, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        D(g, nt * 8 + 2 * t, sign * c[nt][0]);
+        D(g, nt * 8 + 2 * t + 1, sign * c[nt][1]);
+        D(g + 8, nt * 8 + 2 * t, sign * c[nt][2]);
+        D(g + 8, nt * 8 + 2 * t + 1, sign * c[nt][3]);
+    }
+}
+
+// T = (I + A)^-1 for the 64 x 64 strictly-lower A held transposed in sAt (sAt[i][r] = A[r][i]).
+// Diagonal 16 x 16 blocks by right-looking forward substitution (one thread per column), then
+// T_IJ = -T_II (A_IJ T_JJ) for the two 32 x 32 halves and -T_hi (A_ll T_lo) for the lower-left
+// 32 x 32 block, on warp MMAs. The strictly upper part of sT is zero and never written.
+__device__ void unit_lower_inverse64(const float* __restrict__ sAt, float* __restrict__ sT, float* __restrict__ sX,
+                                     int lt, int bar_id) {
+    const int lw = lt >> 5, lane = lt & 31;
+    auto At = [&](int r, int i) { return sAt[i * kLdA + r]; };  // A[r][i]
+    if (lt < 64) {
+        const int base = (lt >> 4) * 16, j = lt & 15;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
+#pragma unroll
+        for (int i = 0; i < 15; ++i)
+#pragma unroll
+            for (int r = i + 1; r < 16; ++r) x[r] = fmaf(-At(base + r, base + i), x[i], x[r]);
+#pragma unroll
+        for (int r = 0; r < 16; ++r) sT[(base + r) * kLdT + base + j] = x[r];
+    }
+    named_bar(bar_id, kPrepThreads);
+    // T_10 = -T_11 (A_10 T_00) (warp 0), T_32 = -T_33 (A_32 T_22) (warp 1)
+    if (lw < 2) {
+        const int I = 2 * lw + 1, J = 2 * lw;
+        float* X = sX + lw * 16 * kLdX;  // 16 x 16 scratch per warp
+        float c[2][4];
+        warp_gemm16(c, [&](int r, int k) { return At(16 * I + r, 16 * J + k); },
+                    [&](int k, int col) { return sT[(16 * J + k) * kLdT + 16 * J + col]; }, 16, lane);
+        warp_store16(c, [&](int r, int col, float v) { X[r * kLdX + col] = v; }, 1.f, lane);
+        __syncwarp();
+        warp_gemm16(c, [&](int r, int k) { return sT[(16 * I + r) * kLdT + 16 * I + k]; },
+                    [&](int k, int col) { return X[k * kLdX + col]; }, 16, lane);
+        warp_store16(c, [&](int r, int col, float v) { sT[(16 * I + r) * kLdT + 16 * J + col] = v; }, -1.f, lane);
+    }
+    named_bar(bar_id, kPrepThreads);
+    // lower-left 32 x 32: Y = A_ll T_lo, then T_ll = -T_hi Y; warp w owns the 16 x 16 quadrant (qr, qc)
+    {
+        const int qr = lw >> 1, qc = lw & 1;
+        float c[2][4];
+        warp_gemm16(c, [&](int r, int k) { return At(32 + 16 * qr + r, k); },
+                    [&](int k, int col) { return sT[k * kLdT + 16 * qc + col]; }, 32, lane);
+        warp_store16(c, [&](int r, int col, float v) { sX[(16 * qr + r) * kLdX + 16 * qc + col] = v; }, 1.f, lane);
+        named_bar(bar_id, kPrepThreads);
+        warp_gemm16(c, [&](int r, int k) { return sT[(32 + 16 * qr + r) * kLdT + 32 + k]; },
+                    [&](int k, int col) { return sX[k * kLdX + 16 * qc + col]; }, 32, lane);
+        warp_store16(c, [&](int r, int col, float v) { sT[(32 + 16 * qr + r) * kLdT + 16 * qc + col] = v; }, -1.f,
+                     lane);
+    }
+    named_bar(bar_id, kPrepThreads);
+}
+
+// One-time set-up of a prep pipeline's shared memory: the zero blocks around T diag(beta) and the
+// strictly upper part of T (never written by the solve).
+__device__ void prep_init(const PrepSmem& ps, int lt) {
+    uint8_t* tbz = ps.base + kPTBZ;
+    for (int i = lt; i < 512; i += kPrepThreads) {                            // 512 x 16 B = 8 KiB
+        reinterpret_cast<uint4*>(tbz)[i] = make_uint4(0, 0, 0, 0);           // first Z
+        reinterpret_cast<uint4*>(tbz + 16384)[i] = make_uint4(0, 0, 0, 0);   // second Z
+    }
+    float* sT = reinterpret_cast<float*>(ps.base + kPT);
+    for (int i = lt; i < 64 * kLdT; i += kPrepThreads) sT[i] = 0.f;
+}
+
+// Computes the hand-off block of chunk c of head (b, h) into `out` (global memory). Executed by the
+// 128 threads of one pipeline; `it` counts the pipeline's previous tasks (mbarrier phase parity).
 template <int MODE>
-__global__ void __launch_bounds__(kPrepThreads)
-chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                  const __nv_bfloat16* __restrict__ v, const float* __restrict__ g, const float* __restrict__ beta,
-                  int T, int H, int NC, uint8_t* __restrict__ ws, int* status) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = align1024(smem_raw);
-    uint8_t* sAG = sm + kPrepAG;
-    uint8_t* sBG = sm + kPrepBG;
-    uint8_t* sKG = sm + kPrepKG;
-    uint8_t* sV = sm + kPrepV;
-    uint8_t* sTB = sm + kPrepTB;
-    float* sGam = reinterpret_cast<float*>(sm + kPrepGam);
-    float* sBeta = reinterpret_cast<float*>(sm + kPrepBeta);
-    __shared__ uint64_t bar;
-    __shared__ uint32_t tmem_base;
-
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+__device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv,
+                           const PrepSmem& ps, int b, int h, int c, uint8_t* __restrict__ out, uint32_t it, int lt) {
+    const int lw = lt >> 5, lane = lt & 31;
+    const uint32_t par = it & 1u;
+    uint8_t* sm = ps.base;
+    uint8_t* sKQ = sm + kPKQ;
+    uint8_t* sV = sm + kPV;
+    uint8_t* sTB = sm + kPTBZ + 8192;
+    float* sAt = reinterpret_cast<float*>(sm + kPA);
+    float* sT = reinterpret_cast<float*>(sm + kPT);
+    float* sX = reinterpret_cast<float*>(sm + kPX);
+    float* sBeta = reinterpret_cast<float*>(sm + kPBeta);
+    float* sGam = reinterpret_cast<float*>(sm + kPGam);
+    uint8_t* sKB = sm + kPKB;
+    uint64_t* barT = ps.bars;
+    uint64_t* barG = ps.bars + 1;
+    uint64_t* barW = ps.bars + 2;
+    const int T = P.T, H = P.H;
     const int c0 = c * kC;
     const int n = min(kC, T - c0);
-    const size_t tok0 = ((size_t)b * T + c0) * H + h;  // row r of the chunk is token tok0 + r * H
-    uint8_t* out = ws + ((size_t)(b * H + h) * NC + c) * kHandoffStride;
+    const size_t tok0 = ((size_t)b * T + c0) * H + h;  // chunk row r is token tok0 + r * H
 
-    if (tid == 0) {
-        mbar_init(&bar, 1);
-        fence_mbar_init();
+    // ---- 1. TMA: K and Q into the two halves of the 128-row [K; Q] tile, V
+    if (lt == 0) {
+        mbar_arrive_expect_tx(barT, 6 * 8192);
+        tma_load_4d(sKQ, mk, 0, h, c0, b, barT);
+        tma_load_4d(sKQ + 16384, mk, 64, h, c0, b, barT);
+        tma_load_4d(sKQ + 8192, mq, 0, h, c0, b, barT);
+        tma_load_4d(sKQ + 24576, mq, 64, h, c0, b, barT);
+        tma_load_4d(sV, mv, 0, h, c0, b, barT);
+        tma_load_4d(sV + 8192, mv, 64, h, c0, b, barT);
     }
-    if (warp == 0) {
-        tmem_alloc(&tmem_base, 256);
-        tmem_relinquish();
-    }
-
-    // ---- beta and the inclusive cumulative log-decay (rows past the tail repeat Gamma_{n-1})
-    if (tid < kC) sBeta[tid] = (tid < n) ? beta[tok0 + (size_t)tid * H] : 0.f;
+    // ---- 2. beta and the cumulative log-decay (log2 units; rows past the tail repeat Gamma_{n-1})
+    if (lt < kC) sBeta[lt] = (lt < n) ? P.beta[tok0 + (size_t)lt * H] : 0.f;
     if (MODE == GDR_DECAY_SCALAR) {
-        if (warp == 0) {
-            float x0 = (lane < n) ? g[tok0 + (size_t)lane * H] : 0.f;
-            float x1 = (lane + 32 < n) ? g[tok0 + (size_t)(lane + 32) * H] : 0.f;
+        if (lw == 0) {
+            float x0 = (lane < n) ? P.g[tok0 + (size_t)lane * H] * kLog2e : 0.f;
+            float x1 = (lane + 32 < n) ? P.g[tok0 + (size_t)(lane + 32) * H] * kLog2e : 0.f;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
@@ -222,355 +279,541 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             sGam[lane + 32] = x1;
         }
     } else if (MODE == GDR_DECAY_CHANNEL) {
+        float gv[kC];
+#pragma unroll
+        for (int r = 0; r < kC; ++r) gv[r] = (r < n) ? P.g[(tok0 + (size_t)r * H) * kD + lt] : 0.f;
         float acc = 0.f;
+#pragma unroll
         for (int r = 0; r < kC; ++r) {
-            if (r < n) acc += g[(tok0 + (size_t)r * H) * kD + tid];
-            sGam[r * kD + tid] = acc;
+            acc = fmaf(gv[r], kLog2e, acc);
+            sGam[r * kD + lt] = acc;
         }
     }
-    __syncthreads();
+    named_bar(ps.bar_id, kPrepThreads);
+    mbar_wait(barT, par, P.status);
 
-    // ---- stage K, Q, V and the decay-scaled operands; write Q*gamma and K*gamma_C/gamma out
-    const int ref = (n - 1) >> 1;  // channel mode: mid-chunk reference row
+    // ---- 3. Q*gamma and K*gamma_C/gamma hand-off images; channel gate: decay-factored Gram operands
+    const int ref = (n - 1) >> 1;
     bool range_bad = false;
-    for (int it = 0; it < 8; ++it) {
-        const int task = tid + kPrepThreads * it;
+    for (int j = 0; j < 8; ++j) {
+        const int task = lt + kPrepThreads * j;
         const int r = task >> 4, col0 = (task & 15) * 8;
-        float kx[8], qx[8], vx[8];
-        if (r < n) {
-            const size_t off = (tok0 + (size_t)r * H) * kD + col0;
-            unpack8(*reinterpret_cast<const uint4*>(k + off), kx);
-            unpack8(*reinterpret_cast<const uint4*>(q + off), qx);
-            unpack8(*reinterpret_cast<const uint4*>(v + off), vx);
+        const uint32_t okr = kmajor_off(r, col0, 128), oqr = kmajor_off(kC + r, col0, 128);
+        float kx[8], qx[8];
+        unpack8bf(ld16(sKQ + okr), kx);
+        unpack8bf(ld16(sKQ + oqr), qx);
+        float qg[8], kt[8];
+        if (MODE == GDR_DECAY_NONE) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                qg[e] = qx[e];
+                kt[e] = kx[e];
+            }
+        } else if (MODE == GDR_DECAY_SCALAR) {
+            const float fr = fast_exp2(sGam[r]), ft = fast_exp2(sGam[kC - 1] - sGam[r]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                qg[e] = qx[e] * fr;
+                kt[e] = kx[e] * ft;
+            }
         } else {
+            float ka[8], qa[8], kb[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) kx[e] = qx[e] = vx[e] = 0.f;
-        }
-        float ka[8], qa[8], kb[8], kg[8], qg[8], kt[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            if (MODE == GDR_DECAY_NONE) {
-                ka[e] = kb[e] = kg[e] = kt[e] = kx[e];
-                qa[e] = qg[e] = qx[e];
-            } else if (MODE == GDR_DECAY_SCALAR) {
-                const float G = sGam[r];
-                const float gr = expf(G), tail = expf(sGam[kC - 1] - G);
-                ka[e] = kb[e] = kx[e];
-                qa[e] = qx[e];
-                kg[e] = kx[e] * gr;
-                qg[e] = qx[e] * gr;
-                kt[e] = kx[e] * tail;
-            } else {
+            for (int e = 0; e < 8; ++e) {
                 const float G = sGam[r * kD + col0 + e];
                 const float Gr = sGam[ref * kD + col0 + e];
                 const float GC = sGam[(kC - 1) * kD + col0 + e];
-                const float up = expf(G - Gr), dn = expf(Gr - G), gr = expf(G);
+                const float up = fast_exp2(G - Gr), dn = fast_exp2(Gr - G);
+                if (!(up < kF16Max && dn < kF16Max)) range_bad = true;
+                qg[e] = qx[e] * fast_exp2(G);
+                kt[e] = kx[e] * fast_exp2(GC - G);
                 ka[e] = kx[e] * up;
                 qa[e] = qx[e] * up;
                 kb[e] = kx[e] * dn;
-                if (!(up < kF16Max && dn < kF16Max)) range_bad = true;
-                kg[e] = kx[e] * gr;
-                qg[e] = qx[e] * gr;
-                kt[e] = kx[e] * expf(GC - G);
             }
+            st16(sKQ + okr, pack8h(ka));
+            st16(sKQ + oqr, pack8h(qa));
+            st16(sKB + kmajor_off(r, col0, 64), pack8h(kb));
         }
-        st16(sAG + kmajor_off(r, col0, 128), pack8(ka));
-        st16(sAG + kmajor_off(kC + r, col0, 128), pack8(qa));
-        st16(sBG + kmajor_off(r, col0, 64), pack8(kb));
-        st16(sKG + kmajor_off(r, col0, 64), pack8(kg));
-        st16(sV + kmajor_off(r, col0, 64), pack8(vx));
-        st16(out + kOffQG + kmajor_off(r, col0, 64), pack8(qg));
-        st16(out + kOffKT + mnmajor_off(r, col0, 64), pack8(kt));
+        st16(out + kOffWQ + oqr, pack8h(qg));
+        st16(out + kOffKT + mnmajor_off(r, col0, 64), pack8h(kt));
     }
-    if (MODE == GDR_DECAY_CHANNEL && range_bad) report_status(status, GDR_ERR_RANGE);
+    if (MODE == GDR_DECAY_CHANNEL && range_bad) report_status(P.status, GDR_ERR_RANGE);
     {
         float gc = 1.f;
-        if (MODE == GDR_DECAY_SCALAR) gc = expf(sGam[kC - 1]);
-        if (MODE == GDR_DECAY_CHANNEL) gc = expf(sGam[(kC - 1) * kD + tid]);
-        reinterpret_cast<float*>(out + kOffGam)[tid] = gc;
+        if (MODE == GDR_DECAY_SCALAR) gc = fast_exp2(sGam[kC - 1]);
+        if (MODE == GDR_DECAY_CHANNEL) gc = fast_exp2(sGam[(kC - 1) * kD + lt]);
+        reinterpret_cast<float*>(out + kOffGam)[lt] = gc;
     }
-    fence_proxy_async_smem();
+    if (MODE == GDR_DECAY_CHANNEL) fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    named_bar(ps.bar_id, kPrepThreads);
     tc_fence_after();
 
-    // ---- Gram products: rows 0-63 K' K''^T, rows 64-127 Q' K''^T (M = 128, N = 64, K = 128)
-    const uint32_t tG = tmem_base, tW = tmem_base + 64, tU = tmem_base + 128;
-    if (tid == 0) {
-        const uint32_t id = idesc_f16(128, 64, false, false);
+    // ---- 4. Gram products: rows 0-63 K' K''^T, rows 64-127 Q' K''^T (M = 128, N = 64, K = 128)
+    const uint32_t tG = ps.tmem + kTG, tW = ps.tmem + kTW, tU = ps.tmem + kTU;
+    if (lt == 0) {
+        if (MODE == GDR_DECAY_CHANNEL) {
+            const uint32_t id = idesc_f16(128, 64, false, false);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-            mma_f16(tG, sdesc(smem_u32(sAG) + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
-                     sdesc(smem_u32(sBG) + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id, ks > 0);
-        mma_commit(&bar);
+            for (int ks = 0; ks < 8; ++ks)
+                mma_f16(tG, sdesc(smem_u32(sKQ) + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                        sdesc(smem_u32(sKB) + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id, ks > 0);
+        } else {
+            const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t d = sdesc(smem_u32(sKQ) + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                mma_f16(tG, d, d, id, ks > 0);  // B = the K rows (first 64 rows) of the same tile
+            }
+        }
+        mma_commit(barG);
     }
     __syncwarp();
-    mbar_wait(&bar, 0, status);
+    mbar_wait(barG, par, P.status);
     tc_fence_after();
 
-    float* sA = reinterpret_cast<float*>(sm + kPrepA);
-    float* sT = reinterpret_cast<float*>(sm + kPrepT);
-    float* sX = reinterpret_cast<float*>(sm + kPrepX);
+    // ---- 5. A (strictly lower, beta_r folded in; stored transposed) and P (causal incl. diagonal)
     {
-        const int rr = (warp & 1) * 32 + lane;  // chunk row of this thread's TMEM lane
-        const uint32_t lane_addr = tG + ((uint32_t)(warp * 32) << 16);
+        const int rr = (lw & 1) * 32 + lane;
+        const uint32_t laddr = tG + ((uint32_t)(lw * 32) << 16);
         const float br = sBeta[rr];
-        float Gr = 0.f;
-        if (MODE == GDR_DECAY_SCALAR) Gr = sGam[rr];
+        const float G2r = (MODE == GDR_DECAY_SCALAR) ? sGam[rr] : 0.f;
         for (int half = 0; half < 2; ++half) {
             float x[32];
-            tmem_ld32(lane_addr + half * 32, x);
+            tmem_ld32(laddr + half * 32, x);
             tmem_ld_wait();
-            float p[32];
+            if (lw < 2) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int i = half * 32 + e;
-                float d = 1.f;
-                if (MODE == GDR_DECAY_SCALAR) d = (i <= rr) ? expf(Gr - sGam[i]) : 0.f;
-                if (warp < 2) {
-                    sA[rr * kLd + i] = (i < rr && rr < n) ? br * x[e] * d : 0.f;
-                } else {
-                    p[e] = (i <= rr && rr < n) ? x[e] * d : 0.f;
+                for (int e = 0; e < 32; ++e) {
+                    const int i = half * 32 + e;
+                    float a = 0.f;
+                    if (i < rr && rr < n) {
+                        a = br * x[e];
+                        if (MODE == GDR_DECAY_SCALAR) a *= fast_exp2(G2r - sGam[i]);
+                    }
+                    sAt[i * kLdA + rr] = a;
                 }
-            }
-            if (warp >= 2) {
+            } else {
+                float p[32];
 #pragma unroll
-                for (int ci = 0; ci < 4; ++ci) st16(out + kOffP + kmajor_off(rr, half * 32 + ci * 8, 64), pack8(p + ci * 8));
+                for (int e = 0; e < 32; ++e) {
+                    const int i = half * 32 + e;
+                    float v = 0.f;
+                    if (i <= rr && rr < n) {
+                        v = x[e];
+                        if (MODE == GDR_DECAY_SCALAR) v *= fast_exp2(G2r - sGam[i]);
+                    }
+                    p[e] = v;
+                }
+#pragma unroll
+                for (int ci = 0; ci < 4; ++ci)
+                    st16(out + kOffP + kmajor_off(rr, half * 32 + ci * 8, 64), pack8h(p + ci * 8));
             }
         }
     }
     tc_fence_before();
-    __syncthreads();
+    named_bar(ps.bar_id, kPrepThreads);
 
-    // ---- UT transform: T = (I + A)^-1, then T diag(beta) as the K-major B operand
-    unit_lower_inverse64(sA, sT, sX, tid);
-    for (int task = tid; task < 64 * 8; task += kPrepThreads) {
+    // ---- 6. K*gamma (in place over the K rows) and V as fp16 operands of the W / U MMAs
+    for (int j = 0; j < 16; ++j) {
+        const int task = lt + kPrepThreads * j;
+        const bool isv = task >= 1024;
+        const int r = (task & 1023) >> 4, col0 = (task & 15) * 8;
+        uint8_t* p = isv ? sV + kmajor_off(r, col0, 64) : sKQ + kmajor_off(r, col0, 128);
+        float x[8];
+        if (!isv && MODE == GDR_DECAY_CHANNEL) {
+            unpack8h(ld16(p), x);  // K' = K e^{Gamma - Gamma_ref}: times e^{Gamma_ref} gives K*gamma
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] *= fast_exp2(sGam[ref * kD + col0 + e]);
+        } else {
+            unpack8bf(ld16(p), x);
+            if (!isv && MODE == GDR_DECAY_SCALAR) {
+                const float fr = fast_exp2(sGam[r]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] *= fr;
+            }
+        }
+        st16(p, pack8h(x));
+    }
+    named_bar(ps.bar_id, kPrepThreads);
+
+    // ---- 7. UT transform T = (I + A)^-1, then T diag(beta) as fp16
+    unit_lower_inverse64(sAt, sT, sX, lt, ps.bar_id);
+    for (int j = 0; j < 4; ++j) {
+        const int task = lt + kPrepThreads * j;
         const int r = task >> 3, i0 = (task & 7) * 8;
         float t8[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t8[e] = sT[r * kLd + i0 + e] * sBeta[i0 + e];
-        st16(sTB + kmajor_off(r, i0, 64), pack8(t8));
+        for (int e = 0; e < 8; ++e) t8[e] = sT[r * kLdT + i0 + e] * sBeta[i0 + e];
+        st16(sTB + kmajor_off(r, i0, 64), pack8h(t8));
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    named_bar(ps.bar_id, kPrepThreads);
     tc_fence_after();
 
-    // ---- W^T = (K*gamma)^T (T diag beta)^T and U^T = V^T (T diag beta)^T (M = 128, N = 64, K = 64)
-    if (tid == 0) {
-        const uint32_t id = idesc_f16(128, 64, true, false);
+    // ---- 8. W = [T diag(beta); 0] (K*gamma) (M = 128, N = 128) and U^T = V^T (T diag(beta))^T (M = 128, N = 64)
+    if (lt == 0) {
+        const uint32_t idW = idesc_f16(128, 128, false, true);
+        const uint32_t idU = idesc_f16(128, 64, true, false);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t bd = sdesc(smem_u32(sTB) + ks * 32, 16, 1024);
-            mma_f16(tW, sdesc(smem_u32(sKG) + ks * 2048, 8192, 1024), bd, id, ks > 0);
-            mma_f16(tU, sdesc(smem_u32(sV) + ks * 2048, 8192, 1024), bd, id, ks > 0);
+            const uint64_t tb = sdesc(smem_u32(sTB) + ks * 32, 16, 1024);
+            mma_f16(tW, tb, sdesc(smem_u32(sKQ) + ks * 2048, 16384, 1024), idW, ks > 0);
+            mma_f16(tU, sdesc(smem_u32(sV) + ks * 2048, 8192, 1024), tb, idU, ks > 0);
         }
-        mma_commit(&bar);
+        mma_commit(barW);
     }
     __syncwarp();
-    mbar_wait(&bar, 1, status);
+    mbar_wait(barW, par, P.status);
     tc_fence_after();
     {
-        const int row = warp * 32 + lane;  // d_k index for W^T, d_v index for U^T
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        for (int half = 0; half < 2; ++half) {
+        const int row = lw * 32 + lane;
+        const uint32_t loff = (uint32_t)(lw * 32) << 16;
+        if (lw < 2) {  // W row r = row (lanes 0-63 of the W accumulator)
+            for (int q4 = 0; q4 < 4; ++q4) {
+                float x[32];
+                tmem_ld32(tW + loff + q4 * 32, x);
+                tmem_ld_wait();
+#pragma unroll
+                for (int ci = 0; ci < 4; ++ci)
+                    st16(out + kOffWQ + kmajor_off(row, q4 * 32 + ci * 8, 128), pack8h(x + ci * 8));
+            }
+        }
+        for (int half = 0; half < 2; ++half) {  // U^T row j = row
             float x[32];
-            tmem_ld32(tW + lane_off + half * 32, x);
+            tmem_ld32(tU + loff + half * 32, x);
             tmem_ld_wait();
 #pragma unroll
             for (int ci = 0; ci < 4; ++ci)
-                st16(out + kOffWT + mnmajor_off(row, half * 32 + ci * 8, 128), pack8(x + ci * 8));
-            tmem_ld32(tU + lane_off + half * 32, x);
-            tmem_ld_wait();
-#pragma unroll
-            for (int ci = 0; ci < 4; ++ci) st16(out + kOffUT + row * 128 + (half * 32 + ci * 8) * 2, pack8(x + ci * 8));
+                st16(out + kOffUT + kmajor_off(row, half * 32 + ci * 8, 128), pack8h(x + ci * 8));
         }
     }
     tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem_base, 256);
+    named_bar(ps.bar_id, kPrepThreads);
 }
 
-// ----------------------------------------------------------------------- state --
+// Standalone prep kernel: one pipeline per CTA, one chunk per CTA, hand-off blocks for all chunks.
+template <int MODE>
+__global__ void __launch_bounds__(kPrepThreads)
+chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                  const __grid_constant__ CUtensorMap mv, PrepArgs P, uint8_t* __restrict__ ws) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t bars[3];
+    __shared__ uint32_t tmem_base;
+    const int lt = threadIdx.x;
+    if (lt == 0) {
+        for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+    }
+    if (lt < 32) {
+        tmem_alloc(&tmem_base, kPrepTmemCols);
+        tmem_relinquish();
+    }
+    PrepSmem ps{align1024(smem_raw), bars, 0, 1};
+    prep_init(ps, lt);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    ps.tmem = tmem_base;
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    uint8_t* out = ws + ((size_t)(b * P.H + h) * P.NC + c) * kHandoffStride;
+    prep_chunk<MODE>(P, &mq, &mk, &mv, ps, b, h, c, out, 0u, lt);
+    tc_fence_before();
+    __syncthreads();
+    if (lt < 32) tmem_dealloc(tmem_base, kPrepTmemCols);
+}
+
+// ------------------------------------------------------------------- state pass --
+constexpr int kStateThreads = 512;
+constexpr uint32_t kSStageA0 = 0;
+constexpr uint32_t kSStageA1 = 58368;
+constexpr uint32_t kSUT = 116736;       // U^T stage (single buffer)
+constexpr uint32_t kSS = 133120;        // S fp16 K-major 128 x 128
+constexpr uint32_t kSDT = 165888;       // Delta^T fp16 K-major 128 x 64
+constexpr uint32_t kSO = 182272;        // output staging: 4 (fp32) or 2 (bf16) TMA boxes of 64 rows x 128 B
+constexpr uint32_t kStateSmem = kSO + 32768 + 1024;
+// TMEM: D1 double-buffered (corr^T | O^T, 128 columns each), D3 (state increment, 128 columns)
+constexpr uint32_t kTD1 = 0, kTD3 = 256, kStateTmemCols = 512;
+
+struct StateArgs {
+    const float* S0;
+    float* S_T;
+    int T, H, NC;
+    float scale;
+    int* status;
+};
+
+template <typename Tout>
+__device__ __forceinline__ void stage_out(uint8_t* sO, int r, int j, float v);
+template <>
+__device__ __forceinline__ void stage_out<float>(uint8_t* sO, int r, int j, float v) {
+    const int box = j >> 5, cc = j & 31;
+    *reinterpret_cast<float*>(sO + box * 8192 + r * 128 + (((cc >> 2) ^ (r & 7)) << 4) + (cc & 3) * 4) = v;
+}
+template <>
+__device__ __forceinline__ void stage_out<__nv_bfloat16>(uint8_t* sO, int r, int j, float v) {
+    const int box = j >> 6, cc = j & 63;
+    *reinterpret_cast<__nv_bfloat16*>(sO + box * 8192 + r * 128 + (((cc >> 3) ^ (r & 7)) << 4) + (cc & 7) * 2) =
+        __float2bfloat16_rn(v);
+}
+
+// Walks the chunks of head (b, h) in order. `src(c)` gives chunk c's hand-off block.
 template <typename Tout>
 __global__ void __launch_bounds__(kStateThreads, 1)
-chunk_state_kernel(const uint8_t* __restrict__ ws, const float* S0, Tout* __restrict__ o, float* S_T, int T, int H,
-                   int NC, float scale, int* status) {
+chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const uint8_t* __restrict__ ws) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
-    uint8_t* stage0 = sm;
-    uint8_t* stage1 = sm + kHandoffStride;
-    uint8_t* sS = sm + kStS;
-    uint8_t* sDT = sm + kStDT;
-    __shared__ uint64_t full[2], barA, barB;
+    uint8_t* stageA[2] = {sm + kSStageA0, sm + kSStageA1};
+    uint8_t* sUT = sm + kSUT;
+    uint8_t* sS = sm + kSS;
+    uint8_t* sDT = sm + kSDT;
+    uint8_t* sO = sm + kSO;
+    __shared__ uint64_t fullA[2], fullU, barA[2], barB, barC;
     __shared__ uint32_t tmem_base;
 
     const int bh = blockIdx.x;
-    const int b = bh / H, h = bh % H;
+    const int b = bh / A.H, h = bh % A.H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
-    const int j = quad * 32 + lane;  // state row (d_v index) = TMEM lane
+    const int quad = warp & 3, cg = warp >> 2;  // TMEM lane quadrant, column group
+    const int j = quad * 32 + lane;             // state row (d_v index) = TMEM lane
+    const int NC = A.NC;
     const uint8_t* src = ws + (size_t)bh * NC * kHandoffStride;
+    constexpr int kOutBoxes = sizeof(Tout) == 4 ? 4 : 2;
+    constexpr int kOutBoxCols = 128 / kOutBoxes;
 
     if (tid == 0) {
-        mbar_init(&full[0], 1);
-        mbar_init(&full[1], 1);
-        mbar_init(&barA, 1);
+        mbar_init(&fullA[0], 1);
+        mbar_init(&fullA[1], 1);
+        mbar_init(&fullU, 1);
+        mbar_init(&barA[0], 1);
+        mbar_init(&barA[1], 1);
         mbar_init(&barB, 1);
+        mbar_init(&barC, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(&tmem_base, 256);
+        tmem_alloc(&tmem_base, kStateTmemCols);
         tmem_relinquish();
     }
-
-    // initial state: this thread holds S[j][64*half .. 64*half + 63] in fp32
-    float s[64];
+    // initial state: this thread holds S[j][32*cg .. 32*cg + 31] in fp32
+    float s[32];
     {
-        const float* s0 = S0 ? S0 + ((size_t)bh * kD + j) * kD + 64 * half : nullptr;
+        const float* s0 = A.S0 ? A.S0 + ((size_t)bh * kD + j) * kD + 32 * cg : nullptr;
 #pragma unroll
-        for (int e = 0; e < 64; e += 4) {
-            float4 t = s0 ? *reinterpret_cast<const float4*>(s0 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int e = 0; e < 32; e += 4) {
+            const float4 t = s0 ? *reinterpret_cast<const float4*>(s0 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
             s[e] = t.x;
             s[e + 1] = t.y;
             s[e + 2] = t.z;
             s[e + 3] = t.w;
         }
 #pragma unroll
-        for (int ci = 0; ci < 8; ++ci) st16(sS + kmajor_off(j, 64 * half + ci * 8, 128), pack8(s + ci * 8));
+        for (int ci = 0; ci < 4; ++ci) st16(sS + kmajor_off(j, 32 * cg + ci * 8, 128), pack8h(s + ci * 8));
     }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tD3 = tmem_base + kTD3;
+    const uint32_t idA = idesc_f16(128, 128, false, false);
+    const uint32_t idC = idesc_f16(128, 128, false, true);
+    const uint32_t idB = idesc_f16(128, 64, false, false);
+
+    auto issue_A = [&](int c) {  // D1[c&1] = S [W; Q*gamma]^T (M = 128, N = 128, K = 128)
+        const uint8_t* st = stageA[c & 1];
+        const uint32_t d = tmem_base + kTD1 + (c & 1) * 128;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+            mma_f16(d, sdesc(smem_u32(sS) + koff, 16, 1024), sdesc(smem_u32(st + kOffWQ) + koff, 16, 1024), idA,
+                    ks > 0);
+        }
+        mma_commit(&barA[c & 1]);
+    };
+
     if (tid == 0) {
         for (int st = 0; st < 2 && st < NC; ++st) {
-            mbar_arrive_expect_tx(&full[st], kHandoffBytes);
-            bulk_g2s(st ? stage1 : stage0, src + (size_t)st * kHandoffStride, kHandoffBytes, &full[st]);
+            mbar_arrive_expect_tx(&fullA[st], kPartA);
+            bulk_g2s(stageA[st], src + (size_t)st * kHandoffStride, kPartA, &fullA[st]);
         }
+        mbar_arrive_expect_tx(&fullU, 16384);
+        bulk_g2s(sUT, src + kOffUT, 16384, &fullU);
+        mbar_wait(&fullA[0], 0, A.status);
+        tc_fence_after();
+        issue_A(0);
     }
-    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t tD1 = tmem_base, tD3 = tmem_base + 128;
-    const int dv = kD;
 
     for (int c = 0; c < NC; ++c) {
-        const int st = c & 1;
-        uint8_t* S_ = st ? stage1 : stage0;
-        mbar_wait(&full[st], (c >> 1) & 1, status);
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
+        const int sb = c & 1;
+        const uint8_t* st = stageA[sb];
+        const uint32_t tD1 = tmem_base + kTD1 + sb * 128;
+        mbar_wait(&fullU, c & 1, A.status);
+        mbar_wait(&barA[sb], (c >> 1) & 1, A.status);
         tc_fence_after();
-        // D1[:, 0:64] = S W^T ; D1[:, 64:128] = S (Q*gamma)^T   (M = 128, N = 64, K = 128)
-        if (tid == 0) {
-            const uint32_t idW = idesc_f16(128, 64, false, true);
-            const uint32_t idQ = idesc_f16(128, 64, false, false);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t ad = sdesc(smem_u32(sS) + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                mma_f16(tD1, ad, sdesc(smem_u32(S_ + kOffWT) + ks * 2048, 16384, 1024), idW, ks > 0);
-                mma_f16(tD1 + 64, ad, sdesc(smem_u32(S_ + kOffQG) + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024),
-                         idQ, ks > 0);
-            }
-            mma_commit(&barA);
-        }
-        __syncwarp();
-        mbar_wait(&barA, c & 1, status);
-        tc_fence_after();
-        // Delta^T[j][r] = U^T[j][r] - (S W^T)[j][r] for r in [32*half, 32*half + 32)
-        {
-            float x[32], u[32];
-            tmem_ld32(tD1 + lane_off + 32 * half, x);
-            const uint8_t* ut = S_ + kOffUT + j * 128 + 64 * half;
-#pragma unroll
-            for (int ci = 0; ci < 4; ++ci) unpack8h(*reinterpret_cast<const uint4*>(ut + ci * 16), u + ci * 8);
+        // ---- output of chunk c-1 (its MMA-B completed before MMA-A of chunk c was issued)
+        if (c > 0) {
+            const uint32_t tO = tmem_base + kTD1 + (sb ^ 1) * 128 + 64;
+            float x[16];
+            tmem_ld16(tO + lane_off + 16 * cg, x);
             tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) u[e] -= x[e];
+            for (int e = 0; e < 16; ++e) stage_out<Tout>(sO, 16 * cg + e, j, A.scale * x[e]);
+        }
+        // ---- Delta^T[j][r] = U^T[j][r] - (S W^T)[j][r], r in [16 cg, 16 cg + 16)
+        {
+            float x[16], u[16];
+            tmem_ld16(tD1 + lane_off + 16 * cg, x);
+            unpack8h(ld16(sUT + kmajor_off(j, 16 * cg, 128)), u);
+            unpack8h(ld16(sUT + kmajor_off(j, 16 * cg + 8, 128)), u + 8);
+            tmem_ld_wait();
 #pragma unroll
-            for (int ci = 0; ci < 4; ++ci) st16(sDT + kmajor_off(j, 32 * half + ci * 8, 128), pack8(u + ci * 8));
+            for (int e = 0; e < 16; ++e) u[e] -= x[e];
+            st16(sDT + kmajor_off(j, 16 * cg, 128), pack8h(u));
+            st16(sDT + kmajor_off(j, 16 * cg + 8, 128), pack8h(u + 8));
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        // D1[:, 64:128] += Delta^T P^T (M = 128, N = 64, K = 64); D3 = Delta^T K~ (M = 128, N = 128, K = 64)
         if (tid == 0) {
-            const uint32_t idP = idesc_f16(128, 64, false, false);
-            const uint32_t idK = idesc_f16(128, 128, false, true);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t ad = sdesc(smem_u32(sDT) + ks * 32, 16, 1024);
-                mma_f16(tD1 + 64, ad, sdesc(smem_u32(S_ + kOffP) + ks * 32, 16, 1024), idP, true);
-                mma_f16(tD3, ad, sdesc(smem_u32(S_ + kOffKT) + ks * 2048, 8192, 1024), idK, ks > 0);
+            if (c > 0) {  // output of chunk c-1
+                for (int bx = 0; bx < kOutBoxes; ++bx)
+                    tma_store_4d(&mo, sO + bx * 8192, bx * kOutBoxCols, h, (c - 1) * kC, b);
+                bulk_commit();
             }
+            if (c + 1 < NC) {  // U^T of chunk c+1 (this chunk's has been consumed)
+                mbar_arrive_expect_tx(&fullU, 16384);
+                bulk_g2s(sUT, src + (size_t)(c + 1) * kHandoffStride + kOffUT, 16384, &fullU);
+            }
+            // D3 = Delta^T K~ (M = 128, N = 128, K = 64), then D1[:, 64:128] += Delta^T P^T (N = 64)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_f16(tmem_base + kTD3, sdesc(smem_u32(sDT) + ks * 32, 16, 1024),
+                        sdesc(smem_u32(st + kOffKT) + ks * 2048, 8192, 1024), idC, ks > 0);
+            mma_commit(&barC);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_f16(tD1 + 64, sdesc(smem_u32(sDT) + ks * 32, 16, 1024),
+                        sdesc(smem_u32(st + kOffP) + ks * 32, 16, 1024), idB, true);
             mma_commit(&barB);
         }
         __syncwarp();
-        mbar_wait(&barB, c & 1, status);
+        mbar_wait(&barC, c & 1, A.status);
         tc_fence_after();
-        // S <- S Diag(gamma_C) + Delta^T K~ (this thread's 64 columns), then its fp16 copy
+        // ---- S <- S Diag(gamma_C) + Delta^T K~ on this thread's 32 columns, and its fp16 copy
         {
-            const float* gam = reinterpret_cast<const float*>(S_ + kOffGam) + 64 * half;
-            for (int q2 = 0; q2 < 2; ++q2) {
-                float x[32];
-                tmem_ld32(tD3 + lane_off + 64 * half + 32 * q2, x);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) s[32 * q2 + e] = fmaf(gam[32 * q2 + e], s[32 * q2 + e], x[e]);
-            }
-#pragma unroll
-            for (int ci = 0; ci < 8; ++ci) st16(sS + kmajor_off(j, 64 * half + ci * 8, 128), pack8(s + ci * 8));
-        }
-        // O rows r in [32*half, 32*half + 32), column j
-        {
+            const float* gam = reinterpret_cast<const float*>(st + kOffGam) + 32 * cg;
             float x[32];
-            tmem_ld32(tD1 + lane_off + 64 + 32 * half, x);
+            tmem_ld32(tD3 + lane_off + 32 * cg, x);
             tmem_ld_wait();
-            const int r0 = c * kC + 32 * half;
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-                if (r0 + e < T) store_f32(o + ((size_t)(b * T + r0 + e) * H + h) * dv + j, scale * x[e]);
+            for (int e = 0; e < 32; ++e) s[e] = fmaf(gam[e], s[e], x[e]);
+#pragma unroll
+            for (int ci = 0; ci < 4; ++ci) st16(sS + kmajor_off(j, 32 * cg + ci * 8, 128), pack8h(s + ci * 8));
         }
+        fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (tid == 0 && c + 2 < NC) {
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(&full[st], kHandoffBytes);
-            bulk_g2s(S_, src + (size_t)(c + 2) * kHandoffStride, kHandoffBytes, &full[st]);
+        tc_fence_after();
+        if (tid == 0) {
+            mbar_wait(&barB, c & 1, A.status);  // MMA-B done: stage A[sb] and the output columns are final
+            bulk_wait_read<0>();                // output staging may be rewritten
+            if (c + 2 < NC) {
+                mbar_arrive_expect_tx(&fullA[sb], kPartA);
+                bulk_g2s(stageA[sb], src + (size_t)(c + 2) * kHandoffStride, kPartA, &fullA[sb]);
+            }
+            if (c + 1 < NC) {
+                mbar_wait(&fullA[sb ^ 1], ((c + 1) >> 1) & 1, A.status);
+                tc_fence_after();
+                issue_A(c + 1);
+            }
         }
     }
-    if (S_T != nullptr) {
-        float* dst = S_T + ((size_t)bh * kD + j) * kD + 64 * half;
+    // ---- output of the last chunk
+    mbar_wait(&barB, (NC - 1) & 1, A.status);
+    tc_fence_after();
+    {
+        const uint32_t tO = tmem_base + kTD1 + ((NC - 1) & 1) * 128 + 64;
+        float x[16];
+        tmem_ld16(tO + lane_off + 16 * cg, x);
+        tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 64; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
+        for (int e = 0; e < 16; ++e) stage_out<Tout>(sO, 16 * cg + e, j, A.scale * x[e]);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        for (int bx = 0; bx < kOutBoxes; ++bx) tma_store_4d(&mo, sO + bx * 8192, bx * kOutBoxCols, h, (NC - 1) * kC, b);
+        bulk_commit();
+        bulk_wait<0>();
+    }
+    if (A.S_T != nullptr) {
+        float* dst = A.S_T + ((size_t)bh * kD + j) * kD + 32 * cg;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + e) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem_base, 256);
+    if (warp == 0) tmem_dealloc(tmem_base, kStateTmemCols);
+}
+
+// ---------------------------------------------------------------------- host --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 4-D map over a [B, T, H, 128] tensor: box of `box_cols` elements x 1 head x 64 tokens x 1 batch,
+// 128-byte swizzle. Tokens past T read as zero and are not written.
+cudaError_t make_map(CUtensorMap* map, const void* base, CUtensorMapDataType type, int esize, int B, int T, int H,
+                     int box_cols) {
+    EncodeTiledFn enc = encode_fn();
+    if (enc == nullptr) return cudaErrorNotSupported;
+    const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)kD * esize, (cuuint64_t)H * kD * esize, (cuuint64_t)T * H * kD * esize};
+    const cuuint32_t box[4] = {(cuuint32_t)box_cols, 1, (cuuint32_t)kC, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    const CUresult r = enc(map, type, 4, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 template <int MODE>
-cudaError_t launch_prep(const ChunkProblem& p, int NC, cudaStream_t stream) {
+cudaError_t launch_prep(const ChunkProblem& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        int NC, cudaStream_t stream) {
     auto kern = chunk_prep_kernel<MODE>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPrepSmem);
+    const uint32_t smem = (MODE == GDR_DECAY_CHANNEL ? kPrepBytesChannel : kPrepBytesScalar) + 1024;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    dim3 grid(NC, p.H, p.B);
-    kern<<<grid, kPrepThreads, kPrepSmem, stream>>>(
-        static_cast<const __nv_bfloat16*>(p.q), static_cast<const __nv_bfloat16*>(p.k),
-        static_cast<const __nv_bfloat16*>(p.v), p.g, p.beta, p.T, p.H, NC, static_cast<uint8_t*>(p.workspace),
-        p.status);
+    PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status};
+    kern<<<dim3(NC, p.H, p.B), kPrepThreads, smem, stream>>>(mq, mk, mv, P, static_cast<uint8_t*>(p.workspace));
     return cudaGetLastError();
 }
 
 template <typename Tout>
-cudaError_t launch_state(const ChunkProblem& p, int NC, cudaStream_t stream) {
+cudaError_t launch_state(const ChunkProblem& p, const CUtensorMap& mo, int NC, cudaStream_t stream) {
     auto kern = chunk_state_kernel<Tout>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem);
     if (err != cudaSuccess) return err;
-    kern<<<p.B * p.H, kStateThreads, kStateSmem, stream>>>(static_cast<const uint8_t*>(p.workspace), p.S0,
-                                                          static_cast<Tout*>(p.o), p.S_T, p.T, p.H, NC, p.scale,
-                                                          p.status);
+    StateArgs A{p.S0, p.S_T, p.T, p.H, NC, p.scale, p.status};
+    kern<<<p.B * p.H, kStateThreads, kStateSmem, stream>>>(mo, A, static_cast<const uint8_t*>(p.workspace));
     return cudaGetLastError();
 }
 
@@ -589,16 +832,25 @@ int chunk_tc_launches(int, int, int, int, int, int, int) { return 2; }
 
 cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream) {
     const int NC = (p.T + kC - 1) / kC;
-    cudaError_t err = cudaSuccess;
+    CUtensorMap mq, mk, mv, mo;
+    cudaError_t err;
+    if ((err = make_map(&mq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, 64)) != cudaSuccess) return err;
+    if ((err = make_map(&mk, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, 64)) != cudaSuccess) return err;
+    if ((err = make_map(&mv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, 64)) != cudaSuccess) return err;
+    if (p.o_dtype == GDR_BF16)
+        err = make_map(&mo, p.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, 64);
+    else
+        err = make_map(&mo, p.o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.B, p.T, p.H, 32);
+    if (err != cudaSuccess) return err;
     switch (p.mode) {
-        case GDR_DECAY_NONE: err = launch_prep<GDR_DECAY_NONE>(p, NC, stream); break;
-        case GDR_DECAY_SCALAR: err = launch_prep<GDR_DECAY_SCALAR>(p, NC, stream); break;
-        case GDR_DECAY_CHANNEL: err = launch_prep<GDR_DECAY_CHANNEL>(p, NC, stream); break;
+        case GDR_DECAY_NONE: err = launch_prep<GDR_DECAY_NONE>(p, mq, mk, mv, NC, stream); break;
+        case GDR_DECAY_SCALAR: err = launch_prep<GDR_DECAY_SCALAR>(p, mq, mk, mv, NC, stream); break;
+        case GDR_DECAY_CHANNEL: err = launch_prep<GDR_DECAY_CHANNEL>(p, mq, mk, mv, NC, stream); break;
         default: return cudaErrorInvalidValue;
     }
     if (err != cudaSuccess) return err;
-    if (p.o_dtype == GDR_BF16) return launch_state<__nv_bfloat16>(p, NC, stream);
-    return launch_state<float>(p, NC, stream);
+    if (p.o_dtype == GDR_BF16) return launch_state<__nv_bfloat16>(p, mo, NC, stream);
+    return launch_state<float>(p, mo, NC, stream);
 }
 
 }  // namespace gdr
