@@ -13,7 +13,7 @@
 //   O  = scale [ (Q*gamma) S^T + P Delta ]
 //   S <- S Diag(gamma_C) + Delta^T (K * gamma_C / gamma)
 //
-// Work split. A prep pass (one 128-thread pipeline per chunk, all chunks independent) computes the
+// Work split. A prep pass (one 256-thread pipeline per chunk, all chunks independent) computes the
 // S-independent factors and writes them as ready-to-use, 128-byte-swizzled fp16 operand images
 // (the "hand-off block"); a state pass (one 512-thread CTA per (b, h)) walks the chunks in order,
 // copies each block into shared memory with bulk copies and runs the S-dependent MMAs; the fp32
@@ -61,7 +61,7 @@ constexpr uint32_t kOffUT = 58368;      // U^T           fp16 K-major, 128 rows 
 constexpr uint32_t kHandoffStride = 74752;  // multiple of 1024
 
 // ------------------------------------------------------------------ prep pipeline --
-constexpr int kPrepThreads = 128;
+constexpr int kPrepThreads = 256;
 // shared memory of one prep pipeline (offsets from a 1024-aligned base)
 constexpr uint32_t kPKQ = 0;          // [K; Q] bf16 (TMA) K-major 128 x 128; K rows become K*gamma (fp16)
 constexpr uint32_t kPV = 32768;       // V bf16 (TMA) K-major 64 x 128, converted in place to fp16
@@ -167,6 +167,7 @@ __device__ __forceinline__ void warp_store16(const float (&c)[2][4], FD D, float
 // 32 x 32 block, on warp MMAs. The strictly upper part of sT is zero and never written.
 __device__ void unit_lower_inverse64(const float* __restrict__ sAt, float* __restrict__ sT, float* __restrict__ sX,
                                      int lt, int bar_id) {
+    // executed by 128 threads (4 warps); bar_id is their named barrier
     const int lw = lt >> 5, lane = lt & 31;
     auto At = [&](int r, int i) { return sAt[i * kLdA + r]; };  // A[r][i]
     if (lt < 64) {
@@ -181,7 +182,7 @@ __device__ void unit_lower_inverse64(const float* __restrict__ sAt, float* __res
 #pragma unroll
         for (int r = 0; r < 16; ++r) sT[(base + r) * kLdT + base + j] = x[r];
     }
-    named_bar(bar_id, kPrepThreads);
+    named_bar(bar_id, 128);
     // T_10 = -T_11 (A_10 T_00) (warp 0), T_32 = -T_33 (A_32 T_22) (warp 1)
     if (lw < 2) {
         const int I = 2 * lw + 1, J = 2 * lw;
@@ -195,7 +196,7 @@ __device__ void unit_lower_inverse64(const float* __restrict__ sAt, float* __res
                     [&](int k, int col) { return X[k * kLdX + col]; }, 16, lane);
         warp_store16(c, [&](int r, int col, float v) { sT[(16 * I + r) * kLdT + 16 * J + col] = v; }, -1.f, lane);
     }
-    named_bar(bar_id, kPrepThreads);
+    named_bar(bar_id, 128);
     // lower-left 32 x 32: Y = A_ll T_lo, then T_ll = -T_hi Y; warp w owns the 16 x 16 quadrant (qr, qc)
     {
         const int qr = lw >> 1, qc = lw & 1;
@@ -203,13 +204,13 @@ __device__ void unit_lower_inverse64(const float* __restrict__ sAt, float* __res
         warp_gemm16(c, [&](int r, int k) { return At(32 + 16 * qr + r, k); },
                     [&](int k, int col) { return sT[k * kLdT + 16 * qc + col]; }, 32, lane);
         warp_store16(c, [&](int r, int col, float v) { sX[(16 * qr + r) * kLdX + 16 * qc + col] = v; }, 1.f, lane);
-        named_bar(bar_id, kPrepThreads);
+        named_bar(bar_id, 128);
         warp_gemm16(c, [&](int r, int k) { return sT[(32 + 16 * qr + r) * kLdT + 32 + k]; },
                     [&](int k, int col) { return sX[k * kLdX + 16 * qc + col]; }, 32, lane);
         warp_store16(c, [&](int r, int col, float v) { sT[(32 + 16 * qr + r) * kLdT + 16 * qc + col] = v; }, -1.f,
                      lane);
     }
-    named_bar(bar_id, kPrepThreads);
+    named_bar(bar_id, 128);
 }
 
 // One-time set-up of a prep pipeline's shared memory: the zero blocks around T diag(beta) and the
@@ -225,11 +226,13 @@ __device__ void prep_init(const PrepSmem& ps, int lt) {
 }
 
 // Computes the hand-off block of chunk c of head (b, h) into `out` (global memory). Executed by the
-// 128 threads of one pipeline; `it` counts the pipeline's previous tasks (mbarrier phase parity).
+// 256 threads of one pipeline (8 warps: TMEM lane quadrant q = warp & 3, column half hf = warp >> 2);
+// `it` counts the pipeline's previous tasks (mbarrier phase parity).
 template <int MODE>
 __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv,
                            const PrepSmem& ps, int b, int h, int c, uint8_t* __restrict__ out, uint32_t it, int lt) {
     const int lw = lt >> 5, lane = lt & 31;
+    const int q = lw & 3, hf = lw >> 2;
     const uint32_t par = it & 1u;
     uint8_t* sm = ps.base;
     uint8_t* sKQ = sm + kPKQ;
@@ -249,7 +252,8 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
     const int n = min(kC, T - c0);
     const size_t tok0 = ((size_t)b * T + c0) * H + h;  // chunk row r is token tok0 + r * H
 
-    // ---- 1. TMA: K and Q into the two halves of the 128-row [K; Q] tile, V
+    // ---- 1. TMA: K and Q into the two halves of the 128-row [K; Q] tile, V; beta and the
+    //         cumulative log-decay (log2 units; rows past the tail repeat Gamma_{n-1}) meanwhile
     if (lt == 0) {
         mbar_arrive_expect_tx(barT, 6 * 8192);
         tma_load_4d(sKQ, mk, 0, h, c0, b, barT);
@@ -259,10 +263,12 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
         tma_load_4d(sV, mv, 0, h, c0, b, barT);
         tma_load_4d(sV + 8192, mv, 64, h, c0, b, barT);
     }
-    // ---- 2. beta and the cumulative log-decay (log2 units; rows past the tail repeat Gamma_{n-1})
-    if (lt < kC) sBeta[lt] = (lt < n) ? P.beta[tok0 + (size_t)lt * H] : 0.f;
+    if (lw == 7) {
+        sBeta[lane] = (lane < n) ? P.beta[tok0 + (size_t)lane * H] : 0.f;
+        sBeta[lane + 32] = (lane + 32 < n) ? P.beta[tok0 + (size_t)(lane + 32) * H] : 0.f;
+    }
     if (MODE == GDR_DECAY_SCALAR) {
-        if (lw == 0) {
+        if (lw == 6) {
             float x0 = (lane < n) ? P.g[tok0 + (size_t)lane * H] * kLog2e : 0.f;
             float x1 = (lane + 32 < n) ? P.g[tok0 + (size_t)(lane + 32) * H] * kLog2e : 0.f;
 #pragma unroll
@@ -279,23 +285,38 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
             sGam[lane + 32] = x1;
         }
     } else if (MODE == GDR_DECAY_CHANNEL) {
-        float gv[kC];
+        if (lt < kD) {
+            float gv[kC];
 #pragma unroll
-        for (int r = 0; r < kC; ++r) gv[r] = (r < n) ? P.g[(tok0 + (size_t)r * H) * kD + lt] : 0.f;
-        float acc = 0.f;
+            for (int r = 0; r < kC; ++r) gv[r] = (r < n) ? P.g[(tok0 + (size_t)r * H) * kD + lt] : 0.f;
+            float acc = 0.f;
 #pragma unroll
-        for (int r = 0; r < kC; ++r) {
-            acc = fmaf(gv[r], kLog2e, acc);
-            sGam[r * kD + lt] = acc;
+            for (int r = 0; r < kC; ++r) {
+                acc = fmaf(gv[r], kLog2e, acc);
+                sGam[r * kD + lt] = acc;
+            }
         }
     }
     named_bar(ps.bar_id, kPrepThreads);
     mbar_wait(barT, par, P.status);
+    const uint32_t tG = ps.tmem + kTG, tW = ps.tmem + kTW, tU = ps.tmem + kTU;
+    // Gram products for the scalar gate / DeltaNet straight from the bf16 tiles
+    if (MODE != GDR_DECAY_CHANNEL && lt == 0) {
+        tc_fence_after();
+        const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t d = sdesc(smem_u32(sKQ) + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+            mma_f16(tG, d, d, id, ks > 0);  // B = the K rows (first 64 rows) of the same tile
+        }
+        mma_commit(barG);
+    }
 
-    // ---- 3. Q*gamma and K*gamma_C/gamma hand-off images; channel gate: decay-factored Gram operands
+    // ---- 2. Q*gamma and K*gamma_C/gamma hand-off images; channel gate: decay-factored Gram operands
     const int ref = (n - 1) >> 1;
     bool range_bad = false;
-    for (int j = 0; j < 8; ++j) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
         const int task = lt + kPrepThreads * j;
         const int r = task >> 4, col0 = (task & 15) * 8;
         const uint32_t okr = kmajor_off(r, col0, 128), oqr = kmajor_off(kC + r, col0, 128);
@@ -339,108 +360,100 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
         st16(out + kOffKT + mnmajor_off(r, col0, 64), pack8h(kt));
     }
     if (MODE == GDR_DECAY_CHANNEL && range_bad) report_status(P.status, GDR_ERR_RANGE);
-    {
+    if (lt < kD) {
         float gc = 1.f;
         if (MODE == GDR_DECAY_SCALAR) gc = fast_exp2(sGam[kC - 1]);
         if (MODE == GDR_DECAY_CHANNEL) gc = fast_exp2(sGam[(kC - 1) * kD + lt]);
         reinterpret_cast<float*>(out + kOffGam)[lt] = gc;
     }
-    if (MODE == GDR_DECAY_CHANNEL) fence_proxy_async_smem();
-    tc_fence_before();
-    named_bar(ps.bar_id, kPrepThreads);
-    tc_fence_after();
-
-    // ---- 4. Gram products: rows 0-63 K' K''^T, rows 64-127 Q' K''^T (M = 128, N = 64, K = 128)
-    const uint32_t tG = ps.tmem + kTG, tW = ps.tmem + kTW, tU = ps.tmem + kTU;
-    if (lt == 0) {
-        if (MODE == GDR_DECAY_CHANNEL) {
+    if (MODE == GDR_DECAY_CHANNEL) {
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar(ps.bar_id, kPrepThreads);
+        tc_fence_after();
+        if (lt == 0) {
             const uint32_t id = idesc_f16(128, 64, false, false);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
                 mma_f16(tG, sdesc(smem_u32(sKQ) + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
                         sdesc(smem_u32(sKB) + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id, ks > 0);
-        } else {
-            const uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t d = sdesc(smem_u32(sKQ) + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                mma_f16(tG, d, d, id, ks > 0);  // B = the K rows (first 64 rows) of the same tile
-            }
+            mma_commit(barG);
         }
-        mma_commit(barG);
     }
     __syncwarp();
     mbar_wait(barG, par, P.status);
     tc_fence_after();
 
-    // ---- 5. A (strictly lower, beta_r folded in; stored transposed) and P (causal incl. diagonal)
+    // ---- 3. A (strictly lower, beta_r folded in; stored transposed) and P (causal incl. diagonal):
+    //         thread (q, hf) takes TMEM lane 32 q + lane (K rows for q < 2, Q rows for q >= 2),
+    //         columns i in [32 hf, 32 hf + 32)
     {
-        const int rr = (lw & 1) * 32 + lane;
-        const uint32_t laddr = tG + ((uint32_t)(lw * 32) << 16);
+        const int rr = (q & 1) * 32 + lane;
+        float x[32];
+        tmem_ld32(tG + ((uint32_t)(q * 32) << 16) + 32 * hf, x);
+        float d[32];
+        if (MODE == GDR_DECAY_SCALAR) {
+            const float G2r = sGam[rr];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) d[e] = fast_exp2(fminf(G2r - sGam[32 * hf + e], 0.f));
+        }
         const float br = sBeta[rr];
-        const float G2r = (MODE == GDR_DECAY_SCALAR) ? sGam[rr] : 0.f;
-        for (int half = 0; half < 2; ++half) {
-            float x[32];
-            tmem_ld32(laddr + half * 32, x);
-            tmem_ld_wait();
-            if (lw < 2) {
+        tmem_ld_wait();
+        if (q < 2) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int i = half * 32 + e;
-                    float a = 0.f;
-                    if (i < rr && rr < n) {
-                        a = br * x[e];
-                        if (MODE == GDR_DECAY_SCALAR) a *= fast_exp2(G2r - sGam[i]);
-                    }
-                    sAt[i * kLdA + rr] = a;
-                }
-            } else {
-                float p[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int i = half * 32 + e;
-                    float v = 0.f;
-                    if (i <= rr && rr < n) {
-                        v = x[e];
-                        if (MODE == GDR_DECAY_SCALAR) v *= fast_exp2(G2r - sGam[i]);
-                    }
-                    p[e] = v;
-                }
-#pragma unroll
-                for (int ci = 0; ci < 4; ++ci)
-                    st16(out + kOffP + kmajor_off(rr, half * 32 + ci * 8, 64), pack8h(p + ci * 8));
+            for (int e = 0; e < 32; ++e) {
+                const int i = 32 * hf + e;
+                float a = (i < rr && rr < n) ? br * x[e] : 0.f;
+                if (MODE == GDR_DECAY_SCALAR) a *= d[e];
+                sAt[i * kLdA + rr] = a;
             }
+        } else {
+            float p[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int i = 32 * hf + e;
+                float v = (i <= rr && rr < n) ? x[e] : 0.f;
+                if (MODE == GDR_DECAY_SCALAR) v *= d[e];
+                p[e] = v;
+            }
+#pragma unroll
+            for (int ci = 0; ci < 4; ++ci) st16(out + kOffP + kmajor_off(rr, 32 * hf + ci * 8, 64), pack8h(p + ci * 8));
         }
     }
     tc_fence_before();
     named_bar(ps.bar_id, kPrepThreads);
 
-    // ---- 6. K*gamma (in place over the K rows) and V as fp16 operands of the W / U MMAs
-    for (int j = 0; j < 16; ++j) {
-        const int task = lt + kPrepThreads * j;
-        const bool isv = task >= 1024;
-        const int r = (task & 1023) >> 4, col0 = (task & 15) * 8;
-        uint8_t* p = isv ? sV + kmajor_off(r, col0, 64) : sKQ + kmajor_off(r, col0, 128);
-        float x[8];
-        if (!isv && MODE == GDR_DECAY_CHANNEL) {
-            unpack8h(ld16(p), x);  // K' = K e^{Gamma - Gamma_ref}: times e^{Gamma_ref} gives K*gamma
+    // ---- 4. warps 0-3: UT transform T = (I + A)^-1;  warps 4-7: K*gamma (in place over the K rows)
+    //         and V as fp16 operands of the W / U MMAs
+    if (lw < 4) {
+        unit_lower_inverse64(sAt, sT, sX, lt, ps.bar_id + 1);
+    } else {
+        const int lt4 = lt - 128;
+        for (int j = 0; j < 16; ++j) {
+            const int task = lt4 + 128 * j;
+            const bool isv = task >= 1024;
+            const int r = (task & 1023) >> 4, col0 = (task & 15) * 8;
+            uint8_t* p = isv ? sV + kmajor_off(r, col0, 64) : sKQ + kmajor_off(r, col0, 128);
+            float x[8];
+            if (!isv && MODE == GDR_DECAY_CHANNEL) {
+                unpack8h(ld16(p), x);  // K' = K e^{Gamma - Gamma_ref}: times e^{Gamma_ref} gives K*gamma
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] *= fast_exp2(sGam[ref * kD + col0 + e]);
-        } else {
-            unpack8bf(ld16(p), x);
-            if (!isv && MODE == GDR_DECAY_SCALAR) {
-                const float fr = fast_exp2(sGam[r]);
+                for (int e = 0; e < 8; ++e) x[e] *= fast_exp2(sGam[ref * kD + col0 + e]);
+            } else {
+                unpack8bf(ld16(p), x);
+                if (!isv && MODE == GDR_DECAY_SCALAR) {
+                    const float fr = fast_exp2(sGam[r]);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] *= fr;
+                    for (int e = 0; e < 8; ++e) x[e] *= fr;
+                }
             }
+            st16(p, pack8h(x));
         }
-        st16(p, pack8h(x));
     }
     named_bar(ps.bar_id, kPrepThreads);
-
-    // ---- 7. UT transform T = (I + A)^-1, then T diag(beta) as fp16
-    unit_lower_inverse64(sAt, sT, sX, lt, ps.bar_id);
-    for (int j = 0; j < 4; ++j) {
+    // T diag(beta) as fp16
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
         const int task = lt + kPrepThreads * j;
         const int r = task >> 3, i0 = (task & 7) * 8;
         float t8[8];
@@ -453,7 +466,7 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
     named_bar(ps.bar_id, kPrepThreads);
     tc_fence_after();
 
-    // ---- 8. W = [T diag(beta); 0] (K*gamma) (M = 128, N = 128) and U^T = V^T (T diag(beta))^T (M = 128, N = 64)
+    // ---- 5. W = [T diag(beta); 0] (K*gamma) (M = 128, N = 128) and U^T = V^T (T diag(beta))^T (M = 128, N = 64)
     if (lt == 0) {
         const uint32_t idW = idesc_f16(128, 128, false, true);
         const uint32_t idU = idesc_f16(128, 64, true, false);
@@ -468,30 +481,40 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
     __syncwarp();
     mbar_wait(barW, par, P.status);
     tc_fence_after();
+    // ---- 6. W rows and U^T rows to staging images (the K / V tiles are free now), bulk-stored out
     {
-        const int row = lw * 32 + lane;
-        const uint32_t loff = (uint32_t)(lw * 32) << 16;
-        if (lw < 2) {  // W row r = row (lanes 0-63 of the W accumulator)
-            for (int q4 = 0; q4 < 4; ++q4) {
+        uint8_t* stW = sKQ;  // W rows 0-63 in the 128-row K-major layout of the [W; Q*gamma] image
+        uint8_t* stU = sV;   // U^T, 128-row K-major (one 64-column block)
+        const uint32_t loff = (uint32_t)(q * 32) << 16;
+        const int row = q * 32 + lane;
+        if (q < 2) {
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
                 float x[32];
-                tmem_ld32(tW + loff + q4 * 32, x);
+                tmem_ld32(tW + loff + 64 * hf + 32 * q2, x);
                 tmem_ld_wait();
 #pragma unroll
                 for (int ci = 0; ci < 4; ++ci)
-                    st16(out + kOffWQ + kmajor_off(row, q4 * 32 + ci * 8, 128), pack8h(x + ci * 8));
+                    st16(stW + kmajor_off(row, 64 * hf + 32 * q2 + ci * 8, 128), pack8h(x + ci * 8));
             }
         }
-        for (int half = 0; half < 2; ++half) {  // U^T row j = row
-            float x[32];
-            tmem_ld32(tU + loff + half * 32, x);
-            tmem_ld_wait();
+        float x[32];
+        tmem_ld32(tU + loff + 32 * hf, x);
+        tmem_ld_wait();
 #pragma unroll
-            for (int ci = 0; ci < 4; ++ci)
-                st16(out + kOffUT + kmajor_off(row, half * 32 + ci * 8, 128), pack8h(x + ci * 8));
+        for (int ci = 0; ci < 4; ++ci) st16(stU + kmajor_off(row, 32 * hf + ci * 8, 128), pack8h(x + ci * 8));
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar(ps.bar_id, kPrepThreads);
+        if (lt == 0) {
+            bulk_s2g(out + kOffWQ, stW, 8192);
+            bulk_s2g(out + kOffWQ + 16384, stW + 16384, 8192);
+            bulk_s2g(out + kOffUT, stU, 16384);
+            bulk_commit();
+            bulk_wait<0>();
         }
+        named_bar(ps.bar_id, kPrepThreads);
     }
-    tc_fence_before();
-    named_bar(ps.bar_id, kPrepThreads);
 }
 
 // Standalone prep kernel: one pipeline per CTA, one chunk per CTA, hand-off blocks for all chunks.
@@ -653,15 +676,6 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const ui
         mbar_wait(&fullU, c & 1, A.status);
         mbar_wait(&barA[sb], (c >> 1) & 1, A.status);
         tc_fence_after();
-        // ---- output of chunk c-1 (its MMA-B completed before MMA-A of chunk c was issued)
-        if (c > 0) {
-            const uint32_t tO = tmem_base + kTD1 + (sb ^ 1) * 128 + 64;
-            float x[16];
-            tmem_ld16(tO + lane_off + 16 * cg, x);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) stage_out<Tout>(sO, 16 * cg + e, j, A.scale * x[e]);
-        }
         // ---- Delta^T[j][r] = U^T[j][r] - (S W^T)[j][r], r in [16 cg, 16 cg + 16)
         {
             float x[16], u[16];
@@ -679,7 +693,19 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const ui
         __syncthreads();
         tc_fence_after();
         if (tid == 0) {
-            if (c > 0) {  // output of chunk c-1
+            // D3 = Delta^T K~ (M = 128, N = 128, K = 64) first: the state update waits on it
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_f16(tmem_base + kTD3, sdesc(smem_u32(sDT) + ks * 32, 16, 1024),
+                        sdesc(smem_u32(st + kOffKT) + ks * 2048, 8192, 1024), idC, ks > 0);
+            mma_commit(&barC);
+            // D1[:, 64:128] += Delta^T P^T (N = 64): the output of chunk c
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_f16(tD1 + 64, sdesc(smem_u32(sDT) + ks * 32, 16, 1024),
+                        sdesc(smem_u32(st + kOffP) + ks * 32, 16, 1024), idB, true);
+            mma_commit(&barB);
+            if (c > 0) {  // output of chunk c-1, staged at the end of the previous iteration
                 for (int bx = 0; bx < kOutBoxes; ++bx)
                     tma_store_4d(&mo, sO + bx * 8192, bx * kOutBoxCols, h, (c - 1) * kC, b);
                 bulk_commit();
@@ -688,17 +714,6 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const ui
                 mbar_arrive_expect_tx(&fullU, 16384);
                 bulk_g2s(sUT, src + (size_t)(c + 1) * kHandoffStride + kOffUT, 16384, &fullU);
             }
-            // D3 = Delta^T K~ (M = 128, N = 128, K = 64), then D1[:, 64:128] += Delta^T P^T (N = 64)
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_f16(tmem_base + kTD3, sdesc(smem_u32(sDT) + ks * 32, 16, 1024),
-                        sdesc(smem_u32(st + kOffKT) + ks * 2048, 8192, 1024), idC, ks > 0);
-            mma_commit(&barC);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_f16(tD1 + 64, sdesc(smem_u32(sDT) + ks * 32, 16, 1024),
-                        sdesc(smem_u32(st + kOffP) + ks * 32, 16, 1024), idB, true);
-            mma_commit(&barB);
         }
         __syncwarp();
         mbar_wait(&barC, c & 1, A.status);
@@ -714,35 +729,32 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const ui
 #pragma unroll
             for (int ci = 0; ci < 4; ++ci) st16(sS + kmajor_off(j, 32 * cg + ci * 8, 128), pack8h(s + ci * 8));
         }
+        if (tid == 0) bulk_wait_read<0>();  // the output store of chunk c-1 has read the staging buffer
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        if (tid == 0) {
-            mbar_wait(&barB, c & 1, A.status);  // MMA-B done: stage A[sb] and the output columns are final
-            bulk_wait_read<0>();                // output staging may be rewritten
-            if (c + 2 < NC) {
-                mbar_arrive_expect_tx(&fullA[sb], kPartA);
-                bulk_g2s(stageA[sb], src + (size_t)(c + 2) * kHandoffStride, kPartA, &fullA[sb]);
-            }
-            if (c + 1 < NC) {
-                mbar_wait(&fullA[sb ^ 1], ((c + 1) >> 1) & 1, A.status);
-                tc_fence_after();
-                issue_A(c + 1);
-            }
+        if (tid == 0 && c + 1 < NC) {
+            mbar_wait(&fullA[sb ^ 1], ((c + 1) >> 1) & 1, A.status);
+            tc_fence_after();
+            issue_A(c + 1);
+        }
+        // ---- output of chunk c, overlapping the next chunk's first MMA (D1 is double-buffered)
+        mbar_wait(&barB, c & 1, A.status);
+        tc_fence_after();
+        {
+            float x[16];
+            tmem_ld16(tD1 + 64 + lane_off + 16 * cg, x);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) stage_out<Tout>(sO, 16 * cg + e, j, A.scale * x[e]);
+        }
+        if (tid == 0 && c + 2 < NC) {  // all MMAs of chunk c are done: refill its stage with chunk c+2
+            mbar_arrive_expect_tx(&fullA[sb], kPartA);
+            bulk_g2s(stageA[sb], src + (size_t)(c + 2) * kHandoffStride, kPartA, &fullA[sb]);
         }
     }
-    // ---- output of the last chunk
-    mbar_wait(&barB, (NC - 1) & 1, A.status);
-    tc_fence_after();
-    {
-        const uint32_t tO = tmem_base + kTD1 + ((NC - 1) & 1) * 128 + 64;
-        float x[16];
-        tmem_ld16(tO + lane_off + 16 * cg, x);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) stage_out<Tout>(sO, 16 * cg + e, j, A.scale * x[e]);
-    }
+    // ---- store the output of the last chunk
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
