@@ -549,16 +549,22 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
 }
 
 // ------------------------------------------------------------------- state pass --
-constexpr int kStateThreads = 512;
+// One CTA per (b, h): 16 epilogue warps (warp w reads TMEM lane quadrant w & 3 and column group
+// w >> 2) and one issuer warp (MMAs, bulk copies, output stores). The fp32 state lives in the
+// epilogue threads' registers; its fp16 copy and Delta^T live in TMEM as the A operands of the
+// MMAs, so the S-dependent products read only their B operands from shared memory. Epilogue
+// warps hand over to the issuer through mbarriers (one arrival per warp).
+constexpr int kEpiWarps = 16;
+constexpr int kStateThreads = (kEpiWarps + 1) * 32;
 constexpr uint32_t kSStageA0 = 0;
 constexpr uint32_t kSStageA1 = 58368;
 constexpr uint32_t kSUT = 116736;       // U^T stage (single buffer)
-constexpr uint32_t kSS = 133120;        // S fp16 K-major 128 x 128
-constexpr uint32_t kSDT = 165888;       // Delta^T fp16 K-major 128 x 64
-constexpr uint32_t kSO = 182272;        // output staging: 4 (fp32) or 2 (bf16) TMA boxes of 64 rows x 128 B
-constexpr uint32_t kStateSmem = kSO + 32768 + 1024;
-// TMEM: D1 double-buffered (corr^T | O^T, 128 columns each), D3 (state increment, 128 columns)
-constexpr uint32_t kTD1 = 0, kTD3 = 256, kStateTmemCols = 512;
+constexpr uint32_t kSO0 = 133120;       // output staging, double-buffered: 4 (fp32) or 2 (bf16) TMA boxes
+constexpr uint32_t kSO1 = 165888;       //   of 64 rows x 128 B each
+constexpr uint32_t kStateSmem = kSO1 + 32768 + 1024;
+// TMEM: D1 double-buffered (corr^T | O^T, 128 columns each), D3 (state increment), the fp16 state
+// copy (128 x 128 -> 64 columns) and Delta^T (128 x 64 fp16 -> 32 columns)
+constexpr uint32_t kTD1 = 0, kTD3 = 256, kTS = 384, kTDelta = 448, kStateTmemCols = 512;
 
 struct StateArgs {
     const float* S0;
@@ -582,7 +588,7 @@ __device__ __forceinline__ void stage_out<__nv_bfloat16>(uint8_t* sO, int r, int
         __float2bfloat16_rn(v);
 }
 
-// Walks the chunks of head (b, h) in order. `src(c)` gives chunk c's hand-off block.
+// Walks the chunks of head (b, h) in order, reading hand-off block c at ws + (bh * NC + c) * stride.
 template <typename Tout>
 __global__ void __launch_bounds__(kStateThreads, 1)
 chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const uint8_t* __restrict__ ws) {
@@ -590,188 +596,212 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const ui
     uint8_t* sm = align1024(smem_raw);
     uint8_t* stageA[2] = {sm + kSStageA0, sm + kSStageA1};
     uint8_t* sUT = sm + kSUT;
-    uint8_t* sS = sm + kSS;
-    uint8_t* sDT = sm + kSDT;
-    uint8_t* sO = sm + kSO;
-    __shared__ uint64_t fullA[2], fullU, barA[2], barB, barC;
+    uint8_t* sO[2] = {sm + kSO0, sm + kSO1};
+    // fullA/fullU: bulk copies landed. barA/barB/barC: MMA groups done. deltaReady/sReady/oStaged:
+    // all epilogue warps wrote Delta^T / the fp16 state (TMEM) / the output staging (shared).
+    // oFree[b]: the output staging buffer b has been read by its store.
+    __shared__ uint64_t fullA[2], fullU, barA[2], barB, barC, deltaReady, sReady, oStaged, oFree[2];
     __shared__ uint32_t tmem_base;
 
     const int bh = blockIdx.x;
     const int b = bh / A.H, h = bh % A.H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, cg = warp >> 2;  // TMEM lane quadrant, column group
-    const int j = quad * 32 + lane;             // state row (d_v index) = TMEM lane
     const int NC = A.NC;
     const uint8_t* src = ws + (size_t)bh * NC * kHandoffStride;
     constexpr int kOutBoxes = sizeof(Tout) == 4 ? 4 : 2;
     constexpr int kOutBoxCols = 128 / kOutBoxes;
 
     if (tid == 0) {
-        mbar_init(&fullA[0], 1);
-        mbar_init(&fullA[1], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&fullA[i], 1);
+            mbar_init(&barA[i], 1);
+            mbar_init(&oFree[i], 1);
+        }
         mbar_init(&fullU, 1);
-        mbar_init(&barA[0], 1);
-        mbar_init(&barA[1], 1);
         mbar_init(&barB, 1);
         mbar_init(&barC, 1);
+        mbar_init(&deltaReady, kEpiWarps);
+        mbar_init(&sReady, kEpiWarps);
+        mbar_init(&oStaged, kEpiWarps);
         fence_mbar_init();
     }
     if (warp == 0) {
         tmem_alloc(&tmem_base, kStateTmemCols);
         tmem_relinquish();
     }
-    // initial state: this thread holds S[j][32*cg .. 32*cg + 31] in fp32
-    float s[32];
-    {
-        const float* s0 = A.S0 ? A.S0 + ((size_t)bh * kD + j) * kD + 32 * cg : nullptr;
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-            const float4 t = s0 ? *reinterpret_cast<const float4*>(s0 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-            s[e] = t.x;
-            s[e + 1] = t.y;
-            s[e + 2] = t.z;
-            s[e + 3] = t.w;
-        }
-#pragma unroll
-        for (int ci = 0; ci < 4; ++ci) st16(sS + kmajor_off(j, 32 * cg + ci * 8, 128), pack8h(s + ci * 8));
-    }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t tD3 = tmem_base + kTD3;
-    const uint32_t idA = idesc_f16(128, 128, false, false);
-    const uint32_t idC = idesc_f16(128, 128, false, true);
-    const uint32_t idB = idesc_f16(128, 64, false, false);
+    const uint32_t tbase = tmem_base;
 
-    auto issue_A = [&](int c) {  // D1[c&1] = S [W; Q*gamma]^T (M = 128, N = 128, K = 128)
-        const uint8_t* st = stageA[c & 1];
-        const uint32_t d = tmem_base + kTD1 + (c & 1) * 128;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-            mma_f16(d, sdesc(smem_u32(sS) + koff, 16, 1024), sdesc(smem_u32(st + kOffWQ) + koff, 16, 1024), idA,
-                    ks > 0);
-        }
-        mma_commit(&barA[c & 1]);
-    };
-
-    if (tid == 0) {
-        for (int st = 0; st < 2 && st < NC; ++st) {
-            mbar_arrive_expect_tx(&fullA[st], kPartA);
-            bulk_g2s(stageA[st], src + (size_t)st * kHandoffStride, kPartA, &fullA[st]);
-        }
-        mbar_arrive_expect_tx(&fullU, 16384);
-        bulk_g2s(sUT, src + kOffUT, 16384, &fullU);
-        mbar_wait(&fullA[0], 0, A.status);
-        tc_fence_after();
-        issue_A(0);
-    }
-
-    for (int c = 0; c < NC; ++c) {
-        const int sb = c & 1;
-        const uint8_t* st = stageA[sb];
-        const uint32_t tD1 = tmem_base + kTD1 + sb * 128;
-        mbar_wait(&fullU, c & 1, A.status);
-        mbar_wait(&barA[sb], (c >> 1) & 1, A.status);
-        tc_fence_after();
-        // ---- Delta^T[j][r] = U^T[j][r] - (S W^T)[j][r], r in [16 cg, 16 cg + 16)
-        {
-            float x[16], u[16];
-            tmem_ld16(tD1 + lane_off + 16 * cg, x);
-            unpack8h(ld16(sUT + kmajor_off(j, 16 * cg, 128)), u);
-            unpack8h(ld16(sUT + kmajor_off(j, 16 * cg + 8, 128)), u + 8);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) u[e] -= x[e];
-            st16(sDT + kmajor_off(j, 16 * cg, 128), pack8h(u));
-            st16(sDT + kmajor_off(j, 16 * cg + 8, 128), pack8h(u + 8));
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (tid == 0) {
-            // D3 = Delta^T K~ (M = 128, N = 128, K = 64) first: the state update waits on it
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_f16(tmem_base + kTD3, sdesc(smem_u32(sDT) + ks * 32, 16, 1024),
-                        sdesc(smem_u32(st + kOffKT) + ks * 2048, 8192, 1024), idC, ks > 0);
-            mma_commit(&barC);
-            // D1[:, 64:128] += Delta^T P^T (N = 64): the output of chunk c
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_f16(tD1 + 64, sdesc(smem_u32(sDT) + ks * 32, 16, 1024),
-                        sdesc(smem_u32(st + kOffP) + ks * 32, 16, 1024), idB, true);
-            mma_commit(&barB);
-            if (c > 0) {  // output of chunk c-1, staged at the end of the previous iteration
-                for (int bx = 0; bx < kOutBoxes; ++bx)
-                    tma_store_4d(&mo, sO + bx * 8192, bx * kOutBoxCols, h, (c - 1) * kC, b);
-                bulk_commit();
+    if (warp == kEpiWarps) {
+        // ------------------------------------------------------------- issuer warp --
+        if (lane == 0) {
+            const uint32_t idA = idesc_f16(128, 128, false, false);
+            const uint32_t idC = idesc_f16(128, 128, false, true);
+            const uint32_t idB = idesc_f16(128, 64, false, false);
+            for (int st = 0; st < 2 && st < NC; ++st) {
+                mbar_arrive_expect_tx(&fullA[st], kPartA);
+                bulk_g2s(stageA[st], src + (size_t)st * kHandoffStride, kPartA, &fullA[st]);
             }
-            if (c + 1 < NC) {  // U^T of chunk c+1 (this chunk's has been consumed)
-                mbar_arrive_expect_tx(&fullU, 16384);
-                bulk_g2s(sUT, src + (size_t)(c + 1) * kHandoffStride + kOffUT, 16384, &fullU);
+            mbar_arrive_expect_tx(&fullU, 16384);
+            bulk_g2s(sUT, src + kOffUT, 16384, &fullU);
+            for (int c = 0; c < NC; ++c) {
+                const int sb = c & 1;
+                const uint8_t* st = stageA[sb];
+                const uint32_t tD1 = tbase + kTD1 + sb * 128;
+                // D1[sb] = S [W; Q*gamma]^T (M = 128, N = 128, K = 128), once the fp16 state is in TMEM
+                mbar_wait(&sReady, c & 1, A.status);
+                mbar_wait(&fullA[sb], (c >> 1) & 1, A.status);
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_f16_ts(tD1, tbase + kTS + ks * 8,
+                               sdesc(smem_u32(st + kOffWQ) + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024), idA,
+                               ks > 0);
+                mma_commit(&barA[sb]);
+                // output of chunk c-1 (staged by the epilogue warps in sO[(c-1)&1])
+                if (c > 0) {
+                    mbar_wait(&oStaged, (c - 1) & 1, A.status);
+                    const uint8_t* so = sO[(c - 1) & 1];
+                    for (int bx = 0; bx < kOutBoxes; ++bx)
+                        tma_store_4d(&mo, so + bx * 8192, bx * kOutBoxCols, h, (c - 1) * kC, b);
+                    bulk_commit();
+                    bulk_wait_read<1>();  // the store of chunk c-2 has read sO[c & 1]
+                    mbar_arrive(&oFree[c & 1]);
+                } else {
+                    mbar_arrive(&oFree[0]);
+                }
+                // D3 = Delta^T K~ (N = 128) and D1[sb][:, 64:128] += Delta^T P^T (N = 64)
+                mbar_wait(&deltaReady, c & 1, A.status);
+                tc_fence_after();
+                if (c + 1 < NC) {  // every epilogue warp has read U^T of chunk c
+                    mbar_arrive_expect_tx(&fullU, 16384);
+                    bulk_g2s(sUT, src + (size_t)(c + 1) * kHandoffStride + kOffUT, 16384, &fullU);
+                }
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16_ts(tbase + kTD3, tbase + kTDelta + ks * 8,
+                               sdesc(smem_u32(st + kOffKT) + ks * 2048, 8192, 1024), idC, ks > 0);
+                mma_commit(&barC);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16_ts(tD1 + 64, tbase + kTDelta + ks * 8, sdesc(smem_u32(st + kOffP) + ks * 32, 16, 1024),
+                               idB, true);
+                mma_commit(&barB);
+                // every MMA of chunk c is done and gamma_C has been read (sReady of chunk c+1 implies
+                // the state update of chunk c is complete): refill the stage with chunk c+2
+                if (c + 2 < NC) {
+                    mbar_wait(&barB, c & 1, A.status);
+                    mbar_wait(&sReady, (c + 1) & 1, A.status);
+                    mbar_arrive_expect_tx(&fullA[sb], kPartA);
+                    bulk_g2s(stageA[sb], src + (size_t)(c + 2) * kHandoffStride, kPartA, &fullA[sb]);
+                }
             }
+            // output of the last chunk
+            mbar_wait(&oStaged, (NC - 1) & 1, A.status);
+            const uint8_t* so = sO[(NC - 1) & 1];
+            for (int bx = 0; bx < kOutBoxes; ++bx) tma_store_4d(&mo, so + bx * 8192, bx * kOutBoxCols, h, (NC - 1) * kC, b);
+            bulk_commit();
+            bulk_wait<0>();
         }
         __syncwarp();
-        mbar_wait(&barC, c & 1, A.status);
-        tc_fence_after();
-        // ---- S <- S Diag(gamma_C) + Delta^T K~ on this thread's 32 columns, and its fp16 copy
+    } else {
+        // ---------------------------------------------------------- epilogue warps --
+        const int quad = warp & 3, cg = warp >> 2;
+        const int j = quad * 32 + lane;  // state row (d_v index) = TMEM lane
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const uint32_t tD3 = tbase + kTD3;
+        // initial state: this thread holds S[j][32 cg .. 32 cg + 31] in fp32
+        float s[32];
         {
-            const float* gam = reinterpret_cast<const float*>(st + kOffGam) + 32 * cg;
-            float x[32];
-            tmem_ld32(tD3 + lane_off + 32 * cg, x);
-            tmem_ld_wait();
+            const float* s0 = A.S0 ? A.S0 + ((size_t)bh * kD + j) * kD + 32 * cg : nullptr;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) s[e] = fmaf(gam[e], s[e], x[e]);
+            for (int e = 0; e < 32; e += 4) {
+                const float4 t = s0 ? *reinterpret_cast<const float4*>(s0 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+                s[e] = t.x;
+                s[e + 1] = t.y;
+                s[e + 2] = t.z;
+                s[e + 3] = t.w;
+            }
+            uint32_t w[16];
 #pragma unroll
-            for (int ci = 0; ci < 4; ++ci) st16(sS + kmajor_off(j, 32 * cg + ci * 8, 128), pack8h(s + ci * 8));
+            for (int e = 0; e < 16; ++e) w[e] = pack2h(s[2 * e], s[2 * e + 1]);
+            tmem_st16(tbase + kTS + lane_off + 16 * cg, w);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sReady);
         }
-        if (tid == 0) bulk_wait_read<0>();  // the output store of chunk c-1 has read the staging buffer
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (tid == 0 && c + 1 < NC) {
-            mbar_wait(&fullA[sb ^ 1], ((c + 1) >> 1) & 1, A.status);
+        for (int c = 0; c < NC; ++c) {
+            const int sb = c & 1;
+            const uint8_t* st = stageA[sb];
+            const uint32_t tD1 = tbase + kTD1 + sb * 128;
+            // ---- Delta^T[j][r] = U^T[j][r] - (S W^T)[j][r], r in [16 cg, 16 cg + 16), into TMEM
+            mbar_wait(&fullU, c & 1, A.status);
+            mbar_wait(&barA[sb], (c >> 1) & 1, A.status);
             tc_fence_after();
-            issue_A(c + 1);
-        }
-        // ---- output of chunk c, overlapping the next chunk's first MMA (D1 is double-buffered)
-        mbar_wait(&barB, c & 1, A.status);
-        tc_fence_after();
-        {
-            float x[16];
-            tmem_ld16(tD1 + 64 + lane_off + 16 * cg, x);
-            tmem_ld_wait();
+            {
+                float x[16], u[16];
+                tmem_ld16(tD1 + lane_off + 16 * cg, x);
+                unpack8h(ld16(sUT + kmajor_off(j, 16 * cg, 128)), u);
+                unpack8h(ld16(sUT + kmajor_off(j, 16 * cg + 8, 128)), u + 8);
+                tmem_ld_wait();
+                uint32_t w[8];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) stage_out<Tout>(sO, 16 * cg + e, j, A.scale * x[e]);
-        }
-        if (tid == 0 && c + 2 < NC) {  // all MMAs of chunk c are done: refill its stage with chunk c+2
-            mbar_arrive_expect_tx(&fullA[sb], kPartA);
-            bulk_g2s(stageA[sb], src + (size_t)(c + 2) * kHandoffStride, kPartA, &fullA[sb]);
-        }
-    }
-    // ---- store the output of the last chunk
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-        for (int bx = 0; bx < kOutBoxes; ++bx) tma_store_4d(&mo, sO + bx * 8192, bx * kOutBoxCols, h, (NC - 1) * kC, b);
-        bulk_commit();
-        bulk_wait<0>();
-    }
-    if (A.S_T != nullptr) {
-        float* dst = A.S_T + ((size_t)bh * kD + j) * kD + 32 * cg;
+                for (int e = 0; e < 8; ++e) w[e] = pack2h(u[2 * e] - x[2 * e], u[2 * e + 1] - x[2 * e + 1]);
+                tmem_st8(tbase + kTDelta + lane_off + 8 * cg, w);
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&deltaReady);
+            // ---- S <- S Diag(gamma_C) + Delta^T K~ on this thread's 32 columns; fp16 copy into TMEM
+            mbar_wait(&barC, c & 1, A.status);
+            tc_fence_after();
+            {
+                const float* gam = reinterpret_cast<const float*>(st + kOffGam) + 32 * cg;
+                float x[32];
+                tmem_ld32(tD3 + lane_off + 32 * cg, x);
+                tmem_ld_wait();
+                uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + e) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
+                for (int e = 0; e < 32; ++e) s[e] = fmaf(gam[e], s[e], x[e]);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) w[e] = pack2h(s[2 * e], s[2 * e + 1]);
+                tmem_st16(tbase + kTS + lane_off + 16 * cg, w);
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sReady);
+            // ---- output of chunk c into the staging buffer sO[sb]
+            mbar_wait(&barB, c & 1, A.status);
+            mbar_wait(&oFree[sb], (c >> 1) & 1, A.status);
+            tc_fence_after();
+            {
+                float x[16];
+                tmem_ld16(tD1 + 64 + lane_off + 16 * cg, x);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) stage_out<Tout>(sO[sb], 16 * cg + e, j, A.scale * x[e]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&oStaged);
+        }
+        if (A.S_T != nullptr) {
+            float* dst = A.S_T + ((size_t)bh * kD + j) * kD + 32 * cg;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4*>(dst + e) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
+        }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem_base, kStateTmemCols);
+    if (warp == 0) tmem_dealloc(tbase, kStateTmemCols);
 }
 
 // ---------------------------------------------------------------------- host --
