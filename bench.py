@@ -58,6 +58,18 @@ def chunk_bytes(w):
     return th * per_th + w.B * w.H * w.dv * w.dk * 4
 
 
+def kernel_bytes(w):
+    """Algorithmic HBM bytes per launch of each kernel of the two-pass tensor-core path: the prep
+    pass reads the method's inputs q, k, v, beta, g once; the state pass writes o and S_T once
+    (and reads S0 when given). The hand-off blocks the passes exchange through the workspace are
+    implementation traffic, not algorithmic bytes (they show up in the ncu DRAM counters)."""
+    eb = 2 if w.dtype == "bf16" else 4
+    th = w.B * w.T * w.H
+    g = 0 if w.mode == "none" else (4 if w.mode == "scalar" else 4 * w.dk)
+    return {"chunk_prep": th * (eb * (2 * w.dk + w.dv) + 4 + g),
+            "chunk_state": th * OUT_BYTES * w.dv + w.B * w.H * w.dv * w.dk * 4}
+
+
 def decode_bytes(w):
     """S read and written once (fp32), q, k, v read, o (fp32) written, beta and g read."""
     eb = 2 if w.dtype == "bf16" else 4
@@ -177,12 +189,25 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The maximum of a per-rank number over all ranks (device tensor under NCCL, host under gloo)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank, ms_per_step, world):
+    """Whole-job rate under weak scaling: every rank processes `units_per_rank` per step and the
+    step time is the slowest rank's (already the max over ranks)."""
+    return world * units_per_rank / (ms_per_step * 1e-3)
+
+
+def rank_seed(base, rank, input_set):
+    """Seed of one rank's input set: each rank runs its own independent batch."""
+    return base + 1000 * rank + input_set
 
 
 # ------------------------------------------------------------------- ours --
@@ -218,15 +243,26 @@ def run_ours(args):
     # two resident input sets, each larger than L2; one seed per rank (weak scaling)
     sets = []
     for s in range(2):
-        x = workload_inputs(w, seed=WORKLOAD_SEEDS[WORKLOAD] + 1000 * rank + s)
+        x = workload_inputs(w, seed=rank_seed(WORKLOAD_SEEDS[WORKLOAD], rank, s))
         sets.append({k: (None if t is None else t.to(dev)) for k, t in x.items()})
     o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=dev)
     st = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
     ws_n = gdr.workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.chunk, w.mode, torch.bfloat16, torch.float32)
     ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev) if ws_n else None
 
+    # per-kernel durations: an event before each step and one the library records after each of
+    # its kernels (gdr_profile_next_call), all on the launching stream
+    kernels_per_step = gdr_kernels_per_step(w)
+    names = ["chunk_prep", "chunk_state"] if kernels_per_step == 2 else [f"kernel{j}" for j in range(kernels_per_step)]
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(kernels_per_step)] for _ in range(args.steps)]
+    for e in ev0 + [e for row in evk for e in row]:
+        e.record(stream)  # creates the event (torch creates them lazily)
+
     def step(i=0):
         x = sets[i & 1]
+        ev0[i].record(stream)
+        gdr.profile_next_call(evk[i])
         gdr.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], mode=w.mode, chunk=w.chunk,
                       out=o, state_out=st, workspace=ws)
 
@@ -241,26 +277,45 @@ def run_ours(args):
     ms = max_over_ranks(ms, world)
     ms_step = ms / args.steps
     tokens = w.B * w.T
-    value = world * tokens / (ms_step * 1e-3)
+    value = job_throughput(tokens, ms_step, world)
 
     nbytes = chunk_bytes(w)
     flops = chunk_flops_per_token_head(w.chunk, w.dk, w.dv) * w.B * w.T * w.H
-    kernels_per_step = gdr_kernels_per_step(w)
     achieved_gbs = nbytes / (ms_step * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved_gbs / peaks["hbm_gbs"], 4), "traffic": traffic_from_profile(),
-                "peak_source": peak_src, "algorithmic_bytes_per_launch": nbytes,
-                "tensor_view": {"flops_per_launch": flops,
+    kb = kernel_bytes(w) if kernels_per_step == 2 else {names[0]: nbytes}
+    kernels = []
+    for j, name in enumerate(names):
+        us = [1e3 * (evk[i][j - 1] if j else ev0[i]).elapsed_time(evk[i][j]) for i in range(args.steps)]
+        us = max_over_ranks(statistics.mean(us), world)
+        gbs = kb[name] / (us * 1e-6) / 1e9
+        kernels.append({"kernel": name, "launch_us": round(us, 2), "share": None,
+                        "algorithmic_bytes_per_launch": kb[name], "achieved_gbs": round(gbs, 1),
+                        "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": traffic_from_profile(name)})
+    tot = sum(k["launch_us"] for k in kernels)
+    for k in kernels:
+        k["share"] = round(k["launch_us"] / tot, 4)
+    dom = max(kernels, key=lambda k: k["launch_us"])
+    roofline = {"bound": "hbm", "achieved": dom["achieved_gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": dom["frac"], "traffic": dom["traffic"], "kernel": dom["kernel"],
+                "launch_us": dom["launch_us"], "algorithmic_bytes_per_launch": dom["algorithmic_bytes_per_launch"],
+                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)" if peak_src == "measured"
+                else "fallback 6650 GB/s",
+                "kernels": kernels,
+                "step": {"achieved": round(achieved_gbs, 1), "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
+                         "algorithmic_bytes": nbytes,
+                         "roofline_us": round(max(nbytes / (peaks["hbm_gbs"] * 1e9),
+                                                  flops / (peaks["bf16_tflops"] * 1e12)) * 1e6, 2)},
+                "tensor_view": {"flops_per_step": flops,
                                 "achieved_tflops": round(flops / (ms_step * 1e-3) / 1e12, 1),
                                 "peak_tflops": peaks["bf16_tflops"],
-                                "frac": round(flops / (ms_step * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)},
-                "roofline_us": round(max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)) * 1e6, 2)}
+                                "frac": round(flops / (ms_step * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}}
 
     if args.only == "fwd":
         if rank == 0:
             print(json.dumps({"metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
                               "ms_per_step": round(ms_step, 5), "config": {"workload": WORKLOAD, "B": w.B},
-                              "roofline_frac": round(nbytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}))
+                              "roofline_frac": round(nbytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                              "kernels": [(k["kernel"], k["launch_us"]) for k in kernels]}))
         return
 
     # end to end: pinned host inputs -> device -> kernels -> host outputs, every step
@@ -287,7 +342,7 @@ def run_ours(args):
                    "decay": w.mode, "inputs": "bf16 q/k/v, fp32 g/beta, fp32 state; S0 = 0; returns o (fp32) and S_T",
                    "l2": "two resident input sets alternated, each 270 MB > 126 MB L2 (no flush)",
                    "parallelism": f"replicas x{world} (independent batches per GPU)"},
-        "e2e": {"value": round(world * tokens / (e2e_ms / e2e_steps * 1e-3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(job_throughput(tokens, e2e_ms / e2e_steps, world), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": kernels_per_step * args.steps,
         "roofline": roofline,
@@ -308,14 +363,21 @@ def gdr_kernels_per_step(w):
     return gdr.launches_per_chunk_fwd(w.B, w.T, w.H, w.dk, w.dv, w.chunk, w.mode, torch.bfloat16, torch.float32)
 
 
-def traffic_from_profile():
-    """DRAM bytes per launch from the committed ncu summary of the current kernel, if recorded."""
+def traffic_from_profile(kernel):
+    """DRAM bytes (read + write) per launch of `kernel` on this workload, from the committed ncu
+    summary (profiles/traffic.json), or None when none was recorded for the current kernel."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(path):
-        with open(path) as f:
-            d = json.load(f)
-        return d.get(WORKLOAD)
-    return None
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    src = os.path.join(ROOT, "gated_delta_rule_143_b200", "csrc", "gdr_chunk_tc.cu")
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    if not sha.startswith(d.get("_kernel_sha256_prefix", "-")):
+        return None  # the kernel changed since the counters were taken
+    return d.get(WORKLOAD, {}).get(kernel)
 
 
 def bench_decode(args, dev, peaks, world):

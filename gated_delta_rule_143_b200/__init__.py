@@ -20,7 +20,8 @@ import torch
 
 from ._lib import DECAY_MODES, DTYPE_BF16, DTYPE_F32, GdrError, check, lib
 
-__all__ = ["chunk_fwd", "decode_step", "sync_status", "workspace_bytes", "launches_per_chunk_fwd", "GdrError", "DECAY_MODES"]
+__all__ = ["chunk_fwd", "decode_step", "sync_status", "workspace_bytes", "launches_per_chunk_fwd", "profile_next_call",
+           "GdrError", "DECAY_MODES"]
 
 
 def _mode(mode) -> int:
@@ -150,3 +151,14 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optional[t
 def sync_status(stream: Optional[torch.cuda.Stream] = None) -> None:
     """Wait for the stream and raise if a kernel recorded a device-side error."""
     check(lib().gdr_sync_status(_stream_handle(stream)))
+
+
+def profile_next_call(events) -> None:
+    """Per-kernel timing: the next ``chunk_fwd`` on this thread records ``events[i]`` (created
+    ``torch.cuda.Event`` objects) right after enqueuing its i-th kernel, on its stream."""
+    import ctypes
+    handles = [int(e.cuda_event) for e in events]
+    if any(h == 0 for h in handles):
+        raise ValueError("record each event once before passing it (torch creates events lazily)")
+    arr = (ctypes.c_void_p * max(len(handles), 1))(*handles)
+    check(lib().gdr_profile_next_call(arr, len(handles)))

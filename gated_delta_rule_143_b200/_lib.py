@@ -30,6 +30,7 @@ SIGNATURES = {
     "gdr_chunk_fwd_launches": (_i, [_i] * 9),
     "gdr_decode_step": (_i, [_vp] * 7 + [_i] * 7 + [_vp]),
     "gdr_chunk_fwd_noalloc": (_i, [_vp] * 8 + [_i] * 9 + [_vp]),
+    "gdr_profile_next_call": (_i, [_vp, _i]),
     "gdr_sync_status": (_i, [_vp]),
     "gdr_last_error": (ctypes.c_char_p, []),
     "gdr_version": (_i, []),

@@ -27,6 +27,29 @@ int ok() {
     return GDR_OK;
 }
 
+// Per-kernel timing events for the next chunked forward on this thread (gdr_profile_next_call).
+// `pending` is set by the caller; the outermost chunk-forward entry point moves it to `active`
+// for the duration of the call and clears both on exit.
+struct ProfileEvents {
+    cudaEvent_t ev[8];
+    int n = 0, next = 0;
+};
+thread_local ProfileEvents g_prof_pending, g_prof_active;
+thread_local int g_prof_depth = 0;
+
+struct ProfileScope {
+    ProfileScope() {
+        if (g_prof_depth++ == 0) {
+            g_prof_active = g_prof_pending;
+            g_prof_active.next = 0;
+            g_prof_pending.n = 0;
+        }
+    }
+    ~ProfileScope() {
+        if (--g_prof_depth == 0) g_prof_active.n = 0;
+    }
+};
+
 // Device status word: kernels record the first device-side error here (a bounded wait that
 // expired). A statically sized __device__ variable, so it needs no allocation; each device
 // that loads the library has its own copy. Host code reaches it through its address.
@@ -93,6 +116,11 @@ int chunk_shape_check(int B, int T, int H, int dk, int dv, int chunk, int mode, 
 }
 
 }  // namespace
+
+void profile_after_launch(cudaStream_t stream) {
+    if (g_prof_active.next < g_prof_active.n) cudaEventRecord(g_prof_active.ev[g_prof_active.next++], stream);
+}
+
 }  // namespace gdr
 
 using namespace gdr;
@@ -100,6 +128,14 @@ using namespace gdr;
 extern "C" {
 
 int gdr_version(void) { return 100; }
+
+int gdr_profile_next_call(void* const* events, int n_events) {
+    if (n_events < 0 || n_events > 8) return fail(GDR_ERR_INVALID_ARG, "n_events = %d (0 .. 8)", n_events);
+    if (n_events > 0 && events == nullptr) return fail(GDR_ERR_INVALID_ARG, "events is NULL");
+    for (int i = 0; i < n_events; ++i) g_prof_pending.ev[i] = static_cast<cudaEvent_t>(events[i]);
+    g_prof_pending.n = n_events;
+    return ok();
+}
 
 const char* gdr_last_error(void) { return g_last_error; }
 
@@ -126,6 +162,7 @@ int gdr_chunk_fwd_launches(int B, int T, int H, int dk, int dv, int chunk, int m
 int gdr_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                   const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk,
                   int mode, int dtype, int o_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    ProfileScope prof_scope;
     if (int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype)) return rc;
     if (!q || !k || !v || !beta || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, beta and o must be non-null");
     if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
@@ -265,6 +302,7 @@ int noalloc_scratch(void** ptr) {
 extern "C" int gdr_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g, const float* beta,
                                      const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv,
                                      int chunk, int mode, int dtype, int o_dtype, void* stream) {
+    ProfileScope prof_scope;
     if (int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype)) return rc;
     if (!chunk_tc_supported(dk, dv, chunk, dtype, o_dtype))
         return fail(GDR_ERR_UNSUPPORTED,

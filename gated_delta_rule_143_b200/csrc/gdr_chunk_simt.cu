@@ -238,6 +238,7 @@ cudaError_t launch_typed(const ChunkProblem& p, cudaStream_t stream) {
     kern<<<grid, kThreads, smem, stream>>>(
         static_cast<const Tin*>(p.q), static_cast<const Tin*>(p.k), static_cast<const Tin*>(p.v), p.g, p.beta,
         p.S0, static_cast<Tout*>(p.o), p.S_T, p.T, p.H, p.dv, p.scale);
+    profile_after_launch(stream);
     return cudaGetLastError();
 }
 

@@ -511,7 +511,7 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
             bulk_s2g(out + kOffWQ + 16384, stW + 16384, 8192);
             bulk_s2g(out + kOffUT, stU, 16384);
             bulk_commit();
-            bulk_wait<0>();
+            bulk_wait_read<0>();  // the staging tiles may be reused; the writes complete on their own
         }
         named_bar(ps.bar_id, kPrepThreads);
     }
@@ -846,6 +846,7 @@ cudaError_t launch_prep(const ChunkProblem& p, const CUtensorMap& mq, const CUte
     if (err != cudaSuccess) return err;
     PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status};
     kern<<<dim3(NC, p.H, p.B), kPrepThreads, smem, stream>>>(mq, mk, mv, P, static_cast<uint8_t*>(p.workspace));
+    profile_after_launch(stream);
     return cudaGetLastError();
 }
 
@@ -856,6 +857,7 @@ cudaError_t launch_state(const ChunkProblem& p, const CUtensorMap& mo, int NC, c
     if (err != cudaSuccess) return err;
     StateArgs A{p.S0, p.S_T, p.T, p.H, NC, p.scale, p.status};
     kern<<<p.B * p.H, kStateThreads, kStateSmem, stream>>>(mo, A, static_cast<const uint8_t*>(p.workspace));
+    profile_after_launch(stream);
     return cudaGetLastError();
 }
 

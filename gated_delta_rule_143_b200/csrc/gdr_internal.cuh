@@ -68,6 +68,11 @@ __device__ __forceinline__ void store_f32<__nv_bfloat16>(__nv_bfloat16* p, float
 
 // CUDA-core fp32 chunked forward (any supported shape, fp32 or bf16 inputs).
 bool chunk_simt_supported(int dk, int dv, int chunk);
+// Records the next caller-supplied profiling event (gdr_profile_next_call) on `stream`, if one is
+// pending for the chunked forward in progress on this host thread. Launchers call it right after
+// each kernel launch.
+void profile_after_launch(cudaStream_t stream);
+
 cudaError_t launch_chunk_simt(const ChunkProblem& p, cudaStream_t stream);
 
 // Tensor-core (tcgen05) chunked forward: bf16, d_k = d_v = 128, chunk = 64.

@@ -138,6 +138,18 @@ int gdr_decode_step(const void* q, const void* k, const void* v, const float* g,
 int gdr_chunk_fwd_launches(int B, int T, int H, int d_k, int d_v, int chunk, int mode, int dtype,
                            int o_dtype);
 
+/* Diagnostics (no counterpart in the method): per-kernel timing of the next chunked forward.
+ * The next gdr_chunk_fwd or gdr_chunk_fwd_noalloc call made on the calling host thread records
+ * events[i] on its stream right after it enqueues its i-th kernel, for i < min(n_events,
+ * launches), then forgets the events; a call that fails validation forgets them too.
+ *   events    n_events cudaEvent_t handles created by the caller (owned by the caller; timing
+ *             events if durations are wanted). An event recorded by the caller before the call
+ *             and events[0] bracket the first kernel, events[i-1] and events[i] the i-th one.
+ *   n_events  0 .. 8; 0 clears a pending request.
+ * Returns GDR_OK, or GDR_ERR_INVALID_ARG for n_events outside 0 .. 8 or a NULL events array
+ * with n_events > 0. Host-only; enqueues nothing by itself. */
+int gdr_profile_next_call(void* const* events, int n_events);
+
 /* Size of the scratch area built into the library for gdr_chunk_fwd_noalloc: 32 MiB of device
  * memory on every GPU that loads the library, held until the process exits. */
 #define GDR_NOALLOC_SCRATCH_BYTES (32u << 20)

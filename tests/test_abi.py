@@ -93,3 +93,11 @@ def test_decode_rejects_bad_arguments_on_host(kw, code):
 def test_error_object_carries_status_name():
     e = _lib.GdrError(-3, "x")
     assert e.status == "GDR_ERR_MISALIGNED" and "x" in str(e)
+
+
+def test_profile_next_call_validates_on_host():
+    L = _lib.lib()
+    assert L.gdr_profile_next_call(None, 9) == -1
+    assert L.gdr_profile_next_call(None, -1) == -1
+    assert L.gdr_profile_next_call(None, 1) == -1
+    assert L.gdr_profile_next_call(None, 0) == 0  # clears; enqueues nothing

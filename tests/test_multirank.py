@@ -1,0 +1,77 @@
+"""Host side of the multi-GPU bench path, on CPU with two gloo ranks.
+
+Under torchrun every rank runs its own independent batch (weak scaling, no data-path collective):
+the only collectives are the barrier around the timed region and the max-over-ranks of the step
+time. These tests run that logic with world_size 2 on the gloo backend, plus the reference arm's
+rank handling (only rank 0 works and prints).
+"""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    import datetime
+
+    import bench
+    from gated_delta_rule_143_b200.inputs import CHUNK_WORKLOADS, WORKLOAD_SEEDS, make_chunk_inputs
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        bench.barrier(world)
+        # a per-rank "step time": the job's time is the slowest rank's
+        ms = bench.max_over_ranks(1.5 + rank, world)
+        w = CHUNK_WORKLOADS[bench.WORKLOAD]
+        seed = bench.rank_seed(WORKLOAD_SEEDS[bench.WORKLOAD], rank, 0)
+        # each rank's batch differs (small shapes stand in for the workload's)
+        x = make_chunk_inputs(1, 64, 2, 32, 32, w.mode, "bf16", seed)
+        digest = float(x["k"].float().sum())
+        bench.barrier(world)
+        with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+            json.dump({"ms": ms, "seed": seed, "digest": digest,
+                       "value": bench.job_throughput(w.B * w.T, ms, world)}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_agree_on_the_max_step_time(tmp_path):
+    world = 2
+    port = _free_port()
+    mp.start_processes(_rank_main, args=(world, port, str(tmp_path)), nprocs=world, join=True, start_method="spawn")
+    res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
+    assert res[0]["ms"] == res[1]["ms"] == 2.5  # max over ranks, seen identically by both
+    assert res[0]["seed"] != res[1]["seed"]
+    assert res[0]["digest"] != res[1]["digest"]  # independent batches per rank
+    # whole-job rate: both ranks' tokens over the slowest rank's time
+    assert res[0]["value"] == pytest.approx(2 * 8 * 4096 / 2.5e-3)
+
+
+def test_job_throughput_is_weak_scaling_sum():
+    import bench
+    assert bench.job_throughput(1000, 2.0, 1) == pytest.approx(5e5)
+    assert bench.job_throughput(1000, 2.0, 4) == pytest.approx(2e6)
+
+
+def test_reference_arm_nonzero_rank_exits_without_work():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""
