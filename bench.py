@@ -253,7 +253,8 @@ def run_ours(args):
     # per-kernel durations: an event before each step and one the library records after each of
     # its kernels (gdr_profile_next_call), all on the launching stream
     kernels_per_step = gdr_kernels_per_step(w)
-    names = ["chunk_prep", "chunk_state"] if kernels_per_step == 2 else [f"kernel{j}" for j in range(kernels_per_step)]
+    names = {1: ["chunk_fused"], 2: ["chunk_prep", "chunk_state"]}.get(kernels_per_step,
+                                                                     [f"kernel{j}" for j in range(kernels_per_step)])
     ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     evk = [[torch.cuda.Event(enable_timing=True) for _ in range(kernels_per_step)] for _ in range(args.steps)]
     for e in ev0 + [e for row in evk for e in row]:

@@ -311,10 +311,9 @@ extern "C" int gdr_chunk_fwd_noalloc(const void* q, const void* k, const void* v
     const size_t need = chunk_tc_workspace_bytes(B, T, H, dk, dv, chunk, mode);
     if (need > (size_t)GDR_NOALLOC_SCRATCH_BYTES)
         return fail(GDR_ERR_UNSUPPORTED,
-                    "this problem needs %zu bytes of scratch but the built-in area holds %zu "
-                    "(B * H * ceil(T / 64) must be <= %zu); use gdr_chunk_fwd with a workspace",
-                    need, (size_t)GDR_NOALLOC_SCRATCH_BYTES,
-                    (size_t)GDR_NOALLOC_SCRATCH_BYTES / (need / ((size_t)B * H * ((T + 63) / 64))));
+                    "this problem needs %zu bytes of scratch but the built-in area holds %zu; "
+                    "use gdr_chunk_fwd with a workspace",
+                    need, (size_t)GDR_NOALLOC_SCRATCH_BYTES);
     void* ws = nullptr;
     if (int rc = noalloc_scratch(&ws)) return rc;
     return gdr_chunk_fwd(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, ws,

@@ -48,6 +48,10 @@ constexpr int kC = 64;    // chunk length
 constexpr int kD = 128;   // d_k = d_v
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kF16Max = 65504.f;
+// Largest within-chunk spread of the cumulative log2-decay for which the scalar gate's pairwise
+// decays are taken as products 2^(G_r - G_ref) 2^(G_ref - G_i) around the mid value (both factors
+// within 2^+-100); beyond it they are computed one by one.
+constexpr float kFactorSpread = 200.f;
 
 // ------------------------------------------------------------------ hand-off block --
 // Per-chunk block in the workspace (byte offsets). Images are laid out exactly as the state
@@ -517,11 +521,285 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
     }
 }
 
-// Standalone prep kernel: one pipeline per CTA, one chunk per CTA, hand-off blocks for all chunks.
+// Optional steps the fused kernel's prep pipelines insert into a task (thread 0, right after the
+// task's TMA loads are issued): publish the previous task's block, then wait until the ring slot
+// of this task is free. All null / unused in the two-pass prep kernel.
+struct PrepHooks {
+    int* pub_flag = nullptr;          // release pub_value here once the previous block is complete
+    int pub_value = 0;
+    const int* slot_counter = nullptr;  // wait until *slot_counter >= slot_target
+    int slot_target = 0;
+    volatile int* go = nullptr;       // shared: 0 once a wait gave up (the task is skipped)
+    volatile int* abort = nullptr;
+};
+
+// Prep of one chunk for DeltaNet and the scalar gate (the channel gate uses prep_chunk): the same
+// hand-off block and step order as prep_chunk, with the tail taken off the pipeline's path: W and U^T
+// are staged in the A^T / T area (dead once T diag(beta) is formed) and bulk-stored without
+// waiting; the next task waits for those reads only before its A / P epilogue writes A^T, so its
+// loads, Gram MMA and output conversions overlap them. The pairwise decays are products of two
+// per-row factors when the chunk's decay spread allows. The caller makes the stores complete
+// (bulk_wait) before publishing or exiting. Returns false if a hook's wait gave up.
 template <int MODE>
-__global__ void __launch_bounds__(kPrepThreads)
+__device__ bool prep_chunk_sg(const PrepArgs& P, const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv,
+                              const PrepSmem& ps, int b, int h, int c, uint8_t* __restrict__ out, uint32_t it, int lt,
+                              const PrepHooks& hk) {
+    static_assert(MODE != GDR_DECAY_CHANNEL, "the channel gate uses prep_chunk");
+    const int lw = lt >> 5, lane = lt & 31;
+    const int q = lw & 3, hf = lw >> 2;
+    const uint32_t par = it & 1u;
+    uint8_t* sm = ps.base;
+    uint8_t* sKQ = sm + kPKQ;
+    uint8_t* sV = sm + kPV;
+    uint8_t* sTB = sm + kPTBZ + 8192;
+    uint8_t* stg = sm + kPA;  // W / U^T staging over A^T and T (32 KiB of 34 KiB)
+    float* sAt = reinterpret_cast<float*>(sm + kPA);
+    float* sT = reinterpret_cast<float*>(sm + kPT);
+    float* sX = reinterpret_cast<float*>(sm + kPX);
+    float* sDu = sX;       // 2^(G_r - G_ref), rows      } read by the A / P epilogue only, before the
+    float* sDv = sX + 64;  // 2^(G_ref - G_i), columns   } solve uses sX as scratch
+    int* sFact = reinterpret_cast<int*>(sX + 128);
+    float* sBeta = reinterpret_cast<float*>(sm + kPBeta);
+    float* sGam = reinterpret_cast<float*>(sm + kPGam);
+    uint64_t* barT = ps.bars;
+    uint64_t* barG = ps.bars + 1;
+    uint64_t* barW = ps.bars + 2;
+    const int T = P.T, H = P.H;
+    const int c0 = c * kC;
+    const int n = min(kC, T - c0);
+    const size_t tok0 = ((size_t)b * T + c0) * H + h;  // chunk row r is token tok0 + r * H
+
+    // ---- 1. TMA loads; beta and the cumulative log2-decay meanwhile (rows past the tail repeat
+    //         Gamma_{n-1}), with the factors of the pairwise decays around the mid value
+    if (lt == 0) {
+        mbar_arrive_expect_tx(barT, 6 * 8192);
+        tma_load_4d(sKQ, mk, 0, h, c0, b, barT);
+        tma_load_4d(sKQ + 16384, mk, 64, h, c0, b, barT);
+        tma_load_4d(sKQ + 8192, mq, 0, h, c0, b, barT);
+        tma_load_4d(sKQ + 24576, mq, 64, h, c0, b, barT);
+        tma_load_4d(sV, mv, 0, h, c0, b, barT);
+        tma_load_4d(sV + 8192, mv, 64, h, c0, b, barT);
+        bool go = true;
+        if (hk.pub_flag != nullptr) {  // the previous block: its bulk stores complete, then release
+            bulk_wait<0>();
+            fence_proxy_async_global();
+            __threadfence();
+            st_release_gpu(hk.pub_flag, hk.pub_value);
+        }
+        if (hk.slot_counter != nullptr) go = flag_wait_geq(hk.slot_counter, hk.slot_target, P.status, hk.abort, 2048);
+        if (hk.go != nullptr) *hk.go = go;
+        bulk_wait_read<0>();  // the previous W / U^T staging (over A^T / T) has been read
+    }
+    if (lw == 7) {
+        sBeta[lane] = (lane < n) ? P.beta[tok0 + (size_t)lane * H] : 0.f;
+        sBeta[lane + 32] = (lane + 32 < n) ? P.beta[tok0 + (size_t)(lane + 32) * H] : 0.f;
+    }
+    if (MODE == GDR_DECAY_SCALAR && lw == 6) {
+        float x0 = (lane < n) ? P.g[tok0 + (size_t)lane * H] * kLog2e : 0.f;
+        float x1 = (lane + 32 < n) ? P.g[tok0 + (size_t)(lane + 32) * H] * kLog2e : 0.f;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
+            const float y1 = __shfl_up_sync(0xffffffffu, x1, off);
+            if (lane >= off) {
+                x0 += y0;
+                x1 += y1;
+            }
+        }
+        x1 += __shfl_sync(0xffffffffu, x0, 31);
+        const float g0 = __shfl_sync(0xffffffffu, x0, 0), gC = __shfl_sync(0xffffffffu, x1, 31);
+        const float gref = 0.5f * (g0 + gC);
+        sGam[lane] = x0;
+        sGam[lane + 32] = x1;
+        sDu[lane] = fast_exp2(x0 - gref);
+        sDu[lane + 32] = fast_exp2(x1 - gref);
+        sDv[lane] = fast_exp2(gref - x0);
+        sDv[lane + 32] = fast_exp2(gref - x1);
+        if (lane == 0) *sFact = (g0 - gC) <= kFactorSpread;
+    }
+    named_bar(ps.bar_id, kPrepThreads);
+    if (hk.go != nullptr && !*hk.go) {
+        if (lt == 0) mbar_wait(barT, par, P.status);  // the loads land before shared memory is reused
+        return false;
+    }
+    mbar_wait(barT, par, P.status);
+    const uint32_t tG = ps.tmem + kTG, tW = ps.tmem + kTW, tU = ps.tmem + kTU;
+    if (lt == 0) {  // Gram products straight from the bf16 tiles
+        tc_fence_after();
+        const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t d = sdesc(smem_u32(sKQ) + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+            mma_f16(tG, d, d, id, ks > 0);  // B = the K rows (first 64 rows) of the same tile
+        }
+        mma_commit(barG);
+    }
+    // ---- 2. while the Gram MMA runs: Q*gamma and K*gamma_C/gamma hand-off images (all 8 warps,
+    //         from the bf16 tiles, which stay unchanged until step 4)
+    {
+        const float GC = MODE == GDR_DECAY_SCALAR ? sGam[kC - 1] : 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int task = lt + kPrepThreads * j;
+            const int r = task >> 4, col0 = (task & 15) * 8;
+            const uint32_t ok = kmajor_off(r, col0, 128), oq = kmajor_off(kC + r, col0, 128);
+            float kx[8], qx[8];
+            unpack8bf(ld16(sKQ + ok), kx);
+            unpack8bf(ld16(sKQ + oq), qx);
+            if (MODE == GDR_DECAY_SCALAR) {
+                const float fr = fast_exp2(sGam[r]), ft = fast_exp2(GC - sGam[r]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    qx[e] *= fr;
+                    kx[e] *= ft;
+                }
+            }
+            st16(out + kOffWQ + oq, pack8h(qx));
+            st16(out + kOffKT + mnmajor_off(r, col0, 64), pack8h(kx));
+        }
+        if (lt < kD) reinterpret_cast<float*>(out + kOffGam)[lt] = MODE == GDR_DECAY_SCALAR ? fast_exp2(GC) : 1.f;
+    }
+    __syncwarp();
+    mbar_wait(barG, par, P.status);
+    tc_fence_after();
+
+    // ---- 3. A (strictly lower, beta_r folded in; stored transposed) and P (causal incl. diagonal):
+    //         thread (q, hf) takes TMEM lane 32 q + lane (K rows for q < 2, Q rows for q >= 2),
+    //         columns i in [32 hf, 32 hf + 32)
+    {
+        const int rr = (q & 1) * 32 + lane;
+        float x[32];
+        tmem_ld32(tG + ((uint32_t)(q * 32) << 16) + 32 * hf, x);
+        const bool factored = MODE == GDR_DECAY_SCALAR && *sFact;
+        const float G2r = MODE == GDR_DECAY_SCALAR ? sGam[rr] : 0.f;
+        const float ur = MODE == GDR_DECAY_SCALAR && factored ? sDu[rr] : 1.f;
+        auto decay = [&](int i) {
+            if (MODE != GDR_DECAY_SCALAR) return 1.f;
+            return factored ? sDv[i] : fast_exp2(fminf(G2r - sGam[i], 0.f));
+        };
+        tmem_ld_wait();
+        if (q < 2) {
+            const float br = sBeta[rr] * ur;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int i = 32 * hf + e;
+                sAt[i * kLdA + rr] = (i < rr && rr < n) ? br * x[e] * decay(i) : 0.f;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int i = 32 * hf + e;
+                x[e] = (i <= rr && rr < n) ? ur * x[e] * decay(i) : 0.f;
+            }
+#pragma unroll
+            for (int ci = 0; ci < 4; ++ci) st16(out + kOffP + kmajor_off(rr, 32 * hf + ci * 8, 64), pack8h(x + ci * 8));
+        }
+    }
+    tc_fence_before();
+    named_bar(ps.bar_id, kPrepThreads);
+
+    // ---- 4. warps 0-3: T = (I + A)^-1;  warps 4-7: K*gamma and V as fp16, in place (the W / U^T
+    //         MMA operands)
+    if (lw < 4) {
+        // the upper blocks of T the solve and TB read as zero held the previous staging
+        for (int i = lt; i < 1536; i += 128) {
+            int r, col;
+            if (i < 256) { r = i >> 4; col = 16 + (i & 15); }                   // T[0:16, 16:32]
+            else if (i < 512) { r = 32 + ((i - 256) >> 4); col = 48 + (i & 15); }  // T[32:48, 48:64]
+            else { r = (i - 512) >> 5; col = 32 + (i & 31); }                  // T[0:32, 32:64]
+            sT[r * kLdT + col] = 0.f;
+        }
+        named_bar(ps.bar_id + 1, 128);
+        unit_lower_inverse64(sAt, sT, sX, lt, ps.bar_id + 1);
+    } else {
+        const int lt4 = lt - 128;
+        for (int j = 0; j < 16; ++j) {
+            const int task = lt4 + 128 * j;
+            const bool isv = task >= 1024;
+            const int r = (task & 1023) >> 4, col0 = (task & 15) * 8;
+            uint8_t* p = isv ? sV + kmajor_off(r, col0, 64) : sKQ + kmajor_off(r, col0, 128);
+            float x[8];
+            unpack8bf(ld16(p), x);
+            if (!isv && MODE == GDR_DECAY_SCALAR) {
+                const float fr = fast_exp2(sGam[r]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] *= fr;
+            }
+            st16(p, pack8h(x));
+        }
+    }
+    named_bar(ps.bar_id, kPrepThreads);
+    // T diag(beta) as fp16
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int task = lt + kPrepThreads * j;
+        const int r = task >> 3, i0 = (task & 7) * 8;
+        float t8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t8[e] = sT[r * kLdT + i0 + e] * sBeta[i0 + e];
+        st16(sTB + kmajor_off(r, i0, 64), pack8h(t8));
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    named_bar(ps.bar_id, kPrepThreads);
+    tc_fence_after();
+
+    // ---- 5. W = [T diag(beta); 0] (K*gamma) (M = 128, N = 128) and U^T = V^T (T diag(beta))^T (M = 128, N = 64)
+    if (lt == 0) {
+        const uint32_t idW = idesc_f16(128, 128, false, true);
+        const uint32_t idU = idesc_f16(128, 64, true, false);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t tb = sdesc(smem_u32(sTB) + ks * 32, 16, 1024);
+            mma_f16(tW, tb, sdesc(smem_u32(sKQ) + ks * 2048, 16384, 1024), idW, ks > 0);
+            mma_f16(tU, sdesc(smem_u32(sV) + ks * 2048, 8192, 1024), tb, idU, ks > 0);
+        }
+        mma_commit(barW);
+    }
+    __syncwarp();
+    mbar_wait(barW, par, P.status);
+    tc_fence_after();
+    // ---- 6. W rows (stg: two 64-row K-major blocks) and U^T (stg + 16 KiB: 128-row K-major) staged
+    //         over A^T / T, then bulk-stored
+    {
+        const uint32_t loff = (uint32_t)(q * 32) << 16;
+        const int row = q * 32 + lane;
+        if (q < 2) {
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+                float x[32];
+                tmem_ld32(tW + loff + 64 * hf + 32 * q2, x);
+                tmem_ld_wait();
+#pragma unroll
+                for (int ci = 0; ci < 4; ++ci)
+                    st16(stg + kmajor_off(row, 64 * hf + 32 * q2 + ci * 8, 64), pack8h(x + ci * 8));
+            }
+        }
+        float x[32];
+        tmem_ld32(tU + loff + 32 * hf, x);
+        tmem_ld_wait();
+#pragma unroll
+        for (int ci = 0; ci < 4; ++ci) st16(stg + 16384 + kmajor_off(row, 32 * hf + ci * 8, 128), pack8h(x + ci * 8));
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar(ps.bar_id, kPrepThreads);
+        if (lt == 0) {
+            bulk_s2g(out + kOffWQ, stg, 8192);
+            bulk_s2g(out + kOffWQ + 16384, stg + 8192, 8192);
+            bulk_s2g(out + kOffUT, stg + 16384, 16384);
+            bulk_commit();
+        }
+    }
+    return true;
+}
+
+// Standalone prep kernel (two-pass path): one pipeline per CTA, persistent over the chunk tasks
+// t = blockIdx.x, blockIdx.x + gridDim.x, ... (t = (b * H + h) * NC + c, the block's index in the
+// workspace). At the start of each task the tiles of the CTA's next task are prefetched into L2.
+template <int MODE>
+__global__ void __launch_bounds__(kPrepThreads, MODE == GDR_DECAY_CHANNEL ? 1 : 2)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-                  const __grid_constant__ CUtensorMap mv, PrepArgs P, uint8_t* __restrict__ ws) {
+                  const __grid_constant__ CUtensorMap mv, PrepArgs P, uint8_t* __restrict__ ws, int n_tasks) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bars[3];
     __shared__ uint32_t tmem_base;
@@ -540,9 +818,25 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     ps.tmem = tmem_base;
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    uint8_t* out = ws + ((size_t)(b * P.H + h) * P.NC + c) * kHandoffStride;
-    prep_chunk<MODE>(P, &mq, &mk, &mv, ps, b, h, c, out, 0u, lt);
+    uint32_t it = 0;
+    for (int t = blockIdx.x; t < n_tasks; t += gridDim.x, ++it) {
+        const int c = t % P.NC, bh = t / P.NC;
+        const int h = bh % P.H, b = bh / P.H;
+        const int tn = t + gridDim.x;
+        if (lt == 0 && tn < n_tasks) {
+            const int cn = tn % P.NC, bhn = tn / P.NC;
+            const int hn = bhn % P.H, bn = bhn / P.H;
+            tma_prefetch_l2_4d(&mk, 0, hn, cn * kC, bn);
+            tma_prefetch_l2_4d(&mk, 64, hn, cn * kC, bn);
+            tma_prefetch_l2_4d(&mq, 0, hn, cn * kC, bn);
+            tma_prefetch_l2_4d(&mq, 64, hn, cn * kC, bn);
+            tma_prefetch_l2_4d(&mv, 0, hn, cn * kC, bn);
+            tma_prefetch_l2_4d(&mv, 64, hn, cn * kC, bn);
+        }
+        uint8_t* out = ws + (size_t)t * kHandoffStride;
+        prep_chunk<MODE>(P, &mq, &mk, &mv, ps, b, h, c, out, it, lt);
+    }
+    if (lt == 0) bulk_wait<0>();
     tc_fence_before();
     __syncthreads();
     if (lt < 32) tmem_dealloc(tmem_base, kPrepTmemCols);
@@ -555,7 +849,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
 // MMAs, so the S-dependent products read only their B operands from shared memory. Epilogue
 // warps hand over to the issuer through mbarriers (one arrival per warp).
 constexpr int kEpiWarps = 16;
-constexpr int kStateThreads = (kEpiWarps + 1) * 32;
+constexpr int kStateThreads = (kEpiWarps + 2) * 32;  // + MMA issuer warp + copy warp
 constexpr uint32_t kSStageA0 = 0;
 constexpr uint32_t kSStageA1 = 58368;
 constexpr uint32_t kSUT = 116736;       // U^T stage (single buffer)
@@ -588,28 +882,50 @@ __device__ __forceinline__ void stage_out<__nv_bfloat16>(uint8_t* sO, int r, int
         __float2bfloat16_rn(v);
 }
 
-// Walks the chunks of head (b, h) in order, reading hand-off block c at ws + (bh * NC + c) * stride.
-template <typename Tout>
-__global__ void __launch_bounds__(kStateThreads, 1)
-chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const uint8_t* __restrict__ ws) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = align1024(smem_raw);
+// Where the state pass finds hand-off block c of its head, when that block is complete, and how it
+// tells the producer that the block has been copied out.
+struct WorkspaceSource {  // two passes: every block was written before the state pass started
+    const uint8_t* base;  // block 0 of this head
+    size_t cstep;         // bytes from block c to block c + 1
+    __device__ const uint8_t* block(int c) const { return base + (size_t)c * cstep; }
+    __device__ bool wait_ready(int, int*, volatile int*) const { return true; }
+    __device__ void release(int) const {}
+};
+
+constexpr int kRing = 8;  // ring slots per head in the fused kernel
+struct RingSource {       // fused kernel: blocks pass through kRing slots per head, flagged by the producers
+    const uint8_t* base;  // slot 0 of this head
+    const int* ready;     // [kRing]: c + 1 once the block of chunk c in that slot is complete
+    int* consumed;        // number of this head's chunks already copied out of the ring
+    __device__ const uint8_t* block(int c) const { return base + (size_t)(c % kRing) * kHandoffStride; }
+    __device__ bool wait_ready(int c, int* status, volatile int* abort) const {
+        if (!flag_wait_geq(ready + c % kRing, c + 1, status, abort, 128)) return false;
+        fence_proxy_async_global();  // the bulk copies that follow read what the acquire made visible
+        return true;
+    }
+    __device__ void release(int c) const { st_release_gpu(consumed, c + 1); }
+};
+
+// The state pass of one head (b, h) = bh, executed by all kStateThreads threads of the CTA, with
+// kStateTmemCols TMEM columns at tbase and kStateSmem bytes of shared memory at sm (1024-aligned).
+// Walks the chunks in order, reading hand-off block c through `src`.
+template <typename Tout, typename Src>
+__device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, const Src& src, uint8_t* sm,
+                           uint32_t tbase, volatile int* abort) {
     uint8_t* stageA[2] = {sm + kSStageA0, sm + kSStageA1};
     uint8_t* sUT = sm + kSUT;
     uint8_t* sO[2] = {sm + kSO0, sm + kSO1};
     // fullA/fullU: bulk copies landed. barA/barB/barC: MMA groups done. deltaReady/sReady/oStaged:
     // all epilogue warps wrote Delta^T / the fp16 state (TMEM) / the output staging (shared).
-    // oFree[b]: the output staging buffer b has been read by its store.
-    __shared__ uint64_t fullA[2], fullU, barA[2], barB, barC, deltaReady, sReady, oStaged, oFree[2];
-    __shared__ uint32_t tmem_base;
+    // oFree[b]: the output staging buffer b has been read by its store. drain: last MMAs complete.
+    __shared__ uint64_t fullA[2], fullU, barA[2], barB, barC, deltaReady, sReady, oStaged, oFree[2], drain;
 
-    const int bh = blockIdx.x;
     const int b = bh / A.H, h = bh % A.H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int NC = A.NC;
-    const uint8_t* src = ws + (size_t)bh * NC * kHandoffStride;
     constexpr int kOutBoxes = sizeof(Tout) == 4 ? 4 : 2;
     constexpr int kOutBoxCols = 128 / kOutBoxes;
+    auto wait = [&](uint64_t* bar, uint32_t parity) { return mbar_wait_abort(bar, parity, A.status, abort); };
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -620,39 +936,74 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const ui
         mbar_init(&fullU, 1);
         mbar_init(&barB, 1);
         mbar_init(&barC, 1);
+        mbar_init(&drain, 1);
         mbar_init(&deltaReady, kEpiWarps);
         mbar_init(&sReady, kEpiWarps);
         mbar_init(&oStaged, kEpiWarps);
         fence_mbar_init();
     }
-    if (warp == 0) {
-        tmem_alloc(&tmem_base, kStateTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
     __syncthreads();
-    tc_fence_after();
-    const uint32_t tbase = tmem_base;
 
-    if (warp == kEpiWarps) {
+    if (warp == kEpiWarps + 1) {
+        // --------------------------------------------------------------- copy warp --
+        // Brings hand-off blocks into shared memory (part A double-buffered, U^T single-buffered)
+        // as soon as both the block is ready and its buffer is free, and hands each ring slot back
+        // once both parts of its chunk are in shared memory: all flag traffic stays off the MMA
+        // issuer's path.
+        if (lane == 0) {
+            int lastA[2] = {-1, -1}, lastU = -1;  // last chunk whose part A / U^T copy was issued
+            bool ok = true;
+            for (int st = 0; st < 2 && st < NC && ok; ++st) {
+                if (!(ok = src.wait_ready(st, A.status, abort))) break;
+                mbar_arrive_expect_tx(&fullA[st], kPartA);
+                bulk_g2s(stageA[st], src.block(st), kPartA, &fullA[st]);
+                lastA[st] = st;
+            }
+            if (ok) {
+                mbar_arrive_expect_tx(&fullU, 16384);
+                bulk_g2s(sUT, src.block(0) + kOffUT, 16384, &fullU);
+                lastU = 0;
+            }
+            for (int c = 0; ok && c < NC; ++c) {
+                const int sb = c & 1;
+                // every epilogue warp has read U^T of chunk c (and waited for it), so both parts of
+                // chunk c are in shared memory: the ring slot goes back; U^T of chunk c + 1 comes in
+                if (!wait(&deltaReady, c & 1)) break;
+                src.release(c);
+                if (c + 1 < NC) {
+                    mbar_arrive_expect_tx(&fullU, 16384);
+                    bulk_g2s(sUT, src.block(c + 1) + kOffUT, 16384, &fullU);
+                    lastU = c + 1;
+                }
+                // stage sb is free once every MMA of chunk c is done and gamma_C has been read
+                // (sReady of chunk c + 1): chunk c + 2 comes in
+                if (c + 2 < NC) {
+                    if (!wait(&barB, c & 1) || !wait(&sReady, (c + 1) & 1)) break;
+                    if (!src.wait_ready(c + 2, A.status, abort)) break;
+                    mbar_arrive_expect_tx(&fullA[sb], kPartA);
+                    bulk_g2s(stageA[sb], src.block(c + 2), kPartA, &fullA[sb]);
+                    lastA[sb] = c + 2;
+                }
+            }
+            // every copy issued lands before shared memory is released
+            for (int sb = 0; sb < 2; ++sb)
+                if (lastA[sb] >= 0) mbar_wait(&fullA[sb], (lastA[sb] >> 1) & 1, A.status);
+            if (lastU >= 0) mbar_wait(&fullU, lastU & 1, A.status);
+        }
+        __syncwarp();
+    } else if (warp == kEpiWarps) {
         // ------------------------------------------------------------- issuer warp --
         if (lane == 0) {
             const uint32_t idA = idesc_f16(128, 128, false, false);
             const uint32_t idC = idesc_f16(128, 128, false, true);
             const uint32_t idB = idesc_f16(128, 64, false, false);
-            for (int st = 0; st < 2 && st < NC; ++st) {
-                mbar_arrive_expect_tx(&fullA[st], kPartA);
-                bulk_g2s(stageA[st], src + (size_t)st * kHandoffStride, kPartA, &fullA[st]);
-            }
-            mbar_arrive_expect_tx(&fullU, 16384);
-            bulk_g2s(sUT, src + kOffUT, 16384, &fullU);
-            for (int c = 0; c < NC; ++c) {
+            int c = 0;
+            for (; c < NC; ++c) {
                 const int sb = c & 1;
                 const uint8_t* st = stageA[sb];
                 const uint32_t tD1 = tbase + kTD1 + sb * 128;
                 // D1[sb] = S [W; Q*gamma]^T (M = 128, N = 128, K = 128), once the fp16 state is in TMEM
-                mbar_wait(&sReady, c & 1, A.status);
-                mbar_wait(&fullA[sb], (c >> 1) & 1, A.status);
+                if (!wait(&sReady, c & 1) || !wait(&fullA[sb], (c >> 1) & 1)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
@@ -662,10 +1013,10 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const ui
                 mma_commit(&barA[sb]);
                 // output of chunk c-1 (staged by the epilogue warps in sO[(c-1)&1])
                 if (c > 0) {
-                    mbar_wait(&oStaged, (c - 1) & 1, A.status);
+                    if (!wait(&oStaged, (c - 1) & 1)) break;
                     const uint8_t* so = sO[(c - 1) & 1];
                     for (int bx = 0; bx < kOutBoxes; ++bx)
-                        tma_store_4d(&mo, so + bx * 8192, bx * kOutBoxCols, h, (c - 1) * kC, b);
+                        tma_store_4d(mo, so + bx * 8192, bx * kOutBoxCols, h, (c - 1) * kC, b);
                     bulk_commit();
                     bulk_wait_read<1>();  // the store of chunk c-2 has read sO[c & 1]
                     mbar_arrive(&oFree[c & 1]);
@@ -673,12 +1024,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const ui
                     mbar_arrive(&oFree[0]);
                 }
                 // D3 = Delta^T K~ (N = 128) and D1[sb][:, 64:128] += Delta^T P^T (N = 64)
-                mbar_wait(&deltaReady, c & 1, A.status);
+                if (!wait(&deltaReady, c & 1)) break;
                 tc_fence_after();
-                if (c + 1 < NC) {  // every epilogue warp has read U^T of chunk c
-                    mbar_arrive_expect_tx(&fullU, 16384);
-                    bulk_g2s(sUT, src + (size_t)(c + 1) * kHandoffStride + kOffUT, 16384, &fullU);
-                }
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma_f16_ts(tbase + kTD3, tbase + kTDelta + ks * 8,
@@ -689,21 +1036,16 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const ui
                     mma_f16_ts(tD1 + 64, tbase + kTDelta + ks * 8, sdesc(smem_u32(st + kOffP) + ks * 32, 16, 1024),
                                idB, true);
                 mma_commit(&barB);
-                // every MMA of chunk c is done and gamma_C has been read (sReady of chunk c+1 implies
-                // the state update of chunk c is complete): refill the stage with chunk c+2
-                if (c + 2 < NC) {
-                    mbar_wait(&barB, c & 1, A.status);
-                    mbar_wait(&sReady, (c + 1) & 1, A.status);
-                    mbar_arrive_expect_tx(&fullA[sb], kPartA);
-                    bulk_g2s(stageA[sb], src + (size_t)(c + 2) * kHandoffStride, kPartA, &fullA[sb]);
-                }
             }
-            // output of the last chunk
-            mbar_wait(&oStaged, (NC - 1) & 1, A.status);
-            const uint8_t* so = sO[(NC - 1) & 1];
-            for (int bx = 0; bx < kOutBoxes; ++bx) tma_store_4d(&mo, so + bx * 8192, bx * kOutBoxCols, h, (NC - 1) * kC, b);
-            bulk_commit();
+            if (c == NC && wait(&oStaged, (NC - 1) & 1)) {  // output of the last chunk
+                const uint8_t* so = sO[(NC - 1) & 1];
+                for (int bx = 0; bx < kOutBoxes; ++bx)
+                    tma_store_4d(mo, so + bx * 8192, bx * kOutBoxCols, h, (NC - 1) * kC, b);
+                bulk_commit();
+            }
             bulk_wait<0>();
+            mma_commit(&drain);
+            mbar_wait(&drain, 0, A.status);
         }
         __syncwarp();
     } else {
@@ -738,8 +1080,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const ui
             const uint8_t* st = stageA[sb];
             const uint32_t tD1 = tbase + kTD1 + sb * 128;
             // ---- Delta^T[j][r] = U^T[j][r] - (S W^T)[j][r], r in [16 cg, 16 cg + 16), into TMEM
-            mbar_wait(&fullU, c & 1, A.status);
-            mbar_wait(&barA[sb], (c >> 1) & 1, A.status);
+            if (!wait(&fullU, c & 1) || !wait(&barA[sb], (c >> 1) & 1)) break;
             tc_fence_after();
             {
                 float x[16], u[16];
@@ -757,7 +1098,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const ui
             __syncwarp();
             if (lane == 0) mbar_arrive(&deltaReady);
             // ---- S <- S Diag(gamma_C) + Delta^T K~ on this thread's 32 columns; fp16 copy into TMEM
-            mbar_wait(&barC, c & 1, A.status);
+            if (!wait(&barC, c & 1)) break;
             tc_fence_after();
             {
                 const float* gam = reinterpret_cast<const float*>(st + kOffGam) + 32 * cg;
@@ -776,8 +1117,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const ui
             __syncwarp();
             if (lane == 0) mbar_arrive(&sReady);
             // ---- output of chunk c into the staging buffer sO[sb]
-            mbar_wait(&barB, c & 1, A.status);
-            mbar_wait(&oFree[sb], (c >> 1) & 1, A.status);
+            if (!wait(&barB, c & 1) || !wait(&oFree[sb], (c >> 1) & 1)) break;
             tc_fence_after();
             {
                 float x[16];
@@ -798,10 +1138,144 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const ui
                 *reinterpret_cast<float4*>(dst + e) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
         }
     }
+}
+
+// Two-pass state kernel: one CTA per (b, h), hand-off blocks from the workspace.
+template <typename Tout>
+__global__ void __launch_bounds__(kStateThreads, 1)
+chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const uint8_t* __restrict__ ws) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) abort_flag = 0;
+    if (warp == 0) {
+        tmem_alloc(&tmem_base, kStateTmemCols);
+        tmem_relinquish();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tbase, kStateTmemCols);
+    const int bh = blockIdx.x;
+    const WorkspaceSource src{ws + (size_t)bh * A.NC * kHandoffStride, kHandoffStride};
+    state_body<Tout>(&mo, A, bh, src, align1024(smem_raw), tmem_base, &abort_flag);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem_base, kStateTmemCols);
+}
+
+// ------------------------------------------------------------------- fused kernel --
+// Both passes in one cooperative launch: CTAs 0 .. BH-1 run the state pass of head bh = blockIdx.x,
+// the other CTAs run two prep pipelines each (warps 0-7 and 8-15; warps 16-17 idle). The prep
+// pipelines claim tasks from a counter in the order the state passes consume them (chunk index
+// outermost: tau = c * BH + bh) and write each hand-off block into ring slot c % kRing of
+// its head, after the head's state pass has copied out chunk c - kRing; a release flag per slot
+// publishes the block. All CTAs are co-resident (cooperative launch), tasks are claimed in
+// increasing order and the state passes consume in order, so the earliest unfinished task can
+// always proceed. The ring stays in L2: the hand-off never makes a round trip to DRAM.
+constexpr uint32_t kPrepPipeBytes = kPrepBytesScalar;  // one pipeline's shared memory (1024-aligned)
+static_assert(kPrepPipeBytes % 1024 == 0, "pipeline shared memory must keep 1024-byte alignment");
+static_assert(2 * (kPrepBytesScalar + 1024 + 1024 + 64) <= 233472, "two prep pipelines per SM");
+constexpr uint32_t kFusedSmem = (2 * kPrepPipeBytes > kStateSmem - 1024 ? 2 * kPrepPipeBytes : kStateSmem - 1024) + 1024;
+constexpr int kFusedMaxHeads = 48;  // B * H above this runs the two-pass path (prep-bound when fused)
+
+struct RingArgs {
+    uint8_t* ring;   // [BH][kRing] hand-off blocks
+    int* ready;      // [BH][kRing]
+    int* consumed;   // [BH]
+    int* next_task;  // prep tasks claimed so far (one counter)
+    int BH;
+};
+
+template <int MODE>
+__device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv, const PrepArgs& P,
+                          const RingArgs& R, uint8_t* sm, uint32_t tbase, volatile int* abort) {
+    __shared__ uint64_t pbars[2][3];
+    __shared__ volatile int go[2];
+    __shared__ volatile int claimed[2];
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int pipe = warp >> 3;  // 0, 1; warps 16-17 have pipe 2 and idle
+    const int lt = tid & 255;
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i)
+            for (int k = 0; k < 3; ++k) mbar_init(&pbars[i][k], 1);
+        fence_mbar_init();
+    }
+    if (pipe < 2) prep_init(PrepSmem{sm + pipe * kPrepPipeBytes, nullptr, 0, 0}, lt);
+    __syncthreads();
+    // a head's chain consumes a chunk about every 2 us and a pipeline prepares one in about 11 us:
+    // 3 CTAs (6 pipelines) per head keep the rings full; more would only wait on ring slots
+    if (pipe >= 2 || (int)blockIdx.x - R.BH >= 3 * R.BH + 4) return;
+    const PrepSmem ps{sm + pipe * kPrepPipeBytes, pbars[pipe], tbase + (uint32_t)pipe * kPrepTmemCols, 1 + 2 * pipe};
+    const int n_tasks = P.NC * R.BH;
+    uint32_t it = 0;
+    int* prev_flag = nullptr;  // the previous task's ready flag, published at the start of the next task
+    int prev_value = 0;
+    for (;; ++it) {
+        // claim the next task in consumption order (a pipeline claims only after finishing its
+        // previous task, so claims, like the state passes' reads, go in increasing order)
+        if (lt == 0) claimed[pipe] = atomicAdd(R.next_task, 1);
+        named_bar(ps.bar_id, kPrepThreads);
+        const int tau = claimed[pipe];
+        named_bar(ps.bar_id, kPrepThreads);  // every thread has read it before the next claim
+        if (tau >= n_tasks) break;
+        const int c = tau / R.BH, bh = tau % R.BH;
+        const int slot = c % kRing;
+        PrepHooks hk;
+        hk.pub_flag = prev_flag;
+        hk.pub_value = prev_value;
+        hk.slot_counter = c >= kRing ? R.consumed + bh : nullptr;
+        hk.slot_target = c - kRing + 1;
+        hk.go = &go[pipe];
+        hk.abort = abort;
+        uint8_t* out = R.ring + ((size_t)bh * kRing + slot) * kHandoffStride;
+        if (!prep_chunk_sg<MODE>(P, mq, mk, mv, ps, bh / P.H, bh % P.H, c, out, it, lt, hk)) {
+            prev_flag = nullptr;
+            break;
+        }
+        prev_flag = R.ready + bh * kRing + slot;
+        prev_value = c + 1;
+    }
+    if (lt == 0) {
+        bulk_wait<0>();
+        if (prev_flag != nullptr) {
+            fence_proxy_async_global();
+            __threadfence();
+            st_release_gpu(prev_flag, prev_value);
+        }
+    }
+}
+
+template <int MODE, typename Tout>
+__global__ void __launch_bounds__(kStateThreads, 1)
+chunk_fused_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                   const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mo, PrepArgs P,
+                   StateArgs A, RingArgs R) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) abort_flag = 0;
+    if (warp == 0) {
+        tmem_alloc(&tmem_base, kStateTmemCols);  // 512: the state pass, or two prep pipelines x 256
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    uint8_t* sm = align1024(smem_raw);
+    if ((int)blockIdx.x < R.BH) {
+        const int bh = blockIdx.x;
+        const RingSource src{R.ring + (size_t)bh * kRing * kHandoffStride, R.ready + bh * kRing, R.consumed + bh};
+        state_body<Tout>(&mo, A, bh, src, sm, tmem_base, &abort_flag);
+    } else {
+        prep_role<MODE>(&mq, &mk, &mv, P, R, sm, tmem_base, &abort_flag);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem_base, kStateTmemCols);
 }
 
 // ---------------------------------------------------------------------- host --
@@ -844,8 +1318,19 @@ cudaError_t launch_prep(const ChunkProblem& p, const CUtensorMap& mq, const CUte
     const uint32_t smem = (MODE == GDR_DECAY_CHANNEL ? kPrepBytesChannel : kPrepBytesScalar) + 1024;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
+    // the whole unified L1 / shared array as shared memory, so that two pipelines fit per SM
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (err != cudaSuccess) return err;
     PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status};
-    kern<<<dim3(NC, p.H, p.B), kPrepThreads, smem, stream>>>(mq, mk, mv, P, static_cast<uint8_t*>(p.workspace));
+    int dev = 0, sms = 0;
+    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+    if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+    // pipelines per SM: two for DeltaNet and the scalar gate (2 x (114,688 + 1,024 reserved + static)
+    // bytes fit in the SM's 228 KiB), one for the channel gate
+    const int per_sm = MODE == GDR_DECAY_CHANNEL ? 1 : 2;
+    const int n_tasks = NC * p.H * p.B;
+    const int grid = n_tasks < sms * per_sm ? n_tasks : sms * per_sm;
+    kern<<<grid, kPrepThreads, smem, stream>>>(mq, mk, mv, P, static_cast<uint8_t*>(p.workspace), n_tasks);
     profile_after_launch(stream);
     return cudaGetLastError();
 }
@@ -861,18 +1346,54 @@ cudaError_t launch_state(const ChunkProblem& p, const CUtensorMap& mo, int NC, c
     return cudaGetLastError();
 }
 
+// The fused kernel serves DeltaNet and the scalar gate for up to kFusedMaxHeads heads; the channel
+// gate (two of its prep pipelines do not fit in shared memory) and larger B * H use two passes.
+bool use_fused(int B, int H, int mode) { return mode != GDR_DECAY_CHANNEL && (size_t)B * H <= kFusedMaxHeads; }
+size_t ring_bytes(int BH) { return (size_t)BH * kRing * kHandoffStride; }
+size_t flag_bytes(int BH) { return ((size_t)(BH * (kRing + 1) + 1) * sizeof(int) + 255) & ~size_t(255); }
+
+template <int MODE, typename Tout>
+cudaError_t launch_fused(const ChunkProblem& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const CUtensorMap& mo, int NC, cudaStream_t stream) {
+    auto kern = chunk_fused_kernel<MODE, Tout>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFusedSmem);
+    if (err != cudaSuccess) return err;
+    int dev = 0, sms = 0, coop = 0, per_sm = 0;
+    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+    if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+    if ((err = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev)) != cudaSuccess) return err;
+    if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kStateThreads, kFusedSmem)) != cudaSuccess)
+        return err;
+    const int BH = p.B * p.H;
+    const int grid = sms * per_sm;
+    if (!coop || per_sm < 1 || grid - BH < 8) return cudaErrorCooperativeLaunchTooLarge;
+    uint8_t* ws = static_cast<uint8_t*>(p.workspace);
+    int* flags = reinterpret_cast<int*>(ws + ring_bytes(BH));
+    RingArgs R{ws, flags, flags + (size_t)BH * kRing, flags + (size_t)BH * (kRing + 1), BH};
+    if ((err = cudaMemsetAsync(flags, 0, flag_bytes(BH), stream)) != cudaSuccess) return err;
+    PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status};
+    StateArgs A{p.S0, p.S_T, p.T, p.H, NC, p.scale, p.status};
+    CUtensorMap aq = mq, ak = mk, av = mv, ao = mo;
+    void* args[] = {&aq, &ak, &av, &ao, &P, &A, &R};
+    err = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(kStateThreads), args,
+                                      kFusedSmem, stream);
+    profile_after_launch(stream);
+    return err;
+}
+
 }  // namespace
 
 bool chunk_tc_supported(int dk, int dv, int chunk, int dtype, int o_dtype) {
     return dtype == GDR_BF16 && (o_dtype == GDR_F32 || o_dtype == GDR_BF16) && dk == kD && dv == kD && chunk == kC;
 }
 
-size_t chunk_tc_workspace_bytes(int B, int T, int H, int, int, int, int) {
+size_t chunk_tc_workspace_bytes(int B, int T, int H, int, int, int, int mode) {
+    if (use_fused(B, H, mode)) return ring_bytes(B * H) + flag_bytes(B * H);
     const size_t NC = (size_t)(T + kC - 1) / kC;
     return (size_t)B * H * NC * kHandoffStride;
 }
 
-int chunk_tc_launches(int, int, int, int, int, int, int) { return 2; }
+int chunk_tc_launches(int B, int, int H, int, int, int, int mode) { return use_fused(B, H, mode) ? 1 : 2; }
 
 cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream) {
     const int NC = (p.T + kC - 1) / kC;
@@ -886,6 +1407,14 @@ cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream) {
     else
         err = make_map(&mo, p.o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.B, p.T, p.H, 32);
     if (err != cudaSuccess) return err;
+    if (use_fused(p.B, p.H, p.mode)) {
+        const bool bf = p.o_dtype == GDR_BF16;
+        if (p.mode == GDR_DECAY_NONE)
+            return bf ? launch_fused<GDR_DECAY_NONE, __nv_bfloat16>(p, mq, mk, mv, mo, NC, stream)
+                      : launch_fused<GDR_DECAY_NONE, float>(p, mq, mk, mv, mo, NC, stream);
+        return bf ? launch_fused<GDR_DECAY_SCALAR, __nv_bfloat16>(p, mq, mk, mv, mo, NC, stream)
+                  : launch_fused<GDR_DECAY_SCALAR, float>(p, mq, mk, mv, mo, NC, stream);
+    }
     switch (p.mode) {
         case GDR_DECAY_NONE: err = launch_prep<GDR_DECAY_NONE>(p, mq, mk, mv, NC, stream); break;
         case GDR_DECAY_SCALAR: err = launch_prep<GDR_DECAY_SCALAR>(p, mq, mk, mv, NC, stream); break;

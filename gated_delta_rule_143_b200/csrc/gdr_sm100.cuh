@@ -70,6 +70,54 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
     }
 }
 
+// As mbar_wait, for warp-specialised kernels: also gives up as soon as another thread of the CTA
+// has set *abort (a wait elsewhere expired), and sets it on its own timeout, so one lost arrival
+// ends every role's loop within one wait limit instead of one limit per remaining wait.
+__device__ __forceinline__ bool mbar_wait_abort(uint64_t* bar, uint32_t parity, int* status, volatile int* abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            report_status(status, kStatusTimeout);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+// ------------------------------------------------------------- global flags --
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Waits until the global counter *flag (written by other CTAs with release semantics) reaches
+// `target`, polling with an exponential back-off of up to max_sleep_ns between reads (short for a
+// wait on the critical path, long where many waiters would otherwise crowd the flag's L2 line).
+// Bounded like mbar_wait_abort: gives up when *abort is set, sets it on its own timeout.
+__device__ __forceinline__ bool flag_wait_geq(const int* flag, int target, int* status, volatile int* abort,
+                                              unsigned max_sleep_ns) {
+    if (ld_acquire_gpu(flag) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    unsigned sleep_ns = 32;
+    while (true) {
+        __nanosleep(sleep_ns);
+        sleep_ns = sleep_ns * 2 < max_sleep_ns ? sleep_ns * 2 : max_sleep_ns;
+        if (ld_acquire_gpu(flag) >= target) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            report_status(status, kStatusTimeout);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
 // --------------------------------------------------------------------- fences --
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -232,6 +280,14 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
         "[%6];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Prefetch of a tiled box (4-D map) into L2 only; no shared memory, no completion to wait for.
+__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* map, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
 }
 
 // Tiled tensor store (4-D map) from shared memory; rows outside the tensor are not written.

@@ -102,6 +102,11 @@ typedef enum {
  *             NULL when that is 0). Contents on entry do not matter; the library does not
  *             keep it after the enqueued work completes. Two calls in flight at the same time
  *             must not share one workspace.
+ * Launches (tensor-core path): DeltaNet and the scalar gate with B * H <= 48 run as one
+ * cooperative kernel with one CTA per SM, in which the per-chunk factor pipelines hand their
+ * blocks to the per-head state passes through a ring of eight blocks per head in the workspace
+ * (0.6 MB per head); otherwise two kernels exchange one block per chunk through it
+ * (73 KB per chunk). gdr_chunk_fwd_launches reports which.
  */
 int gdr_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                   const float* S0, void* o, float* S_T, int B, int T, int H, int d_k, int d_v,
@@ -163,8 +168,9 @@ int gdr_profile_next_call(void* const* events, int n_events);
  * (which may synchronise the device) is not allowed; a program that must not grow its device
  * footprint after start-up. This entry point takes the same arguments as gdr_chunk_fwd minus the
  * workspace and uses a fixed scratch area compiled into the library instead
- * (GDR_NOALLOC_SCRATCH_BYTES, enough for B * H * ceil(T / 64) <= 448 chunks). It allocates
- * nothing on any call.
+ * (GDR_NOALLOC_SCRATCH_BYTES). DeltaNet and the scalar gate with B * H <= 48 need a ring of eight
+ * hand-off blocks per head, which fits at any T; the channel gate and larger B * H need one
+ * block per chunk, which fits for B * H * ceil(T / 64) <= 448. It allocates nothing on any call.
  *
  *  - Shapes: only those that need scratch (bf16 q/k/v, d_k = d_v = 128, chunk = 64); other
  *    shapes need none and are rejected with GDR_ERR_UNSUPPORTED (call gdr_chunk_fwd with a null

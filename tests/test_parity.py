@@ -44,6 +44,22 @@ def test_chunk_small(mode, dtype, d, T, with_s0):
     check_chunk(x, mode, dtype, label=f"{mode}/{dtype}/d{d}/T{T}")
 
 
+@pytest.mark.parametrize("mode", ["none", "scalar"])
+@pytest.mark.parametrize("B,H,T,launches", [
+    (1, 1, 5000, 1),    # one head: the fused kernel with 147 prep CTAs, 79 chunks through the 8-slot ring
+    (3, 16, 333, 1),    # B * H = 48: the largest fused case
+    (7, 7, 191, 2),     # B * H = 49: the smallest two-pass case
+    (4, 16, 130, 2),    # B * H = 64, ragged tail: two passes
+])
+def test_chunk_tensor_core_paths(mode, B, H, T, launches):
+    """The bf16 d = 128 path runs fused (one cooperative kernel, hand-off through a ring) for
+    B * H <= 48 and as two kernels (hand-off through the workspace) above: both against the oracle."""
+    assert gdr.launches_per_chunk_fwd(B, T, H, 128, 128, 64, mode, torch.bfloat16) == launches
+    seed = 4000 + B * 100 + H + T + (1 if mode == "scalar" else 0)
+    x = make_chunk_inputs(B, T, H, 128, 128, mode, "bf16", seed, s0_std=0.05)
+    check_chunk(x, mode, "bf16", label=f"{mode}/B{B}/H{H}/T{T}")
+
+
 @pytest.mark.parametrize("mode", MODES)
 def test_chunk_unequal_head_dims(mode):
     x = make_chunk_inputs(1, 130, 2, 128, 64, mode, "bf16", 77, s0_std=0.05)

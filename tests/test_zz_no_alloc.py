@@ -35,10 +35,13 @@ def _rel(a, b):
 
 
 def test_noalloc_rejects_oversized_problem_on_host():
-    """B * H * ceil(T / 64) = 4096 chunks needs far more than the built-in area: rejected
-    before anything is enqueued (fake, widely spaced addresses; never dereferenced)."""
+    """B * H = 128 heads take the two-pass path, whose scratch holds one block per chunk:
+    B * H * ceil(T / 64) = 8192 chunks needs far more than the built-in area, so the call is
+    rejected before anything is enqueued (fake, widely spaced addresses; never dereferenced)."""
     M = 1 << 30
-    rc = _lib.lib().gdr_chunk_fwd_noalloc(1 * M, 2 * M, 3 * M, 4 * M, 5 * M, None, 6 * M, None, 8, 4096, 8, 128, 128,
+    need = _lib.lib().gdr_chunk_fwd_workspace_bytes(8, 4096, 16, 128, 128, 64, 1, BF16, F32)
+    assert need > (32 << 20)
+    rc = _lib.lib().gdr_chunk_fwd_noalloc(1 * M, 2 * M, 3 * M, 4 * M, 5 * M, None, 6 * M, None, 8, 4096, 16, 128, 128,
                                           64, 1, BF16, F32, None)
     assert rc == -2
     assert b"built-in area" in _lib.lib().gdr_last_error()
