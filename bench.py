@@ -238,6 +238,8 @@ def run_ours(args):
     w = CHUNK_WORKLOADS[WORKLOAD]
     if args.batch:
         w = dataclasses.replace(w, B=args.batch)
+    if args.seq:
+        w = dataclasses.replace(w, T=args.seq)
     stream = torch.cuda.current_stream(dev)
 
     # two resident input sets, each larger than L2; one seed per rank (weak scaling)
@@ -314,7 +316,7 @@ def run_ours(args):
     if args.only == "fwd":
         if rank == 0:
             print(json.dumps({"metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
-                              "ms_per_step": round(ms_step, 5), "config": {"workload": WORKLOAD, "B": w.B},
+                              "ms_per_step": round(ms_step, 5), "config": {"workload": WORKLOAD, "B": w.B, "T": w.T},
                               "roofline_frac": round(nbytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                               "kernels": [(k["kernel"], k["launch_us"]) for k in kernels]}))
         return
@@ -468,6 +470,7 @@ def main():
     ap.add_argument("--only", choices=("all", "fwd"), default="all",
                     help="fwd: time the forward only (no e2e, decode or CPU baseline), for profiling runs")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size (profiling runs)")
+    ap.add_argument("--seq", type=int, default=0, help="override the workload's sequence length (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

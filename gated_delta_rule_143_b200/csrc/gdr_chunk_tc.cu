@@ -48,10 +48,6 @@ constexpr int kC = 64;    // chunk length
 constexpr int kD = 128;   // d_k = d_v
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kF16Max = 65504.f;
-// Largest within-chunk spread of the cumulative log2-decay for which the scalar gate's pairwise
-// decays are taken as products 2^(G_r - G_ref) 2^(G_ref - G_i) around the mid value (both factors
-// within 2^+-100); beyond it they are computed one by one.
-constexpr float kFactorSpread = 200.f;
 
 // ------------------------------------------------------------------ hand-off block --
 // Per-chunk block in the workspace (byte offsets). Images are laid out exactly as the state
@@ -521,278 +517,6 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
     }
 }
 
-// Optional steps the fused kernel's prep pipelines insert into a task (thread 0, right after the
-// task's TMA loads are issued): publish the previous task's block, then wait until the ring slot
-// of this task is free. All null / unused in the two-pass prep kernel.
-struct PrepHooks {
-    int* pub_flag = nullptr;          // release pub_value here once the previous block is complete
-    int pub_value = 0;
-    const int* slot_counter = nullptr;  // wait until *slot_counter >= slot_target
-    int slot_target = 0;
-    volatile int* go = nullptr;       // shared: 0 once a wait gave up (the task is skipped)
-    volatile int* abort = nullptr;
-};
-
-// Prep of one chunk for DeltaNet and the scalar gate (the channel gate uses prep_chunk): the same
-// hand-off block and step order as prep_chunk, with the tail taken off the pipeline's path: W and U^T
-// are staged in the A^T / T area (dead once T diag(beta) is formed) and bulk-stored without
-// waiting; the next task waits for those reads only before its A / P epilogue writes A^T, so its
-// loads, Gram MMA and output conversions overlap them. The pairwise decays are products of two
-// per-row factors when the chunk's decay spread allows. The caller makes the stores complete
-// (bulk_wait) before publishing or exiting. Returns false if a hook's wait gave up.
-template <int MODE>
-__device__ bool prep_chunk_sg(const PrepArgs& P, const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv,
-                              const PrepSmem& ps, int b, int h, int c, uint8_t* __restrict__ out, uint32_t it, int lt,
-                              const PrepHooks& hk) {
-    static_assert(MODE != GDR_DECAY_CHANNEL, "the channel gate uses prep_chunk");
-    const int lw = lt >> 5, lane = lt & 31;
-    const int q = lw & 3, hf = lw >> 2;
-    const uint32_t par = it & 1u;
-    uint8_t* sm = ps.base;
-    uint8_t* sKQ = sm + kPKQ;
-    uint8_t* sV = sm + kPV;
-    uint8_t* sTB = sm + kPTBZ + 8192;
-    uint8_t* stg = sm + kPA;  // W / U^T staging over A^T and T (32 KiB of 34 KiB)
-    float* sAt = reinterpret_cast<float*>(sm + kPA);
-    float* sT = reinterpret_cast<float*>(sm + kPT);
-    float* sX = reinterpret_cast<float*>(sm + kPX);
-    float* sDu = sX;       // 2^(G_r - G_ref), rows      } read by the A / P epilogue only, before the
-    float* sDv = sX + 64;  // 2^(G_ref - G_i), columns   } solve uses sX as scratch
-    int* sFact = reinterpret_cast<int*>(sX + 128);
-    float* sBeta = reinterpret_cast<float*>(sm + kPBeta);
-    float* sGam = reinterpret_cast<float*>(sm + kPGam);
-    uint64_t* barT = ps.bars;
-    uint64_t* barG = ps.bars + 1;
-    uint64_t* barW = ps.bars + 2;
-    const int T = P.T, H = P.H;
-    const int c0 = c * kC;
-    const int n = min(kC, T - c0);
-    const size_t tok0 = ((size_t)b * T + c0) * H + h;  // chunk row r is token tok0 + r * H
-
-    // ---- 1. TMA loads; beta and the cumulative log2-decay meanwhile (rows past the tail repeat
-    //         Gamma_{n-1}), with the factors of the pairwise decays around the mid value
-    if (lt == 0) {
-        mbar_arrive_expect_tx(barT, 6 * 8192);
-        tma_load_4d(sKQ, mk, 0, h, c0, b, barT);
-        tma_load_4d(sKQ + 16384, mk, 64, h, c0, b, barT);
-        tma_load_4d(sKQ + 8192, mq, 0, h, c0, b, barT);
-        tma_load_4d(sKQ + 24576, mq, 64, h, c0, b, barT);
-        tma_load_4d(sV, mv, 0, h, c0, b, barT);
-        tma_load_4d(sV + 8192, mv, 64, h, c0, b, barT);
-        bool go = true;
-        if (hk.pub_flag != nullptr) {  // the previous block: its bulk stores complete, then release
-            bulk_wait<0>();
-            fence_proxy_async_global();
-            __threadfence();
-            st_release_gpu(hk.pub_flag, hk.pub_value);
-        }
-        if (hk.slot_counter != nullptr) go = flag_wait_geq(hk.slot_counter, hk.slot_target, P.status, hk.abort, 2048);
-        if (hk.go != nullptr) *hk.go = go;
-        bulk_wait_read<0>();  // the previous W / U^T staging (over A^T / T) has been read
-    }
-    if (lw == 7) {
-        sBeta[lane] = (lane < n) ? P.beta[tok0 + (size_t)lane * H] : 0.f;
-        sBeta[lane + 32] = (lane + 32 < n) ? P.beta[tok0 + (size_t)(lane + 32) * H] : 0.f;
-    }
-    if (MODE == GDR_DECAY_SCALAR && lw == 6) {
-        float x0 = (lane < n) ? P.g[tok0 + (size_t)lane * H] * kLog2e : 0.f;
-        float x1 = (lane + 32 < n) ? P.g[tok0 + (size_t)(lane + 32) * H] * kLog2e : 0.f;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
-            const float y1 = __shfl_up_sync(0xffffffffu, x1, off);
-            if (lane >= off) {
-                x0 += y0;
-                x1 += y1;
-            }
-        }
-        x1 += __shfl_sync(0xffffffffu, x0, 31);
-        const float g0 = __shfl_sync(0xffffffffu, x0, 0), gC = __shfl_sync(0xffffffffu, x1, 31);
-        const float gref = 0.5f * (g0 + gC);
-        sGam[lane] = x0;
-        sGam[lane + 32] = x1;
-        sDu[lane] = fast_exp2(x0 - gref);
-        sDu[lane + 32] = fast_exp2(x1 - gref);
-        sDv[lane] = fast_exp2(gref - x0);
-        sDv[lane + 32] = fast_exp2(gref - x1);
-        if (lane == 0) *sFact = (g0 - gC) <= kFactorSpread;
-    }
-    named_bar(ps.bar_id, kPrepThreads);
-    if (hk.go != nullptr && !*hk.go) {
-        if (lt == 0) mbar_wait(barT, par, P.status);  // the loads land before shared memory is reused
-        return false;
-    }
-    mbar_wait(barT, par, P.status);
-    const uint32_t tG = ps.tmem + kTG, tW = ps.tmem + kTW, tU = ps.tmem + kTU;
-    if (lt == 0) {  // Gram products straight from the bf16 tiles
-        tc_fence_after();
-        const uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t d = sdesc(smem_u32(sKQ) + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-            mma_f16(tG, d, d, id, ks > 0);  // B = the K rows (first 64 rows) of the same tile
-        }
-        mma_commit(barG);
-    }
-    // ---- 2. while the Gram MMA runs: Q*gamma and K*gamma_C/gamma hand-off images (all 8 warps,
-    //         from the bf16 tiles, which stay unchanged until step 4)
-    {
-        const float GC = MODE == GDR_DECAY_SCALAR ? sGam[kC - 1] : 0.f;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int task = lt + kPrepThreads * j;
-            const int r = task >> 4, col0 = (task & 15) * 8;
-            const uint32_t ok = kmajor_off(r, col0, 128), oq = kmajor_off(kC + r, col0, 128);
-            float kx[8], qx[8];
-            unpack8bf(ld16(sKQ + ok), kx);
-            unpack8bf(ld16(sKQ + oq), qx);
-            if (MODE == GDR_DECAY_SCALAR) {
-                const float fr = fast_exp2(sGam[r]), ft = fast_exp2(GC - sGam[r]);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    qx[e] *= fr;
-                    kx[e] *= ft;
-                }
-            }
-            st16(out + kOffWQ + oq, pack8h(qx));
-            st16(out + kOffKT + mnmajor_off(r, col0, 64), pack8h(kx));
-        }
-        if (lt < kD) reinterpret_cast<float*>(out + kOffGam)[lt] = MODE == GDR_DECAY_SCALAR ? fast_exp2(GC) : 1.f;
-    }
-    __syncwarp();
-    mbar_wait(barG, par, P.status);
-    tc_fence_after();
-
-    // ---- 3. A (strictly lower, beta_r folded in; stored transposed) and P (causal incl. diagonal):
-    //         thread (q, hf) takes TMEM lane 32 q + lane (K rows for q < 2, Q rows for q >= 2),
-    //         columns i in [32 hf, 32 hf + 32)
-    {
-        const int rr = (q & 1) * 32 + lane;
-        float x[32];
-        tmem_ld32(tG + ((uint32_t)(q * 32) << 16) + 32 * hf, x);
-        const bool factored = MODE == GDR_DECAY_SCALAR && *sFact;
-        const float G2r = MODE == GDR_DECAY_SCALAR ? sGam[rr] : 0.f;
-        const float ur = MODE == GDR_DECAY_SCALAR && factored ? sDu[rr] : 1.f;
-        auto decay = [&](int i) {
-            if (MODE != GDR_DECAY_SCALAR) return 1.f;
-            return factored ? sDv[i] : fast_exp2(fminf(G2r - sGam[i], 0.f));
-        };
-        tmem_ld_wait();
-        if (q < 2) {
-            const float br = sBeta[rr] * ur;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int i = 32 * hf + e;
-                sAt[i * kLdA + rr] = (i < rr && rr < n) ? br * x[e] * decay(i) : 0.f;
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int i = 32 * hf + e;
-                x[e] = (i <= rr && rr < n) ? ur * x[e] * decay(i) : 0.f;
-            }
-#pragma unroll
-            for (int ci = 0; ci < 4; ++ci) st16(out + kOffP + kmajor_off(rr, 32 * hf + ci * 8, 64), pack8h(x + ci * 8));
-        }
-    }
-    tc_fence_before();
-    named_bar(ps.bar_id, kPrepThreads);
-
-    // ---- 4. warps 0-3: T = (I + A)^-1;  warps 4-7: K*gamma and V as fp16, in place (the W / U^T
-    //         MMA operands)
-    if (lw < 4) {
-        // the upper blocks of T the solve and TB read as zero held the previous staging
-        for (int i = lt; i < 1536; i += 128) {
-            int r, col;
-            if (i < 256) { r = i >> 4; col = 16 + (i & 15); }                   // T[0:16, 16:32]
-            else if (i < 512) { r = 32 + ((i - 256) >> 4); col = 48 + (i & 15); }  // T[32:48, 48:64]
-            else { r = (i - 512) >> 5; col = 32 + (i & 31); }                  // T[0:32, 32:64]
-            sT[r * kLdT + col] = 0.f;
-        }
-        named_bar(ps.bar_id + 1, 128);
-        unit_lower_inverse64(sAt, sT, sX, lt, ps.bar_id + 1);
-    } else {
-        const int lt4 = lt - 128;
-        for (int j = 0; j < 16; ++j) {
-            const int task = lt4 + 128 * j;
-            const bool isv = task >= 1024;
-            const int r = (task & 1023) >> 4, col0 = (task & 15) * 8;
-            uint8_t* p = isv ? sV + kmajor_off(r, col0, 64) : sKQ + kmajor_off(r, col0, 128);
-            float x[8];
-            unpack8bf(ld16(p), x);
-            if (!isv && MODE == GDR_DECAY_SCALAR) {
-                const float fr = fast_exp2(sGam[r]);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] *= fr;
-            }
-            st16(p, pack8h(x));
-        }
-    }
-    named_bar(ps.bar_id, kPrepThreads);
-    // T diag(beta) as fp16
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const int task = lt + kPrepThreads * j;
-        const int r = task >> 3, i0 = (task & 7) * 8;
-        float t8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) t8[e] = sT[r * kLdT + i0 + e] * sBeta[i0 + e];
-        st16(sTB + kmajor_off(r, i0, 64), pack8h(t8));
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    named_bar(ps.bar_id, kPrepThreads);
-    tc_fence_after();
-
-    // ---- 5. W = [T diag(beta); 0] (K*gamma) (M = 128, N = 128) and U^T = V^T (T diag(beta))^T (M = 128, N = 64)
-    if (lt == 0) {
-        const uint32_t idW = idesc_f16(128, 128, false, true);
-        const uint32_t idU = idesc_f16(128, 64, true, false);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t tb = sdesc(smem_u32(sTB) + ks * 32, 16, 1024);
-            mma_f16(tW, tb, sdesc(smem_u32(sKQ) + ks * 2048, 16384, 1024), idW, ks > 0);
-            mma_f16(tU, sdesc(smem_u32(sV) + ks * 2048, 8192, 1024), tb, idU, ks > 0);
-        }
-        mma_commit(barW);
-    }
-    __syncwarp();
-    mbar_wait(barW, par, P.status);
-    tc_fence_after();
-    // ---- 6. W rows (stg: two 64-row K-major blocks) and U^T (stg + 16 KiB: 128-row K-major) staged
-    //         over A^T / T, then bulk-stored
-    {
-        const uint32_t loff = (uint32_t)(q * 32) << 16;
-        const int row = q * 32 + lane;
-        if (q < 2) {
-#pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                float x[32];
-                tmem_ld32(tW + loff + 64 * hf + 32 * q2, x);
-                tmem_ld_wait();
-#pragma unroll
-                for (int ci = 0; ci < 4; ++ci)
-                    st16(stg + kmajor_off(row, 64 * hf + 32 * q2 + ci * 8, 64), pack8h(x + ci * 8));
-            }
-        }
-        float x[32];
-        tmem_ld32(tU + loff + 32 * hf, x);
-        tmem_ld_wait();
-#pragma unroll
-        for (int ci = 0; ci < 4; ++ci) st16(stg + 16384 + kmajor_off(row, 32 * hf + ci * 8, 128), pack8h(x + ci * 8));
-        fence_proxy_async_smem();
-        tc_fence_before();
-        named_bar(ps.bar_id, kPrepThreads);
-        if (lt == 0) {
-            bulk_s2g(out + kOffWQ, stg, 8192);
-            bulk_s2g(out + kOffWQ + 16384, stg + 8192, 8192);
-            bulk_s2g(out + kOffUT, stg + 16384, 16384);
-            bulk_commit();
-        }
-    }
-    return true;
-}
-
 // Standalone prep kernel (two-pass path): one pipeline per CTA, persistent over the chunk tasks
 // t = blockIdx.x, blockIdx.x + gridDim.x, ... (t = (b * H + h) * NC + c, the block's index in the
 // workspace). At the start of each task the tiles of the CTA's next task are prefetched into L2.
@@ -1210,8 +934,6 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
     const PrepSmem ps{sm + pipe * kPrepPipeBytes, pbars[pipe], tbase + (uint32_t)pipe * kPrepTmemCols, 1 + 2 * pipe};
     const int n_tasks = P.NC * R.BH;
     uint32_t it = 0;
-    int* prev_flag = nullptr;  // the previous task's ready flag, published at the start of the next task
-    int prev_value = 0;
     for (;; ++it) {
         // claim the next task in consumption order (a pipeline claims only after finishing its
         // previous task, so claims, like the state passes' reads, go in increasing order)
@@ -1222,27 +944,17 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
         if (tau >= n_tasks) break;
         const int c = tau / R.BH, bh = tau % R.BH;
         const int slot = c % kRing;
-        PrepHooks hk;
-        hk.pub_flag = prev_flag;
-        hk.pub_value = prev_value;
-        hk.slot_counter = c >= kRing ? R.consumed + bh : nullptr;
-        hk.slot_target = c - kRing + 1;
-        hk.go = &go[pipe];
-        hk.abort = abort;
+        if (lt == 0)
+            go[pipe] = c < kRing || flag_wait_geq(R.consumed + bh, c - kRing + 1, P.status, abort, 2048);
+        named_bar(ps.bar_id, kPrepThreads);
+        if (!go[pipe]) break;
         uint8_t* out = R.ring + ((size_t)bh * kRing + slot) * kHandoffStride;
-        if (!prep_chunk_sg<MODE>(P, mq, mk, mv, ps, bh / P.H, bh % P.H, c, out, it, lt, hk)) {
-            prev_flag = nullptr;
-            break;
-        }
-        prev_flag = R.ready + bh * kRing + slot;
-        prev_value = c + 1;
-    }
-    if (lt == 0) {
-        bulk_wait<0>();
-        if (prev_flag != nullptr) {
+        prep_chunk<MODE>(P, mq, mk, mv, ps, bh / P.H, bh % P.H, c, out, it, lt);
+        if (lt == 0) {  // every write of the block (generic stores before prep_chunk's last barrier, bulk stores)
+            bulk_wait<0>();
             fence_proxy_async_global();
             __threadfence();
-            st_release_gpu(prev_flag, prev_value);
+            st_release_gpu(R.ready + bh * kRing + slot, c + 1);
         }
     }
 }
