@@ -58,16 +58,24 @@ def chunk_bytes(w):
     return th * per_th + w.B * w.H * w.dv * w.dk * 4
 
 
-def kernel_bytes(w):
-    """Algorithmic HBM bytes per launch of each kernel of the two-pass tensor-core path: the prep
-    pass reads the method's inputs q, k, v, beta, g once; the state pass writes o and S_T once
-    (and reads S0 when given). The hand-off blocks the passes exchange through the workspace are
-    implementation traffic, not algorithmic bytes (they show up in the ncu DRAM counters)."""
+def kernel_bytes(w, plan, c1):
+    """Algorithmic HBM bytes per launch of each kernel of the chosen plan, as (name, bytes) in launch
+    order. The inputs q, k, v, beta, g are read once by whichever kernel prepares a chunk; o and
+    S_T are written once by the kernel that runs the state passes. Hand-off blocks exchanged
+    through the workspace or the ring are implementation traffic, not algorithmic bytes (they
+    show up in the ncu DRAM counters)."""
     eb = 2 if w.dtype == "bf16" else 4
     th = w.B * w.T * w.H
     g = 0 if w.mode == "none" else (4 if w.mode == "scalar" else 4 * w.dk)
-    return {"chunk_prep": th * (eb * (2 * w.dk + w.dv) + 4 + g),
-            "chunk_state": th * OUT_BYTES * w.dv + w.B * w.H * w.dv * w.dk * 4}
+    inputs = th * (eb * (2 * w.dk + w.dv) + 4 + g)
+    outputs = th * OUT_BYTES * w.dv + w.B * w.H * w.dv * w.dk * 4
+    if plan == "two_pass":
+        return [("chunk_prep", inputs), ("chunk_state", outputs)]
+    if plan == "prep_fused":
+        nc = -(-w.T // w.chunk)
+        pre = inputs * c1 // nc
+        return [("chunk_prep", pre), ("chunk_fused", inputs - pre + outputs)]
+    return [("chunk_fused" if plan == "fused" else "chunk_simt", inputs + outputs)]
 
 
 def decode_bytes(w):
@@ -255,8 +263,10 @@ def run_ours(args):
     # per-kernel durations: an event before each step and one the library records after each of
     # its kernels (gdr_profile_next_call), all on the launching stream
     kernels_per_step = gdr_kernels_per_step(w)
-    names = {1: ["chunk_fused"], 2: ["chunk_prep", "chunk_state"]}.get(kernels_per_step,
-                                                                     [f"kernel{j}" for j in range(kernels_per_step)])
+    plan, c1 = gdr.chunk_fwd_plan(w.B, w.T, w.H, w.dk, w.dv, w.chunk, w.mode, torch.bfloat16, torch.float32)
+    kb = kernel_bytes(w, plan, c1)
+    assert len(kb) == kernels_per_step, (plan, kernels_per_step)
+    names = [n for n, _ in kb]
     ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     evk = [[torch.cuda.Event(enable_timing=True) for _ in range(kernels_per_step)] for _ in range(args.steps)]
     for e in ev0 + [e for row in evk for e in row]:
@@ -285,7 +295,7 @@ def run_ours(args):
     nbytes = chunk_bytes(w)
     flops = chunk_flops_per_token_head(w.chunk, w.dk, w.dv) * w.B * w.T * w.H
     achieved_gbs = nbytes / (ms_step * 1e-3) / 1e9
-    kb = kernel_bytes(w) if kernels_per_step == 2 else {names[0]: nbytes}
+    kb = dict(kb)
     kernels = []
     for j, name in enumerate(names):
         us = [1e3 * (evk[i][j - 1] if j else ev0[i]).elapsed_time(evk[i][j]) for i in range(args.steps)]
@@ -301,6 +311,7 @@ def run_ours(args):
     roofline = {"bound": "hbm", "achieved": dom["achieved_gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": dom["frac"], "traffic": dom["traffic"], "kernel": dom["kernel"],
                 "launch_us": dom["launch_us"], "algorithmic_bytes_per_launch": dom["algorithmic_bytes_per_launch"],
+                "plan": plan, "precomputed_chunks_per_head": c1,
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)" if peak_src == "measured"
                 else "fallback 6650 GB/s",
                 "kernels": kernels,

@@ -18,9 +18,10 @@ from typing import Optional, Tuple
 
 import torch
 
-from ._lib import DECAY_MODES, DTYPE_BF16, DTYPE_F32, GdrError, check, lib
+from ._lib import DECAY_MODES, DTYPE_BF16, DTYPE_F32, PLANS, GdrError, check, lib
 
-__all__ = ["chunk_fwd", "decode_step", "sync_status", "workspace_bytes", "launches_per_chunk_fwd", "profile_next_call",
+__all__ = ["chunk_fwd", "decode_step", "sync_status", "workspace_bytes", "launches_per_chunk_fwd", "chunk_fwd_plan",
+           "profile_next_call",
            "GdrError", "DECAY_MODES"]
 
 
@@ -65,6 +66,17 @@ def launches_per_chunk_fwd(B: int, T: int, H: int, dk: int, dv: int, chunk: int,
     """Kernel launches one ``chunk_fwd`` makes for this problem (as the library reports)."""
     return int(lib().gdr_chunk_fwd_launches(B, T, H, dk, dv, chunk, _mode(mode), _dtype_code(dtype),
                                             _dtype_code(out_dtype)))
+
+
+def chunk_fwd_plan(B: int, T: int, H: int, dk: int, dv: int, chunk: int, mode, dtype: torch.dtype,
+                   out_dtype: torch.dtype = torch.float32) -> Tuple[str, int]:
+    """How ``chunk_fwd`` runs this problem: ("cuda_core" | "two_pass" | "fused" | "prep_fused" |
+    "invalid", chunks per head prepared before the fused kernel)."""
+    import ctypes
+    c1 = ctypes.c_int(0)
+    code = lib().gdr_chunk_fwd_plan(B, T, H, dk, dv, chunk, _mode(mode), _dtype_code(dtype), _dtype_code(out_dtype),
+                                    ctypes.byref(c1))
+    return PLANS[int(code)], int(c1.value)
 
 
 _ws_cache = {}

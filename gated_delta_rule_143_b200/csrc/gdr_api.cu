@@ -150,6 +150,18 @@ size_t gdr_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int ch
     return 0;
 }
 
+int gdr_chunk_fwd_plan(int B, int T, int H, int dk, int dv, int chunk, int mode, int dtype, int o_dtype,
+                       int* precomputed_chunks) {
+    char saved[sizeof(g_last_error)];
+    memcpy(saved, g_last_error, sizeof(saved));
+    const int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype);
+    memcpy(g_last_error, saved, sizeof(saved));
+    if (precomputed_chunks != nullptr) *precomputed_chunks = 0;
+    if (rc != GDR_OK) return GDR_PLAN_INVALID;
+    if (!chunk_tc_supported(dk, dv, chunk, dtype, o_dtype)) return GDR_PLAN_CUDA_CORE;
+    return chunk_tc_plan(B, T, H, dk, dv, chunk, mode, precomputed_chunks);
+}
+
 int gdr_chunk_fwd_launches(int B, int T, int H, int dk, int dv, int chunk, int mode, int dtype, int o_dtype) {
     char saved[sizeof(g_last_error)];
     memcpy(saved, g_last_error, sizeof(saved));

@@ -517,13 +517,14 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
     }
 }
 
-// Standalone prep kernel (two-pass path): one pipeline per CTA, persistent over the chunk tasks
-// t = blockIdx.x, blockIdx.x + gridDim.x, ... (t = (b * H + h) * NC + c, the block's index in the
-// workspace). At the start of each task the tiles of the CTA's next task are prefetched into L2.
+// Standalone prep kernel: one pipeline per CTA, persistent over the chunk tasks t = blockIdx.x,
+// blockIdx.x + gridDim.x, ... for the first NCp chunks of every head (t = (b * H + h) * NCp + c, the
+// block's index in the workspace; NCp = NC on the two-pass path, the fused kernel's c1 before it).
+// At the start of each task the tiles of the CTA's next task are prefetched into L2.
 template <int MODE>
 __global__ void __launch_bounds__(kPrepThreads, MODE == GDR_DECAY_CHANNEL ? 1 : 2)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-                  const __grid_constant__ CUtensorMap mv, PrepArgs P, uint8_t* __restrict__ ws, int n_tasks) {
+                  const __grid_constant__ CUtensorMap mv, PrepArgs P, uint8_t* __restrict__ ws, int NCp, int n_tasks) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bars[3];
     __shared__ uint32_t tmem_base;
@@ -544,11 +545,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     ps.tmem = tmem_base;
     uint32_t it = 0;
     for (int t = blockIdx.x; t < n_tasks; t += gridDim.x, ++it) {
-        const int c = t % P.NC, bh = t / P.NC;
+        const int c = t % NCp, bh = t / NCp;
         const int h = bh % P.H, b = bh / P.H;
         const int tn = t + gridDim.x;
         if (lt == 0 && tn < n_tasks) {
-            const int cn = tn % P.NC, bhn = tn / P.NC;
+            const int cn = tn % NCp, bhn = tn / NCp;
             const int hn = bhn % P.H, bn = bhn / P.H;
             tma_prefetch_l2_4d(&mk, 0, hn, cn * kC, bn);
             tma_prefetch_l2_4d(&mk, 64, hn, cn * kC, bn);
@@ -617,17 +618,25 @@ struct WorkspaceSource {  // two passes: every block was written before the stat
 };
 
 constexpr int kRing = 8;  // ring slots per head in the fused kernel
-struct RingSource {       // fused kernel: blocks pass through kRing slots per head, flagged by the producers
+struct RingSource {       // fused kernel: chunks c < c1 were written to `pre` by a prep kernel launched
+                          // before; the others pass through kRing slots, flagged by the producers
+    const uint8_t* pre;   // block of chunk 0 of this head among the pre-computed ones (c1 per head)
     const uint8_t* base;  // slot 0 of this head
     const int* ready;     // [kRing]: c + 1 once the block of chunk c in that slot is complete
-    int* consumed;        // number of this head's chunks already copied out of the ring
-    __device__ const uint8_t* block(int c) const { return base + (size_t)(c % kRing) * kHandoffStride; }
+    int* consumed;        // number of this head's chunks already copied out of the ring (counted from 0)
+    int c1;
+    __device__ const uint8_t* block(int c) const {
+        return c < c1 ? pre + (size_t)c * kHandoffStride : base + (size_t)(c % kRing) * kHandoffStride;
+    }
     __device__ bool wait_ready(int c, int* status, volatile int* abort) const {
+        if (c < c1) return true;
         if (!flag_wait_geq(ready + c % kRing, c + 1, status, abort, 128)) return false;
         fence_proxy_async_global();  // the bulk copies that follow read what the acquire made visible
         return true;
     }
-    __device__ void release(int c) const { st_release_gpu(consumed, c + 1); }
+    __device__ void release(int c) const {
+        if (c >= c1) st_release_gpu(consumed, c + 1);
+    }
 };
 
 // The state pass of one head (b, h) = bh, executed by all kStateThreads threads of the CTA, with
@@ -902,14 +911,15 @@ constexpr uint32_t kPrepPipeBytes = kPrepBytesScalar;  // one pipeline's shared 
 static_assert(kPrepPipeBytes % 1024 == 0, "pipeline shared memory must keep 1024-byte alignment");
 static_assert(2 * (kPrepBytesScalar + 1024 + 1024 + 64) <= 233472, "two prep pipelines per SM");
 constexpr uint32_t kFusedSmem = (2 * kPrepPipeBytes > kStateSmem - 1024 ? 2 * kPrepPipeBytes : kStateSmem - 1024) + 1024;
-constexpr int kFusedMaxHeads = 48;  // B * H above this runs the two-pass path (prep-bound when fused)
+constexpr int kFusedMaxHeads = 100;  // B * H above this runs the two-pass path (too few SMs left for prep)
 
 struct RingArgs {
-    uint8_t* ring;   // [BH][kRing] hand-off blocks
-    int* ready;      // [BH][kRing]
-    int* consumed;   // [BH]
-    int* next_task;  // prep tasks claimed so far (one counter)
-    int BH;
+    uint8_t* ring;     // [BH][kRing] hand-off blocks
+    int* ready;        // [BH][kRing]
+    int* consumed;     // [BH]
+    int* next_task;    // prep tasks claimed so far (one counter, counted from task c1 * BH)
+    const uint8_t* pre;  // [BH][c1] blocks of the chunks below c1, written by chunk_prep_kernel before
+    int BH, c1;
 };
 
 template <int MODE>
@@ -937,7 +947,7 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
     for (;; ++it) {
         // claim the next task in consumption order (a pipeline claims only after finishing its
         // previous task, so claims, like the state passes' reads, go in increasing order)
-        if (lt == 0) claimed[pipe] = atomicAdd(R.next_task, 1);
+        if (lt == 0) claimed[pipe] = R.c1 * R.BH + atomicAdd(R.next_task, 1);
         named_bar(ps.bar_id, kPrepThreads);
         const int tau = claimed[pipe];
         named_bar(ps.bar_id, kPrepThreads);  // every thread has read it before the next claim
@@ -945,7 +955,7 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
         const int c = tau / R.BH, bh = tau % R.BH;
         const int slot = c % kRing;
         if (lt == 0)
-            go[pipe] = c < kRing || flag_wait_geq(R.consumed + bh, c - kRing + 1, P.status, abort, 2048);
+            go[pipe] = c - kRing < R.c1 || flag_wait_geq(R.consumed + bh, c - kRing + 1, P.status, abort, 2048);
         named_bar(ps.bar_id, kPrepThreads);
         if (!go[pipe]) break;
         uint8_t* out = R.ring + ((size_t)bh * kRing + slot) * kHandoffStride;
@@ -979,7 +989,8 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     uint8_t* sm = align1024(smem_raw);
     if ((int)blockIdx.x < R.BH) {
         const int bh = blockIdx.x;
-        const RingSource src{R.ring + (size_t)bh * kRing * kHandoffStride, R.ready + bh * kRing, R.consumed + bh};
+        const RingSource src{R.pre + (size_t)bh * R.c1 * kHandoffStride, R.ring + (size_t)bh * kRing * kHandoffStride,
+                             R.ready + bh * kRing, R.consumed + bh, R.c1};
         state_body<Tout>(&mo, A, bh, src, sm, tmem_base, &abort_flag);
     } else {
         prep_role<MODE>(&mq, &mk, &mv, P, R, sm, tmem_base, &abort_flag);
@@ -1025,7 +1036,7 @@ cudaError_t make_map(CUtensorMap* map, const void* base, CUtensorMapDataType typ
 
 template <int MODE>
 cudaError_t launch_prep(const ChunkProblem& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                        int NC, cudaStream_t stream) {
+                        int NC, int NCp, uint8_t* blocks, cudaStream_t stream) {
     auto kern = chunk_prep_kernel<MODE>;
     const uint32_t smem = (MODE == GDR_DECAY_CHANNEL ? kPrepBytesChannel : kPrepBytesScalar) + 1024;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -1040,9 +1051,9 @@ cudaError_t launch_prep(const ChunkProblem& p, const CUtensorMap& mq, const CUte
     // pipelines per SM: two for DeltaNet and the scalar gate (2 x (114,688 + 1,024 reserved + static)
     // bytes fit in the SM's 228 KiB), one for the channel gate
     const int per_sm = MODE == GDR_DECAY_CHANNEL ? 1 : 2;
-    const int n_tasks = NC * p.H * p.B;
+    const int n_tasks = NCp * p.H * p.B;
     const int grid = n_tasks < sms * per_sm ? n_tasks : sms * per_sm;
-    kern<<<grid, kPrepThreads, smem, stream>>>(mq, mk, mv, P, static_cast<uint8_t*>(p.workspace), n_tasks);
+    kern<<<grid, kPrepThreads, smem, stream>>>(mq, mk, mv, P, blocks, NCp, n_tasks);
     profile_after_launch(stream);
     return cudaGetLastError();
 }
@@ -1064,6 +1075,24 @@ bool use_fused(int B, int H, int mode) { return mode != GDR_DECAY_CHANNEL && (si
 size_t ring_bytes(int BH) { return (size_t)BH * kRing * kHandoffStride; }
 size_t flag_bytes(int BH) { return ((size_t)(BH * (kRing + 1) + 1) * sizeof(int) + 255) & ~size_t(255); }
 
+// Chunks per head the fused kernel takes pre-computed from a prep kernel that runs before it on
+// all SMs. In the fused kernel the kSMs - BH prep CTAs must keep up with the BH chains: a chain
+// takes kChainPerTask times as long per chunk as a prep CTA (two pipelines) per task, so they
+// produce the last NC - c1 chunks in time if (NC - c1) * BH <= NC * (kSMs - BH) * kChainPerTask;
+// the remaining chunks are prepared beforehand with every SM. (A fixed SM count keeps the result,
+// and with it the workspace size, a host-only function of the shape.)
+constexpr int kSMs = 148;
+constexpr double kChainPerTask = 0.32;  // measured: chain 2.2-2.6 us per chunk, fused prep CTA 7.2 us per task
+constexpr int kHybridMinHeads = 57;     // below, the fused kernel alone is faster (measured at 48 heads)
+int fused_precomputed_chunks(int BH, int NC) {
+    if (BH < kHybridMinHeads) return 0;
+    const double f = 1.0 - kChainPerTask * (kSMs - BH) / (double)BH;
+    if (f <= 0.0) return 0;
+    const int c1 = (int)(f * NC + 0.999);
+    return c1 < NC ? c1 : NC;
+}
+size_t pre_bytes(int BH, int NC) { return (size_t)BH * fused_precomputed_chunks(BH, NC) * kHandoffStride; }
+
 template <int MODE, typename Tout>
 cudaError_t launch_fused(const ChunkProblem& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const CUtensorMap& mo, int NC, cudaStream_t stream) {
@@ -1079,10 +1108,14 @@ cudaError_t launch_fused(const ChunkProblem& p, const CUtensorMap& mq, const CUt
     const int BH = p.B * p.H;
     const int grid = sms * per_sm;
     if (!coop || per_sm < 1 || grid - BH < 8) return cudaErrorCooperativeLaunchTooLarge;
+    // workspace: [pre-computed blocks, BH x c1][ring, BH x kRing][flags]
     uint8_t* ws = static_cast<uint8_t*>(p.workspace);
-    int* flags = reinterpret_cast<int*>(ws + ring_bytes(BH));
-    RingArgs R{ws, flags, flags + (size_t)BH * kRing, flags + (size_t)BH * (kRing + 1), BH};
+    const int c1 = fused_precomputed_chunks(BH, NC);
+    uint8_t* ring = ws + pre_bytes(BH, NC);
+    int* flags = reinterpret_cast<int*>(ring + ring_bytes(BH));
+    RingArgs R{ring, flags, flags + (size_t)BH * kRing, flags + (size_t)BH * (kRing + 1), ws, BH, c1};
     if ((err = cudaMemsetAsync(flags, 0, flag_bytes(BH), stream)) != cudaSuccess) return err;
+    if (c1 > 0 && (err = launch_prep<MODE>(p, mq, mk, mv, NC, c1, ws, stream)) != cudaSuccess) return err;
     PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status};
     StateArgs A{p.S0, p.S_T, p.T, p.H, NC, p.scale, p.status};
     CUtensorMap aq = mq, ak = mk, av = mv, ao = mo;
@@ -1100,12 +1133,23 @@ bool chunk_tc_supported(int dk, int dv, int chunk, int dtype, int o_dtype) {
 }
 
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int, int, int, int mode) {
-    if (use_fused(B, H, mode)) return ring_bytes(B * H) + flag_bytes(B * H);
-    const size_t NC = (size_t)(T + kC - 1) / kC;
+    const int NC = (T + kC - 1) / kC;
+    if (use_fused(B, H, mode)) return pre_bytes(B * H, NC) + ring_bytes(B * H) + flag_bytes(B * H);
     return (size_t)B * H * NC * kHandoffStride;
 }
 
-int chunk_tc_launches(int B, int, int H, int, int, int, int mode) { return use_fused(B, H, mode) ? 1 : 2; }
+int chunk_tc_plan(int B, int T, int H, int, int, int, int mode, int* precomputed_chunks) {
+    const int NC = (T + kC - 1) / kC;
+    const int c1 = use_fused(B, H, mode) ? fused_precomputed_chunks(B * H, NC) : 0;
+    if (precomputed_chunks != nullptr) *precomputed_chunks = c1;
+    if (!use_fused(B, H, mode)) return GDR_PLAN_TWO_PASS;
+    return c1 > 0 ? GDR_PLAN_PREP_FUSED : GDR_PLAN_FUSED;
+}
+
+int chunk_tc_launches(int B, int T, int H, int, int, int, int mode) {
+    if (!use_fused(B, H, mode)) return 2;
+    return fused_precomputed_chunks(B * H, (T + kC - 1) / kC) > 0 ? 2 : 1;
+}
 
 cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream) {
     const int NC = (p.T + kC - 1) / kC;
@@ -1127,10 +1171,11 @@ cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream) {
         return bf ? launch_fused<GDR_DECAY_SCALAR, __nv_bfloat16>(p, mq, mk, mv, mo, NC, stream)
                   : launch_fused<GDR_DECAY_SCALAR, float>(p, mq, mk, mv, mo, NC, stream);
     }
+    uint8_t* ws = static_cast<uint8_t*>(p.workspace);
     switch (p.mode) {
-        case GDR_DECAY_NONE: err = launch_prep<GDR_DECAY_NONE>(p, mq, mk, mv, NC, stream); break;
-        case GDR_DECAY_SCALAR: err = launch_prep<GDR_DECAY_SCALAR>(p, mq, mk, mv, NC, stream); break;
-        case GDR_DECAY_CHANNEL: err = launch_prep<GDR_DECAY_CHANNEL>(p, mq, mk, mv, NC, stream); break;
+        case GDR_DECAY_NONE: err = launch_prep<GDR_DECAY_NONE>(p, mq, mk, mv, NC, NC, ws, stream); break;
+        case GDR_DECAY_SCALAR: err = launch_prep<GDR_DECAY_SCALAR>(p, mq, mk, mv, NC, NC, ws, stream); break;
+        case GDR_DECAY_CHANNEL: err = launch_prep<GDR_DECAY_CHANNEL>(p, mq, mk, mv, NC, NC, ws, stream); break;
         default: return cudaErrorInvalidValue;
     }
     if (err != cudaSuccess) return err;

@@ -80,6 +80,7 @@ bool chunk_tc_supported(int dk, int dv, int chunk, int dtype, int o_dtype);
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int mode);
 cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream);
 int chunk_tc_launches(int B, int T, int H, int dk, int dv, int chunk, int mode);
+int chunk_tc_plan(int B, int T, int H, int dk, int dv, int chunk, int mode, int* precomputed_chunks);
 
 // Bandwidth-bound decode step.
 bool decode_supported(int dk, int dv);

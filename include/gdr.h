@@ -102,11 +102,13 @@ typedef enum {
  *             NULL when that is 0). Contents on entry do not matter; the library does not
  *             keep it after the enqueued work completes. Two calls in flight at the same time
  *             must not share one workspace.
- * Launches (tensor-core path): DeltaNet and the scalar gate with B * H <= 48 run as one
+ * Launches (tensor-core path): DeltaNet and the scalar gate with B * H <= 100 run as one
  * cooperative kernel with one CTA per SM, in which the per-chunk factor pipelines hand their
  * blocks to the per-head state passes through a ring of eight blocks per head in the workspace
- * (0.6 MB per head); otherwise two kernels exchange one block per chunk through it
- * (73 KB per chunk). gdr_chunk_fwd_launches reports which.
+ * (0.6 MB per head); above 56 heads a prep kernel on every SM first writes the blocks of the
+ * leading chunks of each head (73 KB per chunk) to the workspace. The channel gate and more heads
+ * use two kernels that exchange every block through the workspace. gdr_chunk_fwd_plan reports
+ * which.
  */
 int gdr_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                   const float* S0, void* o, float* S_T, int B, int T, int H, int d_k, int d_v,
@@ -143,6 +145,25 @@ int gdr_decode_step(const void* q, const void* k, const void* v, const float* g,
 int gdr_chunk_fwd_launches(int B, int T, int H, int d_k, int d_v, int chunk, int mode, int dtype,
                            int o_dtype);
 
+/* How gdr_chunk_fwd runs a problem (no counterpart in the method; host-only). */
+typedef enum {
+    GDR_PLAN_INVALID = 0,      /* the call would be rejected */
+    GDR_PLAN_CUDA_CORE = 1,    /* one fp32 CUDA-core kernel */
+    GDR_PLAN_TWO_PASS = 2,     /* tensor cores: prep kernel (all chunks), then state kernel */
+    GDR_PLAN_FUSED = 3,        /* tensor cores: one cooperative kernel (prep and state passes) */
+    GDR_PLAN_PREP_FUSED = 4    /* tensor cores: prep kernel for the first chunks of every head, then
+                                  the cooperative kernel for the rest */
+} gdr_plan;
+
+/* The plan gdr_chunk_fwd uses for this problem (a gdr_plan value). For GDR_PLAN_PREP_FUSED,
+ * *precomputed_chunks (if not NULL) receives the number of leading chunks per head the first
+ * kernel prepares; 0 otherwise. Chosen from the shape alone: B * H <= 56 heads run fused (the
+ * chains are the bound), 57-100 heads prepare the first chunks on every SM so that the fused
+ * kernel's remaining prep CTAs keep up with the chains, more than 100 heads or the channel gate
+ * run two passes. */
+int gdr_chunk_fwd_plan(int B, int T, int H, int d_k, int d_v, int chunk, int mode, int dtype,
+                       int o_dtype, int* precomputed_chunks);
+
 /* Diagnostics (no counterpart in the method): per-kernel timing of the next chunked forward.
  * The next gdr_chunk_fwd or gdr_chunk_fwd_noalloc call made on the calling host thread records
  * events[i] on its stream right after it enqueues its i-th kernel, for i < min(n_events,
@@ -168,9 +189,10 @@ int gdr_profile_next_call(void* const* events, int n_events);
  * (which may synchronise the device) is not allowed; a program that must not grow its device
  * footprint after start-up. This entry point takes the same arguments as gdr_chunk_fwd minus the
  * workspace and uses a fixed scratch area compiled into the library instead
- * (GDR_NOALLOC_SCRATCH_BYTES). DeltaNet and the scalar gate with B * H <= 48 need a ring of eight
- * hand-off blocks per head, which fits at any T; the channel gate and larger B * H need one
- * block per chunk, which fits for B * H * ceil(T / 64) <= 448. It allocates nothing on any call.
+ * (GDR_NOALLOC_SCRATCH_BYTES). DeltaNet and the scalar gate with B * H <= 56 need a ring of eight
+ * hand-off blocks per head, which fits at any T; larger problems also need one block per
+ * pre-computed or exchanged chunk and are accepted while the total fits (see
+ * gdr_chunk_fwd_workspace_bytes). It allocates nothing on any call.
  *
  *  - Shapes: only those that need scratch (bf16 q/k/v, d_k = d_v = 128, chunk = 64); other
  *    shapes need none and are rejected with GDR_ERR_UNSUPPORTED (call gdr_chunk_fwd with a null

@@ -101,3 +101,23 @@ def test_profile_next_call_validates_on_host():
     assert L.gdr_profile_next_call(None, -1) == -1
     assert L.gdr_profile_next_call(None, 1) == -1
     assert L.gdr_profile_next_call(None, 0) == 0  # clears; enqueues nothing
+
+
+def test_plan_query_is_host_only():
+    import torch
+    import gated_delta_rule_143_b200 as gdr
+    bf = torch.bfloat16
+    assert gdr.chunk_fwd_plan(1, 4096, 8, 128, 128, 64, "scalar", bf) == ("fused", 0)
+    assert gdr.chunk_fwd_plan(7, 4096, 8, 128, 128, 64, "none", bf) == ("fused", 0)
+    plan, c1 = gdr.chunk_fwd_plan(8, 4096, 8, 128, 128, 64, "scalar", bf)
+    assert plan == "prep_fused" and 0 < c1 < 64
+    assert gdr.chunk_fwd_plan(13, 4096, 8, 128, 128, 64, "scalar", bf) == ("two_pass", 0)
+    assert gdr.chunk_fwd_plan(1, 4096, 8, 128, 128, 64, "channel", bf) == ("two_pass", 0)
+    assert gdr.chunk_fwd_plan(1, 100, 2, 64, 64, 64, "scalar", torch.float32) == ("cuda_core", 0)
+    assert gdr.chunk_fwd_plan(0, 100, 2, 64, 64, 64, "scalar", torch.float32) == ("invalid", 0)
+    # launches and workspace follow the plan
+    assert gdr.launches_per_chunk_fwd(1, 4096, 8, 128, 128, 64, "scalar", bf) == 1
+    assert gdr.launches_per_chunk_fwd(8, 4096, 8, 128, 128, 64, "scalar", bf) == 2
+    ring = 8 * 8 * 74752  # eight ring slots per head
+    assert gdr.workspace_bytes(1, 4096, 8, 128, 128, 64, "scalar", bf) >= ring
+    assert gdr.workspace_bytes(8, 4096, 8, 128, 128, 64, "scalar", bf) >= 64 * (8 + c1) * 74752

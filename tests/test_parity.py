@@ -45,19 +45,23 @@ def test_chunk_small(mode, dtype, d, T, with_s0):
 
 
 @pytest.mark.parametrize("mode", ["none", "scalar"])
-@pytest.mark.parametrize("B,H,T,launches", [
-    (1, 1, 5000, 1),    # one head: the fused kernel with 147 prep CTAs, 79 chunks through the 8-slot ring
-    (3, 16, 333, 1),    # B * H = 48: the largest fused case
-    (7, 7, 191, 2),     # B * H = 49: the smallest two-pass case
-    (4, 16, 130, 2),    # B * H = 64, ragged tail: two passes
+@pytest.mark.parametrize("B,H,T,plan", [
+    (1, 1, 5000, "fused"),        # one head, 147 prep CTAs, 79 chunks through the 8-slot ring
+    (3, 16, 333, "fused"),        # 48 heads
+    (7, 8, 191, "fused"),         # 56 heads: the largest fused-only case
+    (8, 8, 200, "prep_fused"),    # 64 heads: the first chunks prepared before the fused kernel
+    (8, 8, 1000, "prep_fused"),   # 64 heads, 16 chunks (10 prepared before), ragged tail
+    (13, 8, 130, "two_pass"),     # 104 heads: prep kernel, then state kernel
 ])
-def test_chunk_tensor_core_paths(mode, B, H, T, launches):
-    """The bf16 d = 128 path runs fused (one cooperative kernel, hand-off through a ring) for
-    B * H <= 48 and as two kernels (hand-off through the workspace) above: both against the oracle."""
-    assert gdr.launches_per_chunk_fwd(B, T, H, 128, 128, 64, mode, torch.bfloat16) == launches
+def test_chunk_tensor_core_paths(mode, B, H, T, plan):
+    """The bf16 d = 128 path runs fused (one cooperative kernel, hand-off through a ring), prep +
+    fused, or as two kernels (hand-off through the workspace), by head count: each against the
+    oracle."""
+    got, c1 = gdr.chunk_fwd_plan(B, T, H, 128, 128, 64, mode, torch.bfloat16)
+    assert got == plan and (c1 > 0) == (plan == "prep_fused")
     seed = 4000 + B * 100 + H + T + (1 if mode == "scalar" else 0)
     x = make_chunk_inputs(B, T, H, 128, 128, mode, "bf16", seed, s0_std=0.05)
-    check_chunk(x, mode, "bf16", label=f"{mode}/B{B}/H{H}/T{T}")
+    check_chunk(x, mode, "bf16", label=f"{mode}/B{B}/H{H}/T{T}/{plan}")
 
 
 @pytest.mark.parametrize("mode", MODES)
