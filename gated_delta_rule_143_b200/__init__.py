@@ -127,20 +127,33 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optional[tor
 
 
 def _chunk_fwd_host(q, k, v, g, beta, S0, *, mode, chunk, return_state, out, out_dtype, state_out, stream):
-    """Host-resident inputs: H2D copies, the device call and D2H copies, all on one stream."""
+    """Host-resident tensors: gdr_chunk_fwd_host copies them in, computes and copies the outputs
+    back piece by piece, the copies overlapping the work (device staging from a per-stream cache;
+    outputs in page-locked memory unless given)."""
     dev = torch.device("cuda", torch.cuda.current_device())
     s = stream if stream is not None else torch.cuda.current_stream(dev)
-    with torch.cuda.stream(s):
-        d = [None if t is None else t.to(dev, non_blocking=True) for t in (q, k, v, g, beta, S0)]
-        o_d, s_d = chunk_fwd(*d, mode=mode, chunk=chunk, return_state=return_state,
-                             out_dtype=out.dtype if out is not None else out_dtype, stream=s)
-        if out is None:
-            out = torch.empty(o_d.shape, dtype=o_d.dtype, pin_memory=True)
-        out.copy_(o_d, non_blocking=True)
-        if return_state:
-            if state_out is None:
-                state_out = torch.empty(s_d.shape, dtype=s_d.dtype, pin_memory=True)
-            state_out.copy_(s_d, non_blocking=True)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype(q)
+    m = _mode(mode)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=out_dtype, pin_memory=True)
+    odt = _dtype(out)
+    if return_state and state_out is None:
+        state_out = torch.empty((B, H, dv, dk), dtype=torch.float32, pin_memory=True)
+    for t in (q, k, v, g, beta, S0, out, state_out):
+        if t is not None and (t.device.type != "cpu" or not t.is_contiguous()):
+            raise ValueError("host path: every tensor must be a contiguous CPU tensor")
+    nbytes = int(lib().gdr_chunk_fwd_host_staging_bytes(B, T, H, dk, dv, chunk, m, dt, odt))
+    key = ("staging", dev.index, s.cuda_stream)
+    staging = _ws_cache.get(key)
+    if staging is None or staging.numel() < nbytes:
+        staging = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=dev)
+        _ws_cache[key] = staging
+    rc = lib().gdr_chunk_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(out),
+                                  _ptr(state_out) if return_state else None, B, T, H, dk, dv, chunk, m, dt, odt,
+                                  _ptr(staging), staging.numel(), s.cuda_stream)
+    check(rc)
     return out, (state_out if return_state else None)
 
 

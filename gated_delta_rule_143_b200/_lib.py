@@ -32,6 +32,8 @@ SIGNATURES = {
     "gdr_chunk_fwd_plan": (_i, [_i] * 9 + [_vp]),
     "gdr_decode_step": (_i, [_vp] * 7 + [_i] * 7 + [_vp]),
     "gdr_chunk_fwd_noalloc": (_i, [_vp] * 8 + [_i] * 9 + [_vp]),
+    "gdr_chunk_fwd_host": (_i, [_vp] * 8 + [_i] * 9 + [_vp, _sz, _vp]),
+    "gdr_chunk_fwd_host_staging_bytes": (_sz, [_i] * 9),
     "gdr_profile_next_call": (_i, [_vp, _i]),
     "gdr_sync_status": (_i, [_vp]),
     "gdr_last_error": (ctypes.c_char_p, []),

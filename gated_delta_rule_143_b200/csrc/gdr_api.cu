@@ -331,3 +331,173 @@ extern "C" int gdr_chunk_fwd_noalloc(const void* q, const void* k, const void* v
     return gdr_chunk_fwd(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, ws,
                          (size_t)GDR_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+// ------------------------------------------------------------ host-buffer entry point --
+namespace gdr {
+namespace {
+
+constexpr int kHostMaxPieces = 8;
+
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+// Byte sizes of the per-sequence slices of each tensor.
+struct SeqBytes {
+    size_t q, v, g, beta, s, o;
+};
+SeqBytes seq_bytes(int T, int H, int dk, int dv, int mode, int dtype, int o_dtype) {
+    const size_t ntok = (size_t)T * H, eb = elem_bytes(dtype);
+    SeqBytes r;
+    r.q = ntok * dk * eb;
+    r.v = ntok * dv * eb;
+    r.g = mode == GDR_DECAY_NONE ? 0 : (mode == GDR_DECAY_SCALAR ? ntok * sizeof(float) : ntok * dk * sizeof(float));
+    r.beta = ntok * sizeof(float);
+    r.s = (size_t)H * dv * dk * sizeof(float);
+    r.o = ntok * dv * elem_bytes(o_dtype);
+    return r;
+}
+
+// Sequences per piece and the bytes of one staging slot (inputs, outputs and workspace of a piece).
+void host_plan(int B, int T, int H, int dk, int dv, int chunk, int mode, int dtype, int o_dtype, int* pb,
+               size_t* slot) {
+    const int pieces = B < kHostMaxPieces ? B : kHostMaxPieces;
+    *pb = (B + pieces - 1) / pieces;
+    const SeqBytes sb = seq_bytes(T, H, dk, dv, mode, dtype, o_dtype);
+    const size_t n = (size_t)*pb;
+    const size_t ws = chunk_tc_supported(dk, dv, chunk, dtype, o_dtype)
+                          ? chunk_tc_workspace_bytes(*pb, T, H, dk, dv, chunk, mode)
+                          : 0;
+    *slot = 3 * align256(n * sb.q) + align256(n * sb.g) + align256(n * sb.beta) + 2 * align256(n * sb.s) +
+            align256(n * sb.o) + align256(ws);
+}
+
+struct HostStreams {
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr, in_ready[2] = {}, computed[2] = {}, out_done[2] = {};
+};
+HostStreams g_host[kMaxDevices];
+
+int host_streams(HostStreams** out) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
+    if (dev < 0 || dev >= kMaxDevices) return fail(GDR_ERR_DEVICE, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    HostStreams& hs = g_host[dev];
+    if (hs.h2d == nullptr) {
+        HostStreams t;
+        const unsigned ef = cudaEventDisableTiming;
+        err = cudaStreamCreateWithFlags(&t.h2d, cudaStreamNonBlocking);
+        if (err == cudaSuccess) err = cudaStreamCreateWithFlags(&t.d2h, cudaStreamNonBlocking);
+        if (err == cudaSuccess) err = cudaEventCreateWithFlags(&t.start, ef);
+        for (int i = 0; i < 2 && err == cudaSuccess; ++i) {
+            err = cudaEventCreateWithFlags(&t.in_ready[i], ef);
+            if (err == cudaSuccess) err = cudaEventCreateWithFlags(&t.computed[i], ef);
+            if (err == cudaSuccess) err = cudaEventCreateWithFlags(&t.out_done[i], ef);
+        }
+        if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "copy streams: %s", cudaGetErrorString(err));
+        hs = t;
+    }
+    *out = &hs;
+    return GDR_OK;
+}
+
+}  // namespace
+}  // namespace gdr
+
+extern "C" size_t gdr_chunk_fwd_host_staging_bytes(int B, int T, int H, int dk, int dv, int chunk, int mode,
+                                                   int dtype, int o_dtype) {
+    char saved[sizeof(g_last_error)];
+    memcpy(saved, g_last_error, sizeof(saved));
+    const int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype);
+    memcpy(g_last_error, saved, sizeof(saved));
+    if (rc != GDR_OK) return 0;
+    int pb = 0;
+    size_t slot = 0;
+    host_plan(B, T, H, dk, dv, chunk, mode, dtype, o_dtype, &pb, &slot);
+    return 2 * slot;
+}
+
+extern "C" int gdr_chunk_fwd_host(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                                  const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv,
+                                  int chunk, int mode, int dtype, int o_dtype, void* staging, size_t staging_bytes,
+                                  void* stream) {
+    ProfileScope prof_scope;
+    if (int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype)) return rc;
+    if (!q || !k || !v || !beta || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, beta and o must be non-null");
+    if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
+    int pb = 0;
+    size_t slot = 0;
+    host_plan(B, T, H, dk, dv, chunk, mode, dtype, o_dtype, &pb, &slot);
+    if (staging == nullptr || staging_bytes < 2 * slot)
+        return fail(GDR_ERR_WORKSPACE, "staging of %zu bytes required (got %zu at %p)", 2 * slot, staging_bytes,
+                    staging);
+    if (!aligned16(staging)) return fail(GDR_ERR_MISALIGNED, "staging %p is not 16-byte aligned", staging);
+    int* status = nullptr;
+    int major = 0;
+    if (int rc = device_setup(&status, &major)) return rc;
+    if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
+    HostStreams* hs = nullptr;
+    if (int rc = host_streams(&hs)) return rc;
+
+    const SeqBytes sb = seq_bytes(T, H, dk, dv, mode, dtype, o_dtype);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto cuda_fail = [&](cudaError_t e, const char* what) {
+        return fail(GDR_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    };
+    cudaError_t err = cudaEventRecord(hs->start, s);  // everything below follows the work already on `stream`
+    if (err != cudaSuccess) return cuda_fail(err, "event record");
+    if ((err = cudaStreamWaitEvent(hs->h2d, hs->start, 0)) != cudaSuccess) return cuda_fail(err, "stream wait");
+    const size_t sz = (size_t)pb;
+    int piece = 0;
+    for (int b0 = 0; b0 < B; b0 += pb, ++piece) {
+        const int nb = B - b0 < pb ? B - b0 : pb;
+        const int sl = piece & 1;
+        uint8_t* base = static_cast<uint8_t*>(staging) + sl * slot;
+        uint8_t* dq = base;
+        uint8_t* dk_ = dq + align256(sz * sb.q);
+        uint8_t* dv_ = dk_ + align256(sz * sb.q);
+        uint8_t* dg = dv_ + align256(sz * sb.v);
+        uint8_t* dbeta = dg + align256(sz * sb.g);
+        uint8_t* ds0 = dbeta + align256(sz * sb.beta);
+        uint8_t* dst = ds0 + align256(sz * sb.s);
+        uint8_t* dout = dst + align256(sz * sb.s);
+        uint8_t* dws = dout + align256(sz * sb.o);
+        const size_t ws_bytes = slot - (size_t)(dws - base);
+        // inputs of this piece (after the outputs of the piece that used this slot two steps ago)
+        if (piece >= 2 && (err = cudaStreamWaitEvent(hs->h2d, hs->out_done[sl], 0)) != cudaSuccess)
+            return cuda_fail(err, "stream wait");
+        struct Cp { void* d; const void* h; size_t n; };
+        const Cp in[] = {{dq, static_cast<const uint8_t*>(q) + b0 * sb.q, nb * sb.q},
+                         {dk_, static_cast<const uint8_t*>(k) + b0 * sb.q, nb * sb.q},
+                         {dv_, static_cast<const uint8_t*>(v) + b0 * sb.v, nb * sb.v},
+                         {dg, g ? reinterpret_cast<const uint8_t*>(g) + b0 * sb.g : nullptr, nb * sb.g},
+                         {dbeta, reinterpret_cast<const uint8_t*>(beta) + b0 * sb.beta, nb * sb.beta},
+                         {ds0, S0 ? reinterpret_cast<const uint8_t*>(S0) + b0 * sb.s : nullptr, nb * sb.s}};
+        for (const Cp& c : in)
+            if (c.h != nullptr && c.n > 0 &&
+                (err = cudaMemcpyAsync(c.d, c.h, c.n, cudaMemcpyHostToDevice, hs->h2d)) != cudaSuccess)
+                return cuda_fail(err, "copy in");
+        if ((err = cudaEventRecord(hs->in_ready[sl], hs->h2d)) != cudaSuccess) return cuda_fail(err, "event record");
+        // the piece's forward on `stream`
+        if ((err = cudaStreamWaitEvent(s, hs->in_ready[sl], 0)) != cudaSuccess) return cuda_fail(err, "stream wait");
+        const int rc = gdr_chunk_fwd(dq, dk_, dv_, g ? reinterpret_cast<const float*>(dg) : nullptr,
+                                     reinterpret_cast<const float*>(dbeta), S0 ? reinterpret_cast<const float*>(ds0) : nullptr,
+                                     dout, S_T ? reinterpret_cast<float*>(dst) : nullptr, nb, T, H, dk, dv, chunk, mode,
+                                     dtype, o_dtype, dws, ws_bytes, s);
+        if (rc != GDR_OK) return rc;
+        if ((err = cudaEventRecord(hs->computed[sl], s)) != cudaSuccess) return cuda_fail(err, "event record");
+        // outputs of this piece
+        if ((err = cudaStreamWaitEvent(hs->d2h, hs->computed[sl], 0)) != cudaSuccess) return cuda_fail(err, "stream wait");
+        if ((err = cudaMemcpyAsync(static_cast<uint8_t*>(o) + b0 * sb.o, dout, nb * sb.o, cudaMemcpyDeviceToHost,
+                                   hs->d2h)) != cudaSuccess)
+            return cuda_fail(err, "copy out");
+        if (S_T != nullptr &&
+            (err = cudaMemcpyAsync(reinterpret_cast<uint8_t*>(S_T) + b0 * sb.s, dst, nb * sb.s, cudaMemcpyDeviceToHost,
+                                   hs->d2h)) != cudaSuccess)
+            return cuda_fail(err, "copy out");
+        if ((err = cudaEventRecord(hs->out_done[sl], hs->d2h)) != cudaSuccess) return cuda_fail(err, "event record");
+    }
+    // `stream` completes after the last copy out (the copy-out stream runs the pieces in order)
+    if ((err = cudaStreamWaitEvent(s, hs->out_done[(piece - 1) & 1], 0)) != cudaSuccess) return cuda_fail(err, "stream wait");
+    return ok();
+}

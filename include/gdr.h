@@ -176,6 +176,34 @@ int gdr_chunk_fwd_plan(int B, int T, int H, int d_k, int d_v, int chunk, int mod
  * with n_events > 0. Host-only; enqueues nothing by itself. */
 int gdr_profile_next_call(void* const* events, int n_events);
 
+/*
+ * gdr_chunk_fwd_host -- gdr_chunk_fwd on host-resident tensors, copies overlapped with the work.
+ *
+ * No counterpart in the method: a transfer schedule for callers whose inputs and outputs live
+ * in host memory. Arguments as gdr_chunk_fwd, except that q, k, v, g, beta, S0 (inputs) and o,
+ * S_T (outputs) are HOST pointers, and `staging` is caller-owned device memory of at least
+ * gdr_chunk_fwd_host_staging_bytes(...) bytes (16-byte aligned) in place of the workspace.
+ * The batch is processed in pieces of consecutive sequences (at most 8 pieces): the inputs of
+ * piece i are copied in on one internal stream while piece i-1 computes on `stream` and the
+ * outputs of piece i-2 are copied out on another internal stream; staging holds two pieces.
+ * Page-locked host memory lets the copies run asynchronously and overlap (pageable memory
+ * works but serialises). The call returns once everything is enqueued; all of it is ordered
+ * after the work already on `stream`, and `stream` waits for the last copy: when `stream` has
+ * completed, o and S_T hold the results. The host buffers and staging must stay valid until
+ * then. Two calls in flight at the same time must not share `staging`. The two internal streams
+ * and a few events are created on the first call on each device and kept.
+ * Errors: as gdr_chunk_fwd (validated before anything is enqueued), plus GDR_ERR_WORKSPACE for
+ * a staging area that is missing or too small.
+ */
+int gdr_chunk_fwd_host(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                       const float* S0, void* o, float* S_T, int B, int T, int H, int d_k, int d_v,
+                       int chunk, int mode, int dtype, int o_dtype, void* staging, size_t staging_bytes,
+                       void* stream);
+
+/* Device staging gdr_chunk_fwd_host needs for this problem (bytes; 0 if it would be rejected). */
+size_t gdr_chunk_fwd_host_staging_bytes(int B, int T, int H, int d_k, int d_v, int chunk, int mode,
+                                        int dtype, int o_dtype);
+
 /* Size of the scratch area built into the library for gdr_chunk_fwd_noalloc: 32 MiB of device
  * memory on every GPU that loads the library, held until the process exits. */
 #define GDR_NOALLOC_SCRATCH_BYTES (32u << 20)

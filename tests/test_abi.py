@@ -121,3 +121,15 @@ def test_plan_query_is_host_only():
     ring = 8 * 8 * 74752  # eight ring slots per head
     assert gdr.workspace_bytes(1, 4096, 8, 128, 128, 64, "scalar", bf) >= ring
     assert gdr.workspace_bytes(8, 4096, 8, 128, 128, 64, "scalar", bf) >= 64 * (8 + c1) * 74752
+
+
+def test_host_entry_point_validates_on_host():
+    L = _lib.lib()
+    need = L.gdr_chunk_fwd_host_staging_bytes(8, 4096, 8, 128, 128, 64, 1, 1, 0)
+    assert need > 0
+    assert L.gdr_chunk_fwd_host_staging_bytes(0, 4096, 8, 128, 128, 64, 1, 1, 0) == 0
+    M = 1 << 24  # fake addresses: the missing staging area is rejected before anything is enqueued
+    rc = L.gdr_chunk_fwd_host(1 * M, 2 * M, 3 * M, 4 * M, 5 * M, None, 6 * M, None, 8, 4096, 8, 128, 128, 64, 1, 1, 0,
+                              None, 0, None)
+    assert rc == -4
+    assert b"staging" in L.gdr_last_error()

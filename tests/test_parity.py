@@ -154,6 +154,24 @@ def test_host_tensors_roundtrip():
     assert rel_err(st.double().numpy(), s_ref)[0] <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("B,T,H,d,mode,dtype,with_s0", [
+    (5, 130, 2, 128, "scalar", "bf16", True),    # 5 pieces of one sequence, tensor cores
+    (11, 70, 2, 128, "channel", "bf16", False),  # pieces of 2, the last one of 1
+    (3, 90, 3, 64, "none", "f32", True),         # CUDA-core path
+])
+def test_host_tensors_in_pieces(B, T, H, d, mode, dtype, with_s0):
+    """gdr_chunk_fwd_host: page-locked host inputs, copies overlapped with the pieces' work; every
+    piece against the oracle, with S0 carried in and S_T copied back."""
+    x = make_chunk_inputs(B, T, H, d, d, mode, dtype, 500 + B + T, s0_std=0.1 if with_s0 else None)
+    h = {kk: (None if t is None else t.contiguous().pin_memory()) for kk, t in x.items()}
+    o, st = gdr.chunk_fwd(h["q"], h["k"], h["v"], h["g"], h["beta"], h["S0"], mode=mode)
+    torch.cuda.synchronize()
+    gdr.sync_status()
+    o_ref, s_ref = oracle.recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], mode, S0=x["S0"])
+    assert rel_err(o.double().numpy(), o_ref)[0] <= TOL[dtype]
+    assert rel_err(st.double().numpy(), s_ref)[0] <= TOL[dtype]
+
+
 # ------------------------------------------------------------- decode -----
 def run_decode_steps(w_B, w_H, dk, dv, mode, dtype, steps, seed, s_std=0.02, out_dtype=torch.float32):
     from gated_delta_rule_143_b200.inputs import DecodeWorkload
