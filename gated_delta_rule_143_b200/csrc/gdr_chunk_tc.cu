@@ -57,6 +57,7 @@ constexpr uint32_t kOffP = 32768;       // P             fp16 K-major, 64 rows (
 constexpr uint32_t kOffKT = 40960;      // K*gamma_C/gamma fp16 MN-major, 64 rows (i) x 128 (d_k)
 constexpr uint32_t kOffGam = 57344;     // gamma_C       fp32 [128]
 constexpr uint32_t kPartA = 57856;      // bytes of part A (multiple of 16)
+constexpr uint32_t kPartWQ = kOffP;     // part A splits into [W; Q*gamma] and the rest (P, K~, gamma_C)
 constexpr uint32_t kOffUT = 58368;      // U^T           fp16 K-major, 128 rows (d_v) x 64 (r)
 constexpr uint32_t kHandoffStride = 74752;  // multiple of 1024
 
@@ -65,8 +66,8 @@ constexpr int kPrepThreads = 256;
 // shared memory of one prep pipeline (offsets from a 1024-aligned base)
 constexpr uint32_t kPKQ = 0;          // [K; Q] bf16 (TMA) K-major 128 x 128; K rows become K*gamma (fp16)
 constexpr uint32_t kPV = 32768;       // V bf16 (TMA) K-major 64 x 128, converted in place to fp16
-constexpr uint32_t kPTBZ = 49152;     // [Z | T diag(beta) | Z] fp16 K-major 64-row blocks (3 x 8 KiB)
-constexpr uint32_t kPA = 73728;       // A^T fp32 [64][kLdA]
+constexpr uint32_t kPTBZ = 49152;     // [T diag(beta); Z] fp16 K-major 64-row blocks (2 x 8 KiB)
+constexpr uint32_t kPA = kPTBZ + 16384;  // A^T fp32 [64][kLdA]
 constexpr int kLdA = 68;
 constexpr uint32_t kPT = kPA + 64 * kLdA * 4;   // T fp32 [64][kLdT]
 constexpr int kLdT = 68;
@@ -74,8 +75,9 @@ constexpr uint32_t kPX = kPT + 64 * kLdT * 4;   // merge scratch fp32 [32][kLdX]
 constexpr int kLdX = 36;
 constexpr uint32_t kPBeta = kPX + 32 * kLdX * 4;     // beta [64]
 constexpr uint32_t kPGam = kPBeta + 256;             // Gamma * log2(e): [64] or [64][128] (channel)
+constexpr uint32_t kPInvE = kPGam + 256;             // scalar gate: 2^-Gamma [64], then a "factorable" flag
 constexpr uint32_t kPKB = (kPGam + 32768 + 1023) & ~1023u;  // channel: K'' fp16 K-major 64 x 128
-constexpr uint32_t kPrepBytesScalar = kPGam + 256;
+constexpr uint32_t kPrepBytesScalar = (kPInvE + 512 + 1023) & ~1023u;
 constexpr uint32_t kPrepBytesChannel = kPKB + 16384;
 
 // TMEM columns of one prep pipeline
@@ -176,9 +178,21 @@ __device__ void unit_lower_inverse64(const float* __restrict__ sAt, float* __res
 #pragma unroll
         for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
-        for (int i = 0; i < 15; ++i)
+        for (int i = 0; i < 15; ++i) {
+            // column i of the diagonal block, A[base + r][base + i] for r = 0..15, as four 16-byte loads
+            const float4* col = reinterpret_cast<const float4*>(sAt + (base + i) * kLdA + base);
+            float a[16];
 #pragma unroll
-            for (int r = i + 1; r < 16; ++r) x[r] = fmaf(-At(base + r, base + i), x[i], x[r]);
+            for (int q4 = (i + 1) >> 2; q4 < 4; ++q4) {
+                const float4 t = col[q4];
+                a[4 * q4] = t.x;
+                a[4 * q4 + 1] = t.y;
+                a[4 * q4 + 2] = t.z;
+                a[4 * q4 + 3] = t.w;
+            }
+#pragma unroll
+            for (int r = i + 1; r < 16; ++r) x[r] = fmaf(-a[r], x[i], x[r]);
+        }
 #pragma unroll
         for (int r = 0; r < 16; ++r) sT[(base + r) * kLdT + base + j] = x[r];
     }
@@ -213,14 +227,12 @@ __device__ void unit_lower_inverse64(const float* __restrict__ sAt, float* __res
     named_bar(bar_id, 128);
 }
 
-// One-time set-up of a prep pipeline's shared memory: the zero blocks around T diag(beta) and the
-// strictly upper part of T (never written by the solve).
+// One-time set-up of a prep pipeline's shared memory: the zero block under T diag(beta) (rows
+// 64-127 of the M = 128 operand of the W product) and the strictly upper part of T (never
+// written by the solve).
 __device__ void prep_init(const PrepSmem& ps, int lt) {
-    uint8_t* tbz = ps.base + kPTBZ;
-    for (int i = lt; i < 512; i += kPrepThreads) {                            // 512 x 16 B = 8 KiB
-        reinterpret_cast<uint4*>(tbz)[i] = make_uint4(0, 0, 0, 0);           // first Z
-        reinterpret_cast<uint4*>(tbz + 16384)[i] = make_uint4(0, 0, 0, 0);   // second Z
-    }
+    uint8_t* z = ps.base + kPTBZ + 8192;
+    for (int i = lt; i < 512; i += kPrepThreads) reinterpret_cast<uint4*>(z)[i] = make_uint4(0, 0, 0, 0);  // 8 KiB
     float* sT = reinterpret_cast<float*>(ps.base + kPT);
     for (int i = lt; i < 64 * kLdT; i += kPrepThreads) sT[i] = 0.f;
 }
@@ -237,12 +249,13 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
     uint8_t* sm = ps.base;
     uint8_t* sKQ = sm + kPKQ;
     uint8_t* sV = sm + kPV;
-    uint8_t* sTB = sm + kPTBZ + 8192;
+    uint8_t* sTB = sm + kPTBZ;
     float* sAt = reinterpret_cast<float*>(sm + kPA);
     float* sT = reinterpret_cast<float*>(sm + kPT);
     float* sX = reinterpret_cast<float*>(sm + kPX);
     float* sBeta = reinterpret_cast<float*>(sm + kPBeta);
     float* sGam = reinterpret_cast<float*>(sm + kPGam);
+    float* sInvE = reinterpret_cast<float*>(sm + kPInvE);
     uint8_t* sKB = sm + kPKB;
     uint64_t* barT = ps.bars;
     uint64_t* barG = ps.bars + 1;
@@ -283,6 +296,12 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
             x1 += __shfl_sync(0xffffffffu, x0, 31);
             sGam[lane] = x0;
             sGam[lane + 32] = x1;
+            // pairwise decays 2^(Gamma_r - Gamma_i) as 2^Gamma_r * 2^-Gamma_i when every |Gamma| stays
+            // well inside the normal fp32 exponent range (both factors finite and normal)
+            sInvE[lane] = fast_exp2(-x0);
+            sInvE[lane + 32] = fast_exp2(-x1);
+            const bool fac = __all_sync(0xffffffffu, fabsf(x0) <= 120.f && fabsf(x1) <= 120.f);
+            if (lane == 0) *reinterpret_cast<int*>(sInvE + 64) = fac ? 1 : 0;
         }
     } else if (MODE == GDR_DECAY_CHANNEL) {
         if (lt < kD) {
@@ -394,8 +413,14 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
         float d[32];
         if (MODE == GDR_DECAY_SCALAR) {
             const float G2r = sGam[rr];
+            if (*reinterpret_cast<const int*>(sInvE + 64)) {  // one exponential per thread
+                const float er = fast_exp2(G2r);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) d[e] = fast_exp2(fminf(G2r - sGam[32 * hf + e], 0.f));
+                for (int e = 0; e < 32; ++e) d[e] = er * sInvE[32 * hf + e];
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) d[e] = fast_exp2(fminf(G2r - sGam[32 * hf + e], 0.f));
+            }
         }
         const float br = sBeta[rr];
         tmem_ld_wait();
@@ -429,6 +454,7 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
         unit_lower_inverse64(sAt, sT, sX, lt, ps.bar_id + 1);
     } else {
         const int lt4 = lt - 128;
+#pragma unroll 4
         for (int j = 0; j < 16; ++j) {
             const int task = lt4 + 128 * j;
             const bool isv = task >= 1024;
@@ -593,20 +619,6 @@ struct StateArgs {
     int* status;
 };
 
-template <typename Tout>
-__device__ __forceinline__ void stage_out(uint8_t* sO, int r, int j, float v);
-template <>
-__device__ __forceinline__ void stage_out<float>(uint8_t* sO, int r, int j, float v) {
-    const int box = j >> 5, cc = j & 31;
-    *reinterpret_cast<float*>(sO + box * 8192 + r * 128 + (((cc >> 2) ^ (r & 7)) << 4) + (cc & 3) * 4) = v;
-}
-template <>
-__device__ __forceinline__ void stage_out<__nv_bfloat16>(uint8_t* sO, int r, int j, float v) {
-    const int box = j >> 6, cc = j & 63;
-    *reinterpret_cast<__nv_bfloat16*>(sO + box * 8192 + r * 128 + (((cc >> 3) ^ (r & 7)) << 4) + (cc & 7) * 2) =
-        __float2bfloat16_rn(v);
-}
-
 // Where the state pass finds hand-off block c of its head, when that block is complete, and how it
 // tells the producer that the block has been copied out.
 struct WorkspaceSource {  // two passes: every block was written before the state pass started
@@ -645,13 +657,16 @@ struct RingSource {       // fused kernel: chunks c < c1 were written to `pre` b
 template <typename Tout, typename Src>
 __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, const Src& src, uint8_t* sm,
                            uint32_t tbase, volatile int* abort) {
-    uint8_t* stageA[2] = {sm + kSStageA0, sm + kSStageA1};
+    auto stageA = [sm](int i) { return sm + kSStageA0 + i * (kSStageA1 - kSStageA0); };  // part A stage i
     uint8_t* sUT = sm + kSUT;
-    uint8_t* sO[2] = {sm + kSO0, sm + kSO1};
-    // fullA/fullU: bulk copies landed. barA/barB/barC: MMA groups done. deltaReady/sReady/oStaged:
-    // all epilogue warps wrote Delta^T / the fp16 state (TMEM) / the output staging (shared).
-    // oFree[b]: the output staging buffer b has been read by its store. drain: last MMAs complete.
-    __shared__ uint64_t fullA[2], fullU, barA[2], barB, barC, deltaReady, sReady, oStaged, oFree[2], drain;
+    auto sO = [sm](int i) { return sm + kSO0 + i * (kSO1 - kSO0); };  // output staging buffer i
+    // fullWQ/fullR/fullU: bulk copies of [W; Q*gamma], of the rest of part A and of U^T landed.
+    // barA/barB/barC: MMA groups done; rFree[s]: every MMA reading stage s is done. deltaReady/
+    // sReady/oStaged: all epilogue warps wrote Delta^T / the fp16 state (TMEM) / the output
+    // staging (shared). oFree[b]: the output staging buffer b has been read by its store.
+    // drain: last MMAs complete.
+    __shared__ uint64_t fullWQ[2], fullR[2], fullU, barA[2], rFree[2], barB, barC, deltaReady, sReady, oStaged,
+        oFree[2], drain;
 
     const int b = bh / A.H, h = bh % A.H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -662,8 +677,10 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&fullA[i], 1);
+            mbar_init(&fullWQ[i], 1);
+            mbar_init(&fullR[i], 1);
             mbar_init(&barA[i], 1);
+            mbar_init(&rFree[i], 1);
             mbar_init(&oFree[i], 1);
         }
         mbar_init(&fullU, 1);
@@ -681,16 +698,26 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
         // --------------------------------------------------------------- copy warp --
         // Brings hand-off blocks into shared memory (part A double-buffered, U^T single-buffered)
         // as soon as both the block is ready and its buffer is free, and hands each ring slot back
-        // once both parts of its chunk are in shared memory: all flag traffic stays off the MMA
-        // issuer's path.
+        // once all of its chunk is in shared memory: all flag traffic stays off the MMA issuer's
+        // path. Part A of chunk c + 2 comes in two pieces: [W; Q*gamma] as soon as chunk c's first
+        // product is done (its only reader), the rest once chunk c's last product is done.
         if (lane == 0) {
-            int lastA[2] = {-1, -1}, lastU = -1;  // last chunk whose part A / U^T copy was issued
+            int lastWQ[2] = {-1, -1}, lastR[2] = {-1, -1}, lastU = -1;  // last chunk whose copy was issued
+            auto copy_wq = [&](int c) {
+                mbar_arrive_expect_tx(&fullWQ[c & 1], kPartWQ);
+                bulk_g2s(stageA(c & 1), src.block(c), kPartWQ, &fullWQ[c & 1]);
+                lastWQ[c & 1] = c;
+            };
+            auto copy_r = [&](int c) {
+                mbar_arrive_expect_tx(&fullR[c & 1], kPartA - kPartWQ);
+                bulk_g2s(stageA(c & 1) + kPartWQ, src.block(c) + kPartWQ, kPartA - kPartWQ, &fullR[c & 1]);
+                lastR[c & 1] = c;
+            };
             bool ok = true;
             for (int st = 0; st < 2 && st < NC && ok; ++st) {
                 if (!(ok = src.wait_ready(st, A.status, abort))) break;
-                mbar_arrive_expect_tx(&fullA[st], kPartA);
-                bulk_g2s(stageA[st], src.block(st), kPartA, &fullA[st]);
-                lastA[st] = st;
+                copy_wq(st);
+                copy_r(st);
             }
             if (ok) {
                 mbar_arrive_expect_tx(&fullU, 16384);
@@ -699,8 +726,8 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
             }
             for (int c = 0; ok && c < NC; ++c) {
                 const int sb = c & 1;
-                // every epilogue warp has read U^T of chunk c (and waited for it), so both parts of
-                // chunk c are in shared memory: the ring slot goes back; U^T of chunk c + 1 comes in
+                // every epilogue warp has read U^T of chunk c (and waited for it), so all of chunk c
+                // is in shared memory: the ring slot goes back; U^T of chunk c + 1 comes in
                 if (!wait(&deltaReady, c & 1)) break;
                 src.release(c);
                 if (c + 1 < NC) {
@@ -708,19 +735,22 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
                     bulk_g2s(sUT, src.block(c + 1) + kOffUT, 16384, &fullU);
                     lastU = c + 1;
                 }
-                // stage sb is free once every MMA of chunk c is done and gamma_C has been read
-                // (sReady of chunk c + 1): chunk c + 2 comes in
                 if (c + 2 < NC) {
-                    if (!wait(&barB, c & 1) || !wait(&sReady, (c + 1) & 1)) break;
+                    // chunk c's first product (barA, complete before deltaReady) has read [W; Q*gamma]
+                    // of stage sb; the rest follows once every MMA of chunk c is done (gamma_C was
+                    // read before deltaReady)
+                    if (!wait(&barA[sb], (c >> 1) & 1)) break;
                     if (!src.wait_ready(c + 2, A.status, abort)) break;
-                    mbar_arrive_expect_tx(&fullA[sb], kPartA);
-                    bulk_g2s(stageA[sb], src.block(c + 2), kPartA, &fullA[sb]);
-                    lastA[sb] = c + 2;
+                    copy_wq(c + 2);
+                    if (!wait(&rFree[sb], (c >> 1) & 1)) break;
+                    copy_r(c + 2);
                 }
             }
             // every copy issued lands before shared memory is released
-            for (int sb = 0; sb < 2; ++sb)
-                if (lastA[sb] >= 0) mbar_wait(&fullA[sb], (lastA[sb] >> 1) & 1, A.status);
+            for (int sb = 0; sb < 2; ++sb) {
+                if (lastWQ[sb] >= 0) mbar_wait(&fullWQ[sb], (lastWQ[sb] >> 1) & 1, A.status);
+                if (lastR[sb] >= 0) mbar_wait(&fullR[sb], (lastR[sb] >> 1) & 1, A.status);
+            }
             if (lastU >= 0) mbar_wait(&fullU, lastU & 1, A.status);
         }
         __syncwarp();
@@ -733,21 +763,22 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
             int c = 0;
             for (; c < NC; ++c) {
                 const int sb = c & 1;
-                const uint8_t* st = stageA[sb];
+                const uint8_t* st = stageA(sb);
                 const uint32_t tD1 = tbase + kTD1 + sb * 128;
                 // D1[sb] = S [W; Q*gamma]^T (M = 128, N = 128, K = 128), once the fp16 state is in TMEM
-                if (!wait(&sReady, c & 1) || !wait(&fullA[sb], (c >> 1) & 1)) break;
+                // (one N = 128 product: a tcgen05 MMA step costs the same for N = 64 and N = 128)
+                if (!wait(&sReady, c & 1) || !wait(&fullWQ[sb], (c >> 1) & 1)) break;
                 tc_fence_after();
+                const uint64_t dWQ = sdesc(smem_u32(st + kOffWQ), 16, 1024);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_f16_ts(tD1, tbase + kTS + ks * 8,
-                               sdesc(smem_u32(st + kOffWQ) + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024), idA,
-                               ks > 0);
+                    mma_f16_ts(tD1, tbase + kTS + ks * 8, dWQ + (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4),
+                               idA, ks > 0);
                 mma_commit(&barA[sb]);
                 // output of chunk c-1 (staged by the epilogue warps in sO[(c-1)&1])
                 if (c > 0) {
                     if (!wait(&oStaged, (c - 1) & 1)) break;
-                    const uint8_t* so = sO[(c - 1) & 1];
+                    const uint8_t* so = sO((c - 1) & 1);
                     for (int bx = 0; bx < kOutBoxes; ++bx)
                         tma_store_4d(mo, so + bx * 8192, bx * kOutBoxCols, h, (c - 1) * kC, b);
                     bulk_commit();
@@ -757,21 +788,22 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
                     mbar_arrive(&oFree[0]);
                 }
                 // D3 = Delta^T K~ (N = 128) and D1[sb][:, 64:128] += Delta^T P^T (N = 64)
-                if (!wait(&deltaReady, c & 1)) break;
+                if (!wait(&deltaReady, c & 1) || !wait(&fullR[sb], (c >> 1) & 1)) break;
                 tc_fence_after();
+                const uint64_t dKT = sdesc(smem_u32(st + kOffKT), 8192, 1024);
+                const uint64_t dP = sdesc(smem_u32(st + kOffP), 16, 1024);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_f16_ts(tbase + kTD3, tbase + kTDelta + ks * 8,
-                               sdesc(smem_u32(st + kOffKT) + ks * 2048, 8192, 1024), idC, ks > 0);
+                for (int ks = 0; ks < 4; ++ks)  // accumulates onto gamma_C * S, which D3 holds
+                    mma_f16_ts(tbase + kTD3, tbase + kTDelta + ks * 8, dKT + (uint64_t)(ks * 2048 >> 4), idC, true);
                 mma_commit(&barC);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_f16_ts(tD1 + 64, tbase + kTDelta + ks * 8, sdesc(smem_u32(st + kOffP) + ks * 32, 16, 1024),
-                               idB, true);
+                    mma_f16_ts(tD1 + 64, tbase + kTDelta + ks * 8, dP + (uint64_t)(ks * 32 >> 4), idB, true);
                 mma_commit(&barB);
+                if (c + 2 < NC) mma_commit(&rFree[sb]);  // stage sb may take chunk c + 2
             }
             if (c == NC && wait(&oStaged, (NC - 1) & 1)) {  // output of the last chunk
-                const uint8_t* so = sO[(NC - 1) & 1];
+                const uint8_t* so = sO((NC - 1) & 1);
                 for (int bx = 0; bx < kOutBoxes; ++bx)
                     tma_store_4d(mo, so + bx * 8192, bx * kOutBoxCols, h, (NC - 1) * kC, b);
                 bulk_commit();
@@ -783,34 +815,66 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
         __syncwarp();
     } else {
         // ---------------------------------------------------------- epilogue warps --
+        // The fp32 state lives in TMEM (D3): each chunk's Delta^T K~ product accumulates onto
+        // gamma_C * S there. After that product the epilogue warps read S once and hand its fp16
+        // copy to the next chunk's MMAs; they stage the chunk's output and write gamma_C(next) * S
+        // back into D3 while the next chunk's first product runs, off the chain from one chunk's
+        // products to the next.
         const int quad = warp & 3, cg = warp >> 2;
         const int j = quad * 32 + lane;  // state row (d_v index) = TMEM lane
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const uint32_t tD3 = tbase + kTD3;
-        // initial state: this thread holds S[j][32 cg .. 32 cg + 31] in fp32
-        float s[32];
-        {
-            const float* s0 = A.S0 ? A.S0 + ((size_t)bh * kD + j) * kD + 32 * cg : nullptr;
-#pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-                const float4 t = s0 ? *reinterpret_cast<const float4*>(s0 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-                s[e] = t.x;
-                s[e + 1] = t.y;
-                s[e + 2] = t.z;
-                s[e + 3] = t.w;
-            }
+        const uint32_t tD3 = tbase + kTD3 + lane_off + 32 * cg;  // S[j][32 cg .. 32 cg + 31]
+        const uint32_t tS = tbase + kTS + lane_off + 16 * cg;    // their fp16 copy
+        // S_c (this thread's 32 columns, in x) becomes the fp16 operand of chunk c's MMAs
+        auto hand_over = [&](const float (&x)[32]) {
             uint32_t w[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) w[e] = pack2h(s[2 * e], s[2 * e + 1]);
-            tmem_st16(tbase + kTS + lane_off + 16 * cg, w);
+            for (int e = 0; e < 16; ++e) w[e] = pack2h(x[2 * e], x[2 * e + 1]);
+            tmem_st16(tS, w);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sReady);
+        };
+        // D3 <- gamma_C(c) * S_c, which the state product of chunk c accumulates onto; the store
+        // completes before this thread's Delta hand-off of chunk c (tmem_st_wait there)
+        auto decay = [&](float (&x)[32], int c) -> bool {
+            if (!wait(&fullR[c & 1], (c >> 1) & 1)) return false;
+            const float4* gam = reinterpret_cast<const float4*>(stageA(c & 1) + kOffGam) + 8 * cg;
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4) {
+                const float4 g = gam[q4];
+                x[4 * q4] *= g.x;
+                x[4 * q4 + 1] *= g.y;
+                x[4 * q4 + 2] *= g.z;
+                x[4 * q4 + 3] *= g.w;
+            }
+            tmem_st32(tD3, x);
+            return true;
+        };
+        // output staging: this thread's element of row r sits at ob + r * 128 + ((och ^ (r & 7)) << 4)
+        // (128-byte swizzled TMA boxes of 64 rows); rows r = 16 cg + e, and 16 cg is a multiple of 8
+        const uint32_t ob = (uint32_t)(16 * cg) * 128u +
+                            (sizeof(Tout) == 4 ? (uint32_t)(j >> 5) * 8192u + (uint32_t)(j & 3) * 4u
+                                               : (uint32_t)(j >> 6) * 8192u + (uint32_t)(j & 7) * 2u);
+        const uint32_t och = sizeof(Tout) == 4 ? (uint32_t)((j & 31) >> 2) : (uint32_t)((j & 63) >> 3);
+        bool ok;
+        {
+            float x[32];
+            const float* s0 = A.S0 ? A.S0 + ((size_t)bh * kD + j) * kD + 32 * cg : nullptr;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+                const float4 t = s0 ? *reinterpret_cast<const float4*>(s0 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+                x[e] = t.x;
+                x[e + 1] = t.y;
+                x[e + 2] = t.z;
+                x[e + 3] = t.w;
+            }
+            hand_over(x);
+            ok = decay(x, 0);
         }
-        for (int c = 0; c < NC; ++c) {
+        for (int c = 0; ok && c < NC; ++c) {
             const int sb = c & 1;
-            const uint8_t* st = stageA[sb];
             const uint32_t tD1 = tbase + kTD1 + sb * 128;
             // ---- Delta^T[j][r] = U^T[j][r] - (S W^T)[j][r], r in [16 cg, 16 cg + 16), into TMEM
             if (!wait(&fullU, c & 1) || !wait(&barA[sb], (c >> 1) & 1)) break;
@@ -825,50 +889,46 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
 #pragma unroll
                 for (int e = 0; e < 8; ++e) w[e] = pack2h(u[2 * e] - x[2 * e], u[2 * e + 1] - x[2 * e + 1]);
                 tmem_st8(tbase + kTDelta + lane_off + 8 * cg, w);
-                tmem_st_wait();
+                tmem_st_wait();  // also completes the D3 store of hand_over
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&deltaReady);
-            // ---- S <- S Diag(gamma_C) + Delta^T K~ on this thread's 32 columns; fp16 copy into TMEM
+            // ---- S_{c+1} = gamma_C S_c + Delta^T K~ (D3): on to chunk c + 1, or out as S_T
             if (!wait(&barC, c & 1)) break;
             tc_fence_after();
-            {
-                const float* gam = reinterpret_cast<const float*>(st + kOffGam) + 32 * cg;
-                float x[32];
-                tmem_ld32(tD3 + lane_off + 32 * cg, x);
-                tmem_ld_wait();
-                uint32_t w[16];
+            float x[32];
+            tmem_ld32(tD3, x);
+            tmem_ld_wait();
+            if (c + 1 < NC) {
+                hand_over(x);
+            } else if (A.S_T != nullptr) {
+                float* dst = A.S_T + ((size_t)bh * kD + j) * kD + 32 * cg;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) s[e] = fmaf(gam[e], s[e], x[e]);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) w[e] = pack2h(s[2 * e], s[2 * e + 1]);
-                tmem_st16(tbase + kTS + lane_off + 16 * cg, w);
-                tmem_st_wait();
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4*>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sReady);
-            // ---- output of chunk c into the staging buffer sO[sb]
+            // ---- output of chunk c into the staging buffer sO(sb)
             if (!wait(&barB, c & 1) || !wait(&oFree[sb], (c >> 1) & 1)) break;
             tc_fence_after();
             {
                 float x[16];
                 tmem_ld16(tD1 + 64 + lane_off + 16 * cg, x);
                 tmem_ld_wait();
+                uint8_t* o = sO(sb) + ob;
 #pragma unroll
-                for (int e = 0; e < 16; ++e) stage_out<Tout>(sO[sb], 16 * cg + e, j, A.scale * x[e]);
+                for (int e = 0; e < 16; ++e) {
+                    uint8_t* p = o + e * 128 + ((och ^ (uint32_t)(e & 7)) << 4);
+                    if (sizeof(Tout) == 4) *reinterpret_cast<float*>(p) = A.scale * x[e];
+                    else *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(A.scale * x[e]);
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&oStaged);
-        }
-        if (A.S_T != nullptr) {
-            float* dst = A.S_T + ((size_t)bh * kD + j) * kD + 32 * cg;
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-                *reinterpret_cast<float4*>(dst + e) = make_float4(s[e], s[e + 1], s[e + 2], s[e + 3]);
+            // ---- gamma_C(c + 1) S_{c+1} into D3 while chunk c + 1's first product runs
+            if (c + 1 < NC && !decay(x, c + 1)) break;
         }
     }
 }

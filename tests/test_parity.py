@@ -107,6 +107,18 @@ def test_alpha_zero_resets():
     check_chunk(x, "scalar", "bf16")
 
 
+def test_scalar_decay_strength_mix():
+    """Chunks whose cumulative in-chunk log2-decay stays within 120 units take the factored pairwise
+    decays 2^Gamma_r * 2^-Gamma_i, stronger ones the exact 2^(Gamma_r - Gamma_i): both kinds of
+    chunk (and one right at the limit) in one call, against the oracle."""
+    x = make_chunk_inputs(2, 640, 4, 128, 128, "scalar", "bf16", 96, s0_std=0.05)
+    g = x["g"].clone()
+    g[:, 128:256] = -3.0   # about 277 log2 units across a chunk
+    g[:, 384:448] = -1.3   # 64 * 1.3 * log2(e) = 120.0
+    x["g"] = g
+    check_chunk(x, "scalar", "bf16")
+
+
 def test_channel_constant_equals_scalar():
     x = make_chunk_inputs(2, 192, 2, 128, 128, "scalar", "bf16", 93)
     o1, s1 = run_chunk(x, "scalar")
