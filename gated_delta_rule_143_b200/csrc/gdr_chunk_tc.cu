@@ -268,6 +268,7 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
     // ---- 1. TMA: K and Q into the two halves of the 128-row [K; Q] tile, V; beta and the
     //         cumulative log-decay (log2 units; rows past the tail repeat Gamma_{n-1}) meanwhile
     if (lt == 0) {
+        bulk_wait_read<0>();  // the previous task's W / U^T bulk stores have read the K / V tiles
         mbar_arrive_expect_tx(barT, 6 * 8192);
         tma_load_4d(sKQ, mk, 0, h, c0, b, barT);
         tma_load_4d(sKQ + 16384, mk, 64, h, c0, b, barT);
@@ -532,14 +533,12 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
         fence_proxy_async_smem();
         tc_fence_before();
         named_bar(ps.bar_id, kPrepThreads);
-        if (lt == 0) {
+        if (lt == 0) {  // the next task waits for these reads before its TMA loads into the same tiles
             bulk_s2g(out + kOffWQ, stW, 8192);
             bulk_s2g(out + kOffWQ + 16384, stW + 16384, 8192);
             bulk_s2g(out + kOffUT, stU, 16384);
             bulk_commit();
-            bulk_wait_read<0>();  // the staging tiles may be reused; the writes complete on their own
         }
-        named_bar(ps.bar_id, kPrepThreads);
     }
 }
 

@@ -343,7 +343,11 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 }
 
 // Named barrier over `nthreads` threads (a multiple of 32) of this CTA.
+// bar.sync is the warp-aligned barrier: every lane of a participating warp must reach it together,
+// so the warp reconverges first (a lane still inside a single-thread branch, e.g. waiting on a bulk
+// copy, would otherwise let the warp's other lanes arrive for it).
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
+    __syncwarp();
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
