@@ -628,20 +628,20 @@ struct WorkspaceSource {  // two passes: every block was written before the stat
     __device__ void release(int) const {}
 };
 
-constexpr int kRing = 8;  // ring slots per head in the fused kernel
+constexpr int kRing = 8;  // ring slots per head in the fused kernel when no chunk is pre-computed
 struct RingSource {       // fused kernel: chunks c < c1 were written to `pre` by a prep kernel launched
-                          // before; the others pass through kRing slots, flagged by the producers
+                          // before; the others pass through `depth` slots, flagged by the producers
     const uint8_t* pre;   // block of chunk 0 of this head among the pre-computed ones (c1 per head)
     const uint8_t* base;  // slot 0 of this head
-    const int* ready;     // [kRing]: c + 1 once the block of chunk c in that slot is complete
+    const int* ready;     // [depth]: c + 1 once the block of chunk c in that slot is complete
     int* consumed;        // number of this head's chunks already copied out of the ring (counted from 0)
-    int c1;
+    int c1, depth;
     __device__ const uint8_t* block(int c) const {
-        return c < c1 ? pre + (size_t)c * kHandoffStride : base + (size_t)(c % kRing) * kHandoffStride;
+        return c < c1 ? pre + (size_t)c * kHandoffStride : base + (size_t)(c % depth) * kHandoffStride;
     }
     __device__ bool wait_ready(int c, int* status, volatile int* abort) const {
         if (c < c1) return true;
-        if (!flag_wait_geq(ready + c % kRing, c + 1, status, abort, 128)) return false;
+        if (!flag_wait_geq(ready + c % depth, c + 1, status, abort, 128)) return false;
         fence_proxy_async_global();  // the bulk copies that follow read what the acquire made visible
         return true;
     }
@@ -961,8 +961,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const ui
 // Both passes in one cooperative launch: CTAs 0 .. BH-1 run the state pass of head bh = blockIdx.x,
 // the other CTAs run two prep pipelines each (warps 0-7 and 8-15; warps 16-17 idle). The prep
 // pipelines claim tasks from a counter in the order the state passes consume them (chunk index
-// outermost: tau = c * BH + bh) and write each hand-off block into ring slot c % kRing of
-// its head, after the head's state pass has copied out chunk c - kRing; a release flag per slot
+// outermost: tau = c * BH + bh) and write each hand-off block into ring slot c % depth of
+// its head, after the head's state pass has copied out chunk c - depth; a release flag per slot
 // publishes the block. All CTAs are co-resident (cooperative launch), tasks are claimed in
 // increasing order and the state passes consume in order, so the earliest unfinished task can
 // always proceed. The ring stays in L2: the hand-off never makes a round trip to DRAM.
@@ -973,12 +973,13 @@ constexpr uint32_t kFusedSmem = (2 * kPrepPipeBytes > kStateSmem - 1024 ? 2 * kP
 constexpr int kFusedMaxHeads = 100;  // B * H above this runs the two-pass path (too few SMs left for prep)
 
 struct RingArgs {
-    uint8_t* ring;     // [BH][kRing] hand-off blocks
-    int* ready;        // [BH][kRing]
+    uint8_t* ring;     // [BH][depth] hand-off blocks
+    int* ready;        // [BH][depth]
     int* consumed;     // [BH]
     int* next_task;    // prep tasks claimed so far (one counter, counted from task c1 * BH)
     const uint8_t* pre;  // [BH][c1] blocks of the chunks below c1, written by chunk_prep_kernel before
     int BH, c1;
+    int depth;         // ring slots per head: kRing, or every chunk from c1 on when c1 > 0
 };
 
 template <int MODE>
@@ -1012,18 +1013,18 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
         named_bar(ps.bar_id, kPrepThreads);  // every thread has read it before the next claim
         if (tau >= n_tasks) break;
         const int c = tau / R.BH, bh = tau % R.BH;
-        const int slot = c % kRing;
+        const int slot = c % R.depth;
         if (lt == 0)
-            go[pipe] = c - kRing < R.c1 || flag_wait_geq(R.consumed + bh, c - kRing + 1, P.status, abort, 2048);
+            go[pipe] = c - R.depth < R.c1 || flag_wait_geq(R.consumed + bh, c - R.depth + 1, P.status, abort, 2048);
         named_bar(ps.bar_id, kPrepThreads);
         if (!go[pipe]) break;
-        uint8_t* out = R.ring + ((size_t)bh * kRing + slot) * kHandoffStride;
+        uint8_t* out = R.ring + ((size_t)bh * R.depth + slot) * kHandoffStride;
         prep_chunk<MODE>(P, mq, mk, mv, ps, bh / P.H, bh % P.H, c, out, it, lt);
         if (lt == 0) {  // every write of the block (generic stores before prep_chunk's last barrier, bulk stores)
             bulk_wait<0>();
             fence_proxy_async_global();
             __threadfence();
-            st_release_gpu(R.ready + bh * kRing + slot, c + 1);
+            st_release_gpu(R.ready + bh * R.depth + slot, c + 1);
         }
     }
 }
@@ -1048,8 +1049,9 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     uint8_t* sm = align1024(smem_raw);
     if ((int)blockIdx.x < R.BH) {
         const int bh = blockIdx.x;
-        const RingSource src{R.pre + (size_t)bh * R.c1 * kHandoffStride, R.ring + (size_t)bh * kRing * kHandoffStride,
-                             R.ready + bh * kRing, R.consumed + bh, R.c1};
+        const RingSource src{R.pre + (size_t)bh * R.c1 * kHandoffStride,
+                             R.ring + (size_t)bh * R.depth * kHandoffStride, R.ready + bh * R.depth, R.consumed + bh,
+                             R.c1, R.depth};
         state_body<Tout>(&mo, A, bh, src, sm, tmem_base, &abort_flag);
     } else {
         prep_role<MODE>(&mq, &mk, &mv, P, R, sm, tmem_base, &abort_flag);
@@ -1131,8 +1133,6 @@ cudaError_t launch_state(const ChunkProblem& p, const CUtensorMap& mo, int NC, c
 // The fused kernel serves DeltaNet and the scalar gate for up to kFusedMaxHeads heads; the channel
 // gate (two of its prep pipelines do not fit in shared memory) and larger B * H use two passes.
 bool use_fused(int B, int H, int mode) { return mode != GDR_DECAY_CHANNEL && (size_t)B * H <= kFusedMaxHeads; }
-size_t ring_bytes(int BH) { return (size_t)BH * kRing * kHandoffStride; }
-size_t flag_bytes(int BH) { return ((size_t)(BH * (kRing + 1) + 1) * sizeof(int) + 255) & ~size_t(255); }
 
 // Chunks per head the fused kernel takes pre-computed from a prep kernel that runs before it on
 // all SMs. In the fused kernel the kSMs - BH prep CTAs must keep up with the BH chains: a chain
@@ -1151,6 +1151,17 @@ int fused_precomputed_chunks(int BH, int NC) {
     return c1 < NC ? c1 : NC;
 }
 size_t pre_bytes(int BH, int NC) { return (size_t)BH * fused_precomputed_chunks(BH, NC) * kHandoffStride; }
+// Ring slots per head. With chunks pre-computed, the chains spend their first c1 chunks on those
+// while the fused kernel's prep CTAs run ahead: a slot for every later chunk keeps them from
+// stalling on a full ring in that time (the blocks then mostly live in DRAM, not L2).
+int ring_depth(int BH, int NC) {
+    const int c1 = fused_precomputed_chunks(BH, NC);
+    return c1 > 0 ? NC - c1 : kRing;
+}
+size_t ring_bytes(int BH, int NC) { return (size_t)BH * ring_depth(BH, NC) * kHandoffStride; }
+size_t flag_bytes(int BH, int NC) {
+    return ((size_t)(BH * (ring_depth(BH, NC) + 1) + 1) * sizeof(int) + 255) & ~size_t(255);
+}
 
 template <int MODE, typename Tout>
 cudaError_t launch_fused(const ChunkProblem& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
@@ -1167,13 +1178,13 @@ cudaError_t launch_fused(const ChunkProblem& p, const CUtensorMap& mq, const CUt
     const int BH = p.B * p.H;
     const int grid = sms * per_sm;
     if (!coop || per_sm < 1 || grid - BH < 8) return cudaErrorCooperativeLaunchTooLarge;
-    // workspace: [pre-computed blocks, BH x c1][ring, BH x kRing][flags]
+    // workspace: [pre-computed blocks, BH x c1][ring, BH x depth][flags]
     uint8_t* ws = static_cast<uint8_t*>(p.workspace);
-    const int c1 = fused_precomputed_chunks(BH, NC);
+    const int c1 = fused_precomputed_chunks(BH, NC), depth = ring_depth(BH, NC);
     uint8_t* ring = ws + pre_bytes(BH, NC);
-    int* flags = reinterpret_cast<int*>(ring + ring_bytes(BH));
-    RingArgs R{ring, flags, flags + (size_t)BH * kRing, flags + (size_t)BH * (kRing + 1), ws, BH, c1};
-    if ((err = cudaMemsetAsync(flags, 0, flag_bytes(BH), stream)) != cudaSuccess) return err;
+    int* flags = reinterpret_cast<int*>(ring + ring_bytes(BH, NC));
+    RingArgs R{ring, flags, flags + (size_t)BH * depth, flags + (size_t)BH * (depth + 1), ws, BH, c1, depth};
+    if ((err = cudaMemsetAsync(flags, 0, flag_bytes(BH, NC), stream)) != cudaSuccess) return err;
     if (c1 > 0 && (err = launch_prep<MODE>(p, mq, mk, mv, NC, c1, ws, stream)) != cudaSuccess) return err;
     PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status};
     StateArgs A{p.S0, p.S_T, p.T, p.H, NC, p.scale, p.status};
@@ -1193,7 +1204,7 @@ bool chunk_tc_supported(int dk, int dv, int chunk, int dtype, int o_dtype) {
 
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int, int, int, int mode) {
     const int NC = (T + kC - 1) / kC;
-    if (use_fused(B, H, mode)) return pre_bytes(B * H, NC) + ring_bytes(B * H) + flag_bytes(B * H);
+    if (use_fused(B, H, mode)) return pre_bytes(B * H, NC) + ring_bytes(B * H, NC) + flag_bytes(B * H, NC);
     return (size_t)B * H * NC * kHandoffStride;
 }
 
