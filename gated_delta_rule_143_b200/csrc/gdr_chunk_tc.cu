@@ -602,9 +602,10 @@ constexpr int kEpiWarps = 16;
 constexpr int kStateThreads = (kEpiWarps + 2) * 32;  // + MMA issuer warp + copy warp
 constexpr uint32_t kSStageA0 = 0;
 constexpr uint32_t kSStageA1 = 58368;
-constexpr uint32_t kSUT = 116736;       // U^T stage (single buffer)
-constexpr uint32_t kSO0 = 133120;       // output staging, double-buffered: 4 (fp32) or 2 (bf16) TMA boxes
-constexpr uint32_t kSO1 = 165888;       //   of 64 rows x 128 B each
+constexpr uint32_t kSUT0 = 116736;      // U^T stages (double-buffered, 16 KiB each)
+constexpr uint32_t kSUT1 = 133120;
+constexpr uint32_t kSO0 = 149504;       // output staging, double-buffered: 4 (fp32) or 2 (bf16) TMA boxes
+constexpr uint32_t kSO1 = 182272;       //   of 64 rows x 128 B each
 constexpr uint32_t kStateSmem = kSO1 + 32768 + 1024;
 // TMEM: D1 double-buffered (corr^T | O^T, 128 columns each), D3 (state increment), the fp16 state
 // copy (128 x 128 -> 64 columns) and Delta^T (128 x 64 fp16 -> 32 columns)
@@ -657,14 +658,14 @@ template <typename Tout, typename Src>
 __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, const Src& src, uint8_t* sm,
                            uint32_t tbase, volatile int* abort) {
     auto stageA = [sm](int i) { return sm + kSStageA0 + i * (kSStageA1 - kSStageA0); };  // part A stage i
-    uint8_t* sUT = sm + kSUT;
+    auto sUT = [sm](int i) { return sm + kSUT0 + i * (kSUT1 - kSUT0); };  // U^T stage i
     auto sO = [sm](int i) { return sm + kSO0 + i * (kSO1 - kSO0); };  // output staging buffer i
     // fullWQ/fullR/fullU: bulk copies of [W; Q*gamma], of the rest of part A and of U^T landed.
     // barA/barB/barC: MMA groups done; rFree[s]: every MMA reading stage s is done. deltaReady/
     // sReady/oStaged: all epilogue warps wrote Delta^T / the fp16 state (TMEM) / the output
     // staging (shared). oFree[b]: the output staging buffer b has been read by its store.
     // drain: last MMAs complete.
-    __shared__ uint64_t fullWQ[2], fullR[2], fullU, barA[2], rFree[2], barB, barC, deltaReady, sReady, oStaged,
+    __shared__ uint64_t fullWQ[2], fullR[2], fullU[2], barA[2], rFree[2], barB, barC, deltaReady, sReady, oStaged,
         oFree[2], drain;
 
     const int b = bh / A.H, h = bh % A.H;
@@ -678,11 +679,11 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
         for (int i = 0; i < 2; ++i) {
             mbar_init(&fullWQ[i], 1);
             mbar_init(&fullR[i], 1);
+            mbar_init(&fullU[i], 1);
             mbar_init(&barA[i], 1);
             mbar_init(&rFree[i], 1);
             mbar_init(&oFree[i], 1);
         }
-        mbar_init(&fullU, 1);
         mbar_init(&barB, 1);
         mbar_init(&barC, 1);
         mbar_init(&drain, 1);
@@ -695,13 +696,13 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
 
     if (warp == kEpiWarps + 1) {
         // --------------------------------------------------------------- copy warp --
-        // Brings hand-off blocks into shared memory (part A double-buffered, U^T single-buffered)
-        // as soon as both the block is ready and its buffer is free, and hands each ring slot back
-        // once all of its chunk is in shared memory: all flag traffic stays off the MMA issuer's
-        // path. Part A of chunk c + 2 comes in two pieces: [W; Q*gamma] as soon as chunk c's first
-        // product is done (its only reader), the rest once chunk c's last product is done.
+        // Brings hand-off blocks into shared memory (part A and U^T double-buffered) as soon as both
+        // the block is ready and its buffer is free, and hands each ring slot back once all of its
+        // chunk is in shared memory: all flag traffic stays off the MMA issuer's path. Chunk c + 2
+        // comes in three pieces: U^T and [W; Q*gamma] once chunk c's Delta is done (their readers:
+        // the epilogue warps, chunk c's first product), the rest once chunk c's last product is done.
         if (lane == 0) {
-            int lastWQ[2] = {-1, -1}, lastR[2] = {-1, -1}, lastU = -1;  // last chunk whose copy was issued
+            int lastWQ[2] = {-1, -1}, lastR[2] = {-1, -1}, lastU[2] = {-1, -1};  // last chunk copied
             auto copy_wq = [&](int c) {
                 mbar_arrive_expect_tx(&fullWQ[c & 1], kPartWQ);
                 bulk_g2s(stageA(c & 1), src.block(c), kPartWQ, &fullWQ[c & 1]);
@@ -712,34 +713,31 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
                 bulk_g2s(stageA(c & 1) + kPartWQ, src.block(c) + kPartWQ, kPartA - kPartWQ, &fullR[c & 1]);
                 lastR[c & 1] = c;
             };
+            auto copy_u = [&](int c) {
+                mbar_arrive_expect_tx(&fullU[c & 1], 16384);
+                bulk_g2s(sUT(c & 1), src.block(c) + kOffUT, 16384, &fullU[c & 1]);
+                lastU[c & 1] = c;
+            };
             bool ok = true;
             for (int st = 0; st < 2 && st < NC && ok; ++st) {
                 if (!(ok = src.wait_ready(st, A.status, abort))) break;
+                copy_u(st);
                 copy_wq(st);
                 copy_r(st);
-            }
-            if (ok) {
-                mbar_arrive_expect_tx(&fullU, 16384);
-                bulk_g2s(sUT, src.block(0) + kOffUT, 16384, &fullU);
-                lastU = 0;
             }
             for (int c = 0; ok && c < NC; ++c) {
                 const int sb = c & 1;
                 // every epilogue warp has read U^T of chunk c (and waited for it), so all of chunk c
-                // is in shared memory: the ring slot goes back; U^T of chunk c + 1 comes in
+                // is in shared memory: the ring slot goes back
                 if (!wait(&deltaReady, c & 1)) break;
                 src.release(c);
-                if (c + 1 < NC) {
-                    mbar_arrive_expect_tx(&fullU, 16384);
-                    bulk_g2s(sUT, src.block(c + 1) + kOffUT, 16384, &fullU);
-                    lastU = c + 1;
-                }
                 if (c + 2 < NC) {
                     // chunk c's first product (barA, complete before deltaReady) has read [W; Q*gamma]
                     // of stage sb; the rest follows once every MMA of chunk c is done (gamma_C was
                     // read before deltaReady)
                     if (!wait(&barA[sb], (c >> 1) & 1)) break;
                     if (!src.wait_ready(c + 2, A.status, abort)) break;
+                    copy_u(c + 2);
                     copy_wq(c + 2);
                     if (!wait(&rFree[sb], (c >> 1) & 1)) break;
                     copy_r(c + 2);
@@ -749,8 +747,8 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
             for (int sb = 0; sb < 2; ++sb) {
                 if (lastWQ[sb] >= 0) mbar_wait(&fullWQ[sb], (lastWQ[sb] >> 1) & 1, A.status);
                 if (lastR[sb] >= 0) mbar_wait(&fullR[sb], (lastR[sb] >> 1) & 1, A.status);
+                if (lastU[sb] >= 0) mbar_wait(&fullU[sb], (lastU[sb] >> 1) & 1, A.status);
             }
-            if (lastU >= 0) mbar_wait(&fullU, lastU & 1, A.status);
         }
         __syncwarp();
     } else if (warp == kEpiWarps) {
@@ -876,13 +874,13 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
             const int sb = c & 1;
             const uint32_t tD1 = tbase + kTD1 + sb * 128;
             // ---- Delta^T[j][r] = U^T[j][r] - (S W^T)[j][r], r in [16 cg, 16 cg + 16), into TMEM
-            if (!wait(&fullU, c & 1) || !wait(&barA[sb], (c >> 1) & 1)) break;
+            if (!wait(&fullU[sb], (c >> 1) & 1) || !wait(&barA[sb], (c >> 1) & 1)) break;
             tc_fence_after();
             {
                 float x[16], u[16];
                 tmem_ld16(tD1 + lane_off + 16 * cg, x);
-                unpack8h(ld16(sUT + kmajor_off(j, 16 * cg, 128)), u);
-                unpack8h(ld16(sUT + kmajor_off(j, 16 * cg + 8, 128)), u + 8);
+                unpack8h(ld16(sUT(sb) + kmajor_off(j, 16 * cg, 128)), u);
+                unpack8h(ld16(sUT(sb) + kmajor_off(j, 16 * cg + 8, 128)), u + 8);
                 tmem_ld_wait();
                 uint32_t w[8];
 #pragma unroll
