@@ -118,9 +118,17 @@ def test_plan_query_is_host_only():
     # launches and workspace follow the plan
     assert gdr.launches_per_chunk_fwd(1, 4096, 8, 128, 128, 64, "scalar", bf) == 1
     assert gdr.launches_per_chunk_fwd(8, 4096, 8, 128, 128, 64, "scalar", bf) == 2
-    ring = 8 * 8 * 74752  # eight ring slots per head
-    assert gdr.workspace_bytes(1, 4096, 8, 128, 128, 64, "scalar", bf) >= ring
-    assert gdr.workspace_bytes(8, 4096, 8, 128, 128, 64, "scalar", bf) >= 64 * (8 + c1) * 74752
+    block = 74752  # one hand-off block per chunk of a head
+
+    def flags(heads, slots):  # a ready flag per slot, a consumed counter per head, one task counter
+        return (heads * (slots + 1) + 1) * 4 + 255 & ~255
+
+    # fused alone: a ring of eight slots per head
+    assert gdr.workspace_bytes(1, 4096, 8, 128, 128, 64, "scalar", bf) == 8 * 8 * block + flags(8, 8)
+    # prep + fused: c1 pre-computed blocks and a slot for every later chunk, i.e. one block per chunk
+    assert gdr.workspace_bytes(8, 4096, 8, 128, 128, 64, "scalar", bf) == 64 * 64 * block + flags(64, 64 - c1)
+    # a short sequence keeps eight slots even when it has fewer chunks
+    assert gdr.workspace_bytes(1, 100, 8, 128, 128, 64, "scalar", bf) == 8 * 8 * block + flags(8, 8)
 
 
 def test_host_entry_point_validates_on_host():
