@@ -547,7 +547,7 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
 // block's index in the workspace; NCp = NC on the two-pass path, the fused kernel's c1 before it).
 // At the start of each task the tiles of the CTA's next task are prefetched into L2.
 template <int MODE>
-__global__ void __launch_bounds__(kPrepThreads, MODE == GDR_DECAY_CHANNEL ? 1 : 2)
+__global__ void __maxnreg__(MODE == GDR_DECAY_CHANNEL ? 240 : 96)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                   const __grid_constant__ CUtensorMap mv, PrepArgs P, uint8_t* __restrict__ ws, int NCp, int n_tasks) {
     extern __shared__ uint8_t smem_raw[];
@@ -1139,7 +1139,7 @@ bool use_fused(int B, int H, int mode) { return mode != GDR_DECAY_CHANNEL && (si
 // the remaining chunks are prepared beforehand with every SM. (A fixed SM count keeps the result,
 // and with it the workspace size, a host-only function of the shape.)
 constexpr int kSMs = 148;
-constexpr double kChainPerTask = 0.32;  // measured: chain 2.2-2.6 us per chunk, fused prep CTA 7.2 us per task
+constexpr double kChainPerTask = 0.35;  // measured: chain 2.2-2.6 us per chunk, fused prep CTA 7.2 us per task
 constexpr int kHybridMinHeads = 57;     // below, the fused kernel alone is faster (measured at 48 heads)
 int fused_precomputed_chunks(int BH, int NC) {
     if (BH < kHybridMinHeads) return 0;
