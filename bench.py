@@ -377,20 +377,30 @@ def gdr_kernels_per_step(w):
     return gdr.launches_per_chunk_fwd(w.B, w.T, w.H, w.dk, w.dv, w.chunk, w.mode, torch.bfloat16, torch.float32)
 
 
+def kernel_code_digest(text=None):
+    """sha256 of the tensor-core kernel source (or of `text`) with its comments and blank lines
+    removed: an edit of the code makes recorded counters stale, an edit of a comment does not."""
+    import hashlib
+    import re
+    if text is None:
+        with open(os.path.join(ROOT, "gated_delta_rule_143_b200", "csrc", "gdr_chunk_tc.cu")) as f:
+            text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+    return hashlib.sha256(code.encode()).hexdigest()
+
+
 def traffic_from_profile(kernel):
     """DRAM bytes (read + write) per launch of `kernel` on this workload, from the committed ncu
-    summary (profiles/traffic.json), or None when none was recorded for the current kernel."""
-    import hashlib
+    summary (profiles/traffic.json), or None when none was recorded for the current kernel code."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    src = os.path.join(ROOT, "gated_delta_rule_143_b200", "csrc", "gdr_chunk_tc.cu")
-    with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
-    if not sha.startswith(d.get("_kernel_sha256_prefix", "-")):
-        return None  # the kernel changed since the counters were taken
+    if not kernel_code_digest().startswith(d.get("_kernel_code_sha256_prefix", "-")):
+        return None  # the kernel code changed since the counters were taken
     return d.get(WORKLOAD, {}).get(kernel)
 
 

@@ -75,3 +75,13 @@ def test_reference_arm_nonzero_rank_exits_without_work():
                         "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_kernel_code_digest_ignores_comments_only():
+    """Recorded DRAM counters stay valid across comment edits of the kernel source, not code edits."""
+    import bench
+    a = "int f(int x) {  // doubles\n    return 2 * x;  /* the\n factor */\n}\n"
+    b = "// new header\nint f(int x) {\n\n    return 2 * x;\n}\n"
+    c = "int f(int x) {\n    return 3 * x;\n}\n"
+    assert bench.kernel_code_digest(a) == bench.kernel_code_digest(b)
+    assert bench.kernel_code_digest(a) != bench.kernel_code_digest(c)
