@@ -378,13 +378,17 @@ def gdr_kernels_per_step(w):
 
 
 def kernel_code_digest(text=None):
-    """sha256 of the tensor-core kernel source (or of `text`) with its comments and blank lines
-    removed: an edit of the code makes recorded counters stale, an edit of a comment does not."""
+    """sha256 of the tensor-core kernel sources (gdr_chunk_tc.cu and the device helpers it
+    includes, gdr_sm100.cuh), or of `text`, with comments and blank lines removed: an edit of the
+    code makes recorded counters stale, an edit of a comment does not."""
     import hashlib
     import re
     if text is None:
-        with open(os.path.join(ROOT, "gated_delta_rule_143_b200", "csrc", "gdr_chunk_tc.cu")) as f:
-            text = f.read()
+        csrc = os.path.join(ROOT, "gated_delta_rule_143_b200", "csrc")
+        text = ""
+        for name in ("gdr_chunk_tc.cu", "gdr_sm100.cuh"):
+            with open(os.path.join(csrc, name)) as f:
+                text += f.read() + "\n"
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     text = re.sub(r"//[^\n]*", "", text)
     code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
