@@ -50,7 +50,9 @@ def test_chunk_small(mode, dtype, d, T, with_s0):
     (3, 16, 333, "fused"),        # 48 heads
     (7, 8, 191, "fused"),         # 56 heads: the largest fused-only case
     (8, 8, 200, "prep_fused"),    # 64 heads: the first chunks prepared before the fused kernel
-    (8, 8, 1000, "prep_fused"),   # 64 heads, 16 chunks (10 prepared before), ragged tail
+    (8, 8, 1000, "prep_fused"),   # 64 heads, 16 chunks (9 prepared before, 7 ring slots), ragged tail
+    (8, 8, 50, "prep_fused"),     # 64 heads, one chunk: every chunk prepared before, no ring slot
+    (12, 8, 100, "prep_fused"),   # 96 heads, two chunks, both prepared before
     (13, 8, 130, "two_pass"),     # 104 heads: prep kernel, then state kernel
 ])
 def test_chunk_tensor_core_paths(mode, B, H, T, plan):
