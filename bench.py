@@ -328,6 +328,7 @@ def run_ours(args):
         if rank == 0:
             print(json.dumps({"metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
                               "ms_per_step": round(ms_step, 5), "config": {"workload": WORKLOAD, "B": w.B, "T": w.T},
+                              "plan": plan, "precomputed_chunks_per_head": c1,
                               "roofline_frac": round(nbytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                               "kernels": [(k["kernel"], k["launch_us"]) for k in kernels]}))
         return
@@ -487,6 +488,7 @@ def run_reference(args):
 
 
 def main():
+    global WORKLOAD
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)  # about 0.25 s timed: a dozen clock samples
@@ -496,7 +498,13 @@ def main():
                     help="fwd: time the forward only (no e2e, decode or CPU baseline), for profiling runs")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size (profiling runs)")
     ap.add_argument("--seq", type=int, default=0, help="override the workload's sequence length (profiling runs)")
+    ap.add_argument("--workload", choices=sorted(CHUNK_WORKLOADS), default=WORKLOAD,
+                    help="chunked-forward workload (default: the headline one; others for --only fwd runs)")
     args = ap.parse_args()
+    if args.workload != WORKLOAD:
+        if args.only != "fwd" or args.impl != "ours":
+            ap.error("other workloads are timed with --only fwd (the full line describes the headline one)")
+        WORKLOAD = args.workload
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":
