@@ -228,8 +228,98 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
     }
 }
 
+// ------------------------------------------------------------- short sequences --
+// Up to kRecMaxT tokens the token-by-token recurrence itself beats the chunk form's per-chunk
+// work: one warp per state row (rows of S evolve independently given k, beta and alpha), the row
+// in registers (lane holds columns lane + 32 i). Per token, with alpha = exp(g):
+//   s <- s * alpha;  p = s . k;  s <- s + beta (v_j - p) k;  o_j = scale (s . q)
+// (the delta rule of "Linear Attention & DeltaNet" with the gate of "linear attention and its
+// gated descendants"). Tokens are staged in shared memory kRecTB at a time.
+constexpr int kRecWarps = 8;   // state rows per CTA
+constexpr int kRecTB = 16;     // tokens per staged block
+constexpr int kRecMaxT = 256;  // sequences up to this length run the recurrence
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+    return x;
+}
+
+template <typename Tin, typename Tout, int MODE, int DK>
+__global__ void __launch_bounds__(kRecWarps * 32)
+recurrent_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+                      const float* __restrict__ g, const float* __restrict__ beta, const float* S0,
+                      Tout* __restrict__ o, float* S_T, int T, int H, int dv, float scale) {
+    constexpr int NL = DK / 32;                                  // state columns per lane
+    constexpr int NA = MODE == GDR_DECAY_CHANNEL ? DK : 1;       // decay factors per token
+    __shared__ float sK[kRecTB][DK], sQ[kRecTB][DK], sAl[kRecTB][NA], sV[kRecTB][kRecWarps], sB[kRecTB];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int j0 = blockIdx.x * kRecWarps, j = j0 + warp;       // this warp's state row
+    const int h = blockIdx.y, b = blockIdx.z;
+    const size_t bh = (size_t)b * H + h;
+    const bool active = j < dv;
+    float s[NL];
+#pragma unroll
+    for (int i = 0; i < NL; ++i) s[i] = (active && S0 != nullptr) ? S0[(bh * dv + j) * DK + lane + 32 * i] : 0.f;
+    for (int t0 = 0; t0 < T; t0 += kRecTB) {
+        const int n = min(kRecTB, T - t0);
+        __syncthreads();  // every warp is done with the previous block
+        for (int idx = tid; idx < n * DK; idx += kRecWarps * 32) {
+            const int r = idx / DK, c = idx % DK;
+            const size_t tok = ((size_t)b * T + t0 + r) * H + h;
+            sK[r][c] = load_f32(k + tok * DK + c);
+            sQ[r][c] = load_f32(q + tok * DK + c);
+            if (MODE == GDR_DECAY_CHANNEL) sAl[r][c] = expf(g[tok * DK + c]);
+        }
+        for (int idx = tid; idx < n * kRecWarps; idx += kRecWarps * 32) {
+            const int r = idx / kRecWarps, w = idx % kRecWarps;
+            const size_t tok = ((size_t)b * T + t0 + r) * H + h;
+            sV[r][w] = (j0 + w < dv) ? load_f32(v + tok * dv + j0 + w) : 0.f;
+        }
+        for (int r = tid; r < n; r += kRecWarps * 32) {
+            const size_t tok = ((size_t)b * T + t0 + r) * H + h;
+            sB[r] = beta[tok];
+            if (MODE == GDR_DECAY_SCALAR) sAl[r][0] = expf(g[tok]);
+        }
+        __syncthreads();
+        if (!active) continue;
+        for (int r = 0; r < n; ++r) {
+            float kk[NL], p = 0.f;
+#pragma unroll
+            for (int i = 0; i < NL; ++i) {
+                kk[i] = sK[r][lane + 32 * i];
+                if (MODE == GDR_DECAY_SCALAR) s[i] *= sAl[r][0];
+                if (MODE == GDR_DECAY_CHANNEL) s[i] *= sAl[r][lane + 32 * i];
+                p = fmaf(s[i], kk[i], p);
+            }
+            p = warp_sum(p);
+            const float d = sB[r] * (sV[r][warp] - p);
+            float a = 0.f;
+#pragma unroll
+            for (int i = 0; i < NL; ++i) {
+                s[i] = fmaf(d, kk[i], s[i]);
+                a = fmaf(s[i], sQ[r][lane + 32 * i], a);
+            }
+            a = warp_sum(a);
+            if (lane == 0) store_f32(o + (((size_t)b * T + t0 + r) * H + h) * dv + j, scale * a);
+        }
+    }
+    if (active && S_T != nullptr) {
+#pragma unroll
+        for (int i = 0; i < NL; ++i) S_T[(bh * dv + j) * DK + lane + 32 * i] = s[i];
+    }
+}
+
 template <typename Tin, typename Tout, int MODE, int DK>
 cudaError_t launch_typed(const ChunkProblem& p, cudaStream_t stream) {
+    if (p.T <= kRecMaxT) {
+        dim3 grid((p.dv + kRecWarps - 1) / kRecWarps, p.H, p.B);
+        recurrent_simt_kernel<Tin, Tout, MODE, DK><<<grid, kRecWarps * 32, 0, stream>>>(
+            static_cast<const Tin*>(p.q), static_cast<const Tin*>(p.k), static_cast<const Tin*>(p.v), p.g, p.beta,
+            p.S0, static_cast<Tout*>(p.o), p.S_T, p.T, p.H, p.dv, p.scale);
+        profile_after_launch(stream);
+        return cudaGetLastError();
+    }
     auto kern = chunk_simt_kernel<Tin, Tout, MODE, DK>;
     const size_t smem = SimtSmem<DK>::bytes;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -44,6 +44,16 @@ def test_chunk_small(mode, dtype, d, T, with_s0):
     check_chunk(x, mode, dtype, label=f"{mode}/{dtype}/d{d}/T{T}")
 
 
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("dtype,d", [("f32", 64), ("f32", 32), ("bf16", 64)])
+def test_chunk_cuda_core_chunk_form(mode, dtype, d):
+    """Past 256 tokens the CUDA-core path runs the chunk form (shorter sequences run the token
+    recurrence): several chunks and a ragged tail, with S0, against the oracle."""
+    seed = 5000 + 100 * MODES.index(mode) + d + (3 if dtype == "bf16" else 0)
+    x = make_chunk_inputs(1, 300, 2, d, d, mode, dtype, seed, s0_std=0.1)
+    check_chunk(x, mode, dtype, label=f"chunk form {mode}/{dtype}/d{d}")
+
+
 @pytest.mark.parametrize("mode", ["none", "scalar"])
 @pytest.mark.parametrize("B,H,T,plan", [
     (1, 1, 5000, "fused"),        # one head, 147 prep CTAs, 79 chunks through the 8-slot ring
