@@ -234,7 +234,8 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
 // in registers (lane holds columns lane + 32 i). Per token, with alpha = exp(g):
 //   s <- s * alpha;  p = s . k;  s <- s + beta (v_j - p) k;  o_j = scale (s . q)
 // (the delta rule of "Linear Attention & DeltaNet" with the gate of "linear attention and its
-// gated descendants"). Tokens are staged in shared memory kRecTB at a time.
+// gated descendants"). Tokens are staged in shared memory kRecTB at a time; the next block's
+// loads are in flight while the current one is computed.
 constexpr int kRecWarps = 8;   // state rows per CTA
 constexpr int kRecTB = 16;     // tokens per staged block
 constexpr int kRecMaxT = 256;  // sequences up to this length run the recurrence
@@ -250,58 +251,94 @@ __global__ void __launch_bounds__(kRecWarps * 32)
 recurrent_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                       const float* __restrict__ g, const float* __restrict__ beta, const float* S0,
                       Tout* __restrict__ o, float* S_T, int T, int H, int dv, float scale) {
+    constexpr int NT = kRecWarps * 32;
     constexpr int NL = DK / 32;                                  // state columns per lane
     constexpr int NA = MODE == GDR_DECAY_CHANNEL ? DK : 1;       // decay factors per token
+    constexpr int KPT = kRecTB * DK / NT;                        // staged k (and q) values per thread
+    static_assert(kRecTB * DK % NT == 0 && kRecTB * kRecWarps <= NT && kRecTB <= NT, "staging split");
     __shared__ float sK[kRecTB][DK], sQ[kRecTB][DK], sAl[kRecTB][NA], sV[kRecTB][kRecWarps], sB[kRecTB];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int j0 = blockIdx.x * kRecWarps, j = j0 + warp;       // this warp's state row
     const int h = blockIdx.y, b = blockIdx.z;
     const size_t bh = (size_t)b * H + h;
     const bool active = j < dv;
+    auto tok_of = [&](int t) { return ((size_t)b * T + t) * H + h; };
+
+    // one block's inputs, held in registers between its load and its store into shared memory:
+    // thread tid holds k, q (and the channel gate's g) at flat index tid + NT m of the block, the
+    // value of (token tid / kRecWarps, row j0 + tid % kRecWarps), and beta (and the scalar g) of
+    // token tid
+    float rk[KPT], rq[KPT], rg[KPT], rv = 0.f, rb = 0.f, rs = 0.f;
+    auto load_block = [&](int t0) {
+        const int n = min(kRecTB, T - t0);
+#pragma unroll
+        for (int m = 0; m < KPT; ++m) {
+            const int idx = tid + NT * m, r = idx / DK, c = idx % DK;
+            rk[m] = rq[m] = rg[m] = 0.f;
+            if (r < n) {
+                const size_t tok = tok_of(t0 + r);
+                rk[m] = load_f32(k + tok * DK + c);
+                rq[m] = load_f32(q + tok * DK + c);
+                if (MODE == GDR_DECAY_CHANNEL) rg[m] = g[tok * DK + c];
+            }
+        }
+        const int rr = tid / kRecWarps, w = tid % kRecWarps;
+        rv = (rr < n && j0 + w < dv) ? load_f32(v + tok_of(t0 + rr) * dv + j0 + w) : 0.f;
+        if (tid < n) {
+            rb = beta[tok_of(t0 + tid)];
+            if (MODE == GDR_DECAY_SCALAR) rs = g[tok_of(t0 + tid)];
+        }
+    };
+    auto store_block = [&]() {
+#pragma unroll
+        for (int m = 0; m < KPT; ++m) {
+            const int idx = tid + NT * m, r = idx / DK, c = idx % DK;
+            sK[r][c] = rk[m];
+            sQ[r][c] = rq[m];
+            if (MODE == GDR_DECAY_CHANNEL) sAl[r][c] = expf(rg[m]);
+        }
+        if (tid < kRecTB * kRecWarps) sV[tid / kRecWarps][tid % kRecWarps] = rv;
+        if (tid < kRecTB) {
+            sB[tid] = rb;
+            if (MODE == GDR_DECAY_SCALAR) sAl[tid][0] = expf(rs);
+        }
+    };
+
     float s[NL];
 #pragma unroll
     for (int i = 0; i < NL; ++i) s[i] = (active && S0 != nullptr) ? S0[(bh * dv + j) * DK + lane + 32 * i] : 0.f;
+    load_block(0);
+    store_block();
+    __syncthreads();
     for (int t0 = 0; t0 < T; t0 += kRecTB) {
         const int n = min(kRecTB, T - t0);
-        __syncthreads();  // every warp is done with the previous block
-        for (int idx = tid; idx < n * DK; idx += kRecWarps * 32) {
-            const int r = idx / DK, c = idx % DK;
-            const size_t tok = ((size_t)b * T + t0 + r) * H + h;
-            sK[r][c] = load_f32(k + tok * DK + c);
-            sQ[r][c] = load_f32(q + tok * DK + c);
-            if (MODE == GDR_DECAY_CHANNEL) sAl[r][c] = expf(g[tok * DK + c]);
-        }
-        for (int idx = tid; idx < n * kRecWarps; idx += kRecWarps * 32) {
-            const int r = idx / kRecWarps, w = idx % kRecWarps;
-            const size_t tok = ((size_t)b * T + t0 + r) * H + h;
-            sV[r][w] = (j0 + w < dv) ? load_f32(v + tok * dv + j0 + w) : 0.f;
-        }
-        for (int r = tid; r < n; r += kRecWarps * 32) {
-            const size_t tok = ((size_t)b * T + t0 + r) * H + h;
-            sB[r] = beta[tok];
-            if (MODE == GDR_DECAY_SCALAR) sAl[r][0] = expf(g[tok]);
-        }
-        __syncthreads();
-        if (!active) continue;
-        for (int r = 0; r < n; ++r) {
-            float kk[NL], p = 0.f;
+        if (t0 + kRecTB < T) load_block(t0 + kRecTB);  // in flight while this block is computed
+        if (active) {
+            for (int r = 0; r < n; ++r) {
+                float kk[NL], p = 0.f;
 #pragma unroll
-            for (int i = 0; i < NL; ++i) {
-                kk[i] = sK[r][lane + 32 * i];
-                if (MODE == GDR_DECAY_SCALAR) s[i] *= sAl[r][0];
-                if (MODE == GDR_DECAY_CHANNEL) s[i] *= sAl[r][lane + 32 * i];
-                p = fmaf(s[i], kk[i], p);
-            }
-            p = warp_sum(p);
-            const float d = sB[r] * (sV[r][warp] - p);
-            float a = 0.f;
+                for (int i = 0; i < NL; ++i) {
+                    kk[i] = sK[r][lane + 32 * i];
+                    if (MODE == GDR_DECAY_SCALAR) s[i] *= sAl[r][0];
+                    if (MODE == GDR_DECAY_CHANNEL) s[i] *= sAl[r][lane + 32 * i];
+                    p = fmaf(s[i], kk[i], p);
+                }
+                p = warp_sum(p);
+                const float d = sB[r] * (sV[r][warp] - p);
+                float a = 0.f;
 #pragma unroll
-            for (int i = 0; i < NL; ++i) {
-                s[i] = fmaf(d, kk[i], s[i]);
-                a = fmaf(s[i], sQ[r][lane + 32 * i], a);
+                for (int i = 0; i < NL; ++i) {
+                    s[i] = fmaf(d, kk[i], s[i]);
+                    a = fmaf(s[i], sQ[r][lane + 32 * i], a);
+                }
+                a = warp_sum(a);
+                if (lane == 0) store_f32(o + tok_of(t0 + r) * dv + j, scale * a);
             }
-            a = warp_sum(a);
-            if (lane == 0) store_f32(o + (((size_t)b * T + t0 + r) * H + h) * dv + j, scale * a);
+        }
+        if (t0 + kRecTB < T) {
+            __syncthreads();  // every warp is done with this block
+            store_block();
+            __syncthreads();
         }
     }
     if (active && S_T != nullptr) {
