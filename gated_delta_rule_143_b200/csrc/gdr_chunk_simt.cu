@@ -314,26 +314,37 @@ recurrent_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, cons
         const int n = min(kRecTB, T - t0);
         if (t0 + kRecTB < T) load_block(t0 + kRecTB);  // in flight while this block is computed
         if (active) {
-            for (int r = 0; r < n; ++r) {
-                float kk[NL], p = 0.f;
+            // the state's chain carries one reduction per token (s . k); the lane partials of the
+            // outputs s . q are reduced after the block, 16 independent reductions at once
+            float ap[kRecTB];
 #pragma unroll
-                for (int i = 0; i < NL; ++i) {
-                    kk[i] = sK[r][lane + 32 * i];
-                    if (MODE == GDR_DECAY_SCALAR) s[i] *= sAl[r][0];
-                    if (MODE == GDR_DECAY_CHANNEL) s[i] *= sAl[r][lane + 32 * i];
-                    p = fmaf(s[i], kk[i], p);
-                }
-                p = warp_sum(p);
-                const float d = sB[r] * (sV[r][warp] - p);
-                float a = 0.f;
+            for (int r = 0; r < kRecTB; ++r) {
+                ap[r] = 0.f;
+                if (r < n) {
+                    float kk[NL], p = 0.f;
 #pragma unroll
-                for (int i = 0; i < NL; ++i) {
-                    s[i] = fmaf(d, kk[i], s[i]);
-                    a = fmaf(s[i], sQ[r][lane + 32 * i], a);
+                    for (int i = 0; i < NL; ++i) {
+                        kk[i] = sK[r][lane + 32 * i];
+                        if (MODE == GDR_DECAY_SCALAR) s[i] *= sAl[r][0];
+                        if (MODE == GDR_DECAY_CHANNEL) s[i] *= sAl[r][lane + 32 * i];
+                        p = fmaf(s[i], kk[i], p);
+                    }
+                    p = warp_sum(p);
+                    const float d = sB[r] * (sV[r][warp] - p);
+#pragma unroll
+                    for (int i = 0; i < NL; ++i) {
+                        s[i] = fmaf(d, kk[i], s[i]);
+                        ap[r] = fmaf(s[i], sQ[r][lane + 32 * i], ap[r]);
+                    }
                 }
-                a = warp_sum(a);
-                if (lane == 0) store_f32(o + tok_of(t0 + r) * dv + j, scale * a);
             }
+#pragma unroll
+            for (int r = 0; r < kRecTB; ++r) ap[r] = warp_sum(ap[r]);
+            float mine = 0.f;  // lane r writes the output of token r
+#pragma unroll
+            for (int r = 0; r < kRecTB; ++r)
+                if (lane == r) mine = ap[r];
+            if (lane < n) store_f32(o + tok_of(t0 + lane) * dv + j, scale * mine);
         }
         if (t0 + kRecTB < T) {
             __syncthreads();  // every warp is done with this block
