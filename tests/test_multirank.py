@@ -85,3 +85,16 @@ def test_kernel_code_digest_ignores_comments_only():
     c = "int f(int x) {\n    return 3 * x;\n}\n"
     assert bench.kernel_code_digest(a) == bench.kernel_code_digest(b)
     assert bench.kernel_code_digest(a) != bench.kernel_code_digest(c)
+
+
+@pytest.mark.parametrize("plan", ["fused", "prep_fused", "two_pass", "cuda_core"])
+def test_kernel_bytes_split_the_step_bytes(plan):
+    """The roofline's per-kernel algorithmic bytes add up to the whole step's, on every plan."""
+    import bench
+    from gated_delta_rule_143_b200.inputs import CHUNK_WORKLOADS
+    for w in CHUNK_WORKLOADS.values():
+        nc = -(-w.T // w.chunk)
+        c1 = (nc + 1) // 2 if plan == "prep_fused" else 0  # some chunks pre-computed, some not
+        parts = bench.kernel_bytes(w, plan, c1)
+        assert sum(b for _, b in parts) == bench.chunk_bytes(w)
+        assert all(b > 0 for _, b in parts)
