@@ -45,17 +45,22 @@ def chunk_flops_per_token_head(C, dk, dv):
     return 2 * (C * (3 * dk + 2 * dv) + 3 * dk * dv)
 
 
-OUT_BYTES = 4  # o is written in fp32 (the accumulation precision)
-
-
 def chunk_bytes(w):
-    """Algorithmic HBM bytes of one forward: q, k, v (input dtype) read once, o (fp32)
-    written once, beta and g read once, S_T written once (S0 is null for these workloads)."""
+    """Algorithmic HBM bytes of one forward: q, k, v read once and o written once, all in the input
+    dtype; beta and g read once; S_T written once (S0 is null for these workloads). 1032 bytes per
+    token-head for bf16 Gated DeltaNet at d = 128, plus 64 KiB of S_T per (b, h)."""
     eb = 2 if w.dtype == "bf16" else 4
     th = w.B * w.T * w.H
     g = 0 if w.mode == "none" else (4 if w.mode == "scalar" else 4 * w.dk)
-    per_th = eb * (2 * w.dk + w.dv) + OUT_BYTES * w.dv + 4 + g
+    per_th = eb * (2 * w.dk + w.dv) + eb * w.dv + 4 + g
     return th * per_th + w.B * w.H * w.dv * w.dk * 4
+
+
+def o_fp32_extra_bytes(w):
+    """Bytes the default fp32 output writes beyond an output in the input dtype (implementation
+    traffic of the precision choice, not algorithmic)."""
+    eb = 2 if w.dtype == "bf16" else 4
+    return w.B * w.T * w.H * w.dv * (4 - eb)
 
 
 def kernel_bytes(w, plan, c1):
@@ -68,7 +73,7 @@ def kernel_bytes(w, plan, c1):
     th = w.B * w.T * w.H
     g = 0 if w.mode == "none" else (4 if w.mode == "scalar" else 4 * w.dk)
     inputs = th * (eb * (2 * w.dk + w.dv) + 4 + g)
-    outputs = th * OUT_BYTES * w.dv + w.B * w.H * w.dv * w.dk * 4
+    outputs = th * eb * w.dv + w.B * w.H * w.dv * w.dk * 4
     if plan == "two_pass":
         return [("chunk_prep", inputs), ("chunk_state", outputs)]
     if plan == "prep_fused":
@@ -79,11 +84,12 @@ def kernel_bytes(w, plan, c1):
 
 
 def decode_bytes(w):
-    """S read and written once (fp32), q, k, v read, o (fp32) written, beta and g read."""
+    """S read and written once (fp32); q, k, v read and o written in the input dtype; beta and g
+    read (2 * 4 * d_k * d_v + 1032 bytes per head-step for bf16 Gated DeltaNet at d = 128)."""
     eb = 2 if w.dtype == "bf16" else 4
     nh = w.B * w.H
     g = 0 if w.mode == "none" else (4 if w.mode == "scalar" else 4 * w.dk)
-    return nh * (2 * 4 * w.dk * w.dv + eb * (2 * w.dk + w.dv) + OUT_BYTES * w.dv + 4 + g)
+    return nh * (2 * 4 * w.dk * w.dv + eb * (2 * w.dk + w.dv) + eb * w.dv + 4 + g)
 
 
 def load_peaks():
@@ -96,6 +102,82 @@ def load_peaks():
 
 
 # ------------------------------------------------------------------ clocks --
+class NvmlClockSampler:
+    """SM clock, power and clock-event reasons read through NVML every ~0.5 ms on a host thread, from
+    start() to stop(); summary() keeps the samples taken between mark_begin() and mark_end() (the
+    timed region), so that a region of a few milliseconds still has samples. Reads only."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown"}
+
+    def __init__(self, dev_index: int):
+        import pynvml
+        import threading
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        uuid = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(dev_index).uuid)
+        except Exception:
+            pass
+        h = None
+        if uuid:
+            try:
+                h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                h = None
+        if h is None:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[dev_index]) if vis and vis.split(",")[dev_index].strip().isdigit() else dev_index
+            h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+        self.h = h
+        self.samples = []
+        self.t0 = self.t1 = None
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self.nv
+        getr = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        try:
+            mx = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+        except Exception:
+            mx = None
+        pw, k = 0.0, 0
+        while not self._stop.is_set():
+            try:
+                t = time.perf_counter()
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = getr(self.h)
+                if k % 8 == 0:
+                    pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                k += 1
+                self.samples.append((t, sm, mx, rs, pw))
+            except Exception:
+                pass
+            time.sleep(0.0005)
+
+    def start(self):
+        self._thread.start()
+        time.sleep(0.01)
+
+    def mark_begin(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
+
+    def stop(self):
+        self._stop.set()
+        self._thread.join(timeout=2)
+        rows = [r for r in self.samples if self.t0 is not None and self.t0 <= r[0] <= (self.t1 or r[0])]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": "nvml"}
+        reasons = sorted({name for r in rows for bit, name in self.REASONS.items() if r[3] & bit})
+        return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": max((r[2] or 0) for r in rows) or None,
+                "reasons": reasons, "samples": len(rows), "power_w_max": round(max(r[4] for r in rows), 1),
+                "source": "nvml, every ~0.5 ms during the timed region"}
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled during the timed region."""
 
@@ -279,13 +361,26 @@ def run_ours(args):
         gdr.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], mode=w.mode, chunk=w.chunk,
                       out=o, state_out=st, workspace=ws)
 
-    clocks = ClockSampler(smi_id(dev, local))
+    try:
+        clocks = NvmlClockSampler(local)
+    except Exception:
+        clocks = None
+    if clocks is not None:
+        clocks.start()  # sampling from the start of the warm-up, kept for the timed region only
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    clocks.start()
+    if clocks is None:
+        smi = ClockSampler(smi_id(dev, local))
+        smi.start()
+    else:
+        clocks.mark_begin()
     ms = time_device(step, args.steps, 0, world, stream)
-    clk = clocks.stop()
+    if clocks is None:
+        clk = smi.stop()
+    else:
+        clocks.mark_end()
+        clk = clocks.stop()
     gdr.sync_status()
     ms = max_over_ranks(ms, world)
     ms_step = ms / args.steps
@@ -319,6 +414,10 @@ def run_ours(args):
                          "algorithmic_bytes": nbytes,
                          "roofline_us": round(max(nbytes / (peaks["hbm_gbs"] * 1e9),
                                                   flops / (peaks["bf16_tflops"] * 1e12)) * 1e6, 2)},
+                "bytes_note": "algorithmic bytes count q, k, v and o in the input dtype (bf16); the default "
+                              "call writes o in fp32, o_fp32_extra_bytes_per_step more (see o_bf16 for the "
+                              "bf16-output call)",
+                "o_fp32_extra_bytes_per_step": o_fp32_extra_bytes(w),
                 "tensor_view": {"flops_per_step": flops,
                                 "achieved_tflops": round(flops / (ms_step * 1e-3) / 1e12, 1),
                                 "peak_tflops": peaks["bf16_tflops"],
@@ -332,6 +431,23 @@ def run_ours(args):
                               "roofline_frac": round(nbytes / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                               "kernels": [(k["kernel"], k["launch_us"]) for k in kernels]}))
         return
+
+    # the same forward with o in the input dtype (bf16): the call shape of the C ABI's definition
+    o16 = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.bfloat16, device=dev)
+    ws16_n = gdr.workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.chunk, w.mode, torch.bfloat16, torch.bfloat16)
+    ws16 = ws if (ws is not None and ws16_n <= ws.numel()) else (
+        torch.empty(max(ws16_n, 1), dtype=torch.uint8, device=dev) if ws16_n else None)
+
+    def step16(i=0):
+        x = sets[i & 1]
+        gdr.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], mode=w.mode, chunk=w.chunk,
+                      out=o16, state_out=st, workspace=ws16)
+
+    n16 = max(3, min(args.steps, 200))
+    ms16 = max_over_ranks(time_device(step16, n16, args.warmup, world, stream), world) / n16
+    o_bf16 = {"ms_per_step": round(ms16, 5), "tokens_per_s": round(job_throughput(tokens, ms16, world), 1),
+              "steps": n16, "roofline_frac": round(nbytes / (ms16 * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+              "algorithmic_bytes": nbytes}
 
     # end to end: pinned host inputs -> device -> kernels -> host outputs, every step
     hx = {k: (None if t is None else t.cpu().pin_memory()) for k, t in sets[0].items()}
@@ -348,6 +464,7 @@ def run_ours(args):
     d2h = h_o.numel() * h_o.element_size() + h_s.numel() * h_s.element_size()
 
     dec = bench_decode(args, dev, peaks, world)
+    others = bench_workloads(args, dev, peaks) if world == 1 else None
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -362,8 +479,11 @@ def run_ours(args):
         "gpu_launches": kernels_per_step * args.steps,
         "roofline": roofline,
         "clocks": clk,
+        "o_bf16": o_bf16,
         "decode": dec,
     }
+    if others is not None:
+        line["extra"] = {"workloads": others}
     if rank == 0 and world == 1:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
@@ -435,6 +555,40 @@ def bench_decode(args, dev, peaks, world):
             "l2": "state 537 MB > L2, streamed once per step"}
 
 
+def bench_workloads(args, dev, peaks):
+    """Every named chunked-forward workload, forward only (default call: fp32 o), timed with CUDA
+    events over a few steps after a warm-up: ms per step, tokens/s, the plan, and the fraction of
+    the roofline max(bytes / HBM peak, flops / bf16 peak) with bytes and flops counted as above."""
+    import gated_delta_rule_143_b200 as gdr
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+    for name, w in CHUNK_WORKLOADS.items():
+        x = {k: (None if t is None else t.to(dev)) for k, t in workload_inputs(w).items()}
+        dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=dev)
+        st = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
+        nws = gdr.workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.chunk, w.mode, dt, torch.float32)
+        ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=dev) if nws else None
+
+        def step(i=0):
+            gdr.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], mode=w.mode, chunk=w.chunk,
+                          out=o, state_out=st, workspace=ws)
+
+        n = 50 if w.B * w.T * w.H <= (1 << 20) else 10
+        ms = time_device(step, n, 3, 1, stream) / n
+        nbytes = chunk_bytes(w)
+        flops = chunk_flops_per_token_head(w.chunk, w.dk, w.dv) * w.B * w.T * w.H
+        roof_us = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)) * 1e6
+        plan, c1 = gdr.chunk_fwd_plan(w.B, w.T, w.H, w.dk, w.dv, w.chunk, w.mode, dt, torch.float32)
+        out[name] = {"ms_per_step": round(ms, 5), "tokens_per_s": round(w.B * w.T / (ms * 1e-3), 1), "steps": n,
+                     "plan": plan, "precomputed_chunks_per_head": c1, "roofline_us": round(roof_us, 2),
+                     "roofline_frac": round(roof_us / (ms * 1e3), 4), "algorithmic_bytes": nbytes,
+                     "flops": flops}
+        del x, o, st, ws
+    gdr.sync_status()
+    return out
+
+
 # ------------------------------------------------------------------- oracle --
 def _oracle_sample(w, b_count=1):
     """A bounded sample of the workload for the CPU oracle: the first b_count sequences
@@ -494,8 +648,9 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)  # about 0.25 s timed: a dozen clock samples
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--only", choices=("all", "fwd"), default="all",
-                    help="fwd: time the forward only (no e2e, decode or CPU baseline), for profiling runs")
+    ap.add_argument("--only", choices=("all", "fwd", "decode"), default="all",
+                    help="fwd: time the forward only (no e2e, decode or CPU baseline); decode: the decode step "
+                         "only; both for profiling runs")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size (profiling runs)")
     ap.add_argument("--seq", type=int, default=0, help="override the workload's sequence length (profiling runs)")
     ap.add_argument("--workload", choices=sorted(CHUNK_WORKLOADS), default=WORKLOAD,
@@ -509,6 +664,11 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.only == "decode":
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        peaks, _ = load_peaks()
+        print(json.dumps({"metric": "decode step", "decode": bench_decode(args, dev, peaks, 1)}))
     else:
         run_ours(args)
 

@@ -84,6 +84,25 @@ def test_chunk_unequal_head_dims(mode):
     check_chunk(x, mode, "f32")
 
 
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("dk,dv", [(64, 32), (32, 128)])
+@pytest.mark.parametrize("T", [200, 300])
+def test_chunk_cuda_core_unequal_head_dims(mode, dk, dv, T):
+    """d_k != d_v in both directions on the fp32 CUDA-core path: T = 200 runs the token recurrence
+    (a ragged last block of 16 tokens), T = 300 the chunk form (ragged last chunk), both with S0."""
+    seed = 6000 + 10 * MODES.index(mode) + dk + dv + T
+    x = make_chunk_inputs(1, T, 2, dk, dv, mode, "f32", seed, s0_std=0.1)
+    check_chunk(x, mode, "f32", label=f"{mode}/dk{dk}/dv{dv}/T{T}")
+
+
+def test_chunk_cuda_core_chunk_form_gdn_small_workload_shape():
+    """The chunk form at the small Gated DeltaNet workload's shape (fp32, B = 1, H = 2, d = 64) with a
+    sequence long enough to leave the token recurrence (T = 320, five chunks): the workload itself
+    (T = 256) is served by the recurrence, so this keeps the fp32 chunk form covered at that shape."""
+    x = make_chunk_inputs(1, 320, 2, 64, 64, "scalar", "f32", 6100)
+    check_chunk(x, "scalar", "f32", label="gdn f32 B1 H2 d64 T320")
+
+
 @pytest.mark.parametrize("name", list(CHUNK_WORKLOADS))
 def test_chunk_full_workload(name):
     """Every named workload at full size, whole output against the oracle."""
