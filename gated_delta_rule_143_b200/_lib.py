@@ -36,6 +36,7 @@ SIGNATURES = {
     "gdr_chunk_fwd_host_staging_bytes": (_sz, [_i] * 9),
     "gdr_profile_next_call": (_i, [_vp, _i]),
     "gdr_sync_status": (_i, [_vp]),
+    "gdr_selftest_bounded_wait": (_i, [ctypes.c_uint, _vp, _vp]),
     "gdr_last_error": (ctypes.c_char_p, []),
     "gdr_version": (_i, []),
 }

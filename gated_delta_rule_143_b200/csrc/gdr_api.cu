@@ -271,9 +271,26 @@ int gdr_sync_status(void* stream) {
     if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "reading the status word: %s", cudaGetErrorString(err));
     if (h == GDR_ERR_TIMEOUT) return fail(GDR_ERR_TIMEOUT, "a kernel's bounded wait expired; its outputs are invalid");
     if (h == GDR_ERR_RANGE)
-        return fail(GDR_ERR_RANGE, "a decay factor left the fp16 operand range (channel gate spread within a chunk)");
+        return fail(GDR_ERR_RANGE, "a value left the range a kernel supports");
     if (h != 0) return fail(h, "device reported status %d", h);
     return ok();
+}
+
+int gdr_selftest_bounded_wait(unsigned limit_us, unsigned long long* elapsed_ns, void* stream) {
+    if (limit_us == 0 || limit_us > 1000000u)
+        return fail(GDR_ERR_INVALID_ARG, "limit_us = %u (1 .. 1000000)", limit_us);
+    int* status = nullptr;
+    int major = 0;
+    if (int rc = device_setup(&status, &major)) return rc;
+    if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
+    const int before = gdr_sync_status(stream);  // an idle stream and a clear status word to start from
+    if (before == GDR_ERR_CUDA) return before;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t err = launch_bounded_wait_selftest(status, (uint64_t)limit_us * 1000ull, s);
+    if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "self-test launch: %s", cudaGetErrorString(err));
+    const int rc = gdr_sync_status(stream);
+    if (elapsed_ns != nullptr && read_bounded_wait_selftest_elapsed(elapsed_ns) != cudaSuccess) *elapsed_ns = 0;
+    return rc;
 }
 
 }  // extern "C"
@@ -375,12 +392,16 @@ struct HostStreams {
     cudaEvent_t start = nullptr, in_ready[2] = {}, computed[2] = {}, out_done[2] = {};
 };
 HostStreams g_host[kMaxDevices];
+// Held by a gdr_chunk_fwd_host call while it enqueues: the copy streams and events above are
+// shared by every call on the device, so two threads must not interleave their records and waits.
+std::mutex g_host_enqueue[kMaxDevices];
 
-int host_streams(HostStreams** out) {
+int host_streams(HostStreams** out, int* device) {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
     if (dev < 0 || dev >= kMaxDevices) return fail(GDR_ERR_DEVICE, "device ordinal %d out of range", dev);
+    *device = dev;
     std::lock_guard<std::mutex> lock(g_dev_mutex);
     HostStreams& hs = g_host[dev];
     if (hs.h2d == nullptr) {
@@ -437,7 +458,10 @@ extern "C" int gdr_chunk_fwd_host(const void* q, const void* k, const void* v, c
     if (int rc = device_setup(&status, &major)) return rc;
     if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
     HostStreams* hs = nullptr;
-    if (int rc = host_streams(&hs)) return rc;
+    int hdev = 0;
+    if (int rc = host_streams(&hs, &hdev)) return rc;
+    // the whole enqueue sequence below uses the device's shared copy streams and events
+    std::lock_guard<std::mutex> enqueue_lock(g_host_enqueue[hdev]);
 
     const SeqBytes sb = seq_bytes(T, H, dk, dv, mode, dtype, o_dtype);
     cudaStream_t s = static_cast<cudaStream_t>(stream);

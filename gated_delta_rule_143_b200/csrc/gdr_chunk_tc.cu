@@ -28,10 +28,13 @@
 //
 // Decay handling: the scalar gate's Gram products are scaled elementwise by exp(Gamma_r - Gamma_i)
 // <= 1 (safe for any g <= 0), computed as exp(Gamma_r) * exp(-Gamma_i) while every |Gamma| of the
-// chunk stays within 120 log2 units (both factors normal fp32) and directly beyond that. The channel gate's factors are folded into the operands around a
-// mid-chunk reference: (K e^{Gamma - Gamma_ref})(K e^{Gamma_ref - Gamma})^T; a factor beyond the
-// fp16 range (a within-chunk spread of the cumulative log-decay above about 22 on one channel) is
-// reported as GDR_ERR_RANGE through the status word.
+// chunk stays within 120 log2 units (both factors normal fp32) and directly beyond that. The channel
+// gate's factors are folded into the Gram operands around a mid-chunk reference,
+// (K e^{Gamma - Gamma_ref})(K e^{Gamma_ref - Gamma})^T, for every key channel whose cumulative
+// log-decay varies by at most kStrongSpread log2 units inside the chunk (factors within 2^14, far
+// inside fp16); the other ("strong") channels are left out of the tensor-core product and their
+// terms k_r,d k_i,d 2^(Gamma_r,d - Gamma_i,d) (each factor <= 1) are added to the Gram on the CUDA
+// cores, in fp32, from a second copy of the bf16 tiles. Any g <= 0 is computed exactly.
 //
 // Operands are fp16, not bf16: with bf16 operands the rounding of the intermediate factors alone
 // exceeded the 2e-2 * rms(o) parity bar; fp16 holds the bf16 inputs exactly at these ranges and
@@ -48,7 +51,6 @@ using namespace sm100;
 constexpr int kC = 64;    // chunk length
 constexpr int kD = 128;   // d_k = d_v
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kF16Max = 65504.f;
 
 // ------------------------------------------------------------------ hand-off block --
 // Per-chunk block in the workspace (byte offsets). Images are laid out exactly as the state
@@ -79,7 +81,10 @@ constexpr uint32_t kPGam = kPBeta + 256;             // Gamma * log2(e): [64] or
 constexpr uint32_t kPInvE = kPGam + 256;             // scalar gate: 2^-Gamma [64], then a "factorable" flag
 constexpr uint32_t kPKB = (kPGam + 32768 + 1023) & ~1023u;  // channel: K'' fp16 K-major 64 x 128
 constexpr uint32_t kPrepBytesScalar = (kPInvE + 512 + 1023) & ~1023u;
-constexpr uint32_t kPrepBytesChannel = kPKB + 16384;
+constexpr uint32_t kPKQ2 = kPKB + 16384;  // channel: second copy of the bf16 [K; Q] tile (TMA), 32 KiB
+constexpr uint32_t kPStrong = kPKQ2 + 32768;  // channel: int flags [128], then per-warp lists [4][32] + counts [4]
+constexpr uint32_t kPrepBytesChannel = kPStrong + 1024 + 1024;
+constexpr float kStrongSpread = 14.f;  // log2 units: a larger within-chunk spread makes a channel "strong"
 
 // TMEM columns of one prep pipeline
 constexpr uint32_t kTG = 0, kTW = 64, kTU = 192, kPrepTmemCols = 256;
@@ -270,7 +275,14 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
     //         cumulative log-decay (log2 units; rows past the tail repeat Gamma_{n-1}) meanwhile
     if (lt == 0) {
         bulk_wait_read<0>();  // the previous task's W / U^T bulk stores have read the K / V tiles
-        mbar_arrive_expect_tx(barT, 6 * 8192);
+        mbar_arrive_expect_tx(barT, (MODE == GDR_DECAY_CHANNEL ? 10 : 6) * 8192);
+        if (MODE == GDR_DECAY_CHANNEL) {  // the copy the strong channels and K*gamma are computed from
+            uint8_t* sKQ2 = sm + kPKQ2;
+            tma_load_4d(sKQ2, mk, 0, h, c0, b, barT);
+            tma_load_4d(sKQ2 + 16384, mk, 64, h, c0, b, barT);
+            tma_load_4d(sKQ2 + 8192, mq, 0, h, c0, b, barT);
+            tma_load_4d(sKQ2 + 24576, mq, 64, h, c0, b, barT);
+        }
         tma_load_4d(sKQ, mk, 0, h, c0, b, barT);
         tma_load_4d(sKQ + 16384, mk, 64, h, c0, b, barT);
         tma_load_4d(sKQ + 8192, mq, 0, h, c0, b, barT);
@@ -310,12 +322,22 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
             float gv[kC];
 #pragma unroll
             for (int r = 0; r < kC; ++r) gv[r] = (r < n) ? P.g[(tok0 + (size_t)r * H) * kD + lt] : 0.f;
-            float acc = 0.f;
+            float acc = 0.f, lo = 0.f, hi = 0.f;
 #pragma unroll
             for (int r = 0; r < kC; ++r) {
                 acc = fmaf(gv[r], kLog2e, acc);
                 sGam[r * kD + lt] = acc;
+                lo = fminf(lo, acc);
+                hi = fmaxf(hi, acc);
             }
+            // a channel whose cumulative log-decay spreads wider than kStrongSpread inside the chunk
+            // stays out of the factored tensor-core product (its factors could leave fp16's range)
+            const bool strong = hi - lo > kStrongSpread;
+            int* sStrong = reinterpret_cast<int*>(sm + kPStrong);
+            sStrong[lt] = strong ? 1 : 0;
+            const unsigned m = __ballot_sync(0xffffffffu, strong);
+            if (strong) sStrong[128 + 32 * lw + __popc(m & ((1u << lane) - 1u))] = lt;
+            if (lane == 0) sStrong[256 + lw] = __popc(m);
         }
     }
     named_bar(ps.bar_id, kPrepThreads);
@@ -335,7 +357,6 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
 
     // ---- 2. Q*gamma and K*gamma_C/gamma hand-off images; channel gate: decay-factored Gram operands
     const int ref = (n - 1) >> 1;
-    bool range_bad = false;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int task = lt + kPrepThreads * j;
@@ -365,8 +386,9 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
                 const float G = sGam[r * kD + col0 + e];
                 const float Gr = sGam[ref * kD + col0 + e];
                 const float GC = sGam[(kC - 1) * kD + col0 + e];
-                const float up = fast_exp2(G - Gr), dn = fast_exp2(Gr - G);
-                if (!(up < kF16Max && dn < kF16Max)) range_bad = true;
+                // factors within 2^kStrongSpread; a strong channel's terms are added on the CUDA cores
+                const bool weak = reinterpret_cast<const int*>(sm + kPStrong)[col0 + e] == 0;
+                const float up = weak ? fast_exp2(G - Gr) : 0.f, dn = weak ? fast_exp2(Gr - G) : 0.f;
                 qg[e] = qx[e] * fast_exp2(G);
                 kt[e] = kx[e] * fast_exp2(GC - G);
                 ka[e] = kx[e] * up;
@@ -380,7 +402,6 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
         st16(out + kOffWQ + oqr, pack8h(qg));
         st16(out + kOffKT + mnmajor_off(r, col0, 64), pack8h(kt));
     }
-    if (MODE == GDR_DECAY_CHANNEL && range_bad) report_status(P.status, GDR_ERR_RANGE);
     if (lt < kD) {
         float gc = 1.f;
         if (MODE == GDR_DECAY_SCALAR) gc = fast_exp2(sGam[kC - 1]);
@@ -426,6 +447,32 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
         }
         const float br = sBeta[rr];
         tmem_ld_wait();
+        if (MODE == GDR_DECAY_CHANNEL) {
+            // the strong channels' terms, left out of the tensor-core product: k_r,d k_i,d
+            // 2^(Gamma_r,d - Gamma_i,d) (or q_r,d ...) from the bf16 copy of the tiles, fp32
+            const int* sStrong = reinterpret_cast<const int*>(sm + kPStrong);
+            const uint8_t* sKQ2 = sm + kPKQ2;
+            const int row = q * 32 + lane;  // tile row: K rows 0-63, Q rows 64-127
+#pragma unroll 1
+            for (int w4 = 0; w4 < 4; ++w4) {
+                const int cnt = sStrong[256 + w4];
+#pragma unroll 1
+                for (int kk = 0; kk < cnt; ++kk) {
+                    const int dch = sStrong[128 + 32 * w4 + kk];
+                    const float a = __bfloat162float(
+                        *reinterpret_cast<const __nv_bfloat16*>(sKQ2 + kmajor_off(row, dch, 128)));
+                    const float Gr = sGam[rr * kD + dch];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int i = 32 * hf + e;
+                        const float ki = __bfloat162float(
+                            *reinterpret_cast<const __nv_bfloat16*>(sKQ2 + kmajor_off(i, dch, 128)));
+                        const float f = (i <= rr) ? fast_exp2(Gr - sGam[i * kD + dch]) : 0.f;
+                        x[e] = fmaf(a * ki, f, x[e]);
+                    }
+                }
+            }
+        }
         if (q < 2) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
@@ -464,9 +511,10 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
             uint8_t* p = isv ? sV + kmajor_off(r, col0, 64) : sKQ + kmajor_off(r, col0, 128);
             float x[8];
             if (!isv && MODE == GDR_DECAY_CHANNEL) {
-                unpack8h(ld16(p), x);  // K' = K e^{Gamma - Gamma_ref}: times e^{Gamma_ref} gives K*gamma
+                // K*gamma straight from the bf16 copy (every factor <= 1, any decay)
+                unpack8bf(ld16(sm + kPKQ2 + kmajor_off(r, col0, 128)), x);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] *= fast_exp2(sGam[ref * kD + col0 + e]);
+                for (int e = 0; e < 8; ++e) x[e] *= fast_exp2(sGam[r * kD + col0 + e]);
             } else {
                 unpack8bf(ld16(p), x);
                 if (!isv && MODE == GDR_DECAY_SCALAR) {

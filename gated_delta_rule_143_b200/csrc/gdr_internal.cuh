@@ -82,6 +82,11 @@ cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream);
 int chunk_tc_launches(int B, int T, int H, int dk, int dv, int chunk, int mode);
 int chunk_tc_plan(int B, int T, int H, int dk, int dv, int chunk, int mode, int* precomputed_chunks);
 
+// Self-test of the bounded waits (gdr_selftest_bounded_wait): one CTA whose roles wait on a flag
+// that nothing sets, with a wait bound of limit_ns; then the time it ran, read after the stream.
+cudaError_t launch_bounded_wait_selftest(int* status, uint64_t limit_ns, cudaStream_t stream);
+cudaError_t read_bounded_wait_selftest_elapsed(unsigned long long* elapsed_ns);
+
 // Bandwidth-bound decode step.
 bool decode_supported(int dk, int dv);
 cudaError_t launch_decode(const DecodeProblem& p, cudaStream_t stream);

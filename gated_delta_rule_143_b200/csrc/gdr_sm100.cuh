@@ -58,12 +58,13 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 // Waits for the phase with the given parity to complete. Returns false (and records a
 // timeout) if it does not complete within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             report_status(status, kStatusTimeout);
             return false;
         }
@@ -73,13 +74,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
 // As mbar_wait, for warp-specialised kernels: also gives up as soon as another thread of the CTA
 // has set *abort (a wait elsewhere expired), and sets it on its own timeout, so one lost arrival
 // ends every role's loop within one wait limit instead of one limit per remaining wait.
-__device__ __forceinline__ bool mbar_wait_abort(uint64_t* bar, uint32_t parity, int* status, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait_abort(uint64_t* bar, uint32_t parity, int* status, volatile int* abort,
+                                                uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             report_status(status, kStatusTimeout);
             *abort = 1;
             return false;
@@ -101,7 +103,7 @@ __device__ __forceinline__ void st_release_gpu(int* p, int v) {
 // wait on the critical path, long where many waiters would otherwise crowd the flag's L2 line).
 // Bounded like mbar_wait_abort: gives up when *abort is set, sets it on its own timeout.
 __device__ __forceinline__ bool flag_wait_geq(const int* flag, int target, int* status, volatile int* abort,
-                                              unsigned max_sleep_ns) {
+                                              unsigned max_sleep_ns, uint64_t limit_ns = kWaitLimitNs) {
     if (ld_acquire_gpu(flag) >= target) return true;
     const uint64_t t0 = globaltimer_ns();
     unsigned sleep_ns = 32;
@@ -110,7 +112,7 @@ __device__ __forceinline__ bool flag_wait_geq(const int* flag, int target, int* 
         sleep_ns = sleep_ns * 2 < max_sleep_ns ? sleep_ns * 2 : max_sleep_ns;
         if (ld_acquire_gpu(flag) >= target) return true;
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             report_status(status, kStatusTimeout);
             *abort = 1;
             return false;

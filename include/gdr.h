@@ -45,8 +45,8 @@ typedef enum {
     GDR_ERR_CUDA = -5,         /* a CUDA runtime call or launch failed (message has the CUDA error) */
     GDR_ERR_TIMEOUT = -6,      /* a device-side bounded wait expired (reported by gdr_sync_status) */
     GDR_ERR_DEVICE = -7,       /* the current device is not an sm_100 part */
-    GDR_ERR_RANGE = -8         /* device-side: a value left the range the kernel supports (the
-                                  channel gate's within-chunk log-decay spread; see gdr_chunk_fwd) */
+    GDR_ERR_RANGE = -8         /* device-side: a value left the range a kernel supports (kept for
+                                  ABI stability; no current kernel reports it) */
 } gdr_status;
 
 typedef enum {
@@ -94,10 +94,11 @@ typedef enum {
  *             tensor cores (tcgen05); otherwise d_k, d_v in {32, 64, 128} run on an fp32
  *             CUDA-core path (fp32 accumulation, no TF32). Anything else: GDR_ERR_UNSUPPORTED.
  *   chunk     chunk size C; 64 is the supported value.
- *   Range: on the tensor-core path the channel gate's decay factors are applied to fp16 operands
- *             around a mid-chunk reference, so per key channel the cumulative log-decay may vary by
- *             at most about 22 within one chunk (e.g. g >= -0.35 per token on average); beyond that
- *             the call reports GDR_ERR_RANGE through gdr_sync_status and its outputs are invalid.
+ *   Decay range: any g <= 0 (alpha in [0, 1]), including alpha = 0 (g far below zero). On the
+ *             tensor-core path the channel gate folds its decay factors into fp16 operands around a
+ *             mid-chunk reference for the key channels whose cumulative log-decay stays within a
+ *             narrow band inside the chunk; the other channels' terms are added exactly on the CUDA
+ *             cores (slower when many channels decay strongly, never out of range).
  *   workspace device scratch of at least gdr_chunk_fwd_workspace_bytes(...) bytes (may be
  *             NULL when that is 0). Contents on entry do not matter; the library does not
  *             keep it after the enqueued work completes. Two calls in flight at the same time
@@ -192,7 +193,9 @@ int gdr_profile_next_call(void* const* events, int n_events);
  * after the work already on `stream`, and `stream` waits for the last copy: when `stream` has
  * completed, o and S_T hold the results. The host buffers and staging must stay valid until
  * then. Two calls in flight at the same time must not share `staging`. The two internal streams
- * and a few events are created on the first call on each device and kept.
+ * and a few events are created on the first call on each device and kept; they are shared by all
+ * calls on the device, so calls made from several host threads at once are serialised while they
+ * enqueue (a per-device lock), and their work is ordered as enqueued.
  * Errors: as gdr_chunk_fwd (validated before anything is enqueued), plus GDR_ERR_WORKSPACE for
  * a staging area that is missing or too small.
  */
@@ -242,12 +245,25 @@ int gdr_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const flo
 
 /* Waits for `stream`, then reads and clears the calling device's status word. Returns
  * GDR_OK, GDR_ERR_TIMEOUT (a kernel's bounded wait expired; its outputs are invalid),
- * GDR_ERR_RANGE (see gdr_chunk_fwd) or GDR_ERR_CUDA (the stream reported a CUDA error). */
+ * GDR_ERR_RANGE (a value out of a kernel's range) or GDR_ERR_CUDA (the stream reported a CUDA
+ * error). */
 int gdr_sync_status(void* stream);
 
 /* Message for the last non-zero return on the calling thread ("" if none). The pointer stays
  * valid until the next gdr_* call on the same thread. */
 const char* gdr_last_error(void);
+
+/* Self-test of the device-side bounded waits (no counterpart in the method; a diagnostic). Runs one
+ * small kernel whose roles are laid out like the state pass's -- a copy role waiting on a ring flag,
+ * an MMA-issue role waiting on the copy role, epilogue warps waiting on the issue role -- where the
+ * ring flag is one that nothing ever sets. The copy role's wait is bounded by limit_us microseconds
+ * (instead of the kernels' 2 s), the other roles' by 100 times that: the copy role's wait expires,
+ * records GDR_ERR_TIMEOUT and releases the other roles through the CTA's abort flag, so the run ends
+ * after about limit_us. Synchronous: waits for `stream` before and after, clears the status
+ * word, and returns what gdr_sync_status returns for the run (GDR_ERR_TIMEOUT when the bounded waits
+ * work). *elapsed_ns (if not NULL) receives the kernel's own measure of how long its roles waited.
+ * limit_us must be in 1 .. 1000000. Nothing faults or traps; the stream stays usable. */
+int gdr_selftest_bounded_wait(unsigned limit_us, unsigned long long* elapsed_ns, void* stream);
 
 /* Library ABI version (major * 10000 + minor * 100 + patch). */
 int gdr_version(void);

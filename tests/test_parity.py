@@ -160,6 +160,45 @@ def test_channel_constant_equals_scalar():
     assert rel_err(s2, s1)[0] <= TOL["bf16"]
 
 
+# log-decay per token that makes a channel's cumulative log2-decay spread by about `spread` over a
+# full chunk of 64 tokens: 63 * |g| * log2(e)
+def _g_for_spread(spread):
+    return -spread / (63 * 1.4426950408889634)
+
+
+def test_channel_gate_strong_decays_mixed():
+    """Channel gate with a within-chunk log2-decay spread of about 5, 15, 21 and 40 on four groups of
+    channels and alpha = 0 (g = -1e4) on a fifth, the rest at the workload's mild decay: channels
+    beyond the factored operands' range take the exact CUDA-core terms, the others the tensor-core
+    product; several chunks, a ragged tail and S0, against the oracle."""
+    x = make_chunk_inputs(2, 300, 3, 128, 128, "channel", "bf16", 201, s0_std=0.05)
+    g = x["g"].clone()
+    for c0, spread in ((0, 5.0), (8, 15.0), (16, 21.0), (24, 40.0)):
+        g[..., c0:c0 + 8] = _g_for_spread(spread)
+    g[..., 40:44] = -1e4
+    x["g"] = g
+    check_chunk(x, "channel", "bf16", label="channel spreads 5/15/21/40 + alpha=0")
+
+
+@pytest.mark.parametrize("gval", [-1.0, -1e4])
+def test_channel_gate_every_channel_strong(gval):
+    """Every key channel beyond the factored range (g = -1: a spread of about 91 log2 units per chunk;
+    g = -1e4: alpha = 0, the state resets every token)."""
+    x = make_chunk_inputs(1, 200, 2, 128, 128, "channel", "bf16", 202, s0_std=0.05)
+    x["g"] = torch.full_like(x["g"], gval)
+    check_chunk(x, "channel", "bf16", label=f"channel g={gval} everywhere")
+
+
+def test_channel_gate_strong_decays_full_workload_shape():
+    """The channel-gate workload's shape at a quarter of its length (B=4, H=16, T=2048, d=128) with
+    strong decays on a quarter of the channels: the two-pass plan at full width against the oracle."""
+    x = make_chunk_inputs(4, 2048, 16, 128, 128, "channel", "bf16", 203)
+    g = x["g"].clone()
+    g[..., 96:128] = _g_for_spread(30.0)
+    x["g"] = g
+    check_chunk(x, "channel", "bf16", label="KDA B4 H16 T2048, 32 strong channels")
+
+
 def test_zero_beta_output_is_decayed_initial_state():
     x = make_chunk_inputs(1, 128, 2, 128, 128, "channel", "bf16", 94, s0_std=0.1)
     x["beta"] = torch.zeros_like(x["beta"])
@@ -289,3 +328,42 @@ def test_device_errors_are_codes_not_faults():
         gdr.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, mode="scalar", chunk=48)
     assert e.value.code == -2
     gdr.sync_status()
+
+
+def test_host_tensors_two_threads():
+    """gdr_chunk_fwd_host from two host threads at once, each with its own stream and staging: the
+    calls share the device's copy streams and events (serialised while enqueueing); every result
+    matches the oracle."""
+    import threading
+
+    cases = [make_chunk_inputs(3, 150, 2, 128, 128, "scalar", "bf16", 700 + i, s0_std=0.05) for i in range(2)]
+    pinned = [{kk: (None if t is None else t.contiguous().pin_memory()) for kk, t in x.items()} for x in cases]
+    results, errors = [None, None], []
+    dev = torch.cuda.current_device()
+
+    def worker(i):
+        try:
+            torch.cuda.set_device(dev)
+            s = torch.cuda.Stream()
+            outs = []
+            with torch.cuda.stream(s):
+                for _ in range(3):
+                    h = pinned[i]
+                    outs.append(gdr.chunk_fwd(h["q"], h["k"], h["v"], h["g"], h["beta"], h["S0"], mode="scalar"))
+            s.synchronize()
+            results[i] = outs
+        except Exception as e:  # reported on the main thread
+            errors.append(e)
+
+    ts = [threading.Thread(target=worker, args=(i,)) for i in range(2)]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    assert not errors, errors
+    gdr.sync_status()
+    for i, x in enumerate(cases):
+        o_ref, s_ref = oracle.recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], "scalar", S0=x["S0"])
+        for o, st in results[i]:
+            assert rel_err(o.double().numpy(), o_ref)[0] <= TOL["bf16"]
+            assert rel_err(st.double().numpy(), s_ref)[0] <= TOL["bf16"]
