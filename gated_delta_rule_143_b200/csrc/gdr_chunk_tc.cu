@@ -98,7 +98,7 @@ struct PrepArgs {
 
 struct PrepSmem {
     uint8_t* base;
-    uint64_t* bars;  // [3]: TMA, Gram, W/U
+    uint64_t* bars;  // [4]: TMA, Gram, W/U, TMA of the channel gate's tile copy
     uint32_t tmem;
     int bar_id;      // named barrier of this pipeline's 128 threads
 };
@@ -248,7 +248,8 @@ __device__ void prep_init(const PrepSmem& ps, int lt) {
 // `it` counts the pipeline's previous tasks (mbarrier phase parity).
 template <int MODE>
 __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv,
-                           const PrepSmem& ps, int b, int h, int c, uint8_t* __restrict__ out, uint32_t it, int lt) {
+                           const PrepSmem& ps, int b, int h, int c, uint8_t* __restrict__ out, uint32_t it, int lt,
+                           uint32_t& n_copies) {
     const int lw = lt >> 5, lane = lt & 31;
     const int q = lw & 3, hf = lw >> 2;
     const uint32_t par = it & 1u;
@@ -275,14 +276,7 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
     //         cumulative log-decay (log2 units; rows past the tail repeat Gamma_{n-1}) meanwhile
     if (lt == 0) {
         bulk_wait_read<0>();  // the previous task's W / U^T bulk stores have read the K / V tiles
-        mbar_arrive_expect_tx(barT, (MODE == GDR_DECAY_CHANNEL ? 10 : 6) * 8192);
-        if (MODE == GDR_DECAY_CHANNEL) {  // the copy the strong channels and K*gamma are computed from
-            uint8_t* sKQ2 = sm + kPKQ2;
-            tma_load_4d(sKQ2, mk, 0, h, c0, b, barT);
-            tma_load_4d(sKQ2 + 16384, mk, 64, h, c0, b, barT);
-            tma_load_4d(sKQ2 + 8192, mq, 0, h, c0, b, barT);
-            tma_load_4d(sKQ2 + 24576, mq, 64, h, c0, b, barT);
-        }
+        mbar_arrive_expect_tx(barT, 6 * 8192);
         tma_load_4d(sKQ, mk, 0, h, c0, b, barT);
         tma_load_4d(sKQ + 16384, mk, 64, h, c0, b, barT);
         tma_load_4d(sKQ + 8192, mq, 0, h, c0, b, barT);
@@ -341,6 +335,22 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
         }
     }
     named_bar(ps.bar_id, kPrepThreads);
+    // channel gate: the number of strong channels in this chunk; if any, a second copy of the bf16 K
+    // and Q tiles (which step 2 overwrites) for their exact terms and for K*gamma
+    int n_strong = 0;
+    uint64_t* barT2 = ps.bars + 3;
+    if (MODE == GDR_DECAY_CHANNEL) {
+        const int* sStrong = reinterpret_cast<const int*>(sm + kPStrong);
+        n_strong = sStrong[256] + sStrong[257] + sStrong[258] + sStrong[259];
+        if (n_strong > 0 && lt == 0) {
+            uint8_t* sKQ2 = sm + kPKQ2;
+            mbar_arrive_expect_tx(barT2, 4 * 8192);
+            tma_load_4d(sKQ2, mk, 0, h, c0, b, barT2);
+            tma_load_4d(sKQ2 + 16384, mk, 64, h, c0, b, barT2);
+            tma_load_4d(sKQ2 + 8192, mq, 0, h, c0, b, barT2);
+            tma_load_4d(sKQ2 + 24576, mq, 64, h, c0, b, barT2);
+        }
+    }
     mbar_wait(barT, par, P.status);
     const uint32_t tG = ps.tmem + kTG, tW = ps.tmem + kTW, tU = ps.tmem + kTU;
     // Gram products for the scalar gate / DeltaNet straight from the bf16 tiles
@@ -357,6 +367,15 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
 
     // ---- 2. Q*gamma and K*gamma_C/gamma hand-off images; channel gate: decay-factored Gram operands
     const int ref = (n - 1) >> 1;
+    // channel gate: strong flags of this thread's 8 columns (the same in each of its 4 tasks)
+    bool weak8[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) weak8[e] = true;
+    if (MODE == GDR_DECAY_CHANNEL && n_strong > 0) {
+        const int* fl = reinterpret_cast<const int*>(sm + kPStrong) + (lt & 15) * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) weak8[e] = fl[e] == 0;
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int task = lt + kPrepThreads * j;
@@ -387,8 +406,7 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
                 const float Gr = sGam[ref * kD + col0 + e];
                 const float GC = sGam[(kC - 1) * kD + col0 + e];
                 // factors within 2^kStrongSpread; a strong channel's terms are added on the CUDA cores
-                const bool weak = reinterpret_cast<const int*>(sm + kPStrong)[col0 + e] == 0;
-                const float up = weak ? fast_exp2(G - Gr) : 0.f, dn = weak ? fast_exp2(Gr - G) : 0.f;
+                const float up = weak8[e] ? fast_exp2(G - Gr) : 0.f, dn = weak8[e] ? fast_exp2(Gr - G) : 0.f;
                 qg[e] = qx[e] * fast_exp2(G);
                 kt[e] = kx[e] * fast_exp2(GC - G);
                 ka[e] = kx[e] * up;
@@ -447,9 +465,10 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
         }
         const float br = sBeta[rr];
         tmem_ld_wait();
-        if (MODE == GDR_DECAY_CHANNEL) {
+        if (MODE == GDR_DECAY_CHANNEL && n_strong > 0) {
             // the strong channels' terms, left out of the tensor-core product: k_r,d k_i,d
             // 2^(Gamma_r,d - Gamma_i,d) (or q_r,d ...) from the bf16 copy of the tiles, fp32
+            mbar_wait(barT2, n_copies & 1u, P.status);
             const int* sStrong = reinterpret_cast<const int*>(sm + kPStrong);
             const uint8_t* sKQ2 = sm + kPKQ2;
             const int row = q * 32 + lane;  // tile row: K rows 0-63, Q rows 64-127
@@ -511,10 +530,21 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
             uint8_t* p = isv ? sV + kmajor_off(r, col0, 64) : sKQ + kmajor_off(r, col0, 128);
             float x[8];
             if (!isv && MODE == GDR_DECAY_CHANNEL) {
-                // K*gamma straight from the bf16 copy (every factor <= 1, any decay)
-                unpack8bf(ld16(sm + kPKQ2 + kmajor_off(r, col0, 128)), x);
+                // K' = K 2^(Gamma - Gamma_ref) times 2^Gamma_ref gives K*gamma on the other channels; a
+                // strong channel's K' is zero, its K*gamma comes from the bf16 copy (every factor <= 1)
+                unpack8h(ld16(p), x);
+                if (n_strong > 0) {
+                    const int* fl = reinterpret_cast<const int*>(sm + kPStrong) + col0;
+                    float kc[8];
+                    unpack8bf(ld16(sm + kPKQ2 + kmajor_off(r, col0, 128)), kc);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] *= fast_exp2(sGam[r * kD + col0 + e]);
+                    for (int e = 0; e < 8; ++e)
+                        x[e] = fl[e] ? kc[e] * fast_exp2(sGam[r * kD + col0 + e])
+                                     : x[e] * fast_exp2(sGam[ref * kD + col0 + e]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] *= fast_exp2(sGam[ref * kD + col0 + e]);
+                }
             } else {
                 unpack8bf(ld16(p), x);
                 if (!isv && MODE == GDR_DECAY_SCALAR) {
@@ -582,6 +612,7 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
         fence_proxy_async_smem();
         tc_fence_before();
         named_bar(ps.bar_id, kPrepThreads);
+        if (MODE == GDR_DECAY_CHANNEL && n_strong > 0) ++n_copies;
         if (lt == 0) {  // the next task waits for these reads before its TMA loads into the same tiles
             bulk_s2g(out + kOffWQ, stW, 8192);
             bulk_s2g(out + kOffWQ + 16384, stW + 16384, 8192);
@@ -602,11 +633,11 @@ __global__ void __maxnreg__(MODE == GDR_DECAY_CHANNEL ? 240 : 96)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                   const __grid_constant__ CUtensorMap mv, PrepArgs P, uint8_t* __restrict__ ws, int NCp, int n_tasks) {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ uint64_t bars[3];
+    __shared__ uint64_t bars[4];
     __shared__ uint32_t tmem_base;
     const int lt = threadIdx.x;
     if (lt == 0) {
-        for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
     }
     if (lt < 32) {
@@ -619,7 +650,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     ps.tmem = tmem_base;
-    uint32_t it = 0;
+    uint32_t it = 0, n_copies = 0;  // tasks so far; channel-gate tile copies so far (mbarrier parities)
     for (int t = blockIdx.x; t < n_tasks; t += gridDim.x, ++it) {
         const int c = t % NCp, bh = t / NCp;
         const int h = bh % P.H, b = bh / P.H;
@@ -635,7 +666,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
             tma_prefetch_l2_4d(&mv, 64, hn, cn * kC, bn);
         }
         uint8_t* out = ws + (size_t)t * kHandoffStride;
-        prep_chunk<MODE>(P, &mq, &mk, &mv, ps, b, h, c, out, it, lt);
+        prep_chunk<MODE>(P, &mq, &mk, &mv, ps, b, h, c, out, it, lt, n_copies);
     }
     if (lt == 0) bulk_wait<0>();
     tc_fence_before();
@@ -1035,7 +1066,7 @@ struct RingArgs {
 template <int MODE>
 __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv, const PrepArgs& P,
                           const RingArgs& R, uint8_t* sm, uint32_t tbase, volatile int* abort) {
-    __shared__ uint64_t pbars[2][3];
+    __shared__ uint64_t pbars[2][4];
     __shared__ volatile int go[2];
     __shared__ volatile int claimed[2];
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -1043,7 +1074,7 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
     const int lt = tid & 255;
     if (tid == 0) {
         for (int i = 0; i < 2; ++i)
-            for (int k = 0; k < 3; ++k) mbar_init(&pbars[i][k], 1);
+            for (int k = 0; k < 4; ++k) mbar_init(&pbars[i][k], 1);
         fence_mbar_init();
     }
     if (pipe < 2) prep_init(PrepSmem{sm + pipe * kPrepPipeBytes, nullptr, 0, 0}, lt);
@@ -1053,7 +1084,7 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
     if (pipe >= 2 || (int)blockIdx.x - R.BH >= 3 * R.BH + 4) return;
     const PrepSmem ps{sm + pipe * kPrepPipeBytes, pbars[pipe], tbase + (uint32_t)pipe * kPrepTmemCols, 1 + 2 * pipe};
     const int n_tasks = P.NC * R.BH;
-    uint32_t it = 0;
+    uint32_t it = 0, n_copies = 0;  // tasks so far; channel-gate tile copies so far (mbarrier parities)
     for (;; ++it) {
         // claim the next task in consumption order (a pipeline claims only after finishing its
         // previous task, so claims, like the state passes' reads, go in increasing order)
@@ -1069,7 +1100,7 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
         named_bar(ps.bar_id, kPrepThreads);
         if (!go[pipe]) break;
         uint8_t* out = R.ring + ((size_t)bh * R.depth + slot) * kHandoffStride;
-        prep_chunk<MODE>(P, mq, mk, mv, ps, bh / P.H, bh % P.H, c, out, it, lt);
+        prep_chunk<MODE>(P, mq, mk, mv, ps, bh / P.H, bh % P.H, c, out, it, lt, n_copies);
         if (lt == 0) {  // every write of the block (generic stores before prep_chunk's last barrier, bulk stores)
             bulk_wait<0>();
             fence_proxy_async_global();
