@@ -131,3 +131,63 @@ def decode_step(q, k, v, g, beta, S, mode: str, *, scale: Optional[float] = None
     o, st = recurrent(tok(q), tok(k), tok(v), tok(g), tok(beta), mode, S0=S, scale=scale,
                       f64_inputs=f64_inputs, threads=threads)
     return o[:, 0], st
+
+
+def _sigmoid(x: np.ndarray) -> np.ndarray:
+    """Logistic function 1 / (1 + e^-x) in float64, evaluated on the side where the
+    exponential cannot overflow (e^x / (1 + e^x) for negative x)."""
+    out = np.empty_like(x)
+    pos = x >= 0
+    out[pos] = 1.0 / (1.0 + np.exp(-x[pos]))
+    e = np.exp(x[~pos])
+    out[~pos] = e / (1.0 + e)
+    return out
+
+
+def _softplus(x: np.ndarray) -> np.ndarray:
+    """softplus(x) = log(1 + e^x) in float64, written as max(x, 0) + log1p(e^-|x|)."""
+    return np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x)))
+
+
+def prologue(q, k, beta, g, mode: str, *, l2norm_qk: bool = False, beta_sigmoid: bool = False,
+             gate_softplus: bool = False, gate_scale=None):
+    """The mixer layer's steps in front of the recurrence, in float64.
+
+    Follows the pages' recurrent reference form ("Linear Attention & DeltaNet",
+    minimal pseudocode): q and k pass through a feature map, the write strength is
+    beta = sigmoid(logit) and the decay gate is a squashed logit. The three steps, each
+    applied only when its flag is set, are:
+
+    - ``l2norm_qk``: every (b, t, h) vector of q and of k is divided by its Euclidean
+      norm (no epsilon; an all-zero vector stays zero).
+    - ``beta_sigmoid``: ``beta`` holds logits; the write strength is their sigmoid.
+    - ``gate_softplus``: ``g`` holds gate logits a ([B,T,H] or [B,T,H,dk]); the
+      log-decay is g = -A_h * softplus(a) with A = ``gate_scale`` [H] (1 if None).
+      With A_h = 0.05 this is the decay exp(-0.05 softplus(.)) of the small
+      Gated DeltaNet workload; with A_h = 1 and a = -x it is alpha = sigmoid(x), the
+      pseudocode's gate, since log sigmoid(x) = -softplus(-x).
+
+    Inputs are read as float32 (exact for bf16 / fp32 data). Returns float64
+    ``(q, k, beta, g)`` to hand to ``recurrent(..., f64_inputs=True)``; arguments
+    whose step is off come back unchanged (widened).
+    """
+    # widen through float32, as the library reads them
+    qa, ka = _arr(_arr(q, False), True), _arr(_arr(k, False), True)
+    ba = _arr(_arr(beta, False), True)
+    ga = None if g is None else _arr(_arr(g, False), True)
+    if l2norm_qk:
+        out = []
+        for a in (qa, ka):
+            n = np.sqrt(np.sum(a * a, axis=-1, keepdims=True))
+            out.append(np.divide(a, n, out=np.zeros_like(a), where=n > 0))
+        qa, ka = out
+    if beta_sigmoid:
+        ba = _sigmoid(ba)
+    if gate_softplus:
+        if mode == "none" or ga is None:
+            raise ValueError("gate_softplus needs a decay mode and gate logits")
+        H = ba.shape[2]
+        A = np.ones(H) if gate_scale is None else _arr(_arr(gate_scale, False), True).reshape(H)
+        Ab = A.reshape((1, 1, H)) if mode == "scalar" else A.reshape((1, 1, H, 1))
+        ga = -Ab * _softplus(ga)
+    return qa, ka, ba, ga

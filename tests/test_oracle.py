@@ -359,3 +359,100 @@ def test_bad_arguments_raise():
         _run(q, k, v, g[..., None].repeat(4, -1), beta, "scalar")
     with pytest.raises(ValueError):
         _run(q, k, v, g, beta, "bogus")
+
+
+# ---- the mixer prologue (q/k L2 normalisation, beta = sigmoid(logit), softplus decay gate)
+
+def test_prologue_l2norm_worked_and_invariants():
+    # worked example: (3, 4) / 5; a zero vector stays zero; every (b, t, h) vector of q and of k
+    # comes out with unit norm and the same direction, whatever its input scale
+    q = np.zeros((1, 2, 2, 2))
+    q[0, 0, 0] = (3.0, 4.0)
+    q[0, 0, 1] = (-6.0, 8.0)
+    q[0, 1, 0] = (0.0, 0.0)
+    q[0, 1, 1] = (1e-3, 0.0)
+    k = q[:, ::-1].copy()
+    qn, kn, _, _ = oracle.prologue(q, k, np.zeros((1, 2, 2)), None, "none", l2norm_qk=True)
+    assert np.array_equal(qn[0, 0, 0], [0.6, 0.8])
+    assert np.array_equal(qn[0, 0, 1], [-0.6, 0.8])
+    assert np.array_equal(qn[0, 1, 0], [0.0, 0.0])
+    assert np.array_equal(qn[0, 1, 1], [1.0, 0.0])
+    assert np.array_equal(kn, qn[:, ::-1])
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((2, 5, 3, 16)) * 10.0 ** rng.integers(-3, 4, (2, 5, 3, 1))
+    xn, _, _, _ = oracle.prologue(x, x, np.zeros((2, 5, 3)), None, "none", l2norm_qk=True)
+    np.testing.assert_allclose(np.linalg.norm(xn, axis=-1), 1.0, rtol=0, atol=1e-15)
+    x32 = x.astype(np.float32).astype(np.float64)  # the oracle reads inputs as float32
+    np.testing.assert_allclose(xn * np.linalg.norm(x32, axis=-1, keepdims=True), x32, rtol=1e-14, atol=0)
+    # flags off: values pass through (widened from float32)
+    xo, _, bo, _ = oracle.prologue(x, x, np.full((2, 5, 3), 0.25), None, "none")
+    assert np.array_equal(xo, x32) and np.all(bo == 0.25)
+
+
+def test_prologue_beta_sigmoid_closed_forms():
+    b = np.array([0.0, np.log(3.0), -np.log(3.0), 800.0, -800.0, 2.5, -2.5]).reshape(1, 7, 1)
+    _, _, s, _ = oracle.prologue(np.ones((1, 7, 1, 2)), np.ones((1, 7, 1, 2)), b, None, "none", beta_sigmoid=True)
+    s = s.ravel()
+    b32 = b.ravel().astype(np.float32).astype(np.float64)
+    assert s[0] == 0.5
+    np.testing.assert_allclose(s[1], 1.0 / (1.0 + np.exp(-b32[1])), rtol=1e-15)  # ~0.75
+    assert abs(s[1] - 0.75) < 1e-7 and abs(s[2] - 0.25) < 1e-7  # ln 3 rounded to float32
+    assert s[3] == 1.0 and 0.0 <= s[4] < 1e-300 and np.all(np.isfinite(s))
+    np.testing.assert_allclose(s[5] + s[6], 1.0, rtol=0, atol=1e-15)  # sigma(x) + sigma(-x) = 1
+    np.testing.assert_allclose(s[5], np.exp(2.5) / (1.0 + np.exp(2.5)), rtol=1e-15)
+
+
+@pytest.mark.parametrize("mode", ["scalar", "channel"])
+def test_prologue_softplus_gate_closed_forms(mode):
+    # a = 0 gives g = -A ln 2; a = ln(e^2 - 1) gives g = -2 A; a = 40 gives -40 A (to 1e-17
+    # relative); a = -40 gives -A e^-40; per-head A broadcasts over tokens (and channels)
+    vals = np.array([0.0, np.log(np.e ** 2 - 1.0), 40.0, -40.0], dtype=np.float32).astype(np.float64)
+    A = np.array([0.05, 1.0, 3.0])
+    H = 3
+    shape = (1, 4, H) if mode == "scalar" else (1, 4, H, 2)
+    a = np.broadcast_to(vals.reshape((1, 4, 1) + ((1,) if mode == "channel" else ())), shape).copy()
+    _, _, _, g = oracle.prologue(np.ones((1, 4, H, 2)), np.ones((1, 4, H, 2)), np.zeros((1, 4, H)), a, mode,
+                                 gate_softplus=True, gate_scale=A)
+    sp = np.array([np.log(2.0), np.log1p(np.exp(vals[1])), 40.0 + np.log1p(np.exp(-40.0)), np.exp(-40.0)])
+    A32 = A.astype(np.float32).astype(np.float64)  # gate_scale is read as float32 too
+    for h in range(H):
+        gh = g[0, :, h] if mode == "scalar" else g[0, :, h, 1]
+        np.testing.assert_allclose(gh, -A32[h] * sp, rtol=1e-15)
+    assert abs(sp[1] - 2.0) < 1e-6  # ln(e^2 - 1) rounded to float32
+    # the pages' gate alpha = sigmoid(x) is A = 1, a = -x: exp(g) = sigmoid(x)
+    x = np.linspace(-30, 30, 61).reshape(1, 61, 1)
+    _, _, _, g1 = oracle.prologue(np.ones((1, 61, 1, 2)), np.ones((1, 61, 1, 2)), np.zeros((1, 61, 1)), -x, "scalar",
+                                  gate_softplus=True)
+    x32 = x.astype(np.float32).astype(np.float64)
+    np.testing.assert_allclose(np.exp(g1), 1.0 / (1.0 + np.exp(-x32)), rtol=1e-14)
+    # the small Gated DeltaNet workload's decay exp(-0.05 softplus(z))
+    z = np.random.default_rng(3).standard_normal((1, 50, 1))
+    _, _, _, g2 = oracle.prologue(np.ones((1, 50, 1, 2)), np.ones((1, 50, 1, 2)), np.zeros((1, 50, 1)), z, "scalar",
+                                  gate_softplus=True, gate_scale=np.array([0.05]))
+    z32 = z.astype(np.float32).astype(np.float64)
+    a05 = float(np.float32(0.05))
+    np.testing.assert_allclose(np.exp(g2), np.exp(-a05 * np.log(1.0 + np.exp(z32))), rtol=1e-14)
+    with pytest.raises(ValueError):
+        oracle.prologue(np.ones((1, 1, 1, 2)), np.ones((1, 1, 1, 2)), np.zeros((1, 1, 1)), None, "none",
+                        gate_softplus=True)
+
+
+def test_prologue_then_recurrence_exact_recall_with_raw_keys():
+    # orthogonal keys of arbitrary lengths (rows of an 8 x 8 Hadamard matrix times lengths that
+    # float32 holds exactly), beta logits large enough that sigmoid rounds to 1, no decay: after
+    # the prologue, S_T k_i / |k_i| = v_i for every i (exact recall)
+    rng = np.random.default_rng(5)
+    dk, T = 8, 6
+    Hd = np.array([[1.0]])
+    for _ in range(3):
+        Hd = np.block([[Hd, Hd], [Hd, -Hd]])
+    lengths = np.array([0.1, 0.3, 2.5, 7.0, 10.0, 0.7], dtype=np.float32).astype(np.float64)
+    k = (Hd[:T] * lengths[:, None]).reshape(1, T, 1, dk)
+    v = rng.standard_normal((1, T, 1, 3))
+    q, kk, b, _ = oracle.prologue(k, k, np.full((1, T, 1), 60.0), None, "none", l2norm_qk=True, beta_sigmoid=True)
+    assert np.all(b == 1.0)
+    _, S = oracle.recurrent(q, kk, v, None, b, "none", f64_inputs=True)
+    k32 = k.astype(np.float32).astype(np.float64)
+    for i in range(T):
+        ki = k32[0, i, 0] / np.linalg.norm(k32[0, i, 0])
+        np.testing.assert_allclose(S[0, 0] @ ki, v[0, i, 0], rtol=0, atol=1e-12)
