@@ -465,6 +465,7 @@ def run_ours(args):
 
     dec = bench_decode(args, dev, peaks, world)
     others = bench_workloads(args, dev, peaks) if world == 1 else None
+    pro = bench_prologue(args, w, dev, ws, o, st, stream, world, rank, ms_step)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -481,6 +482,7 @@ def run_ours(args):
         "clocks": clk,
         "o_bf16": o_bf16,
         "decode": dec,
+        "prologue": pro,
     }
     if others is not None:
         line["extra"] = {"workloads": others}
@@ -491,6 +493,50 @@ def run_ours(args):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def bench_prologue(args, w, dev, ws, o, st, stream, world, rank, ms_plain):
+    """The same step on raw inputs (q/k unnormalised, beta and gate logits), with the mixer prologue
+    fused into the kernels (gdr_chunk_fwd_ex), against the prologue as separate torch ops (F.normalize,
+    sigmoid, softplus: library kernels, for comparison only) followed by the plain call."""
+    import torch.nn.functional as F
+
+    import gated_delta_rule_143_b200 as gdr
+    from gated_delta_rule_143_b200.inputs import make_raw_chunk_inputs
+
+    sets = []
+    for s in range(2):
+        x = make_raw_chunk_inputs(w.B, w.T, w.H, w.dk, w.dv, w.mode, w.dtype, rank_seed(97, rank, s))
+        sets.append({k: (None if t is None else t.to(dev)) for k, t in x.items()})
+    gate = w.mode != "none"
+
+    def fused(i=0):
+        x = sets[i & 1]
+        gdr.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, mode=w.mode, chunk=w.chunk, out=o,
+                      state_out=st, workspace=ws, l2norm_qk=True, beta_sigmoid=True, gate_softplus=gate,
+                      gate_scale=x["gate_scale"])
+
+    def unfused(i=0):
+        x = sets[i & 1]
+        q = F.normalize(x["q"].float(), dim=-1, eps=0.0).to(x["q"].dtype)
+        k = F.normalize(x["k"].float(), dim=-1, eps=0.0).to(x["k"].dtype)
+        b = torch.sigmoid(x["beta"])
+        g = None
+        if gate:
+            A = x["gate_scale"].view((1, 1, -1) + ((1,) if w.mode == "channel" else ()))
+            g = -A * F.softplus(x["g"])
+        gdr.chunk_fwd(q, k, x["v"], g, b, None, mode=w.mode, chunk=w.chunk, out=o, state_out=st, workspace=ws)
+
+    n = max(3, min(args.steps, 100))
+    ms_f = max_over_ranks(time_device(fused, n, args.warmup, world, stream), world) / n
+    ms_u = max_over_ranks(time_device(unfused, n, args.warmup, world, stream), world) / n
+    gdr.sync_status()
+    tokens = w.B * w.T
+    return {"fused_ms_per_step": round(ms_f, 5), "fused_tokens_per_s": round(job_throughput(tokens, ms_f, world), 1),
+            "torch_ops_then_call_ms_per_step": round(ms_u, 5), "plain_step_ms": round(ms_plain, 5),
+            "steps": n, "fused_gpu_launches_per_step": gdr_kernels_per_step(w),
+            "note": "raw q/k (unnormalised, bf16), beta logits, gate logits and A [H]; fused = "
+                    "l2norm_qk + beta_sigmoid + gate_softplus in the library's kernels"}
 
 
 def gdr_kernels_per_step(w):

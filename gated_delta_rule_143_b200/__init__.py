@@ -8,6 +8,10 @@ CUDA kernels; PyTorch provides device memory and streams. The two operations:
   Kimi Delta Attention ("channel");
 * ``decode_step`` -- one recurrent token step on a batch of fp32 states, in place.
 
+Both can apply the mixer layer's input steps inside their kernels (keyword
+arguments ``l2norm_qk``, ``beta_sigmoid``, ``gate_softplus`` / ``gate_scale``):
+q and k then hold raw vectors, ``beta`` logits and ``g`` gate logits.
+
 Both take device tensors. ``chunk_fwd`` also accepts host (CPU) tensors: it
 then copies them to the current device on the current stream, runs, and copies
 the outputs back (the end-to-end path a host-resident caller uses).
@@ -18,7 +22,8 @@ from typing import Optional, Tuple
 
 import torch
 
-from ._lib import DECAY_MODES, DTYPE_BF16, DTYPE_F32, PLANS, GdrError, check, lib
+from ._lib import (DECAY_MODES, DTYPE_BF16, DTYPE_F32, PLANS, PRO_BETA_SIGMOID, PRO_GATE_SOFTPLUS, PRO_L2NORM_QK,
+                   GdrError, check, lib)
 
 __all__ = ["chunk_fwd", "decode_step", "sync_status", "workspace_bytes", "launches_per_chunk_fwd", "chunk_fwd_plan",
            "profile_next_call",
@@ -47,6 +52,11 @@ def _dtype(t: torch.Tensor) -> int:
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
+
+
+def _prologue(l2norm_qk: bool, beta_sigmoid: bool, gate_softplus: bool) -> int:
+    return ((PRO_L2NORM_QK if l2norm_qk else 0) | (PRO_BETA_SIGMOID if beta_sigmoid else 0)
+            | (PRO_GATE_SOFTPLUS if gate_softplus else 0))
 
 
 def _stream_handle(stream: Optional[torch.cuda.Stream]) -> int:
@@ -98,13 +108,21 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optional[tor
               return_state: bool = True, out: Optional[torch.Tensor] = None,
               out_dtype: torch.dtype = torch.float32,
               state_out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-              stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+              stream: Optional[torch.cuda.Stream] = None, l2norm_qk: bool = False, beta_sigmoid: bool = False,
+              gate_softplus: bool = False,
+              gate_scale: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunked forward. q, k [B,T,H,dk]; v [B,T,H,dv] (bf16 or fp32, same dtype);
     g fp32 [B,T,H] ("scalar") / [B,T,H,dk] ("channel") / None ("none"); beta fp32
     [B,T,H]; S0 fp32 [B,H,dv,dk] or None. Returns (o [B,T,H,dv], S_T or None).
     o is fp32 by default (``out_dtype``, or the dtype of ``out``; bf16 allowed for bf16
-    inputs). ``state_out`` may be ``S0`` itself (in-place carry)."""
+    inputs). ``state_out`` may be ``S0`` itself (in-place carry).
+    Prologue (device tensors only, gdr_chunk_fwd_ex): ``l2norm_qk`` divides every q and k
+    vector by its norm, ``beta_sigmoid`` reads ``beta`` as logits, ``gate_softplus`` reads
+    ``g`` as gate logits a with g = -gate_scale[h] * softplus(a) (``gate_scale`` fp32 [H] or None = 1)."""
+    pro = _prologue(l2norm_qk, beta_sigmoid, gate_softplus)
     if q.device.type == "cpu":
+        if pro:
+            raise ValueError("the fused prologue takes device tensors")
         return _chunk_fwd_host(q, k, v, g, beta, S0, mode=mode, chunk=chunk, return_state=return_state,
                                out=out, out_dtype=out_dtype, state_out=state_out, stream=stream)
     B, T, H, dk = q.shape
@@ -119,9 +137,14 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optional[tor
     if workspace is None:
         workspace = _workspace(lib().gdr_chunk_fwd_workspace_bytes(B, T, H, dk, dv, chunk, m, dt, odt), q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = lib().gdr_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(out),
-                             _ptr(state_out) if return_state else None, B, T, H, dk, dv, chunk, m, dt, odt,
-                             _ptr(workspace), ws_bytes, _stream_handle(stream))
+    if pro:
+        rc = lib().gdr_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(out),
+                                    _ptr(state_out) if return_state else None, B, T, H, dk, dv, chunk, m, dt, odt,
+                                    pro, _ptr(gate_scale), _ptr(workspace), ws_bytes, _stream_handle(stream))
+    else:
+        rc = lib().gdr_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(out),
+                                 _ptr(state_out) if return_state else None, B, T, H, dk, dv, chunk, m, dt, odt,
+                                 _ptr(workspace), ws_bytes, _stream_handle(stream))
     check(rc)
     return out, (state_out if return_state else None)
 
@@ -160,15 +183,23 @@ def _chunk_fwd_host(q, k, v, g, beta, S0, *, mode, chunk, return_state, out, out
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optional[torch.Tensor],
                 beta: torch.Tensor, S: torch.Tensor, *, mode="scalar", out: Optional[torch.Tensor] = None,
                 out_dtype: torch.dtype = torch.float32,
-                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+                stream: Optional[torch.cuda.Stream] = None, l2norm_qk: bool = False, beta_sigmoid: bool = False,
+                gate_softplus: bool = False, gate_scale: Optional[torch.Tensor] = None) -> torch.Tensor:
     """One recurrent step: q, k [B,H,dk], v [B,H,dv], g [B,H] / [B,H,dk] / None,
-    beta [B,H], S fp32 [B,H,dv,dk] updated in place. Returns o [B,H,dv] (fp32 by default)."""
+    beta [B,H], S fp32 [B,H,dv,dk] updated in place. Returns o [B,H,dv] (fp32 by default).
+    The prologue keywords are those of ``chunk_fwd`` (gdr_decode_step_ex)."""
     B, H, dk = q.shape
     dv = v.shape[-1]
     if out is None:
         out = torch.empty((B, H, dv), dtype=out_dtype, device=q.device)
-    rc = lib().gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(out), B, H, dk, dv,
-                               _mode(mode), _dtype(q), _dtype(out), _stream_handle(stream))
+    pro = _prologue(l2norm_qk, beta_sigmoid, gate_softplus)
+    if pro:
+        rc = lib().gdr_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(out), B, H, dk,
+                                      dv, _mode(mode), _dtype(q), _dtype(out), pro, _ptr(gate_scale),
+                                      _stream_handle(stream))
+    else:
+        rc = lib().gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(out), B, H, dk,
+                                   dv, _mode(mode), _dtype(q), _dtype(out), _stream_handle(stream))
     check(rc)
     return out
 

@@ -22,6 +22,7 @@ STATUS_NAMES = {
 DECAY_MODES = {"none": 0, "scalar": 1, "channel": 2}
 DTYPE_F32, DTYPE_BF16 = 0, 1
 PLANS = {0: "invalid", 1: "cuda_core", 2: "two_pass", 3: "fused", 4: "prep_fused"}
+PRO_L2NORM_QK, PRO_BETA_SIGMOID, PRO_GATE_SOFTPLUS = 1, 2, 4  # gdr_prologue flags
 
 # Every symbol the header declares: name -> (restype, argtypes).
 _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -30,7 +31,9 @@ SIGNATURES = {
     "gdr_chunk_fwd_workspace_bytes": (_sz, [_i] * 9),
     "gdr_chunk_fwd_launches": (_i, [_i] * 9),
     "gdr_chunk_fwd_plan": (_i, [_i] * 9 + [_vp]),
+    "gdr_chunk_fwd_ex": (_i, [_vp] * 8 + [_i] * 10 + [_vp, _vp, _sz, _vp]),
     "gdr_decode_step": (_i, [_vp] * 7 + [_i] * 7 + [_vp]),
+    "gdr_decode_step_ex": (_i, [_vp] * 7 + [_i] * 8 + [_vp, _vp]),
     "gdr_chunk_fwd_noalloc": (_i, [_vp] * 8 + [_i] * 9 + [_vp]),
     "gdr_chunk_fwd_host": (_i, [_vp] * 8 + [_i] * 9 + [_vp, _sz, _vp]),
     "gdr_chunk_fwd_host_staging_bytes": (_sz, [_i] * 9),

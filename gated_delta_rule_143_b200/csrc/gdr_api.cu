@@ -115,6 +115,14 @@ int chunk_shape_check(int B, int T, int H, int dk, int dv, int chunk, int mode, 
     return GDR_OK;
 }
 
+int prologue_check(int prologue, int mode) {
+    const int all = GDR_PRO_L2NORM_QK | GDR_PRO_BETA_SIGMOID | GDR_PRO_GATE_SOFTPLUS;
+    if (prologue & ~all) return fail(GDR_ERR_INVALID_ARG, "unknown prologue flags 0x%x", prologue & ~all);
+    if ((prologue & GDR_PRO_GATE_SOFTPLUS) && mode == GDR_DECAY_NONE)
+        return fail(GDR_ERR_INVALID_ARG, "GDR_PRO_GATE_SOFTPLUS needs a gated decay mode");
+    return GDR_OK;
+}
+
 }  // namespace
 
 void profile_after_launch(cudaStream_t stream) {
@@ -171,14 +179,17 @@ int gdr_chunk_fwd_launches(int B, int T, int H, int dk, int dv, int chunk, int m
     return chunk_tc_supported(dk, dv, chunk, dtype, o_dtype) ? chunk_tc_launches(B, T, H, dk, dv, chunk, mode) : 1;
 }
 
-int gdr_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                  const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk,
-                  int mode, int dtype, int o_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+int gdr_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                     const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk,
+                     int mode, int dtype, int o_dtype, int prologue, const float* gate_scale, void* workspace,
+                     size_t workspace_bytes, void* stream) {
     ProfileScope prof_scope;
     if (int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype)) return rc;
+    if (int rc = prologue_check(prologue, mode)) return rc;
+    if (!(prologue & GDR_PRO_GATE_SOFTPLUS)) gate_scale = nullptr;
     if (!q || !k || !v || !beta || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, beta and o must be non-null");
     if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
-    const void* ptrs[] = {q, k, v, g, beta, S0, o, S_T, workspace};
+    const void* ptrs[] = {q, k, v, g, beta, S0, o, S_T, workspace, gate_scale};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return fail(GDR_ERR_MISALIGNED, "pointer %p is not 16-byte aligned", p);
     const size_t ntok = (size_t)B * T * H;
@@ -189,7 +200,7 @@ int gdr_chunk_fwd(const void* q, const void* k, const void* v, const float* g, c
     const size_t bs = (size_t)B * H * dv * dk * sizeof(float);
     struct Span { const void* p; size_t n; const char* name; };
     const Span ins[] = {{q, bq, "q"}, {k, bq, "k"}, {v, bv, "v"}, {mode == GDR_DECAY_NONE ? nullptr : g, bg, "g"},
-                        {beta, bb, "beta"}, {S0, bs, "S0"}};
+                        {beta, bb, "beta"}, {S0, bs, "S0"}, {gate_scale, H * sizeof(float), "gate_scale"}};
     for (const Span& s : ins) {
         if (overlap(o, bo, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "o overlaps input %s", s.name);
         if (S_T != S0 && overlap(S_T, bs, s.p, s.n))
@@ -213,7 +224,8 @@ int gdr_chunk_fwd(const void* q, const void* k, const void* v, const float* g, c
     if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
 
     ChunkProblem p{q, k, v, mode == GDR_DECAY_NONE ? nullptr : g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode,
-                   dtype, o_dtype, workspace, workspace_bytes, status, (float)(1.0 / sqrt((double)dk))};
+                   dtype, o_dtype, workspace, workspace_bytes, status, (float)(1.0 / sqrt((double)dk)), prologue,
+                   gate_scale};
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const cudaError_t err = use_tc ? launch_chunk_tc(p, s) : launch_chunk_simt(p, s);
     if (err != cudaSuccess)
@@ -221,9 +233,19 @@ int gdr_chunk_fwd(const void* q, const void* k, const void* v, const float* g, c
     return ok();
 }
 
-int gdr_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta, float* S,
-                    void* o, int B, int H, int dk, int dv, int mode, int dtype, int o_dtype, void* stream) {
+int gdr_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                  const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk,
+                  int mode, int dtype, int o_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    return gdr_chunk_fwd_ex(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, GDR_PRO_NONE,
+                            nullptr, workspace, workspace_bytes, stream);
+}
+
+int gdr_decode_step_ex(const void* q, const void* k, const void* v, const float* g, const float* beta, float* S,
+                       void* o, int B, int H, int dk, int dv, int mode, int dtype, int o_dtype, int prologue,
+                       const float* gate_scale, void* stream) {
     if (int rc = check_enums(mode, dtype, o_dtype)) return rc;
+    if (int rc = prologue_check(prologue, mode)) return rc;
+    if (!(prologue & GDR_PRO_GATE_SOFTPLUS)) gate_scale = nullptr;
     if (B <= 0 || H <= 0 || dk <= 0 || dv <= 0)
         return fail(GDR_ERR_INVALID_ARG, "sizes must be positive (B=%d H=%d d_k=%d d_v=%d)", B, H, dk, dv);
     if ((size_t)B * H > 0x7fffffffu) return fail(GDR_ERR_UNSUPPORTED, "B*H too large");
@@ -231,7 +253,7 @@ int gdr_decode_step(const void* q, const void* k, const void* v, const float* g,
         return fail(GDR_ERR_UNSUPPORTED, "unsupported d_k=%d (supported: 32, 64, 128, 256)", dk);
     if (!q || !k || !v || !beta || !S || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, beta, S and o must be non-null");
     if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
-    const void* ptrs[] = {q, k, v, g, beta, S, o};
+    const void* ptrs[] = {q, k, v, g, beta, S, o, gate_scale};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return fail(GDR_ERR_MISALIGNED, "pointer %p is not 16-byte aligned", p);
     const size_t nh = (size_t)B * H, eb = elem_bytes(dtype);
@@ -240,7 +262,7 @@ int gdr_decode_step(const void* q, const void* k, const void* v, const float* g,
     const Span ins[] = {{q, nh * dk * eb, "q"}, {k, nh * dk * eb, "k"}, {v, nh * dv * eb, "v"},
                         {mode == GDR_DECAY_NONE ? nullptr : g,
                          mode == GDR_DECAY_CHANNEL ? nh * dk * sizeof(float) : nh * sizeof(float), "g"},
-                        {beta, nh * sizeof(float), "beta"}};
+                        {beta, nh * sizeof(float), "beta"}, {gate_scale, H * sizeof(float), "gate_scale"}};
     for (const Span& s : ins) {
         if (overlap(S, bs, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "S overlaps input %s", s.name);
         if (overlap(o, bo, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "o overlaps input %s", s.name);
@@ -251,10 +273,16 @@ int gdr_decode_step(const void* q, const void* k, const void* v, const float* g,
     if (int rc = device_setup(&status, &major)) return rc;
     if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
     DecodeProblem p{q, k, v, mode == GDR_DECAY_NONE ? nullptr : g, beta, S, o, B, H, dk, dv, mode, dtype, o_dtype,
-                    status, (float)(1.0 / sqrt((double)dk))};
+                    status, (float)(1.0 / sqrt((double)dk)), prologue, gate_scale};
     const cudaError_t err = launch_decode(p, static_cast<cudaStream_t>(stream));
     if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
     return ok();
+}
+
+int gdr_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta, float* S,
+                    void* o, int B, int H, int dk, int dv, int mode, int dtype, int o_dtype, void* stream) {
+    return gdr_decode_step_ex(q, k, v, g, beta, S, o, B, H, dk, dv, mode, dtype, o_dtype, GDR_PRO_NONE, nullptr,
+                              stream);
 }
 
 int gdr_sync_status(void* stream) {

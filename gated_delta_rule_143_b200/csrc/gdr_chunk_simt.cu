@@ -45,7 +45,8 @@ template <typename Tin, typename Tout, int MODE, int DK>
 __global__ void __launch_bounds__(kThreads)
 chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                   const float* __restrict__ g, const float* __restrict__ beta, const float* S0,
-                  Tout* __restrict__ o, float* S_T, int T, int H, int dv, float scale) {
+                  Tout* __restrict__ o, float* S_T, int T, int H, int dv, float scale, int pro,
+                  const float* __restrict__ gate_scale) {
     using L = SimtSmem<DK>;
     extern __shared__ float smem[];
     float* sK = smem;
@@ -65,6 +66,8 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
     const int b = blockIdx.z;
     const int nrows = min(kDVS, dv - j0);
     const size_t bh = (size_t)b * H + h;
+    const bool gate = (pro & GDR_PRO_GATE_SOFTPLUS) != 0;
+    const float A = (gate && gate_scale != nullptr) ? gate_scale[h] : 1.f;
 
     // initial state slice
     for (int idx = tid; idx < kDVS * DK; idx += kThreads) {
@@ -89,12 +92,16 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
             const size_t tok = ((size_t)b * T + c0 + r) * H + h;
             sR[r * L::kLdV + j] = (j < nrows) ? load_f32(v + tok * dv + j0 + j) : 0.f;
         }
-        for (int r = tid; r < n; r += kThreads) sBeta[r] = beta[((size_t)b * T + c0 + r) * H + h];
+        for (int r = tid; r < n; r += kThreads) {
+            const float x = beta[((size_t)b * T + c0 + r) * H + h];
+            sBeta[r] = (pro & GDR_PRO_BETA_SIGMOID) ? pro_sigmoid(x) : x;
+        }
         if (MODE == GDR_DECAY_SCALAR) {
             if (tid == 0) {
                 float acc = 0.f;
                 for (int r = 0; r < n; ++r) {
-                    acc += g[((size_t)b * T + c0 + r) * H + h];
+                    const float x = g[((size_t)b * T + c0 + r) * H + h];
+                    acc += gate ? pro_gate(x, A) : x;
                     sG[r * L::kLd] = acc;
                 }
             }
@@ -102,12 +109,26 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
             for (int c = tid; c < DK; c += kThreads) {
                 float acc = 0.f;
                 for (int r = 0; r < n; ++r) {
-                    acc += g[(((size_t)b * T + c0 + r) * H + h) * DK + c];
+                    const float x = g[(((size_t)b * T + c0 + r) * H + h) * DK + c];
+                    acc += gate ? pro_gate(x, A) : x;
                     sG[r * L::kLd + c] = acc;
                 }
             }
         }
         __syncthreads();
+        if (pro & GDR_PRO_L2NORM_QK) {  // one warp per row of K and of Q
+            const int lane = tid & 31;
+            for (int rr = tid >> 5; rr < 2 * n; rr += kThreads / 32) {
+                float* row = (rr < n ? sK : sQ) + (rr % n) * L::kLd;
+                float ss = 0.f;
+                for (int c = lane; c < DK; c += 32) ss = fmaf(row[c], row[c], ss);
+#pragma unroll
+                for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+                const float inv = pro_inv_norm(ss);
+                for (int c = lane; c < DK; c += 32) row[c] *= inv;
+            }
+            __syncthreads();
+        }
         if (MODE == GDR_DECAY_SCALAR) {
             for (int i = tid; i < n; i += kThreads) sTail[i] = expf(sG[(n - 1) * L::kLd] - sG[i * L::kLd]);
         }
@@ -250,7 +271,8 @@ template <typename Tin, typename Tout, int MODE, int DK>
 __global__ void __launch_bounds__(kRecWarps * 32)
 recurrent_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                       const float* __restrict__ g, const float* __restrict__ beta, const float* S0,
-                      Tout* __restrict__ o, float* S_T, int T, int H, int dv, float scale) {
+                      Tout* __restrict__ o, float* S_T, int T, int H, int dv, float scale, int pro,
+                      const float* __restrict__ gate_scale) {
     constexpr int NT = kRecWarps * 32;
     constexpr int NL = DK / 32;                                  // state columns per lane
     constexpr int NA = MODE == GDR_DECAY_CHANNEL ? DK : 1;       // decay factors per token
@@ -263,6 +285,8 @@ recurrent_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, cons
     const size_t bh = (size_t)b * H + h;
     const bool active = j < dv;
     auto tok_of = [&](int t) { return ((size_t)b * T + t) * H + h; };
+    const bool gate = (pro & GDR_PRO_GATE_SOFTPLUS) != 0;
+    const float A = (gate && gate_scale != nullptr) ? gate_scale[h] : 1.f;
 
     // one block's inputs, held in registers between its load and its store into shared memory:
     // thread tid holds k, q (and the channel gate's g) at flat index tid + NT m of the block, the
@@ -295,14 +319,34 @@ recurrent_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, cons
             const int idx = tid + NT * m, r = idx / DK, c = idx % DK;
             sK[r][c] = rk[m];
             sQ[r][c] = rq[m];
-            if (MODE == GDR_DECAY_CHANNEL) sAl[r][c] = expf(rg[m]);
+            if (MODE == GDR_DECAY_CHANNEL) sAl[r][c] = expf(gate ? pro_gate(rg[m], A) : rg[m]);
         }
         if (tid < kRecTB * kRecWarps) sV[tid / kRecWarps][tid % kRecWarps] = rv;
         if (tid < kRecTB) {
-            sB[tid] = rb;
-            if (MODE == GDR_DECAY_SCALAR) sAl[tid][0] = expf(rs);
+            sB[tid] = (pro & GDR_PRO_BETA_SIGMOID) ? pro_sigmoid(rb) : rb;
+            if (MODE == GDR_DECAY_SCALAR) sAl[tid][0] = expf(gate ? pro_gate(rs, A) : rs);
         }
     };
+    // L2 normalisation of the staged k and q vectors (rows past the sequence are zero and stay so):
+    // warp w takes tokens w and w + kRecWarps; each warp rescales only its own rows
+    auto normalise_block = [&]() {
+#pragma unroll
+        for (int r = warp; r < kRecTB; r += kRecWarps) {
+            float sk = 0.f, sq = 0.f;
+#pragma unroll
+            for (int i = 0; i < NL; ++i) {
+                sk = fmaf(sK[r][lane + 32 * i], sK[r][lane + 32 * i], sk);
+                sq = fmaf(sQ[r][lane + 32 * i], sQ[r][lane + 32 * i], sq);
+            }
+            const float nk = pro_inv_norm(warp_sum(sk)), nq = pro_inv_norm(warp_sum(sq));
+#pragma unroll
+            for (int i = 0; i < NL; ++i) {
+                sK[r][lane + 32 * i] *= nk;
+                sQ[r][lane + 32 * i] *= nq;
+            }
+        }
+    };
+    const bool norm = (pro & GDR_PRO_L2NORM_QK) != 0;
 
     float s[NL];
 #pragma unroll
@@ -310,6 +354,10 @@ recurrent_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, cons
     load_block(0);
     store_block();
     __syncthreads();
+    if (norm) {
+        normalise_block();
+        __syncthreads();
+    }
     for (int t0 = 0; t0 < T; t0 += kRecTB) {
         const int n = min(kRecTB, T - t0);
         if (t0 + kRecTB < T) load_block(t0 + kRecTB);  // in flight while this block is computed
@@ -350,6 +398,10 @@ recurrent_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, cons
             __syncthreads();  // every warp is done with this block
             store_block();
             __syncthreads();
+            if (norm) {
+                normalise_block();
+                __syncthreads();
+            }
         }
     }
     if (active && S_T != nullptr) {
@@ -364,7 +416,7 @@ cudaError_t launch_typed(const ChunkProblem& p, cudaStream_t stream) {
         dim3 grid((p.dv + kRecWarps - 1) / kRecWarps, p.H, p.B);
         recurrent_simt_kernel<Tin, Tout, MODE, DK><<<grid, kRecWarps * 32, 0, stream>>>(
             static_cast<const Tin*>(p.q), static_cast<const Tin*>(p.k), static_cast<const Tin*>(p.v), p.g, p.beta,
-            p.S0, static_cast<Tout*>(p.o), p.S_T, p.T, p.H, p.dv, p.scale);
+            p.S0, static_cast<Tout*>(p.o), p.S_T, p.T, p.H, p.dv, p.scale, p.prologue, p.gate_scale);
         profile_after_launch(stream);
         return cudaGetLastError();
     }
@@ -375,7 +427,7 @@ cudaError_t launch_typed(const ChunkProblem& p, cudaStream_t stream) {
     dim3 grid((p.dv + kDVS - 1) / kDVS, p.H, p.B);
     kern<<<grid, kThreads, smem, stream>>>(
         static_cast<const Tin*>(p.q), static_cast<const Tin*>(p.k), static_cast<const Tin*>(p.v), p.g, p.beta,
-        p.S0, static_cast<Tout*>(p.o), p.S_T, p.T, p.H, p.dv, p.scale);
+        p.S0, static_cast<Tout*>(p.o), p.S_T, p.T, p.H, p.dv, p.scale, p.prologue, p.gate_scale);
     profile_after_launch(stream);
     return cudaGetLastError();
 }

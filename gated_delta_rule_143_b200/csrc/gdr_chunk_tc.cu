@@ -36,6 +36,12 @@
 // terms k_r,d k_i,d 2^(Gamma_r,d - Gamma_i,d) (each factor <= 1) are added to the Gram on the CUDA
 // cores, in fp32, from a second copy of the bf16 tiles. Any g <= 0 is computed exactly.
 //
+// Prologue (gdr_chunk_fwd_ex): beta = sigmoid(logit) and g = -A softplus(a) are applied where the prep
+// loads beta and g. For the L2 normalisation of q and k the prep takes the inverse norms of the 128
+// rows of the [K; Q] tile after its TMA load and folds them in as row factors: into the hand-off
+// images and the operands it builds from the tiles, and into the epilogue of the Gram products,
+// which run on the raw bf16 tiles (x_ri * n_r * n_i), so no normalised copy is ever stored.
+//
 // Operands are fp16, not bf16: with bf16 operands the rounding of the intermediate factors alone
 // exceeded the 2e-2 * rms(o) parity bar; fp16 holds the bf16 inputs exactly at these ranges and
 // runs at the same tensor-core rate.
@@ -94,7 +100,17 @@ struct PrepArgs {
     const float* beta;
     int T, H, NC;
     int* status;
+    int pro;                  // gdr_prologue flags
+    const float* gate_scale;  // [H] or NULL
 };
+
+// Inverse L2 norms of the 128 rows of the [K; Q] tile (prologue GDR_PRO_L2NORM_QK), fp32 [128]:
+// in the slack after the scalar gate's 2^-Gamma table, or after the channel gate's strong lists.
+__host__ __device__ constexpr uint32_t nrm_off(int mode) {
+    return mode == GDR_DECAY_CHANNEL ? kPStrong + 1280 : kPInvE + 512;
+}
+static_assert(kPInvE + 512 + 512 <= kPrepBytesScalar, "norm table fits the scalar layout");
+static_assert(kPStrong + 1280 + 512 <= kPrepBytesChannel, "norm table fits the channel layout");
 
 struct PrepSmem {
     uint8_t* base;
@@ -246,7 +262,7 @@ __device__ void prep_init(const PrepSmem& ps, int lt) {
 // Computes the hand-off block of chunk c of head (b, h) into `out` (global memory). Executed by the
 // 256 threads of one pipeline (8 warps: TMEM lane quadrant q = warp & 3, column half hf = warp >> 2);
 // `it` counts the pipeline's previous tasks (mbarrier phase parity).
-template <int MODE>
+template <int MODE, bool PRO>
 __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv,
                            const PrepSmem& ps, int b, int h, int c, uint8_t* __restrict__ out, uint32_t it, int lt,
                            uint32_t& n_copies) {
@@ -271,6 +287,9 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
     const int c0 = c * kC;
     const int n = min(kC, T - c0);
     const size_t tok0 = ((size_t)b * T + c0) * H + h;  // chunk row r is token tok0 + r * H
+    // prologue steps: compiled only into the PRO instantiations, so the plain call's code is unchanged
+    const bool norm = PRO && (P.pro & GDR_PRO_L2NORM_QK) != 0, gate = PRO && (P.pro & GDR_PRO_GATE_SOFTPLUS) != 0;
+    float* sNrm = reinterpret_cast<float*>(sm + nrm_off(MODE));
 
     // ---- 1. TMA: K and Q into the two halves of the 128-row [K; Q] tile, V; beta and the
     //         cumulative log-decay (log2 units; rows past the tail repeat Gamma_{n-1}) meanwhile
@@ -285,13 +304,26 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
         tma_load_4d(sV + 8192, mv, 64, h, c0, b, barT);
     }
     if (lw == 7) {
-        sBeta[lane] = (lane < n) ? P.beta[tok0 + (size_t)lane * H] : 0.f;
-        sBeta[lane + 32] = (lane + 32 < n) ? P.beta[tok0 + (size_t)(lane + 32) * H] : 0.f;
+        const bool sig = PRO && (P.pro & GDR_PRO_BETA_SIGMOID) != 0;
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            const int r = lane + 32 * m;
+            float x = (r < n) ? P.beta[tok0 + (size_t)r * H] : 0.f;
+            if (sig && r < n) x = pro_sigmoid(x);
+            sBeta[r] = x;
+        }
     }
+    const float A = (gate && P.gate_scale != nullptr) ? P.gate_scale[h] : 1.f;
     if (MODE == GDR_DECAY_SCALAR) {
         if (lw == 6) {
-            float x0 = (lane < n) ? P.g[tok0 + (size_t)lane * H] * kLog2e : 0.f;
-            float x1 = (lane + 32 < n) ? P.g[tok0 + (size_t)(lane + 32) * H] * kLog2e : 0.f;
+            float x0 = (lane < n) ? P.g[tok0 + (size_t)lane * H] : 0.f;
+            float x1 = (lane + 32 < n) ? P.g[tok0 + (size_t)(lane + 32) * H] : 0.f;
+            if (gate) {
+                x0 = (lane < n) ? pro_gate(x0, A) : 0.f;
+                x1 = (lane + 32 < n) ? pro_gate(x1, A) : 0.f;
+            }
+            x0 *= kLog2e;
+            x1 *= kLog2e;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
@@ -316,6 +348,10 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
             float gv[kC];
 #pragma unroll
             for (int r = 0; r < kC; ++r) gv[r] = (r < n) ? P.g[(tok0 + (size_t)r * H) * kD + lt] : 0.f;
+            if (gate) {
+#pragma unroll
+                for (int r = 0; r < kC; ++r) gv[r] = (r < n) ? pro_gate(gv[r], A) : 0.f;
+            }
             float acc = 0.f, lo = 0.f, hi = 0.f;
 #pragma unroll
             for (int r = 0; r < kC; ++r) {
@@ -353,6 +389,23 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
     }
     mbar_wait(barT, par, P.status);
     const uint32_t tG = ps.tmem + kTG, tW = ps.tmem + kTW, tU = ps.tmem + kTU;
+    if (norm) {
+        // inverse L2 norms of the 128 tile rows (K rows 0-63, Q rows 64-127; rows past the tail are
+        // zero and get 0), two threads per row; the Gram products below run on the raw tiles and
+        // are rescaled in their epilogue
+        const int row = lt >> 1, half = lt & 1;
+        float ss = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float f[8];
+            unpack8bf(ld16(sKQ + kmajor_off(row, 64 * half + 8 * j, 128)), f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+        }
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        if (half == 0) sNrm[row] = pro_inv_norm(ss);
+        named_bar(ps.bar_id, kPrepThreads);
+    }
     // Gram products for the scalar gate / DeltaNet straight from the bf16 tiles
     if (MODE != GDR_DECAY_CHANNEL && lt == 0) {
         tc_fence_after();
@@ -384,6 +437,14 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
         float kx[8], qx[8];
         unpack8bf(ld16(sKQ + okr), kx);
         unpack8bf(ld16(sKQ + oqr), qx);
+        if (norm) {
+            const float nk = sNrm[r], nq = sNrm[kC + r];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                kx[e] *= nk;
+                qx[e] *= nq;
+            }
+        }
         float qg[8], kt[8];
         if (MODE == GDR_DECAY_NONE) {
 #pragma unroll
@@ -465,6 +526,11 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
         }
         const float br = sBeta[rr];
         tmem_ld_wait();
+        if (MODE != GDR_DECAY_CHANNEL && norm) {  // the Gram of the raw tiles, rescaled
+            const float nr = sNrm[q * 32 + lane];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] *= nr * sNrm[32 * hf + e];
+        }
         if (MODE == GDR_DECAY_CHANNEL && n_strong > 0) {
             // the strong channels' terms, left out of the tensor-core product: k_r,d k_i,d
             // 2^(Gamma_r,d - Gamma_i,d) (or q_r,d ...) from the bf16 copy of the tiles, fp32
@@ -478,14 +544,14 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
 #pragma unroll 1
                 for (int kk = 0; kk < cnt; ++kk) {
                     const int dch = sStrong[128 + 32 * w4 + kk];
-                    const float a = __bfloat162float(
-                        *reinterpret_cast<const __nv_bfloat16*>(sKQ2 + kmajor_off(row, dch, 128)));
+                    const float a = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                                        sKQ2 + kmajor_off(row, dch, 128))) * (norm ? sNrm[row] : 1.f);
                     const float Gr = sGam[rr * kD + dch];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int i = 32 * hf + e;
-                        const float ki = __bfloat162float(
-                            *reinterpret_cast<const __nv_bfloat16*>(sKQ2 + kmajor_off(i, dch, 128)));
+                        const float ki = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                                             sKQ2 + kmajor_off(i, dch, 128))) * (norm ? sNrm[i] : 1.f);
                         const float f = (i <= rr) ? fast_exp2(Gr - sGam[i * kD + dch]) : 0.f;
                         x[e] = fmaf(a * ki, f, x[e]);
                     }
@@ -537,9 +603,10 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
                     const int* fl = reinterpret_cast<const int*>(sm + kPStrong) + col0;
                     float kc[8];
                     unpack8bf(ld16(sm + kPKQ2 + kmajor_off(r, col0, 128)), kc);
+                    const float nk = norm ? sNrm[r] : 1.f;
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
-                        x[e] = fl[e] ? kc[e] * fast_exp2(sGam[r * kD + col0 + e])
+                        x[e] = fl[e] ? kc[e] * nk * fast_exp2(sGam[r * kD + col0 + e])
                                      : x[e] * fast_exp2(sGam[ref * kD + col0 + e]);
                 } else {
 #pragma unroll
@@ -547,8 +614,9 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
                 }
             } else {
                 unpack8bf(ld16(p), x);
-                if (!isv && MODE == GDR_DECAY_SCALAR) {
-                    const float fr = fast_exp2(sGam[r]);
+                if (!isv && (MODE == GDR_DECAY_SCALAR || norm)) {
+                    float fr = MODE == GDR_DECAY_SCALAR ? fast_exp2(sGam[r]) : 1.f;
+                    if (norm) fr *= sNrm[r];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) x[e] *= fr;
                 }
@@ -628,7 +696,7 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
 // At the start of each task the tiles of the CTA's next task are prefetched into L2. The scalar
 // and DeltaNet variants run at 96 registers per thread (no spills; measured 1-2.5 % faster than
 // the 128 two CTAs per SM would allow).
-template <int MODE>
+template <int MODE, bool PRO>
 __global__ void __maxnreg__(MODE == GDR_DECAY_CHANNEL ? 240 : 96)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                   const __grid_constant__ CUtensorMap mv, PrepArgs P, uint8_t* __restrict__ ws, int NCp, int n_tasks) {
@@ -666,7 +734,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
             tma_prefetch_l2_4d(&mv, 64, hn, cn * kC, bn);
         }
         uint8_t* out = ws + (size_t)t * kHandoffStride;
-        prep_chunk<MODE>(P, &mq, &mk, &mv, ps, b, h, c, out, it, lt, n_copies);
+        prep_chunk<MODE, PRO>(P, &mq, &mk, &mv, ps, b, h, c, out, it, lt, n_copies);
     }
     if (lt == 0) bulk_wait<0>();
     tc_fence_before();
@@ -1063,7 +1131,7 @@ struct RingArgs {
     int depth;         // ring slots per head: kRing, or every chunk from c1 on when c1 > 0
 };
 
-template <int MODE>
+template <int MODE, bool PRO>
 __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv, const PrepArgs& P,
                           const RingArgs& R, uint8_t* sm, uint32_t tbase, volatile int* abort) {
     __shared__ uint64_t pbars[2][4];
@@ -1100,7 +1168,7 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
         named_bar(ps.bar_id, kPrepThreads);
         if (!go[pipe]) break;
         uint8_t* out = R.ring + ((size_t)bh * R.depth + slot) * kHandoffStride;
-        prep_chunk<MODE>(P, mq, mk, mv, ps, bh / P.H, bh % P.H, c, out, it, lt, n_copies);
+        prep_chunk<MODE, PRO>(P, mq, mk, mv, ps, bh / P.H, bh % P.H, c, out, it, lt, n_copies);
         if (lt == 0) {  // every write of the block (generic stores before prep_chunk's last barrier, bulk stores)
             bulk_wait<0>();
             fence_proxy_async_global();
@@ -1110,7 +1178,7 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
     }
 }
 
-template <int MODE, typename Tout>
+template <int MODE, typename Tout, bool PRO>
 __global__ void __launch_bounds__(kStateThreads, 1)
 chunk_fused_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                    const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mo, PrepArgs P,
@@ -1135,7 +1203,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                              R.c1, R.depth};
         state_body<Tout>(&mo, A, bh, src, sm, tmem_base, &abort_flag);
     } else {
-        prep_role<MODE>(&mq, &mk, &mv, P, R, sm, tmem_base, &abort_flag);
+        prep_role<MODE, PRO>(&mq, &mk, &mv, P, R, sm, tmem_base, &abort_flag);
     }
     tc_fence_before();
     __syncthreads();
@@ -1176,17 +1244,17 @@ cudaError_t make_map(CUtensorMap* map, const void* base, CUtensorMapDataType typ
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int MODE>
+template <int MODE, bool PRO>
 cudaError_t launch_prep(const ChunkProblem& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                         int NC, int NCp, uint8_t* blocks, cudaStream_t stream) {
-    auto kern = chunk_prep_kernel<MODE>;
+    auto kern = chunk_prep_kernel<MODE, PRO>;
     const uint32_t smem = (MODE == GDR_DECAY_CHANNEL ? kPrepBytesChannel : kPrepBytesScalar) + 1024;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     // the whole unified L1 / shared array as shared memory, so that two pipelines fit per SM
     err = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (err != cudaSuccess) return err;
-    PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status};
+    PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status, p.prologue, p.gate_scale};
     int dev = 0, sms = 0;
     if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
     if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
@@ -1244,10 +1312,10 @@ size_t flag_bytes(int BH, int NC) {
     return ((size_t)(BH * (ring_depth(BH, NC) + 1) + 1) * sizeof(int) + 255) & ~size_t(255);
 }
 
-template <int MODE, typename Tout>
+template <int MODE, typename Tout, bool PRO>
 cudaError_t launch_fused(const ChunkProblem& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const CUtensorMap& mo, int NC, cudaStream_t stream) {
-    auto kern = chunk_fused_kernel<MODE, Tout>;
+    auto kern = chunk_fused_kernel<MODE, Tout, PRO>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFusedSmem);
     if (err != cudaSuccess) return err;
     int dev = 0, sms = 0, coop = 0, per_sm = 0;
@@ -1266,8 +1334,8 @@ cudaError_t launch_fused(const ChunkProblem& p, const CUtensorMap& mq, const CUt
     int* flags = reinterpret_cast<int*>(ring + ring_bytes(BH, NC));
     RingArgs R{ring, flags, flags + (size_t)BH * depth, flags + (size_t)BH * (depth + 1), ws, BH, c1, depth};
     if ((err = cudaMemsetAsync(flags, 0, flag_bytes(BH, NC), stream)) != cudaSuccess) return err;
-    if (c1 > 0 && (err = launch_prep<MODE>(p, mq, mk, mv, NC, c1, ws, stream)) != cudaSuccess) return err;
-    PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status};
+    if (c1 > 0 && (err = launch_prep<MODE, PRO>(p, mq, mk, mv, NC, c1, ws, stream)) != cudaSuccess) return err;
+    PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status, p.prologue, p.gate_scale};
     StateArgs A{p.S0, p.S_T, p.T, p.H, NC, p.scale, p.status};
     CUtensorMap aq = mq, ak = mk, av = mv, ao = mo;
     void* args[] = {&aq, &ak, &av, &ao, &P, &A, &R};
@@ -1275,6 +1343,28 @@ cudaError_t launch_fused(const ChunkProblem& p, const CUtensorMap& mq, const CUt
                                       kFusedSmem, stream);
     profile_after_launch(stream);
     return err;
+}
+
+template <bool PRO>
+cudaError_t launch_fused_mode(const ChunkProblem& p, const CUtensorMap& mq, const CUtensorMap& mk,
+                              const CUtensorMap& mv, const CUtensorMap& mo, int NC, cudaStream_t stream) {
+    const bool bf = p.o_dtype == GDR_BF16;
+    if (p.mode == GDR_DECAY_NONE)
+        return bf ? launch_fused<GDR_DECAY_NONE, __nv_bfloat16, PRO>(p, mq, mk, mv, mo, NC, stream)
+                  : launch_fused<GDR_DECAY_NONE, float, PRO>(p, mq, mk, mv, mo, NC, stream);
+    return bf ? launch_fused<GDR_DECAY_SCALAR, __nv_bfloat16, PRO>(p, mq, mk, mv, mo, NC, stream)
+              : launch_fused<GDR_DECAY_SCALAR, float, PRO>(p, mq, mk, mv, mo, NC, stream);
+}
+
+template <bool PRO>
+cudaError_t launch_prep_mode(const ChunkProblem& p, const CUtensorMap& mq, const CUtensorMap& mk,
+                             const CUtensorMap& mv, int NC, uint8_t* ws, cudaStream_t stream) {
+    switch (p.mode) {
+        case GDR_DECAY_NONE: return launch_prep<GDR_DECAY_NONE, PRO>(p, mq, mk, mv, NC, NC, ws, stream);
+        case GDR_DECAY_SCALAR: return launch_prep<GDR_DECAY_SCALAR, PRO>(p, mq, mk, mv, NC, NC, ws, stream);
+        case GDR_DECAY_CHANNEL: return launch_prep<GDR_DECAY_CHANNEL, PRO>(p, mq, mk, mv, NC, NC, ws, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
@@ -1314,21 +1404,12 @@ cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream) {
     else
         err = make_map(&mo, p.o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.B, p.T, p.H, 32);
     if (err != cudaSuccess) return err;
-    if (use_fused(p.B, p.H, p.mode)) {
-        const bool bf = p.o_dtype == GDR_BF16;
-        if (p.mode == GDR_DECAY_NONE)
-            return bf ? launch_fused<GDR_DECAY_NONE, __nv_bfloat16>(p, mq, mk, mv, mo, NC, stream)
-                      : launch_fused<GDR_DECAY_NONE, float>(p, mq, mk, mv, mo, NC, stream);
-        return bf ? launch_fused<GDR_DECAY_SCALAR, __nv_bfloat16>(p, mq, mk, mv, mo, NC, stream)
-                  : launch_fused<GDR_DECAY_SCALAR, float>(p, mq, mk, mv, mo, NC, stream);
-    }
+    if (use_fused(p.B, p.H, p.mode))
+        return p.prologue ? launch_fused_mode<true>(p, mq, mk, mv, mo, NC, stream)
+                          : launch_fused_mode<false>(p, mq, mk, mv, mo, NC, stream);
     uint8_t* ws = static_cast<uint8_t*>(p.workspace);
-    switch (p.mode) {
-        case GDR_DECAY_NONE: err = launch_prep<GDR_DECAY_NONE>(p, mq, mk, mv, NC, NC, ws, stream); break;
-        case GDR_DECAY_SCALAR: err = launch_prep<GDR_DECAY_SCALAR>(p, mq, mk, mv, NC, NC, ws, stream); break;
-        case GDR_DECAY_CHANNEL: err = launch_prep<GDR_DECAY_CHANNEL>(p, mq, mk, mv, NC, NC, ws, stream); break;
-        default: return cudaErrorInvalidValue;
-    }
+    err = p.prologue ? launch_prep_mode<true>(p, mq, mk, mv, NC, ws, stream)
+                     : launch_prep_mode<false>(p, mq, mk, mv, NC, ws, stream);
     if (err != cudaSuccess) return err;
     if (p.o_dtype == GDR_BF16) return launch_state<__nv_bfloat16>(p, mo, NC, stream);
     return launch_state<float>(p, mo, NC, stream);

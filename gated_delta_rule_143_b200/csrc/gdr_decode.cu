@@ -55,7 +55,7 @@ template <typename Tin, typename Tout, int MODE, int DK>
 __global__ void __launch_bounds__(kThreads)
 decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
               const float* __restrict__ g, const float* __restrict__ beta, float* __restrict__ S,
-              Tout* __restrict__ o, int dv, float scale) {
+              Tout* __restrict__ o, int dv, float scale, int H, int pro, const float* __restrict__ gate_scale) {
     constexpr int EPL = DK / kLanesPerRow;  // floats of a row per lane
     const size_t bh = blockIdx.x;
     const int sub = threadIdx.x & (kLanesPerRow - 1);
@@ -65,11 +65,31 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
     float kr[EPL], qr[EPL], al[EPL];
     load_vec(k + bh * DK + c0, kr);
     load_vec(q + bh * DK + c0, qr);
+    if (pro & GDR_PRO_L2NORM_QK) {  // the 8 lanes of a row group hold all of k and q
+        float sk = 0.f, sq = 0.f;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            sk = fmaf(kr[i], kr[i], sk);
+            sq = fmaf(qr[i], qr[i], sq);
+        }
+        const float nk = pro_inv_norm(group8_sum(sk)), nq = pro_inv_norm(group8_sum(sq));
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            kr[i] *= nk;
+            qr[i] *= nq;
+        }
+    }
+    const bool gate = (pro & GDR_PRO_GATE_SOFTPLUS) != 0;
+    const float A = (gate && gate_scale != nullptr) ? gate_scale[bh % (size_t)H] : 1.f;
     if (MODE == GDR_DECAY_CHANNEL) {
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) al[i] = expf(g[bh * DK + c0 + i]);
+        for (int i = 0; i < EPL; ++i) {
+            const float x = g[bh * DK + c0 + i];
+            al[i] = expf(gate ? pro_gate(x, A) : x);
+        }
     } else {
-        const float a = (MODE == GDR_DECAY_SCALAR) ? expf(g[bh]) : 1.f;
+        float a = 1.f;
+        if (MODE == GDR_DECAY_SCALAR) a = expf(gate ? pro_gate(g[bh], A) : g[bh]);
 #pragma unroll
         for (int i = 0; i < EPL; ++i) al[i] = a;
     }
@@ -77,7 +97,7 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
 #pragma unroll
     for (int i = 0; i < EPL; ++i) kq = fmaf(kr[i], qr[i], kq);
     kq = group8_sum(kq);
-    const float bt = beta[bh];
+    const float bt = (pro & GDR_PRO_BETA_SIGMOID) ? pro_sigmoid(beta[bh]) : beta[bh];
     float* Sh = S + bh * (size_t)dv * DK;
 
     // Loop bounds are uniform across a warp (its 4 rows share `jb`), so every lane reaches the
@@ -134,10 +154,10 @@ cudaError_t launch_mode(const DecodeProblem& p, cudaStream_t stream) {
     const Tin* v = static_cast<const Tin*>(p.v);
     Tout* o = static_cast<Tout*>(p.o);
     switch (p.dk) {
-        case 32: decode_kernel<Tin, Tout, MODE, 32><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale); break;
-        case 64: decode_kernel<Tin, Tout, MODE, 64><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale); break;
-        case 128: decode_kernel<Tin, Tout, MODE, 128><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale); break;
-        case 256: decode_kernel<Tin, Tout, MODE, 256><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale); break;
+        case 32: decode_kernel<Tin, Tout, MODE, 32><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale, p.H, p.prologue, p.gate_scale); break;
+        case 64: decode_kernel<Tin, Tout, MODE, 64><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale, p.H, p.prologue, p.gate_scale); break;
+        case 128: decode_kernel<Tin, Tout, MODE, 128><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale, p.H, p.prologue, p.gate_scale); break;
+        case 256: decode_kernel<Tin, Tout, MODE, 256><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale, p.H, p.prologue, p.gate_scale); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();

@@ -26,6 +26,8 @@ struct ChunkProblem {
     size_t workspace_bytes;
     int* status;  // device status word (first error wins)
     float scale;
+    int prologue;             // gdr_prologue flags: steps of the mixer layer done on the inputs in-kernel
+    const float* gate_scale;  // [H] A of g = -A softplus(a) (GDR_PRO_GATE_SOFTPLUS), NULL = 1
 };
 
 struct DecodeProblem {
@@ -39,7 +41,16 @@ struct DecodeProblem {
     int B, H, dk, dv, mode, dtype, o_dtype;
     int* status;
     float scale;
+    int prologue;             // as ChunkProblem
+    const float* gate_scale;
 };
+
+// The prologue's elementwise steps (gdr_prologue), in fp32 with CUDA's math functions.
+__device__ __forceinline__ float pro_sigmoid(float x) { return 1.f / (1.f + expf(-x)); }
+// g = -A softplus(a), softplus(a) = max(a, 0) + log(1 + e^-|a|)
+__device__ __forceinline__ float pro_gate(float a, float A) { return -A * (fmaxf(a, 0.f) + log1pf(expf(-fabsf(a)))); }
+// 1 / |x| from the sum of squares; an all-zero vector (or one whose squares underflow) stays zero
+__device__ __forceinline__ float pro_inv_norm(float sum_sq) { return sum_sq > 0.f ? rsqrtf(sum_sq) : 0.f; }
 
 // Device status codes written by kernels (mirror gdr_status).
 constexpr int kStatusTimeout = GDR_ERR_TIMEOUT;

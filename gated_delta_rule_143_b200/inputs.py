@@ -154,6 +154,56 @@ def make_chunk_inputs(
     }
 
 
+def make_raw_chunk_inputs(
+    B: int,
+    T: int,
+    H: int,
+    dk: int,
+    dv: int,
+    mode: str,
+    dtype: str,
+    seed: int,
+    s0_std: Optional[float] = None,
+) -> Dict[str, Optional[torch.Tensor]]:
+    """Seeded CPU tensors for a chunked forward whose prologue runs in the kernels: the draws
+    before any squashing or normalisation.
+
+    ``q, k`` [B,T,H,dk]: N(0, 1) vectors, each times a length drawn from U(0.25, 4) (so that
+    their norms differ); ``v`` [B,T,H,dv] N(0, 1); ``beta`` [B,T,H] fp32 logits N(0, 1);
+    ``g`` fp32 gate logits N(0, 1) ([B,T,H] scalar, [B,T,H,dk] channel, None for "none");
+    ``gate_scale`` [H] fp32 from U(0.02, 1); ``S0`` as in ``make_chunk_inputs``. Draw order:
+    q, k, v, beta-logit, g-logit, S0, the q lengths, the k lengths, gate_scale.
+    """
+    if mode not in DECAY_MODES:
+        raise ValueError(f"unknown decay mode {mode!r}")
+    gen = torch.Generator().manual_seed(int(seed))
+    q = torch.randn(B, T, H, dk, generator=gen)
+    k = torch.randn(B, T, H, dk, generator=gen)
+    v = torch.randn(B, T, H, dv, generator=gen)
+    beta_logit = torch.randn(B, T, H, generator=gen)
+    a = None
+    if mode == "scalar":
+        a = torch.randn(B, T, H, generator=gen)
+    elif mode == "channel":
+        a = torch.randn(B, T, H, dk, generator=gen)
+    S0 = None
+    if s0_std is not None:
+        S0 = s0_std * torch.randn(B, H, dv, dk, generator=gen)
+    q = q * (0.25 + 3.75 * torch.rand(B, T, H, 1, generator=gen))
+    k = k * (0.25 + 3.75 * torch.rand(B, T, H, 1, generator=gen))
+    gate_scale = 0.02 + 0.98 * torch.rand(H, generator=gen)
+    td = _torch_dtype(dtype)
+    return {
+        "q": q.to(td).contiguous(),
+        "k": k.to(td).contiguous(),
+        "v": v.to(td).contiguous(),
+        "beta": beta_logit.contiguous(),
+        "g": None if a is None else a.contiguous(),
+        "S0": None if S0 is None else S0.contiguous(),
+        "gate_scale": gate_scale.contiguous(),
+    }
+
+
 def workload_inputs(w: ChunkWorkload, seed: Optional[int] = None) -> Dict[str, Optional[torch.Tensor]]:
     """Inputs of a named chunked workload (its fixed seed unless overridden)."""
     s = WORKLOAD_SEEDS.get(w.name, 0) if seed is None else seed

@@ -123,6 +123,43 @@ size_t gdr_chunk_fwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int 
                                      int dtype, int o_dtype);
 
 /*
+ * gdr_chunk_fwd_ex -- gdr_chunk_fwd with the mixer layer's input steps done inside the kernels.
+ *
+ * Defined by: "Linear Attention & DeltaNet", minimal pseudocode (recurrent reference form): before
+ * the recurrence, q and k pass through a feature map, the write strength is beta = sigmoid of a
+ * projection, and the decay gate is a squashed projection. Each step below is applied, in fp32, to
+ * the values as the kernels read them, so that no separate pass writes and re-reads them:
+ *
+ *   GDR_PRO_L2NORM_QK     q and k hold raw vectors: each (b, t, h) vector of q and of k is divided
+ *                         by its Euclidean norm (no epsilon). An all-zero vector stays zero, and so
+ *                         does one whose squared norm underflows fp32 (norm below about 1e-19).
+ *   GDR_PRO_BETA_SIGMOID  beta holds logits x; the write strength is 1 / (1 + e^-x).
+ *   GDR_PRO_GATE_SOFTPLUS g holds gate logits a (same shape as g); the log-decay is
+ *                         g = -A_h softplus(a) = -A_h log(1 + e^a), with A = gate_scale [H] fp32
+ *                         (NULL: A_h = 1). A_h >= 0 keeps g <= 0. A_h = 0.05 gives the decay
+ *                         exp(-0.05 softplus(.)) of the small Gated DeltaNet workload; A_h = 1 with
+ *                         a = -x gives alpha = sigmoid(x), the pseudocode's gate. Needs mode SCALAR
+ *                         or CHANNEL.
+ *
+ *   prologue    bitwise OR of gdr_prologue flags (0 = gdr_chunk_fwd).
+ *   gate_scale  device pointer, [H] fp32, 16-byte aligned, or NULL; read only with
+ *               GDR_PRO_GATE_SOFTPLUS.
+ * Every other argument, the paths and the errors are as gdr_chunk_fwd; a prologue bit outside the
+ * three above is GDR_ERR_INVALID_ARG. The workspace size and the plan do not depend on `prologue`.
+ */
+typedef enum {
+    GDR_PRO_NONE = 0,
+    GDR_PRO_L2NORM_QK = 1,
+    GDR_PRO_BETA_SIGMOID = 2,
+    GDR_PRO_GATE_SOFTPLUS = 4
+} gdr_prologue;
+
+int gdr_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                     const float* S0, void* o, float* S_T, int B, int T, int H, int d_k, int d_v,
+                     int chunk, int mode, int dtype, int o_dtype, int prologue,
+                     const float* gate_scale, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * gdr_decode_step -- one recurrent step for a batch of states (the decoding view).
  *
  * Defined by: "linear attention and its gated descendants", Recurrent Linear Attention for
@@ -141,6 +178,12 @@ size_t gdr_chunk_fwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int 
 int gdr_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta,
                     float* S, void* o, int B, int H, int d_k, int d_v, int mode, int dtype,
                     int o_dtype, void* stream);
+
+/* gdr_decode_step with the prologue steps of gdr_chunk_fwd_ex applied to q, k (per (b, h) vector),
+ * beta and g in-kernel; arguments and errors otherwise as gdr_decode_step. */
+int gdr_decode_step_ex(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                       float* S, void* o, int B, int H, int d_k, int d_v, int mode, int dtype,
+                       int o_dtype, int prologue, const float* gate_scale, void* stream);
 
 /* Number of kernel launches one gdr_chunk_fwd call makes for this problem (0 if it would be
  * rejected). Host-only. */

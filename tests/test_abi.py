@@ -141,3 +141,26 @@ def test_host_entry_point_validates_on_host():
                               None, 0, None)
     assert rc == -4
     assert b"staging" in L.gdr_last_error()
+
+
+@pytest.mark.parametrize("pro,mode,gs,code", [
+    (8, 1, None, -1),             # unknown prologue bit
+    (4, 0, None, -1),             # gate logits without a gated decay mode
+    (4, 1, (7 << 24) + 4, -3),    # misaligned gate_scale
+    (4, 1, (1 << 24) + 64, -1),   # the output o placed over gate_scale
+])
+def test_chunk_fwd_ex_validates_prologue_on_host(pro, mode, gs, code):
+    M = 1 << 24
+    o = 6 * M
+    if code == -1 and gs is not None:
+        o = gs  # o starts at gate_scale: an output overlapping an input
+    rc = _lib.lib().gdr_chunk_fwd_ex(1 * M, 2 * M, 3 * M, 4 * M, 5 * M, None, o, None, 1, 64, 1, 128, 128, 64, mode, 1, 0,
+                                     pro, gs, None, 0, None)
+    assert rc == code
+    assert len(_lib.lib().gdr_last_error()) > 0
+
+
+@pytest.mark.parametrize("pro,mode,code", [(16, 1, -1), (4, 0, -1), (3, 5, -1)])
+def test_decode_ex_validates_prologue_on_host(pro, mode, code):
+    rc = _lib.lib().gdr_decode_step_ex(16, 32, 48, 64, 80, 1 << 20, 1 << 21, 2, 2, 128, 128, mode, 1, 0, pro, None, None)
+    assert rc == code
