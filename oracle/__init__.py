@@ -50,6 +50,10 @@ def _load():
                 ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
                 ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
             lib.gdr_oracle_max_threads.restype = ctypes.c_int
+            lib.gdr_oracle_backward.restype = ctypes.c_int
+            lib.gdr_oracle_backward.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 4 + [
+                ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_double] + [
+                ctypes.c_void_p] * 8 + [ctypes.c_int]
             _lib = lib
     return _lib
 
@@ -116,6 +120,52 @@ def recurrent(q, k, v, g, beta, mode: str, S0=None, *, erase=None, write=None,
     if rc != 0:
         raise RuntimeError(f"oracle failed with status {rc}")
     return o, st
+
+
+def backward(q, k, v, g, beta, mode: str, dO, S0=None, dS_T=None, *, scale: Optional[float] = None,
+             f64_inputs: bool = False, threads: int = 0):
+    """Gradients of the mixer recurrence (``recurrent`` with erase = write = beta) for a loss
+    whose gradients with respect to o [B,T,H,dv] and S_T [B,H,dv,dk] are ``dO`` and ``dS_T``
+    (None: zero). Reverse-mode differentiation of the token recurrence in float64 (see
+    ``gdr_oracle_backward`` in ``gdr_oracle.c``). Returns a dict of float64 arrays: ``dq``, ``dk``
+    [B,T,H,dk], ``dv`` [B,T,H,dv], ``dbeta`` [B,T,H], ``dg`` (shape of g; None for "none") and
+    ``dS0`` [B,H,dv,dk]."""
+    lib = _load()
+    if mode not in _MODES:
+        raise ValueError(f"unknown decay mode {mode!r}")
+    qa, ka, va = _arr(q, f64_inputs), _arr(k, f64_inputs), _arr(v, f64_inputs)
+    B, T, H, dk = qa.shape
+    dv = va.shape[-1]
+    if ka.shape != (B, T, H, dk) or va.shape != (B, T, H, dv):
+        raise ValueError("q, k, v shapes disagree")
+    ba = _arr(beta, f64_inputs)
+    if ba.shape != (B, T, H):
+        raise ValueError("beta must be [B,T,H]")
+    ga = None
+    if mode != "none":
+        ga = _arr(g, f64_inputs)
+        want = (B, T, H) if mode == "scalar" else (B, T, H, dk)
+        if ga.shape != want:
+            raise ValueError(f"g must be {want} for mode {mode}")
+    s0 = None if S0 is None else _arr(S0, True)
+    do = _arr(dO, True)
+    if do.shape != (B, T, H, dv):
+        raise ValueError("dO must be [B,T,H,dv]")
+    dst = None if dS_T is None else _arr(dS_T, True)
+    for name, a in (("S0", s0), ("dS_T", dst)):
+        if a is not None and a.shape != (B, H, dv, dk):
+            raise ValueError(f"{name} must be [B,H,dv,dk]")
+    out = {"dq": np.empty((B, T, H, dk)), "dk": np.empty((B, T, H, dk)), "dv": np.empty((B, T, H, dv)),
+           "dbeta": np.empty((B, T, H)), "dg": None if ga is None else np.empty(ga.shape),
+           "dS0": np.empty((B, H, dv, dk))}
+    sc = (1.0 / np.sqrt(dk)) if scale is None else float(scale)
+    rc = lib.gdr_oracle_backward(B, T, H, dk, dv, _ptr(qa), _ptr(ka), _ptr(va), _ptr(ga), _MODES[mode], _ptr(ba),
+                                 int(bool(f64_inputs)), _ptr(s0), sc, _ptr(do), _ptr(dst), _ptr(out["dq"]),
+                                 _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
+                                 _ptr(out["dS0"]), int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle backward failed with status {rc}")
+    return out
 
 
 def decode_step(q, k, v, g, beta, S, mode: str, *, scale: Optional[float] = None,

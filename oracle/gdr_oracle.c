@@ -140,3 +140,144 @@ int gdr_oracle_recurrent(int B, int T, int H, int dk, int dv,
     }
     return status;
 }
+
+/*
+ * Gradients of the mixer recurrence (e_t = w_t = beta_t) for a loss whose gradients with respect
+ * to the outputs are dO [B,T,H,d_v] and dS_T [B,H,d_v,d_k] (NULL: zero). Reverse-mode
+ * differentiation of the row form above, written out step by step: a forward sweep keeps the state
+ * before every token, then the tokens are taken from the last to the first. With ds the gradient
+ * of row j of the state after token t, the forward steps
+ *     s_bar = s (.) a ;  p = s_bar . k ;  delta = beta (v_j - p) ;  s' = s_bar + delta k ;
+ *     o_j = scale (s' . q)
+ * give, in reverse order,
+ *     ds'    = ds + scale do_j q            dq += scale do_j s'
+ *     ddelta = ds' . k                      dk += delta ds'
+ *     dbeta += ddelta (v_j - p)             dv_j = beta ddelta
+ *     dp     = -beta ddelta
+ *     ds_bar = ds' + dp k                   dk += dp s_bar
+ *     ds     = ds_bar (.) a                 dg += ds_bar (.) s_bar   (a = exp(g): da/dg = a)
+ * summed over the rows j for dq, dk, dbeta and dg (over the channels too for the scalar gate).
+ * Outputs: dq, dk [B,T,H,d_k]; dv [B,T,H,d_v]; dbeta [B,T,H]; dg [B,T,H] (scalar) or [B,T,H,d_k]
+ * (channel), unused for NONE (may be NULL); dS0 [B,H,d_v,d_k] or NULL. All fp64.
+ * Returns 0, -1 on an invalid argument, -2 on allocation failure.
+ */
+int gdr_oracle_backward(int B, int T, int H, int dk, int dv,
+                        const void* q, const void* k, const void* v, const void* g, int mode,
+                        const void* beta, int in_f64, const double* S0, double scale,
+                        const double* dO, const double* dST,
+                        double* dq, double* dk_out, double* dv_out, double* dg, double* dbeta,
+                        double* dS0, int nthreads) {
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+    if (mode != ORACLE_MODE_NONE && mode != ORACLE_MODE_SCALAR && mode != ORACLE_MODE_CHANNEL) return -1;
+    if (mode != ORACLE_MODE_NONE && (g == NULL || dg == NULL)) return -1;
+    if (T > 0 && (q == NULL || k == NULL || v == NULL || beta == NULL || dO == NULL || dq == NULL ||
+                  dk_out == NULL || dv_out == NULL || dbeta == NULL))
+        return -1;
+    const long nhead = (long)B * H;
+    int status = 0;
+    if (nthreads <= 0) nthreads = gdr_oracle_max_threads();
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long bh = 0; bh < nhead; ++bh) {
+        const int h = (int)(bh % H);
+        const int b = (int)(bh / H);
+        const size_t sz = (size_t)dv * dk;
+        double* hist = (double*)malloc(sizeof(double) * sz * (size_t)(T > 0 ? T : 1));
+        double* s = (double*)malloc(sizeof(double) * sz);
+        double* ds = (double*)malloc(sizeof(double) * sz);
+        double* vec = (double*)malloc(sizeof(double) * (size_t)dk * 8);
+        if (!hist || !s || !ds || !vec) {
+            free(hist); free(s); free(ds); free(vec);
+#pragma omp atomic write
+            status = -2;
+            continue;
+        }
+        double *kt = vec, *qt = vec + dk, *at = vec + 2 * dk, *sbar = vec + 3 * dk, *dsp = vec + 4 * dk;
+        double *gq = vec + 5 * dk, *gk = vec + 6 * dk, *gg = vec + 7 * dk;
+        for (size_t i = 0; i < sz; ++i) {
+            s[i] = S0 ? S0[(size_t)bh * sz + i] : 0.0;
+            ds[i] = dST ? dST[(size_t)bh * sz + i] : 0.0;
+        }
+        /* forward sweep: the state before each token */
+        for (int t = 0; t < T; ++t) {
+            const size_t tok = ((size_t)b * T + t) * H + h;
+            memcpy(hist + (size_t)t * sz, s, sizeof(double) * sz);
+            const double bt = ld_in(beta, tok, in_f64);
+            for (int c = 0; c < dk; ++c) {
+                kt[c] = ld_in(k, tok * dk + c, in_f64);
+                if (mode == ORACLE_MODE_NONE) at[c] = 1.0;
+                else if (mode == ORACLE_MODE_SCALAR) at[c] = exp(ld_in(g, tok, in_f64));
+                else at[c] = exp(ld_in(g, tok * dk + c, in_f64));
+            }
+            for (int j = 0; j < dv; ++j) {
+                double* sj = s + (size_t)j * dk;
+                double p = 0.0;
+                for (int c = 0; c < dk; ++c) {
+                    sj[c] *= at[c];
+                    p += sj[c] * kt[c];
+                }
+                const double delta = bt * (ld_in(v, tok * dv + j, in_f64) - p);
+                for (int c = 0; c < dk; ++c) sj[c] += delta * kt[c];
+            }
+        }
+        /* reverse sweep */
+        for (int t = T - 1; t >= 0; --t) {
+            const size_t tok = ((size_t)b * T + t) * H + h;
+            const double bt = ld_in(beta, tok, in_f64);
+            for (int c = 0; c < dk; ++c) {
+                kt[c] = ld_in(k, tok * dk + c, in_f64);
+                qt[c] = ld_in(q, tok * dk + c, in_f64);
+                if (mode == ORACLE_MODE_NONE) at[c] = 1.0;
+                else if (mode == ORACLE_MODE_SCALAR) at[c] = exp(ld_in(g, tok, in_f64));
+                else at[c] = exp(ld_in(g, tok * dk + c, in_f64));
+                gq[c] = gk[c] = gg[c] = 0.0;
+            }
+            double gb = 0.0;
+            for (int j = 0; j < dv; ++j) {
+                const double* sj = hist + (size_t)t * sz + (size_t)j * dk;
+                double* dsj = ds + (size_t)j * dk;
+                const double vj = ld_in(v, tok * dv + j, in_f64);
+                const double doj = dO[tok * dv + j];
+                double p = 0.0;
+                for (int c = 0; c < dk; ++c) {
+                    sbar[c] = sj[c] * at[c];
+                    p += sbar[c] * kt[c];
+                }
+                const double delta = bt * (vj - p);
+                double ddelta = 0.0;
+                for (int c = 0; c < dk; ++c) {
+                    const double spc = sbar[c] + delta * kt[c];
+                    dsp[c] = dsj[c] + scale * doj * qt[c];
+                    gq[c] += scale * doj * spc;
+                    gk[c] += delta * dsp[c];
+                    ddelta += dsp[c] * kt[c];
+                }
+                gb += ddelta * (vj - p);
+                dv_out[tok * dv + j] = bt * ddelta;
+                const double dp = -bt * ddelta;
+                for (int c = 0; c < dk; ++c) {
+                    const double dsb = dsp[c] + dp * kt[c];
+                    gk[c] += dp * sbar[c];
+                    gg[c] += dsb * sbar[c];
+                    dsj[c] = dsb * at[c];
+                }
+            }
+            for (int c = 0; c < dk; ++c) {
+                dq[tok * dk + c] = gq[c];
+                dk_out[tok * dk + c] = gk[c];
+            }
+            dbeta[tok] = gb;
+            if (mode == ORACLE_MODE_SCALAR) {
+                double sum = 0.0;
+                for (int c = 0; c < dk; ++c) sum += gg[c];
+                dg[tok] = sum;
+            } else if (mode == ORACLE_MODE_CHANNEL) {
+                for (int c = 0; c < dk; ++c) dg[tok * dk + c] = gg[c];
+            }
+        }
+        if (dS0)
+            for (size_t i = 0; i < sz; ++i) dS0[(size_t)bh * sz + i] = ds[i];
+        free(hist); free(s); free(ds); free(vec);
+    }
+    return status;
+}

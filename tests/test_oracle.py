@@ -456,3 +456,62 @@ def test_prologue_then_recurrence_exact_recall_with_raw_keys():
     for i in range(T):
         ki = k32[0, i, 0] / np.linalg.norm(k32[0, i, 0])
         np.testing.assert_allclose(S[0, 0] @ ki, v[0, i, 0], rtol=0, atol=1e-12)
+
+
+# ---- the backward pass (reverse-mode gradients of the recurrence)
+
+def _loss_and_grads(x, mode, R1, R2, S0):
+    o, st = oracle.recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], mode, S0=S0, f64_inputs=True)
+    return float(np.sum(o * R1) + np.sum(st * R2))
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("with_dst", [True, False])
+def test_backward_matches_central_differences(mode, with_dst):
+    """Every gradient (q, k, v, g, beta, S0) of L = <o, R1> + <S_T, R2> against central finite
+    differences of the forward oracle, h = 1e-6, on a tiny problem (error O(h^2) + rounding)."""
+    rng = np.random.default_rng(21 + MODES.index(mode) + (10 if with_dst else 0))
+    B, T, H, dk, dv = 1, 5, 2, 3, 2
+    q, k, v, g, beta = _rand_problem(rng, B, T, H, dk, dv, mode, unit_keys=False, g_scale=0.7)
+    S0 = 0.5 * rng.standard_normal((B, H, dv, dk))
+    R1 = rng.standard_normal((B, T, H, dv))
+    R2 = rng.standard_normal((B, H, dv, dk)) if with_dst else np.zeros((B, H, dv, dk))
+    x = {"q": q, "k": k, "v": v, "g": g, "beta": beta}
+    grads = oracle.backward(q, k, v, g, beta, mode, R1, S0=S0, dS_T=R2 if with_dst else None, f64_inputs=True)
+    h = 1e-6
+    targets = [("q", "dq"), ("k", "dk"), ("v", "dv"), ("beta", "dbeta")] + ([("g", "dg")] if mode != "none" else [])
+    for name, gname in targets:
+        base = x[name]
+        fd = np.zeros_like(base)
+        for idx in np.ndindex(base.shape):
+            xp = dict(x); xm = dict(x)
+            xp[name] = base.copy(); xm[name] = base.copy()
+            xp[name][idx] += h
+            xm[name][idx] -= h
+            fd[idx] = (_loss_and_grads(xp, mode, R1, R2, S0) - _loss_and_grads(xm, mode, R1, R2, S0)) / (2 * h)
+        np.testing.assert_allclose(grads[gname], fd, rtol=1e-6, atol=1e-7, err_msg=name)
+    fd = np.zeros_like(S0)
+    for idx in np.ndindex(S0.shape):
+        sp = S0.copy(); sm = S0.copy()
+        sp[idx] += h
+        sm[idx] -= h
+        fd[idx] = (_loss_and_grads(x, mode, R1, R2, sp) - _loss_and_grads(x, mode, R1, R2, sm)) / (2 * h)
+    np.testing.assert_allclose(grads["dS0"], fd, rtol=1e-6, atol=1e-7, err_msg="S0")
+
+
+def test_backward_no_write_closed_form():
+    """beta = 0 and alpha = 1: the state stays S0, o_t = scale S0 q_t, so dq_t = scale S0^T do_t,
+    dk = dv = 0 and dS0 = dS_T + scale sum_t do_t q_t^T (closed forms)."""
+    rng = np.random.default_rng(33)
+    B, T, H, dk, dv = 2, 7, 2, 4, 3
+    q, k, v, _, _ = _rand_problem(rng, B, T, H, dk, dv, "none")
+    beta = np.zeros((B, T, H))
+    S0 = rng.standard_normal((B, H, dv, dk))
+    dO = rng.standard_normal((B, T, H, dv))
+    dST = rng.standard_normal((B, H, dv, dk))
+    gr = oracle.backward(q, k, v, None, beta, "none", dO, S0=S0, dS_T=dST, f64_inputs=True)
+    sc = 1.0 / np.sqrt(dk)
+    np.testing.assert_allclose(gr["dq"], sc * np.einsum("bhjc,bthj->bthc", S0, dO), rtol=1e-13, atol=1e-13)
+    assert np.all(gr["dk"] == 0) and np.all(gr["dv"] == 0)
+    np.testing.assert_allclose(gr["dS0"], dST + sc * np.einsum("bthj,bthc->bhjc", dO, q), rtol=1e-13, atol=1e-13)
+    assert gr["dg"] is None
