@@ -466,6 +466,7 @@ def run_ours(args):
     dec = bench_decode(args, dev, peaks, world)
     others = bench_workloads(args, dev, peaks) if world == 1 else None
     pro = bench_prologue(args, w, dev, ws, o, st, stream, world, rank, ms_step)
+    bwd = bench_backward(args, w, sets[0], dev, peaks, stream, world)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -483,6 +484,7 @@ def run_ours(args):
         "o_bf16": o_bf16,
         "decode": dec,
         "prologue": pro,
+        "backward": bwd,
     }
     if others is not None:
         line["extra"] = {"workloads": others}
@@ -537,6 +539,37 @@ def bench_prologue(args, w, dev, ws, o, st, stream, world, rank, ms_plain):
             "steps": n, "fused_gpu_launches_per_step": gdr_kernels_per_step(w),
             "note": "raw q/k (unnormalised, bf16), beta logits, gate logits and A [H]; fused = "
                     "l2norm_qk + beta_sigmoid + gate_softplus in the library's kernels"}
+
+
+def bench_backward(args, w, x, dev, peaks, stream, world):
+    """gdr_chunk_bwd on the same workload (all gradients, dS0 included): device time per call and
+    the bytes its two kernels must move (inputs and dO read twice, the per-token state history
+    written once and read once, gradients written)."""
+    import gated_delta_rule_143_b200 as gdr
+
+    gen = torch.Generator().manual_seed(4242)
+    dO = torch.randn(w.B, w.T, w.H, w.dv, generator=gen).to(torch.bfloat16).to(dev)
+    ws_n = gdr._lib.lib().gdr_chunk_bwd_workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, gdr._mode(w.mode), 1)
+    ws_b = torch.empty(ws_n, dtype=torch.uint8, device=dev)
+
+    def step(i=0):
+        gdr.chunk_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], dO, S0=x["S0"], mode=w.mode, workspace=ws_b)
+
+    n = max(3, min(args.steps, 10))
+    ms = max_over_ranks(time_device(step, n, min(args.warmup, 3), world, stream), world) / n
+    gdr.sync_status()
+    ntok = w.B * w.T * w.H
+    hist = w.B * w.H * w.T * w.dv * w.dk * 4
+    gbytes = w.dk * 4 if w.mode == "channel" else (4 if w.mode == "scalar" else 0)
+    nbytes = (2 * ntok * (2 * w.dk * 2 + w.dv * 2 + 4 + gbytes) + ntok * w.dv * 2  # q, k, v, beta, g twice; dO
+              + 2 * hist  # the state history, written and read
+              + ntok * (2 * w.dk + w.dv + 1) * 4 + ntok * gbytes + w.B * w.H * w.dv * w.dk * 4)  # gradients
+    del ws_b
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"ms_per_call": round(ms, 4), "tokens_per_s": round(job_throughput(w.B * w.T, ms, world), 1),
+            "calls": n, "gpu_launches_per_call": 2, "bytes_per_call": nbytes,
+            "achieved_gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+            "note": "fp32 CUDA-core backward: state-history kernel + reverse kernel, one CTA per head"}
 
 
 def gdr_kernels_per_step(w):

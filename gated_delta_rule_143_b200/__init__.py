@@ -25,7 +25,7 @@ import torch
 from ._lib import (DECAY_MODES, DTYPE_BF16, DTYPE_F32, PLANS, PRO_BETA_SIGMOID, PRO_GATE_SOFTPLUS, PRO_L2NORM_QK,
                    GdrError, check, lib)
 
-__all__ = ["chunk_fwd", "decode_step", "sync_status", "workspace_bytes", "launches_per_chunk_fwd", "chunk_fwd_plan",
+__all__ = ["chunk_fwd", "chunk_bwd", "decode_step", "sync_status", "workspace_bytes", "launches_per_chunk_fwd", "chunk_fwd_plan",
            "profile_next_call",
            "GdrError", "DECAY_MODES"]
 
@@ -200,6 +200,33 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optional[t
     else:
         rc = lib().gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(out), B, H, dk,
                                    dv, _mode(mode), _dtype(q), _dtype(out), _stream_handle(stream))
+    check(rc)
+    return out
+
+
+def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optional[torch.Tensor], beta: torch.Tensor,
+              dO: torch.Tensor, S0: Optional[torch.Tensor] = None, dS_T: Optional[torch.Tensor] = None, *,
+              mode="scalar", want_dS0: bool = True, workspace: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """Gradients of ``chunk_fwd`` (gdr_chunk_bwd) for upstream gradients dO [B,T,H,dv] (the dtype of
+    q) and dS_T [B,H,dv,dk] fp32 (None: zero). Returns fp32 device tensors ``dq``, ``dk`` [B,T,H,dk],
+    ``dv`` [B,T,H,dv], ``dbeta`` [B,T,H], ``dg`` (shape of g, None for "none"), ``dS0`` (or None)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    m = _mode(mode)
+    dt = _dtype(q)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    out = {"dq": torch.empty((B, T, H, dk), **f32), "dk": torch.empty((B, T, H, dk), **f32),
+           "dv": torch.empty((B, T, H, dv), **f32), "dbeta": torch.empty((B, T, H), **f32),
+           "dg": None if g is None or m == 0 else torch.empty(g.shape, **f32),
+           "dS0": torch.empty((B, H, dv, dk), **f32) if want_dS0 else None}
+    if workspace is None:
+        workspace = _workspace(lib().gdr_chunk_bwd_workspace_bytes(B, T, H, dk, dv, m, dt), q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().gdr_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(dO), _ptr(dS_T),
+                             _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
+                             _ptr(out["dS0"]), B, T, H, dk, dv, m, dt, _ptr(workspace), ws_bytes,
+                             _stream_handle(stream))
     check(rc)
     return out
 

@@ -285,6 +285,70 @@ int gdr_decode_step(const void* q, const void* k, const void* v, const float* g,
                               stream);
 }
 
+size_t gdr_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int mode, int dtype) {
+    if (B <= 0 || T <= 0 || H <= 0 || !bwd_supported(dk, dv)) return 0;
+    if (mode != GDR_DECAY_NONE && mode != GDR_DECAY_SCALAR && mode != GDR_DECAY_CHANNEL) return 0;
+    if (dtype != GDR_F32 && dtype != GDR_BF16) return 0;
+    return bwd_workspace_bytes(B, T, H, dk, dv);
+}
+
+int gdr_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta, const float* S0,
+                  const void* dO, const float* dS_T, float* dq, float* dk_out, float* dv_out, float* dg,
+                  float* dbeta, float* dS0, int B, int T, int H, int dk, int dv, int mode, int dtype,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+    if (mode != GDR_DECAY_NONE && mode != GDR_DECAY_SCALAR && mode != GDR_DECAY_CHANNEL)
+        return fail(GDR_ERR_INVALID_ARG, "unknown decay mode %d", mode);
+    if (dtype != GDR_F32 && dtype != GDR_BF16) return fail(GDR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+    if (B <= 0 || T <= 0 || H <= 0 || dk <= 0 || dv <= 0)
+        return fail(GDR_ERR_INVALID_ARG, "sizes must be positive (B=%d T=%d H=%d d_k=%d d_v=%d)", B, T, H, dk, dv);
+    if (H > 65535 || (size_t)B * H > 0x7fffffffu) return fail(GDR_ERR_UNSUPPORTED, "B * H too large");
+    if (!bwd_supported(dk, dv))
+        return fail(GDR_ERR_UNSUPPORTED, "unsupported d_k=%d d_v=%d (supported: 32, 64, 128 each)", dk, dv);
+    if (!q || !k || !v || !beta || !dO || !dq || !dk_out || !dv_out || !dbeta)
+        return fail(GDR_ERR_INVALID_ARG, "q, k, v, beta, dO, dq, dk, dv and dbeta must be non-null");
+    if (mode != GDR_DECAY_NONE && (!g || !dg))
+        return fail(GDR_ERR_INVALID_ARG, "g and dg must be non-null for a gated decay mode");
+    if (mode == GDR_DECAY_NONE) g = nullptr, dg = nullptr;
+    const void* ptrs[] = {q, k, v, g, beta, S0, dO, dS_T, dq, dk_out, dv_out, dg, dbeta, dS0, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return fail(GDR_ERR_MISALIGNED, "pointer %p is not 16-byte aligned", p);
+    const size_t ntok = (size_t)B * T * H, eb = elem_bytes(dtype);
+    const size_t bs = (size_t)B * H * dv * dk * sizeof(float);
+    const size_t bgd = mode == GDR_DECAY_CHANNEL ? ntok * dk * sizeof(float) : ntok * sizeof(float);
+    struct Span { const void* p; size_t n; const char* name; };
+    const Span ins[] = {{q, ntok * dk * eb, "q"}, {k, ntok * dk * eb, "k"}, {v, ntok * dv * eb, "v"},
+                        {g, bgd, "g"}, {beta, ntok * sizeof(float), "beta"}, {S0, bs, "S0"},
+                        {dO, ntok * dv * eb, "dO"}, {dS_T, bs, "dS_T"}};
+    const Span outs[] = {{dq, ntok * dk * sizeof(float), "dq"}, {dk_out, ntok * dk * sizeof(float), "dk"},
+                         {dv_out, ntok * dv * sizeof(float), "dv"}, {dg, bgd, "dg"},
+                         {dbeta, ntok * sizeof(float), "dbeta"}, {dS0, bs, "dS0"}};
+    const size_t need = bwd_workspace_bytes(B, T, H, dk, dv);
+    if (workspace == nullptr || workspace_bytes < need)
+        return fail(GDR_ERR_WORKSPACE, "workspace of %zu bytes required (got %zu at %p)", need, workspace_bytes,
+                    workspace);
+    for (size_t i = 0; i < sizeof(outs) / sizeof(outs[0]); ++i) {
+        for (const Span& s : ins)
+            if (overlap(outs[i].p, outs[i].n, s.p, s.n))
+                return fail(GDR_ERR_INVALID_ARG, "%s overlaps input %s", outs[i].name, s.name);
+        for (size_t j = i + 1; j < sizeof(outs) / sizeof(outs[0]); ++j)
+            if (overlap(outs[i].p, outs[i].n, outs[j].p, outs[j].n))
+                return fail(GDR_ERR_INVALID_ARG, "%s overlaps %s", outs[i].name, outs[j].name);
+        if (overlap(workspace, need, outs[i].p, outs[i].n))
+            return fail(GDR_ERR_INVALID_ARG, "workspace overlaps %s", outs[i].name);
+    }
+    for (const Span& s : ins)
+        if (overlap(workspace, need, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "workspace overlaps %s", s.name);
+    int* status = nullptr;
+    int major = 0;
+    if (int rc = device_setup(&status, &major)) return rc;
+    if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
+    BwdProblem p{q, k, v, g, beta, S0, dO, dS_T, dq, dk_out, dv_out, dg, dbeta, dS0, workspace,
+                 B, T, H, dk, dv, mode, dtype, (float)(1.0 / sqrt((double)dk))};
+    const cudaError_t err = launch_bwd(p, static_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "backward launch: %s", cudaGetErrorString(err));
+    return ok();
+}
+
 int gdr_sync_status(void* stream) {
     int* status = nullptr;
     int major = 0;

@@ -45,6 +45,27 @@ struct DecodeProblem {
     const float* gate_scale;
 };
 
+// Everything one backward call needs (gdr_chunk_bwd). Pointers are device pointers.
+struct BwdProblem {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* g;
+    const float* beta;
+    const float* S0;
+    const void* dO;
+    const float* dST;
+    float* dq;
+    float* dk;
+    float* dv;
+    float* dg;
+    float* dbeta;
+    float* dS0;
+    void* workspace;
+    int B, T, H, dk_dim, dv_dim, mode, dtype;
+    float scale;
+};
+
 // The prologue's elementwise steps (gdr_prologue), in fp32 with CUDA's math functions.
 __device__ __forceinline__ float pro_sigmoid(float x) { return 1.f / (1.f + expf(-x)); }
 // g = -A softplus(a), softplus(a) = max(a, 0) + log(1 + e^-|a|)
@@ -97,6 +118,11 @@ int chunk_tc_plan(int B, int T, int H, int dk, int dv, int chunk, int mode, int*
 // that nothing sets, with a wait bound of limit_ns; then the time it ran, read after the stream.
 cudaError_t launch_bounded_wait_selftest(int* status, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t read_bounded_wait_selftest_elapsed(unsigned long long* elapsed_ns);
+
+// Backward of the forward (fp32 CUDA cores): state history, then the reverse sweep.
+bool bwd_supported(int dk, int dv);
+size_t bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
+cudaError_t launch_bwd(const BwdProblem& p, cudaStream_t stream);
 
 // Bandwidth-bound decode step.
 bool decode_supported(int dk, int dv);

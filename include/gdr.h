@@ -185,6 +185,40 @@ int gdr_decode_step_ex(const void* q, const void* k, const void* v, const float*
                        float* S, void* o, int B, int H, int d_k, int d_v, int mode, int dtype,
                        int o_dtype, int prologue, const float* gate_scale, void* stream);
 
+/*
+ * gdr_chunk_bwd -- gradients of gdr_chunk_fwd (the training backward pass).
+ *
+ * Defined by: the forward above (its value is the token recurrence of "Linear Attention & DeltaNet",
+ * How it works, items 3-4, with the decay of "linear attention and its gated descendants", Gated
+ * DeltaNet and Kimi Delta Attention), differentiated in reverse mode. For a loss L with dO = dL/do
+ * and dS_T = dL/dS_T, the call returns dL/dq, dL/dk, dL/dv, dL/dg, dL/dbeta and dL/dS0, where g, beta,
+ * q, k are the values gdr_chunk_fwd reads (no prologue). Per row j of the state, in reverse token
+ * order (s_bar = s (.) alpha, p = s_bar . k, delta = beta (v_j - p), s' = s_bar + delta k):
+ *     ds' = ds + scale do_j q;  ddelta = ds' . k;  dv_j = beta ddelta;  ds_bar = ds' - beta ddelta k;
+ *     ds = ds_bar (.) alpha;  dq += scale do_j s';  dk += delta ds' - beta ddelta s_bar;
+ *     dbeta += ddelta (v_j - p);  dg += ds_bar (.) s_bar  (summed over channels for SCALAR).
+ *
+ *   q, k, v, g, beta, S0  the forward's inputs, as for gdr_chunk_fwd (S0 may be NULL: zero)
+ *   dO        [B, T, H, d_v] dtype (the type of q, k, v)
+ *   dS_T      [B, H, d_v, d_k] fp32, or NULL (zero)
+ *   dq, dk    [B, T, H, d_k] fp32 (written);  dv [B, T, H, d_v] fp32 (written)
+ *   dg        fp32 in the shape of g (written; NULL for NONE);  dbeta [B, T, H] fp32 (written)
+ *   dS0       [B, H, d_v, d_k] fp32 (written), or NULL
+ *   d_k, d_v  in {32, 64, 128}; dtype F32 or BF16; arithmetic fp32 on the CUDA cores.
+ *   workspace at least gdr_chunk_bwd_workspace_bytes(...) bytes: the state before every token,
+ *             B * H * T * d_v * d_k * 4 bytes (the reverse sweep reads it back instead of
+ *             recomputing). Not kept after the enqueued work completes.
+ * Launches: two kernels, one CTA of 512 threads per (b, h). No output may overlap an input, another
+ * output or the workspace. Errors as gdr_chunk_fwd.
+ */
+int gdr_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                  const float* S0, const void* dO, const float* dS_T, float* dq, float* dk, float* dv,
+                  float* dg, float* dbeta, float* dS0, int B, int T, int H, int d_k, int d_v, int mode,
+                  int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace gdr_chunk_bwd needs (0 for arguments it would reject). Host-only. */
+size_t gdr_chunk_bwd_workspace_bytes(int B, int T, int H, int d_k, int d_v, int mode, int dtype);
+
 /* Number of kernel launches one gdr_chunk_fwd call makes for this problem (0 if it would be
  * rejected). Host-only. */
 int gdr_chunk_fwd_launches(int B, int T, int H, int d_k, int d_v, int chunk, int mode, int dtype,

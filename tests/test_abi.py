@@ -164,3 +164,33 @@ def test_chunk_fwd_ex_validates_prologue_on_host(pro, mode, gs, code):
 def test_decode_ex_validates_prologue_on_host(pro, mode, code):
     rc = _lib.lib().gdr_decode_step_ex(16, 32, 48, 64, 80, 1 << 20, 1 << 21, 2, 2, 128, 128, mode, 1, 0, pro, None, None)
     assert rc == code
+
+
+def _bwd(**kw):
+    """Calls gdr_chunk_bwd with fake, widely spaced addresses; used only with argument errors."""
+    M = 1 << 26
+    a = dict(q=1 * M, k=2 * M, v=3 * M, g=4 * M, beta=5 * M, S0=None, dO=6 * M, dST=None, dq=7 * M, dk=8 * M,
+             dv=9 * M, dg=10 * M, dbeta=11 * M, dS0=None, B=1, T=16, H=1, d_k=64, d_v=64, mode=1, dtype=0,
+             ws=12 * M, wsb=1 << 26)
+    a.update(kw)
+    return _lib.lib().gdr_chunk_bwd(a["q"], a["k"], a["v"], a["g"], a["beta"], a["S0"], a["dO"], a["dST"], a["dq"],
+                                    a["dk"], a["dv"], a["dg"], a["dbeta"], a["dS0"], a["B"], a["T"], a["H"], a["d_k"],
+                                    a["d_v"], a["mode"], a["dtype"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), -1), (dict(mode=9), -1), (dict(dtype=4), -1), (dict(d_k=256), -2), (dict(d_v=40), -2),
+    (dict(g=None), -1), (dict(dg=None), -1), (dict(dO=None), -1), (dict(dq=None), -1),
+    (dict(dk=(8 << 26) + 8), -3), (dict(wsb=100), -4), (dict(ws=None), -4),
+    (dict(dv=(1 << 26) + 256), -1),  # dv (an output) over q
+    (dict(dbeta=8 << 26), -1),       # two outputs overlap
+])
+def test_chunk_bwd_rejects_bad_arguments_on_host(kw, code):
+    assert _bwd(**kw) == code
+    assert len(_lib.lib().gdr_last_error()) > 0
+
+
+def test_chunk_bwd_workspace_query():
+    lib = _lib.lib()
+    assert lib.gdr_chunk_bwd_workspace_bytes(2, 100, 3, 64, 32, 1, 0) == 2 * 3 * 100 * 64 * 32 * 4
+    assert lib.gdr_chunk_bwd_workspace_bytes(2, 100, 3, 48, 32, 1, 0) == 0
