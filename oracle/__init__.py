@@ -50,6 +50,8 @@ def _load():
                 ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
                 ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
             lib.gdr_oracle_max_threads.restype = ctypes.c_int
+            lib.gdr_oracle_recurrent_gdn2.restype = ctypes.c_int
+            lib.gdr_oracle_recurrent_gdn2.argtypes = lib.gdr_oracle_recurrent.argtypes
             lib.gdr_oracle_backward.restype = ctypes.c_int
             lib.gdr_oracle_backward.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 4 + [
                 ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_double] + [
@@ -117,6 +119,43 @@ def recurrent(q, k, v, g, beta, mode: str, S0=None, *, erase=None, write=None,
     rc = lib.gdr_oracle_recurrent(B, T, H, dk, dv, _ptr(qa), _ptr(ka), _ptr(va), _ptr(ga), _MODES[mode],
                                   _ptr(ea), _ptr(wa), int(bool(f64_inputs)), _ptr(s0), sc,
                                   _ptr(o), _ptr(st), int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle failed with status {rc}")
+    return o, st
+
+
+def recurrent_gdn2(q, k, v, g, erase, write, mode: str, S0=None, *, scale: Optional[float] = None,
+                   f64_inputs: bool = False, threads: int = 0,
+                   want_state: bool = True) -> Tuple[np.ndarray, Optional[np.ndarray]]:
+    """Gated DeltaNet-2 token recurrence (``gdr_oracle_recurrent_gdn2``): channel-wise erase gate
+    ``erase`` [B,T,H,dk] on the key side and write gate ``write`` [B,T,H,dv] on the value side,
+    decay g as in ``recurrent``. Returns ``(o, S_T)`` in float64."""
+    lib = _load()
+    if mode not in _MODES:
+        raise ValueError(f"unknown decay mode {mode!r}")
+    qa, ka, va = _arr(q, f64_inputs), _arr(k, f64_inputs), _arr(v, f64_inputs)
+    B, T, H, dk = qa.shape
+    dv = va.shape[-1]
+    if ka.shape != (B, T, H, dk) or va.shape != (B, T, H, dv):
+        raise ValueError("q, k, v shapes disagree")
+    ea, wa = _arr(erase, f64_inputs), _arr(write, f64_inputs)
+    if ea.shape != (B, T, H, dk) or wa.shape != (B, T, H, dv):
+        raise ValueError("erase must be [B,T,H,dk] and write [B,T,H,dv]")
+    ga = None
+    if mode != "none":
+        ga = _arr(g, f64_inputs)
+        want = (B, T, H) if mode == "scalar" else (B, T, H, dk)
+        if ga.shape != want:
+            raise ValueError(f"g must be {want} for mode {mode}")
+    s0 = None if S0 is None else _arr(S0, True)
+    if s0 is not None and s0.shape != (B, H, dv, dk):
+        raise ValueError("S0 must be [B,H,dv,dk]")
+    o = np.empty((B, T, H, dv), dtype=np.float64)
+    st = np.empty((B, H, dv, dk), dtype=np.float64) if want_state else None
+    sc = (1.0 / np.sqrt(dk)) if scale is None else float(scale)
+    rc = lib.gdr_oracle_recurrent_gdn2(B, T, H, dk, dv, _ptr(qa), _ptr(ka), _ptr(va), _ptr(ga), _MODES[mode],
+                                       _ptr(ea), _ptr(wa), int(bool(f64_inputs)), _ptr(s0), sc, _ptr(o), _ptr(st),
+                                       int(threads))
     if rc != 0:
         raise RuntimeError(f"oracle failed with status {rc}")
     return o, st

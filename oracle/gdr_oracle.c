@@ -281,3 +281,82 @@ int gdr_oracle_backward(int B, int T, int H, int dk, int dv,
     }
     return status;
 }
+
+/*
+ * Gated DeltaNet-2: the delta rule with a channel-wise erase gate on the key side and a
+ * channel-wise write gate on the value side ("Linear Attention Architectures: Mechanisms,
+ * Trade-offs, and Cross-Layer Routing", Sec. 3, the Gated DeltaNet-2 paragraph and its gate
+ * definitions). With the decay-adjusted memory S_bar = S_{t-1} Diag(alpha_t), the gated erase
+ * direction e_t (.) k_t and the gated write target w_t (.) v_t, the residual written to memory is
+ * r_t = w_t (.) v_t - S_bar (e_t (.) k_t), and
+ *
+ *     S_t = S_bar + r_t k_t^T ,    o_t = scale * S_t q_t .
+ *
+ * (The page's formulas are stripped; this is the reading under which one residual is written
+ * along k_t, e_t = w_t = beta_t 1 gives Kimi Delta Attention and a scalar alpha then gives Gated
+ * DeltaNet, as the page states.) Row form: s_bar = s_j (.) alpha ; p = s_bar . (e (.) k) ;
+ * s_j = s_bar + (w_j v_{t,j} - p) k ; o_{t,j} = scale (s_j . q).
+ * erase: [B,T,H,d_k]; write: [B,T,H,d_v]; other arguments as gdr_oracle_recurrent.
+ */
+int gdr_oracle_recurrent_gdn2(int B, int T, int H, int dk, int dv,
+                              const void* q, const void* k, const void* v,
+                              const void* g, int mode,
+                              const void* erase, const void* write, int in_f64,
+                              const double* S0, double scale,
+                              double* o, double* S_T, int nthreads) {
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+    if (mode != ORACLE_MODE_NONE && mode != ORACLE_MODE_SCALAR && mode != ORACLE_MODE_CHANNEL) return -1;
+    if (mode != ORACLE_MODE_NONE && g == NULL) return -1;
+    if ((T > 0) && (q == NULL || k == NULL || v == NULL || erase == NULL || write == NULL || o == NULL)) return -1;
+    const long nhead = (long)B * H;
+    int status = 0;
+    if (nthreads <= 0) nthreads = gdr_oracle_max_threads();
+
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long bh = 0; bh < nhead; ++bh) {
+        const int h = (int)(bh % H);
+        const int b = (int)(bh / H);
+        double* s = (double*)malloc(sizeof(double) * (size_t)dv * dk);
+        double* vec = (double*)malloc(sizeof(double) * (size_t)dk * 4);
+        if (!s || !vec) {
+            free(s); free(vec);
+#pragma omp atomic write
+            status = -2;
+            continue;
+        }
+        double *kt = vec, *qt = vec + dk, *at = vec + 2 * dk, *ek = vec + 3 * dk;
+        for (size_t i = 0; i < (size_t)dv * dk; ++i) s[i] = S0 ? S0[(size_t)bh * dv * dk + i] : 0.0;
+        for (int t = 0; t < T; ++t) {
+            const size_t tok = ((size_t)b * T + t) * H + h;
+            for (int c = 0; c < dk; ++c) {
+                kt[c] = ld_in(k, tok * dk + c, in_f64);
+                qt[c] = ld_in(q, tok * dk + c, in_f64);
+                ek[c] = ld_in(erase, tok * dk + c, in_f64) * kt[c]; /* gated erase direction */
+                if (mode == ORACLE_MODE_NONE) at[c] = 1.0;
+                else if (mode == ORACLE_MODE_SCALAR) at[c] = exp(ld_in(g, tok, in_f64));
+                else at[c] = exp(ld_in(g, tok * dk + c, in_f64));
+            }
+            for (int j = 0; j < dv; ++j) {
+                double* sj = s + (size_t)j * dk;
+                /* decay-adjusted memory, then its prediction along the gated erase direction */
+                double p = 0.0;
+                for (int c = 0; c < dk; ++c) {
+                    sj[c] *= at[c];
+                    p += sj[c] * ek[c];
+                }
+                /* residual: gated write target minus that prediction, written along k_t */
+                const double r = ld_in(write, tok * dv + j, in_f64) * ld_in(v, tok * dv + j, in_f64) - p;
+                double a = 0.0;
+                for (int c = 0; c < dk; ++c) {
+                    sj[c] += r * kt[c];
+                    a += sj[c] * qt[c];
+                }
+                o[tok * dv + j] = scale * a;
+            }
+        }
+        if (S_T)
+            for (size_t i = 0; i < (size_t)dv * dk; ++i) S_T[(size_t)bh * dv * dk + i] = s[i];
+        free(s); free(vec);
+    }
+    return status;
+}

@@ -57,3 +57,21 @@ def states_by_kron(S0, As, Bs):
         x = np.kron(A.T, np.eye(dv)) @ x + Bm.reshape(-1, order="F")
         out.append(x.reshape(dv, dk, order="F"))
     return out
+
+
+def transitions_gdn2(k, v, g, mode, erase, write):
+    """Gated DeltaNet-2 per-token (A_t, B_t) for one head: A_t = Diag(alpha_t)(I - (e_t * k_t) k_t^T)
+    and B_t = (w_t * v_t) k_t^T, with erase e_t [dk] and write w_t [dv] channel-wise gates."""
+    T, dk = k.shape
+    As, Bs = [], []
+    for t in range(T):
+        if mode == "none":
+            alpha = np.ones(dk)
+        elif mode == "scalar":
+            alpha = np.full(dk, np.exp(g[t]))
+        else:
+            alpha = np.exp(g[t])
+        kt = k[t][:, None]
+        As.append(np.diag(alpha) @ (np.eye(dk) - (erase[t][:, None] * kt) @ kt.T))
+        Bs.append((write[t] * v[t])[:, None] @ kt.T)
+    return As, Bs

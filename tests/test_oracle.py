@@ -515,3 +515,82 @@ def test_backward_no_write_closed_form():
     assert np.all(gr["dk"] == 0) and np.all(gr["dv"] == 0)
     np.testing.assert_allclose(gr["dS0"], dST + sc * np.einsum("bthj,bthc->bhjc", dO, q), rtol=1e-13, atol=1e-13)
     assert gr["dg"] is None
+
+
+# ---- Gated DeltaNet-2 (channel-wise erase and write gates)
+
+def _gdn2_problem(rng, B, T, H, dk, dv, mode):
+    q, k, v, g, _ = _rand_problem(rng, B, T, H, dk, dv, mode, unit_keys=True, g_scale=0.5)
+    erase = rng.uniform(0.0, 1.0, (B, T, H, dk))
+    write = rng.uniform(0.0, 1.0, (B, T, H, dv))
+    return q, k, v, g, erase, write
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_gdn2_matches_transition_products(mode):
+    """S_T from explicit products and from the Kronecker-form linear system of the transitions
+    A_t = Diag(alpha_t)(I - (e_t k_t) k_t^T), B_t = (w_t v_t) k_t^T; o_t = scale S_t q_t."""
+    from brute import transitions_gdn2
+    rng = np.random.default_rng(41 + MODES.index(mode))
+    B, T, H, dk, dv = 1, 6, 2, 4, 3
+    q, k, v, g, e, w = _gdn2_problem(rng, B, T, H, dk, dv, mode)
+    S0 = rng.standard_normal((B, H, dv, dk))
+    o, st = oracle.recurrent_gdn2(q, k, v, g, e, w, mode, S0=S0, f64_inputs=True)
+    sc = 1.0 / np.sqrt(dk)
+    for h in range(H):
+        gh = None if g is None else g[0, :, h]
+        As, Bs = transitions_gdn2(k[0, :, h], v[0, :, h], gh, mode, e[0, :, h], w[0, :, h])
+        by_prod = states_by_product(S0[0, h], As, Bs)
+        by_kron = states_by_kron(S0[0, h], As, Bs)
+        for t in range(T):
+            np.testing.assert_allclose(by_prod[t], by_kron[t], rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(o[0, t, h], sc * by_prod[t] @ q[0, t, h], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(st[0, h], by_prod[-1], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_gdn2_equal_gates_is_the_delta_rule(mode):
+    """e_t = w_t = beta_t 1 gives the delta rule with the same decay (Kimi Delta Attention for the
+    channel gate, Gated DeltaNet for the scalar one, DeltaNet without decay)."""
+    rng = np.random.default_rng(51 + MODES.index(mode))
+    B, T, H, dk, dv = 2, 9, 2, 5, 3
+    q, k, v, g, beta = _rand_problem(rng, B, T, H, dk, dv, mode)
+    S0 = rng.standard_normal((B, H, dv, dk))
+    e = np.repeat(beta[..., None], dk, axis=-1)
+    w = np.repeat(beta[..., None], dv, axis=-1)
+    o2, s2 = oracle.recurrent_gdn2(q, k, v, g, e, w, mode, S0=S0, f64_inputs=True)
+    o1, s1 = _run(q, k, v, g, beta, mode, S0=S0)
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(s2, s1, rtol=1e-12, atol=1e-13)
+
+
+def test_gdn2_erase_free_is_gated_linear_attention():
+    """e = 0, alpha = 1: nothing is erased and o_t = scale sum_{i<=t} (k_i . q_t) (w_i v_i) (closed form)."""
+    rng = np.random.default_rng(61)
+    B, T, H, dk, dv = 1, 7, 2, 4, 3
+    q, k, v, g, e, w = _gdn2_problem(rng, B, T, H, dk, dv, "none")
+    e = np.zeros_like(e)
+    o, st = oracle.recurrent_gdn2(q, k, v, None, e, w, "none", f64_inputs=True)
+    sc = 1.0 / np.sqrt(dk)
+    for t in range(T):
+        ref = sc * sum((k[0, i] * q[0, t]).sum(-1)[:, None] * (w[0, i] * v[0, i]) for i in range(t + 1))
+        np.testing.assert_allclose(o[0, t], ref, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(st[0], np.einsum("thj,thc->hjc", w[0] * v[0], k[0]), rtol=1e-12, atol=1e-13)
+
+
+def test_gdn2_erase_only_projects_out_written_keys():
+    """w = 0, e = 1, alpha = 1, orthonormal keys: each token projects its key direction out of the
+    memory, so S_T k_i = 0 for every key written and S_T x = S0 x for x orthogonal to all of them."""
+    rng = np.random.default_rng(71)
+    dk, dv, T = 6, 3, 4
+    Qm, _ = np.linalg.qr(rng.standard_normal((dk, dk)))
+    k = Qm[:T].reshape(1, T, 1, dk)
+    q = rng.standard_normal((1, T, 1, dk))
+    v = rng.standard_normal((1, T, 1, dv))
+    S0 = rng.standard_normal((1, 1, dv, dk))
+    _, st = oracle.recurrent_gdn2(q, k, v, None, np.ones((1, T, 1, dk)), np.zeros((1, T, 1, dv)), "none", S0=S0,
+                                  f64_inputs=True)
+    for i in range(T):
+        np.testing.assert_allclose(st[0, 0] @ Qm[i], 0.0, atol=1e-13)
+    for i in range(T, dk):
+        np.testing.assert_allclose(st[0, 0] @ Qm[i], S0[0, 0] @ Qm[i], atol=1e-13)
