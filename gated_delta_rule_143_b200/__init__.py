@@ -25,7 +25,7 @@ import torch
 from ._lib import (DECAY_MODES, DTYPE_BF16, DTYPE_F32, PLANS, PRO_BETA_SIGMOID, PRO_GATE_SOFTPLUS, PRO_L2NORM_QK,
                    GdrError, check, lib)
 
-__all__ = ["chunk_fwd", "chunk_bwd", "decode_step", "sync_status", "workspace_bytes", "launches_per_chunk_fwd", "chunk_fwd_plan",
+__all__ = ["chunk_fwd", "chunk_bwd", "chunk_fwd_gdn2", "decode_step", "decode_step_gdn2", "sync_status", "workspace_bytes", "launches_per_chunk_fwd", "chunk_fwd_plan",
            "profile_next_call",
            "GdrError", "DECAY_MODES"]
 
@@ -200,6 +200,42 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optional[t
     else:
         rc = lib().gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(out), B, H, dk,
                                    dv, _mode(mode), _dtype(q), _dtype(out), _stream_handle(stream))
+    check(rc)
+    return out
+
+
+def chunk_fwd_gdn2(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optional[torch.Tensor],
+                   erase: torch.Tensor, write: torch.Tensor, S0: Optional[torch.Tensor] = None, *, mode="channel",
+                   chunk: int = 64, return_state: bool = True, out: Optional[torch.Tensor] = None,
+                   out_dtype: torch.dtype = torch.float32, state_out: Optional[torch.Tensor] = None,
+                   stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Gated DeltaNet-2 forward (gdr_chunk_fwd_gdn2): ``erase`` fp32 [B,T,H,dk] and ``write`` fp32
+    [B,T,H,dv] gates in place of beta; other arguments as ``chunk_fwd``."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=out_dtype, device=q.device)
+    if return_state and state_out is None:
+        state_out = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device)
+    rc = lib().gdr_chunk_fwd_gdn2(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(erase), _ptr(write), _ptr(S0), _ptr(out),
+                                  _ptr(state_out) if return_state else None, B, T, H, dk, dv, chunk, _mode(mode),
+                                  _dtype(q), _dtype(out), _stream_handle(stream))
+    check(rc)
+    return out, (state_out if return_state else None)
+
+
+def decode_step_gdn2(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optional[torch.Tensor],
+                     erase: torch.Tensor, write: torch.Tensor, S: torch.Tensor, *, mode="channel",
+                     out: Optional[torch.Tensor] = None, out_dtype: torch.dtype = torch.float32,
+                     stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """One Gated DeltaNet-2 decode step (gdr_decode_step_gdn2): erase [B,H,dk], write [B,H,dv] fp32;
+    S updated in place."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=out_dtype, device=q.device)
+    rc = lib().gdr_decode_step_gdn2(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(erase), _ptr(write), _ptr(S), _ptr(out),
+                                    B, H, dk, dv, _mode(mode), _dtype(q), _dtype(out), _stream_handle(stream))
     check(rc)
     return out
 

@@ -285,6 +285,81 @@ int gdr_decode_step(const void* q, const void* k, const void* v, const float* g,
                               stream);
 }
 
+int gdr_chunk_fwd_gdn2(const void* q, const void* k, const void* v, const float* g, const float* erase,
+                       const float* write, const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv,
+                       int chunk, int mode, int dtype, int o_dtype, void* stream) {
+    if (int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype)) return rc;
+    if (!chunk_simt_supported(dk, dv, chunk))
+        return fail(GDR_ERR_UNSUPPORTED, "Gated DeltaNet-2: d_k, d_v in {32, 64, 128} and chunk 64 (got %d, %d, %d)", dk,
+                    dv, chunk);
+    if (!q || !k || !v || !erase || !write || !o)
+        return fail(GDR_ERR_INVALID_ARG, "q, k, v, erase, write and o must be non-null");
+    if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
+    if (mode == GDR_DECAY_NONE) g = nullptr;
+    const void* ptrs[] = {q, k, v, g, erase, write, S0, o, S_T};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return fail(GDR_ERR_MISALIGNED, "pointer %p is not 16-byte aligned", p);
+    const size_t ntok = (size_t)B * T * H, eb = elem_bytes(dtype);
+    const size_t bo = ntok * dv * elem_bytes(o_dtype), bs = (size_t)B * H * dv * dk * sizeof(float);
+    struct Span { const void* p; size_t n; const char* name; };
+    const Span ins[] = {{q, ntok * dk * eb, "q"}, {k, ntok * dk * eb, "k"}, {v, ntok * dv * eb, "v"},
+                        {g, mode == GDR_DECAY_CHANNEL ? ntok * dk * 4 : ntok * 4, "g"}, {erase, ntok * dk * 4, "erase"},
+                        {write, ntok * dv * 4, "write"}, {S0, bs, "S0"}};
+    for (const Span& s : ins) {
+        if (overlap(o, bo, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "o overlaps input %s", s.name);
+        if (S_T != S0 && overlap(S_T, bs, s.p, s.n))
+            return fail(GDR_ERR_INVALID_ARG, "S_T overlaps input %s (only S_T == S0 is allowed)", s.name);
+    }
+    if (overlap(o, bo, S_T, bs)) return fail(GDR_ERR_INVALID_ARG, "o overlaps S_T");
+    int* status = nullptr;
+    int major = 0;
+    if (int rc = device_setup(&status, &major)) return rc;
+    if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
+    ChunkProblem p{q, k, v, g, nullptr, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, nullptr, 0, status,
+                   (float)(1.0 / sqrt((double)dk)), GDR_PRO_NONE, nullptr, erase, write};
+    const cudaError_t err = launch_chunk_simt(p, static_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "Gated DeltaNet-2 launch: %s", cudaGetErrorString(err));
+    return ok();
+}
+
+int gdr_decode_step_gdn2(const void* q, const void* k, const void* v, const float* g, const float* erase,
+                         const float* write, float* S, void* o, int B, int H, int dk, int dv, int mode, int dtype,
+                         int o_dtype, void* stream) {
+    if (int rc = check_enums(mode, dtype, o_dtype)) return rc;
+    if (B <= 0 || H <= 0 || dk <= 0 || dv <= 0)
+        return fail(GDR_ERR_INVALID_ARG, "sizes must be positive (B=%d H=%d d_k=%d d_v=%d)", B, H, dk, dv);
+    if ((size_t)B * H > 0x7fffffffu) return fail(GDR_ERR_UNSUPPORTED, "B*H too large");
+    if (!decode_supported(dk, dv))
+        return fail(GDR_ERR_UNSUPPORTED, "unsupported d_k=%d (supported: 32, 64, 128, 256)", dk);
+    if (!q || !k || !v || !erase || !write || !S || !o)
+        return fail(GDR_ERR_INVALID_ARG, "q, k, v, erase, write, S and o must be non-null");
+    if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
+    if (mode == GDR_DECAY_NONE) g = nullptr;
+    const void* ptrs[] = {q, k, v, g, erase, write, S, o};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return fail(GDR_ERR_MISALIGNED, "pointer %p is not 16-byte aligned", p);
+    const size_t nh = (size_t)B * H, eb = elem_bytes(dtype);
+    const size_t bs = nh * dv * dk * sizeof(float), bo = nh * dv * elem_bytes(o_dtype);
+    struct Span { const void* p; size_t n; const char* name; };
+    const Span ins[] = {{q, nh * dk * eb, "q"}, {k, nh * dk * eb, "k"}, {v, nh * dv * eb, "v"},
+                        {g, mode == GDR_DECAY_CHANNEL ? nh * dk * 4 : nh * 4, "g"}, {erase, nh * dk * 4, "erase"},
+                        {write, nh * dv * 4, "write"}};
+    for (const Span& s : ins) {
+        if (overlap(S, bs, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "S overlaps input %s", s.name);
+        if (overlap(o, bo, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "o overlaps input %s", s.name);
+    }
+    if (overlap(o, bo, S, bs)) return fail(GDR_ERR_INVALID_ARG, "o overlaps S");
+    int* status = nullptr;
+    int major = 0;
+    if (int rc = device_setup(&status, &major)) return rc;
+    if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
+    DecodeProblem p{q, k, v, g, nullptr, S, o, B, H, dk, dv, mode, dtype, o_dtype, status,
+                    (float)(1.0 / sqrt((double)dk)), GDR_PRO_NONE, nullptr, erase, write};
+    const cudaError_t err = launch_decode(p, static_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
+    return ok();
+}
+
 size_t gdr_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int mode, int dtype) {
     if (B <= 0 || T <= 0 || H <= 0 || !bwd_supported(dk, dv)) return 0;
     if (mode != GDR_DECAY_NONE && mode != GDR_DECAY_SCALAR && mode != GDR_DECAY_CHANNEL) return 0;

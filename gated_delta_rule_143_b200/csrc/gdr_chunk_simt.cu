@@ -17,6 +17,13 @@
 // Parallel Form) with the WY/UT compact form of a chunk of delta-rule updates ("Linear
 // Attention & DeltaNet", item 3): (I + A)^-1 applied to R gives U - W S^T directly.
 // Pairwise decays exp(Gamma_r - Gamma_i) with i <= r never exceed 1, so any g <= 0 is safe.
+//
+// Gated DeltaNet-2 (EW = true; "Linear Attention Architectures: Mechanisms, Trade-offs, and
+// Cross-Layer Routing", Sec. 3): a channel-wise erase gate e on the key side and write gate w on the
+// value side replace beta, S_t = S_bar + (w (.) v - S_bar (e (.) k)) k^T with S_bar = S_{t-1} Diag(alpha).
+// In the chunk form the erase direction E = e (.) K takes the place of diag(beta) K on the left of the
+// Gram and of the state read, and the write target w (.) V that of diag(beta) V:
+//   A_ri = sum_c E_rc k_ic exp(Gamma_rc - Gamma_ic) (i < r),  R = w (.) V - (E*gamma) S^T.
 #include "gdr_internal.cuh"
 
 namespace gdr {
@@ -26,7 +33,7 @@ constexpr int kC = 64;        // chunk length
 constexpr int kDVS = 32;      // state rows per CTA
 constexpr int kThreads = 256;
 
-template <int DK>
+template <int DK, bool EW = false>
 struct SimtSmem {
     static constexpr int kLd = DK + 1;        // padded row stride of K, Q, Gamma, S
     static constexpr int kLdC = kC + 1;       // padded stride of A, P
@@ -37,17 +44,19 @@ struct SimtSmem {
         + kDVS * kLd          // S slice
         + 2 * kC * kLdV       // R/Delta, O_inter
         + 2 * kC * kLdC       // A, P
-        + 2 * kC;             // beta, tail decay (scalar)
+        + 2 * kC              // beta, tail decay (scalar)
+        + (EW ? kC * kLd : 0);  // erase directions e (.) k (Gated DeltaNet-2)
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
-template <typename Tin, typename Tout, int MODE, int DK>
+template <typename Tin, typename Tout, int MODE, int DK, bool EW>
 __global__ void __launch_bounds__(kThreads)
 chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                   const float* __restrict__ g, const float* __restrict__ beta, const float* S0,
                   Tout* __restrict__ o, float* S_T, int T, int H, int dv, float scale, int pro,
-                  const float* __restrict__ gate_scale) {
-    using L = SimtSmem<DK>;
+                  const float* __restrict__ gate_scale, const float* __restrict__ erase,
+                  const float* __restrict__ write) {
+    using L = SimtSmem<DK, EW>;
     extern __shared__ float smem[];
     float* sK = smem;
     float* sQ = sK + kC * L::kLd;
@@ -59,6 +68,7 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
     float* sP = sA + kC * L::kLdC;
     float* sBeta = sP + kC * L::kLdC;
     float* sTail = sBeta + kC;
+    float* sE = sTail + kC;  // EW only: e (.) k, [kC][kLd]
 
     const int tid = threadIdx.x;
     const int j0 = blockIdx.x * kDVS;           // first state row of this CTA
@@ -84,16 +94,23 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
         for (int idx = tid; idx < n * DK; idx += kThreads) {
             const int r = idx / DK, c = idx % DK;
             const size_t tok = ((size_t)b * T + c0 + r) * H + h;
-            sK[r * L::kLd + c] = load_f32(k + tok * DK + c);
+            const float kv = load_f32(k + tok * DK + c);
+            sK[r * L::kLd + c] = kv;
             sQ[r * L::kLd + c] = load_f32(q + tok * DK + c);
+            if (EW) sE[r * L::kLd + c] = erase[tok * DK + c] * kv;
         }
         for (int idx = tid; idx < n * kDVS; idx += kThreads) {
             const int r = idx / kDVS, j = idx % kDVS;
             const size_t tok = ((size_t)b * T + c0 + r) * H + h;
-            sR[r * L::kLdV + j] = (j < nrows) ? load_f32(v + tok * dv + j0 + j) : 0.f;
+            float x = 0.f;
+            if (j < nrows) {
+                x = load_f32(v + tok * dv + j0 + j);
+                if (EW) x *= write[tok * dv + j0 + j];  // the gated write target
+            }
+            sR[r * L::kLdV + j] = x;
         }
         for (int r = tid; r < n; r += kThreads) {
-            const float x = beta[((size_t)b * T + c0 + r) * H + h];
+            const float x = EW ? 1.f : beta[((size_t)b * T + c0 + r) * H + h];
             sBeta[r] = (pro & GDR_PRO_BETA_SIGMOID) ? pro_sigmoid(x) : x;
         }
         if (MODE == GDR_DECAY_SCALAR) {
@@ -138,7 +155,7 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
             const int r = idx / kC, i = idx % kC;
             float a = 0.f, p = 0.f;
             if (r < n && i <= r) {
-                const float* kr = sK + r * L::kLd;
+                const float* kr = (EW ? sE : sK) + r * L::kLd;  // erase direction of row r
                 const float* ki = sK + i * L::kLd;
                 const float* qr = sQ + r * L::kLd;
                 if (MODE == GDR_DECAY_CHANNEL) {
@@ -169,7 +186,7 @@ chunk_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
         // ---- R = diag(beta)(V - (K*gamma) S^T) and O_inter = (Q*gamma) S^T
         for (int idx = tid; idx < n * kDVS; idx += kThreads) {
             const int r = idx / kDVS, j = idx % kDVS;
-            const float* kr = sK + r * L::kLd;
+            const float* kr = (EW ? sE : sK) + r * L::kLd;  // the state is read along the erase direction
             const float* qr = sQ + r * L::kLd;
             const float* sj = sS + j * L::kLd;
             float x = 0.f, y = 0.f;
@@ -267,18 +284,21 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
-template <typename Tin, typename Tout, int MODE, int DK>
+template <typename Tin, typename Tout, int MODE, int DK, bool EW>
 __global__ void __launch_bounds__(kRecWarps * 32)
 recurrent_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                       const float* __restrict__ g, const float* __restrict__ beta, const float* S0,
                       Tout* __restrict__ o, float* S_T, int T, int H, int dv, float scale, int pro,
-                      const float* __restrict__ gate_scale) {
+                      const float* __restrict__ gate_scale, const float* __restrict__ erase,
+                      const float* __restrict__ write) {
     constexpr int NT = kRecWarps * 32;
     constexpr int NL = DK / 32;                                  // state columns per lane
     constexpr int NA = MODE == GDR_DECAY_CHANNEL ? DK : 1;       // decay factors per token
     constexpr int KPT = kRecTB * DK / NT;                        // staged k (and q) values per thread
     static_assert(kRecTB * DK % NT == 0 && kRecTB * kRecWarps <= NT && kRecTB <= NT, "staging split");
+    constexpr int NE = EW ? DK : 1;  // Gated DeltaNet-2: erase directions e (.) k
     __shared__ float sK[kRecTB][DK], sQ[kRecTB][DK], sAl[kRecTB][NA], sV[kRecTB][kRecWarps], sB[kRecTB];
+    __shared__ float sE[kRecTB][NE];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int j0 = blockIdx.x * kRecWarps, j = j0 + warp;       // this warp's state row
     const int h = blockIdx.y, b = blockIdx.z;
@@ -292,24 +312,26 @@ recurrent_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, cons
     // thread tid holds k, q (and the channel gate's g) at flat index tid + NT m of the block, the
     // value of (token tid / kRecWarps, row j0 + tid % kRecWarps), and beta (and the scalar g) of
     // token tid
-    float rk[KPT], rq[KPT], rg[KPT], rv = 0.f, rb = 0.f, rs = 0.f;
+    float rk[KPT], rq[KPT], rg[KPT], re[KPT], rv = 0.f, rb = 0.f, rs = 0.f;
     auto load_block = [&](int t0) {
         const int n = min(kRecTB, T - t0);
 #pragma unroll
         for (int m = 0; m < KPT; ++m) {
             const int idx = tid + NT * m, r = idx / DK, c = idx % DK;
-            rk[m] = rq[m] = rg[m] = 0.f;
+            rk[m] = rq[m] = rg[m] = re[m] = 0.f;
             if (r < n) {
                 const size_t tok = tok_of(t0 + r);
                 rk[m] = load_f32(k + tok * DK + c);
                 rq[m] = load_f32(q + tok * DK + c);
                 if (MODE == GDR_DECAY_CHANNEL) rg[m] = g[tok * DK + c];
+                if (EW) re[m] = erase[tok * DK + c];
             }
         }
         const int rr = tid / kRecWarps, w = tid % kRecWarps;
         rv = (rr < n && j0 + w < dv) ? load_f32(v + tok_of(t0 + rr) * dv + j0 + w) : 0.f;
+        if (EW && rr < n && j0 + w < dv) rv *= write[tok_of(t0 + rr) * dv + j0 + w];  // gated write target
         if (tid < n) {
-            rb = beta[tok_of(t0 + tid)];
+            rb = EW ? 1.f : beta[tok_of(t0 + tid)];
             if (MODE == GDR_DECAY_SCALAR) rs = g[tok_of(t0 + tid)];
         }
     };
@@ -319,6 +341,7 @@ recurrent_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, cons
             const int idx = tid + NT * m, r = idx / DK, c = idx % DK;
             sK[r][c] = rk[m];
             sQ[r][c] = rq[m];
+            if (EW) sE[r][c] = re[m] * rk[m];
             if (MODE == GDR_DECAY_CHANNEL) sAl[r][c] = expf(gate ? pro_gate(rg[m], A) : rg[m]);
         }
         if (tid < kRecTB * kRecWarps) sV[tid / kRecWarps][tid % kRecWarps] = rv;
@@ -375,7 +398,7 @@ recurrent_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, cons
                         kk[i] = sK[r][lane + 32 * i];
                         if (MODE == GDR_DECAY_SCALAR) s[i] *= sAl[r][0];
                         if (MODE == GDR_DECAY_CHANNEL) s[i] *= sAl[r][lane + 32 * i];
-                        p = fmaf(s[i], kk[i], p);
+                        p = fmaf(s[i], EW ? sE[r][(lane + 32 * i) % NE] : kk[i], p);  // read along e (.) k
                     }
                     p = warp_sum(p);
                     const float d = sB[r] * (sV[r][warp] - p);
@@ -410,26 +433,33 @@ recurrent_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, cons
     }
 }
 
-template <typename Tin, typename Tout, int MODE, int DK>
-cudaError_t launch_typed(const ChunkProblem& p, cudaStream_t stream) {
+template <typename Tin, typename Tout, int MODE, int DK, bool EW>
+cudaError_t launch_typed_ew(const ChunkProblem& p, cudaStream_t stream) {
     if (p.T <= kRecMaxT) {
         dim3 grid((p.dv + kRecWarps - 1) / kRecWarps, p.H, p.B);
-        recurrent_simt_kernel<Tin, Tout, MODE, DK><<<grid, kRecWarps * 32, 0, stream>>>(
+        recurrent_simt_kernel<Tin, Tout, MODE, DK, EW><<<grid, kRecWarps * 32, 0, stream>>>(
             static_cast<const Tin*>(p.q), static_cast<const Tin*>(p.k), static_cast<const Tin*>(p.v), p.g, p.beta,
-            p.S0, static_cast<Tout*>(p.o), p.S_T, p.T, p.H, p.dv, p.scale, p.prologue, p.gate_scale);
+            p.S0, static_cast<Tout*>(p.o), p.S_T, p.T, p.H, p.dv, p.scale, p.prologue, p.gate_scale, p.erase,
+            p.write);
         profile_after_launch(stream);
         return cudaGetLastError();
     }
-    auto kern = chunk_simt_kernel<Tin, Tout, MODE, DK>;
-    const size_t smem = SimtSmem<DK>::bytes;
+    auto kern = chunk_simt_kernel<Tin, Tout, MODE, DK, EW>;
+    const size_t smem = SimtSmem<DK, EW>::bytes;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     dim3 grid((p.dv + kDVS - 1) / kDVS, p.H, p.B);
     kern<<<grid, kThreads, smem, stream>>>(
         static_cast<const Tin*>(p.q), static_cast<const Tin*>(p.k), static_cast<const Tin*>(p.v), p.g, p.beta,
-        p.S0, static_cast<Tout*>(p.o), p.S_T, p.T, p.H, p.dv, p.scale, p.prologue, p.gate_scale);
+        p.S0, static_cast<Tout*>(p.o), p.S_T, p.T, p.H, p.dv, p.scale, p.prologue, p.gate_scale, p.erase, p.write);
     profile_after_launch(stream);
     return cudaGetLastError();
+}
+
+template <typename Tin, typename Tout, int MODE, int DK>
+cudaError_t launch_typed(const ChunkProblem& p, cudaStream_t stream) {
+    return p.erase != nullptr ? launch_typed_ew<Tin, Tout, MODE, DK, true>(p, stream)
+                              : launch_typed_ew<Tin, Tout, MODE, DK, false>(p, stream);
 }
 
 template <typename Tin, typename Tout, int MODE>

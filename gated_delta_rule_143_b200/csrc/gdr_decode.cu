@@ -13,6 +13,10 @@
 // loads, so a warp touches 4 whole rows per instruction, fully coalesced); the two dot
 // products are reduced across those 8 lanes with three xor-shuffles. One CTA of 256 threads
 // per (b, h); each thread carries two rows in flight. S is streamed with evict-first hints.
+//
+// Gated DeltaNet-2 (EW; "Linear Attention Architectures: Mechanisms, Trade-offs, and Cross-Layer
+// Routing", Sec. 3): an erase gate e [d_k] and a write gate w [d_v] replace beta:
+//   p = s_bar . (e (.) k);  delta = w_j v_j - p;  s_j <- s_bar + delta k;  o_j = scale (a + delta (k . q)).
 #include "gdr_internal.cuh"
 
 namespace gdr {
@@ -51,11 +55,12 @@ __device__ __forceinline__ float group8_sum(float x) {
     return x;
 }
 
-template <typename Tin, typename Tout, int MODE, int DK>
+template <typename Tin, typename Tout, int MODE, int DK, bool EW>
 __global__ void __launch_bounds__(kThreads)
 decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
               const float* __restrict__ g, const float* __restrict__ beta, float* __restrict__ S,
-              Tout* __restrict__ o, int dv, float scale, int H, int pro, const float* __restrict__ gate_scale) {
+              Tout* __restrict__ o, int dv, float scale, int H, int pro, const float* __restrict__ gate_scale,
+              const float* __restrict__ erase, const float* __restrict__ write) {
     constexpr int EPL = DK / kLanesPerRow;  // floats of a row per lane
     const size_t bh = blockIdx.x;
     const int sub = threadIdx.x & (kLanesPerRow - 1);
@@ -97,7 +102,14 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
 #pragma unroll
     for (int i = 0; i < EPL; ++i) kq = fmaf(kr[i], qr[i], kq);
     kq = group8_sum(kq);
-    const float bt = (pro & GDR_PRO_BETA_SIGMOID) ? pro_sigmoid(beta[bh]) : beta[bh];
+    float bt = 1.f;
+    float er[EPL];  // the erase direction e (.) k (Gated DeltaNet-2)
+    if (EW) {
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) er[i] = erase[bh * DK + c0 + i] * kr[i];
+    } else {
+        bt = (pro & GDR_PRO_BETA_SIGMOID) ? pro_sigmoid(beta[bh]) : beta[bh];
+    }
     float* Sh = S + bh * (size_t)dv * DK;
 
     // Loop bounds are uniform across a warp (its 4 rows share `jb`), so every lane reaches the
@@ -114,16 +126,21 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
         for (int i = 0; i < EPL; ++i) { s1[i] = 0.f; s2[i] = 0.f; }
         if (ok1) load_row(Sh + (size_t)j * DK + c0, s1);
         if (ok2) load_row(Sh + (size_t)j2 * DK + c0, s2);
-        const float v1 = ok1 ? load_f32(v + bh * dv + j) : 0.f;
-        const float v2 = ok2 ? load_f32(v + bh * dv + j2) : 0.f;
+        float v1 = ok1 ? load_f32(v + bh * dv + j) : 0.f;
+        float v2 = ok2 ? load_f32(v + bh * dv + j2) : 0.f;
+        if (EW) {  // the gated write target
+            if (ok1) v1 *= write[bh * dv + j];
+            if (ok2) v2 *= write[bh * dv + j2];
+        }
         float p1 = 0.f, a1 = 0.f, p2 = 0.f, a2 = 0.f;
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
+            const float rd = EW ? er[i] : kr[i];  // read direction of the prediction
             s1[i] *= al[i];
-            p1 = fmaf(s1[i], kr[i], p1);
+            p1 = fmaf(s1[i], rd, p1);
             a1 = fmaf(s1[i], qr[i], a1);
             s2[i] *= al[i];
-            p2 = fmaf(s2[i], kr[i], p2);
+            p2 = fmaf(s2[i], rd, p2);
             a2 = fmaf(s2[i], qr[i], a2);
         }
         p1 = group8_sum(p1);
@@ -146,21 +163,27 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
     }
 }
 
-template <typename Tin, typename Tout, int MODE>
-cudaError_t launch_mode(const DecodeProblem& p, cudaStream_t stream) {
+template <typename Tin, typename Tout, int MODE, bool EW>
+cudaError_t launch_mode_ew(const DecodeProblem& p, cudaStream_t stream) {
     const dim3 grid((unsigned)((size_t)p.B * p.H));
     const Tin* q = static_cast<const Tin*>(p.q);
     const Tin* k = static_cast<const Tin*>(p.k);
     const Tin* v = static_cast<const Tin*>(p.v);
     Tout* o = static_cast<Tout*>(p.o);
     switch (p.dk) {
-        case 32: decode_kernel<Tin, Tout, MODE, 32><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale, p.H, p.prologue, p.gate_scale); break;
-        case 64: decode_kernel<Tin, Tout, MODE, 64><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale, p.H, p.prologue, p.gate_scale); break;
-        case 128: decode_kernel<Tin, Tout, MODE, 128><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale, p.H, p.prologue, p.gate_scale); break;
-        case 256: decode_kernel<Tin, Tout, MODE, 256><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale, p.H, p.prologue, p.gate_scale); break;
+        case 32: decode_kernel<Tin, Tout, MODE, 32, EW><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale, p.H, p.prologue, p.gate_scale, p.erase, p.write); break;
+        case 64: decode_kernel<Tin, Tout, MODE, 64, EW><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale, p.H, p.prologue, p.gate_scale, p.erase, p.write); break;
+        case 128: decode_kernel<Tin, Tout, MODE, 128, EW><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale, p.H, p.prologue, p.gate_scale, p.erase, p.write); break;
+        case 256: decode_kernel<Tin, Tout, MODE, 256, EW><<<grid, kThreads, 0, stream>>>(q, k, v, p.g, p.beta, p.S, o, p.dv, p.scale, p.H, p.prologue, p.gate_scale, p.erase, p.write); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
+}
+
+template <typename Tin, typename Tout, int MODE>
+cudaError_t launch_mode(const DecodeProblem& p, cudaStream_t stream) {
+    return p.erase != nullptr ? launch_mode_ew<Tin, Tout, MODE, true>(p, stream)
+                              : launch_mode_ew<Tin, Tout, MODE, false>(p, stream);
 }
 
 template <typename Tin, typename Tout>

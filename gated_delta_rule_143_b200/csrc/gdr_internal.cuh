@@ -28,6 +28,8 @@ struct ChunkProblem {
     float scale;
     int prologue;             // gdr_prologue flags: steps of the mixer layer done on the inputs in-kernel
     const float* gate_scale;  // [H] A of g = -A softplus(a) (GDR_PRO_GATE_SOFTPLUS), NULL = 1
+    const float* erase;       // Gated DeltaNet-2: [B,T,H,d_k] erase gate (NULL: the delta rule with beta)
+    const float* write;       // Gated DeltaNet-2: [B,T,H,d_v] write gate
 };
 
 struct DecodeProblem {
@@ -43,6 +45,8 @@ struct DecodeProblem {
     float scale;
     int prologue;             // as ChunkProblem
     const float* gate_scale;
+    const float* erase;       // Gated DeltaNet-2: [B,H,d_k] erase gate, NULL for the delta rule
+    const float* write;       // Gated DeltaNet-2: [B,H,d_v] write gate
 };
 
 // Everything one backward call needs (gdr_chunk_bwd). Pointers are device pointers.

@@ -204,6 +204,14 @@ def make_raw_chunk_inputs(
     }
 
 
+def make_gdn2_gates(B: int, T: int, H: int, dk: int, dv: int, seed: int) -> Dict[str, torch.Tensor]:
+    """Seeded Gated DeltaNet-2 gates: ``erase`` [B,T,H,dk] and ``write`` [B,T,H,dv], fp32 draws
+    from U(0, 1) (the range of a sigmoid gate). Draw order: erase, write."""
+    gen = torch.Generator().manual_seed(int(seed))
+    return {"erase": torch.rand(B, T, H, dk, generator=gen).contiguous(),
+            "write": torch.rand(B, T, H, dv, generator=gen).contiguous()}
+
+
 def workload_inputs(w: ChunkWorkload, seed: Optional[int] = None) -> Dict[str, Optional[torch.Tensor]]:
     """Inputs of a named chunked workload (its fixed seed unless overridden)."""
     s = WORKLOAD_SEEDS.get(w.name, 0) if seed is None else seed

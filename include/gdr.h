@@ -186,6 +186,37 @@ int gdr_decode_step_ex(const void* q, const void* k, const void* v, const float*
                        int o_dtype, int prologue, const float* gate_scale, void* stream);
 
 /*
+ * gdr_chunk_fwd_gdn2 / gdr_decode_step_gdn2 -- Gated DeltaNet-2: separate channel-wise erase and
+ * write gates in place of the single write strength beta.
+ *
+ * Defined by: "Linear Attention Architectures: Mechanisms, Trade-offs, and Cross-Layer Routing",
+ * Sec. 3 (Gated DeltaNet-2 and the gate definitions before it): the decay-adjusted memory
+ * S_bar = S_{t-1} Diag(alpha_t), a gated erase direction e_t (.) k_t on the key side, a gated write
+ * target w_t (.) v_t on the value side, and one residual written along k_t:
+ *
+ *     S_t = S_bar + (w_t (.) v_t - S_bar (e_t (.) k_t)) k_t^T ,   o_t = S_t q_t / sqrt(d_k).
+ *
+ * The page's formulas are stripped; this reading keeps a single rank-one residual per token and
+ * reduces to gdr_chunk_fwd for e_t = beta_t 1, w_t = beta_t 1 (Kimi Delta Attention with the channel
+ * decay, Gated DeltaNet with the scalar one), as the page states.
+ *
+ *   erase   [B, T, H, d_k] fp32 (decode: [B, H, d_k]); usually in [0, 1]
+ *   write   [B, T, H, d_v] fp32 (decode: [B, H, d_v]); usually in [0, 1]
+ *   the other arguments as gdr_chunk_fwd / gdr_decode_step (no beta; any decay mode).
+ * Runs on the fp32 CUDA-core kernels (the chunk form of gdr_chunk_fwd's CUDA-core path with
+ * A_ri = sum_c e_rc k_rc k_ic exp(Gamma_rc - Gamma_ic) and R = w (.) V - ((e (.) K) * gamma) S^T);
+ * needs no workspace. Chunked: d_k, d_v in {32, 64, 128}, chunk 64; decode: as gdr_decode_step.
+ * Errors as gdr_chunk_fwd / gdr_decode_step.
+ */
+int gdr_chunk_fwd_gdn2(const void* q, const void* k, const void* v, const float* g, const float* erase,
+                       const float* write, const float* S0, void* o, float* S_T, int B, int T, int H,
+                       int d_k, int d_v, int chunk, int mode, int dtype, int o_dtype, void* stream);
+
+int gdr_decode_step_gdn2(const void* q, const void* k, const void* v, const float* g, const float* erase,
+                         const float* write, float* S, void* o, int B, int H, int d_k, int d_v, int mode,
+                         int dtype, int o_dtype, void* stream);
+
+/*
  * gdr_chunk_bwd -- gradients of gdr_chunk_fwd (the training backward pass).
  *
  * Defined by: the forward above (its value is the token recurrence of "Linear Attention & DeltaNet",

@@ -194,3 +194,16 @@ def test_chunk_bwd_workspace_query():
     lib = _lib.lib()
     assert lib.gdr_chunk_bwd_workspace_bytes(2, 100, 3, 64, 32, 1, 0) == 2 * 3 * 100 * 64 * 32 * 4
     assert lib.gdr_chunk_bwd_workspace_bytes(2, 100, 3, 48, 32, 1, 0) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(erase=None), -1), (dict(write=None), -1), (dict(dk=256), -2), (dict(chunk=32), -2),
+    (dict(erase=(4 << 24) + 8), -3), (dict(o=(5 << 24) + 64), -1),
+])
+def test_chunk_fwd_gdn2_rejects_bad_arguments_on_host(kw, code):
+    M = 1 << 24
+    a = dict(q=1 * M, k=2 * M, v=3 * M, g=6 * M, erase=4 * M, write=5 * M, o=7 * M, dk=64, chunk=64)
+    a.update(kw)
+    rc = _lib.lib().gdr_chunk_fwd_gdn2(a["q"], a["k"], a["v"], a["g"], a["erase"], a["write"], None, a["o"], None, 1,
+                                       16, 1, a["dk"], 64, a["chunk"], 2, 0, 0, None)
+    assert rc == code
