@@ -25,7 +25,7 @@ import torch
 from ._lib import (DECAY_MODES, DTYPE_BF16, DTYPE_F32, PLANS, PRO_BETA_SIGMOID, PRO_GATE_SOFTPLUS, PRO_L2NORM_QK,
                    GdrError, check, lib)
 
-__all__ = ["chunk_fwd", "chunk_bwd", "chunk_fwd_gdn2", "decode_step", "decode_step_gdn2", "sync_status", "workspace_bytes", "launches_per_chunk_fwd", "chunk_fwd_plan",
+__all__ = ["chunk_fwd", "chunk_bwd", "chunk_fwd_gdn2", "chunk_fwd_scan", "decode_step", "decode_step_gdn2", "sync_status", "workspace_bytes", "launches_per_chunk_fwd", "chunk_fwd_plan",
            "profile_next_call",
            "GdrError", "DECAY_MODES"]
 
@@ -202,6 +202,34 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optional[t
                                    dv, _mode(mode), _dtype(q), _dtype(out), _stream_handle(stream))
     check(rc)
     return out
+
+
+def chunk_fwd_scan(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optional[torch.Tensor],
+                   beta: torch.Tensor, S0: Optional[torch.Tensor] = None, *, n_seg: int, mode="scalar",
+                   chunk: int = 64, return_state: bool = True, out: Optional[torch.Tensor] = None,
+                   out_dtype: torch.dtype = torch.float32, state_out: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None,
+                   stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """``chunk_fwd`` with every sequence split into ``n_seg`` segments run in parallel
+    (gdr_chunk_fwd_scan); bf16 q/k/v with d_k = d_v = 128 and T a multiple of 64 * n_seg."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    m = _mode(mode)
+    dt = _dtype(q)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=out_dtype, device=q.device)
+    odt = _dtype(out)
+    if return_state and state_out is None:
+        state_out = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = _workspace(lib().gdr_chunk_fwd_scan_workspace_bytes(B, T, H, dk, dv, chunk, m, dt, odt, n_seg),
+                               q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().gdr_chunk_fwd_scan(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(out),
+                                  _ptr(state_out) if return_state else None, B, T, H, dk, dv, chunk, m, dt, odt, n_seg,
+                                  _ptr(workspace), ws_bytes, _stream_handle(stream))
+    check(rc)
+    return out, (state_out if return_state else None)
 
 
 def chunk_fwd_gdn2(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optional[torch.Tensor],

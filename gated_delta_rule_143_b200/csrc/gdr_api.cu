@@ -123,6 +123,68 @@ int prologue_check(int prologue, int mode) {
     return GDR_OK;
 }
 
+// The chunked forward behind gdr_chunk_fwd_ex (n_seg = 0) and gdr_chunk_fwd_scan (n_seg >= 2).
+int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g, const float* beta, const float* S0,
+                   void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk, int mode, int dtype,
+                   int o_dtype, int prologue, const float* gate_scale, int n_seg, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+    ProfileScope prof_scope;
+    if (int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype)) return rc;
+    if (n_seg != 0 && !scan_supported(B, T, H, dk, dv, chunk, dtype, o_dtype, n_seg))
+        return fail(GDR_ERR_UNSUPPORTED,
+                    "segment scan: bf16 q/k/v, d_k = d_v = 128, chunk 64, n_seg >= 2 and T a multiple of "
+                    "n_seg * chunk (got T=%d, n_seg=%d)", T, n_seg);
+    if (int rc = prologue_check(prologue, mode)) return rc;
+    if (!(prologue & GDR_PRO_GATE_SOFTPLUS)) gate_scale = nullptr;
+    if (!q || !k || !v || !beta || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, beta and o must be non-null");
+    if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
+    const void* ptrs[] = {q, k, v, g, beta, S0, o, S_T, workspace, gate_scale};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return fail(GDR_ERR_MISALIGNED, "pointer %p is not 16-byte aligned", p);
+    const size_t ntok = (size_t)B * T * H;
+    const size_t eb = elem_bytes(dtype);
+    const size_t bq = ntok * dk * eb, bv = ntok * dv * eb, bb = ntok * sizeof(float);
+    const size_t bo = ntok * dv * elem_bytes(o_dtype);
+    const size_t bg = mode == GDR_DECAY_NONE ? 0 : (mode == GDR_DECAY_SCALAR ? bb : ntok * dk * sizeof(float));
+    const size_t bs = (size_t)B * H * dv * dk * sizeof(float);
+    struct Span { const void* p; size_t n; const char* name; };
+    const Span ins[] = {{q, bq, "q"}, {k, bq, "k"}, {v, bv, "v"}, {mode == GDR_DECAY_NONE ? nullptr : g, bg, "g"},
+                        {beta, bb, "beta"}, {S0, bs, "S0"}, {gate_scale, H * sizeof(float), "gate_scale"}};
+    for (const Span& s : ins) {
+        if (overlap(o, bo, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "o overlaps input %s", s.name);
+        if (S_T != S0 && overlap(S_T, bs, s.p, s.n))
+            return fail(GDR_ERR_INVALID_ARG, "S_T overlaps input %s (only S_T == S0 is allowed)", s.name);
+    }
+    if (overlap(o, bo, S_T, bs)) return fail(GDR_ERR_INVALID_ARG, "o overlaps S_T");
+    const bool use_tc = chunk_tc_supported(dk, dv, chunk, dtype, o_dtype);
+    const size_t need = n_seg != 0 ? scan_workspace_bytes(B, T, H, mode, n_seg, o_dtype)
+                                   : (use_tc ? chunk_tc_workspace_bytes(B, T, H, dk, dv, chunk, mode) : 0);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+        return fail(GDR_ERR_WORKSPACE, "workspace of %zu bytes required (got %zu at %p)", need, workspace_bytes,
+                    workspace);
+    if (need > 0) {
+        for (const Span& s : ins)
+            if (overlap(workspace, need, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "workspace overlaps %s", s.name);
+        if (overlap(workspace, need, o, bo) || overlap(workspace, need, S_T, bs))
+            return fail(GDR_ERR_INVALID_ARG, "workspace overlaps an output");
+    }
+    int* status = nullptr;
+    int major = 0;
+    if (int rc = device_setup(&status, &major)) return rc;
+    if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
+
+    ChunkProblem p{q, k, v, mode == GDR_DECAY_NONE ? nullptr : g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode,
+                   dtype, o_dtype, workspace, workspace_bytes, status, (float)(1.0 / sqrt((double)dk)), prologue,
+                   gate_scale};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t err = n_seg != 0 ? launch_scan(p, n_seg, s) : (use_tc ? launch_chunk_tc(p, s) : launch_chunk_simt(p, s));
+    if (err != cudaSuccess)
+        return fail(GDR_ERR_CUDA, "%s chunk launch: %s", n_seg ? "segment-scan" : (use_tc ? "tensor-core" : "fp32"),
+                    cudaGetErrorString(err));
+    return ok();
+}
+
+
 }  // namespace
 
 void profile_after_launch(cudaStream_t stream) {
@@ -183,54 +245,27 @@ int gdr_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* g
                      const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk,
                      int mode, int dtype, int o_dtype, int prologue, const float* gate_scale, void* workspace,
                      size_t workspace_bytes, void* stream) {
-    ProfileScope prof_scope;
-    if (int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype)) return rc;
-    if (int rc = prologue_check(prologue, mode)) return rc;
-    if (!(prologue & GDR_PRO_GATE_SOFTPLUS)) gate_scale = nullptr;
-    if (!q || !k || !v || !beta || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, beta and o must be non-null");
-    if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
-    const void* ptrs[] = {q, k, v, g, beta, S0, o, S_T, workspace, gate_scale};
-    for (const void* p : ptrs)
-        if (p && !aligned16(p)) return fail(GDR_ERR_MISALIGNED, "pointer %p is not 16-byte aligned", p);
-    const size_t ntok = (size_t)B * T * H;
-    const size_t eb = elem_bytes(dtype);
-    const size_t bq = ntok * dk * eb, bv = ntok * dv * eb, bb = ntok * sizeof(float);
-    const size_t bo = ntok * dv * elem_bytes(o_dtype);
-    const size_t bg = mode == GDR_DECAY_NONE ? 0 : (mode == GDR_DECAY_SCALAR ? bb : ntok * dk * sizeof(float));
-    const size_t bs = (size_t)B * H * dv * dk * sizeof(float);
-    struct Span { const void* p; size_t n; const char* name; };
-    const Span ins[] = {{q, bq, "q"}, {k, bq, "k"}, {v, bv, "v"}, {mode == GDR_DECAY_NONE ? nullptr : g, bg, "g"},
-                        {beta, bb, "beta"}, {S0, bs, "S0"}, {gate_scale, H * sizeof(float), "gate_scale"}};
-    for (const Span& s : ins) {
-        if (overlap(o, bo, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "o overlaps input %s", s.name);
-        if (S_T != S0 && overlap(S_T, bs, s.p, s.n))
-            return fail(GDR_ERR_INVALID_ARG, "S_T overlaps input %s (only S_T == S0 is allowed)", s.name);
-    }
-    if (overlap(o, bo, S_T, bs)) return fail(GDR_ERR_INVALID_ARG, "o overlaps S_T");
-    const bool use_tc = chunk_tc_supported(dk, dv, chunk, dtype, o_dtype);
-    const size_t need = use_tc ? chunk_tc_workspace_bytes(B, T, H, dk, dv, chunk, mode) : 0;
-    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
-        return fail(GDR_ERR_WORKSPACE, "workspace of %zu bytes required (got %zu at %p)", need, workspace_bytes,
-                    workspace);
-    if (need > 0) {
-        for (const Span& s : ins)
-            if (overlap(workspace, need, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "workspace overlaps %s", s.name);
-        if (overlap(workspace, need, o, bo) || overlap(workspace, need, S_T, bs))
-            return fail(GDR_ERR_INVALID_ARG, "workspace overlaps an output");
-    }
-    int* status = nullptr;
-    int major = 0;
-    if (int rc = device_setup(&status, &major)) return rc;
-    if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
+    return chunk_fwd_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, prologue,
+                          gate_scale, 0, workspace, workspace_bytes, stream);
+}
 
-    ChunkProblem p{q, k, v, mode == GDR_DECAY_NONE ? nullptr : g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode,
-                   dtype, o_dtype, workspace, workspace_bytes, status, (float)(1.0 / sqrt((double)dk)), prologue,
-                   gate_scale};
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const cudaError_t err = use_tc ? launch_chunk_tc(p, s) : launch_chunk_simt(p, s);
-    if (err != cudaSuccess)
-        return fail(GDR_ERR_CUDA, "%s chunk launch: %s", use_tc ? "tensor-core" : "fp32", cudaGetErrorString(err));
-    return ok();
+int gdr_chunk_fwd_scan(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                       const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk,
+                       int mode, int dtype, int o_dtype, int n_seg, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+    if (n_seg < 2) return fail(GDR_ERR_INVALID_ARG, "n_seg = %d (at least 2)", n_seg);
+    return chunk_fwd_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, GDR_PRO_NONE,
+                          nullptr, n_seg, workspace, workspace_bytes, stream);
+}
+
+size_t gdr_chunk_fwd_scan_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int mode, int dtype,
+                                          int o_dtype, int n_seg) {
+    char saved[sizeof(g_last_error)];
+    memcpy(saved, g_last_error, sizeof(saved));
+    const int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype);
+    memcpy(g_last_error, saved, sizeof(saved));
+    if (rc != GDR_OK || !scan_supported(B, T, H, dk, dv, chunk, dtype, o_dtype, n_seg)) return 0;
+    return scan_workspace_bytes(B, T, H, mode, n_seg, o_dtype);
 }
 
 int gdr_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,

@@ -118,6 +118,13 @@ cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream);
 int chunk_tc_launches(int B, int T, int H, int dk, int dv, int chunk, int mode);
 int chunk_tc_plan(int B, int T, int H, int dk, int dv, int chunk, int mode, int* precomputed_chunks);
 
+// Segment scan (sequence-parallel forward) on the tensor-core path: the chunked forward on the
+// [B * n_seg, T / n_seg, H] view twice (data from a zero state; identity state with v = 0), a carry
+// of the incoming states across the segments and a tensor-core correction of the outputs.
+bool scan_supported(int B, int T, int H, int dk, int dv, int chunk, int dtype, int o_dtype, int n_seg);
+size_t scan_workspace_bytes(int B, int T, int H, int mode, int n_seg, int o_dtype);
+cudaError_t launch_scan(const ChunkProblem& p, int n_seg, cudaStream_t stream);
+
 // Self-test of the bounded waits (gdr_selftest_bounded_wait): one CTA whose roles wait on a flag
 // that nothing sets, with a wait bound of limit_ns; then the time it ran, read after the stream.
 cudaError_t launch_bounded_wait_selftest(int* status, uint64_t limit_ns, cudaStream_t stream);

@@ -186,6 +186,38 @@ int gdr_decode_step_ex(const void* q, const void* k, const void* v, const float*
                        int o_dtype, int prologue, const float* gate_scale, void* stream);
 
 /*
+ * gdr_chunk_fwd_scan -- gdr_chunk_fwd with each sequence split into n_seg segments that run in
+ * parallel (sequence-level parallelism for few heads and long sequences).
+ *
+ * Defined by: "linear attention and its gated descendants", Hardware Performance (with few
+ * sequences x heads there is not enough parallel work; sequence-level parallelism) and the closing
+ * summary of the gated variants (the update is a transition plus a write, S_t = S_{t-1} A_t + B_t,
+ * with A_t = Diag(alpha_t)(I - beta_t k_t k_t^T) and B_t = beta_t v_t k_t^T in this library's
+ * orientation, and such maps compose associatively). With segments of T / n_seg tokens, M(i) the
+ * product of the A_t of segment i and ^0 a run from a zero state:
+ *     S_in(i + 1) = S_in(i) M(i) + S_end^0(i),   S_in(0) = S0,   S_T = S_in(n_seg),
+ *     o_t = o_t^0 + S_in(i) (scale * prod_{u <= t in segment i} A_u) q_t.
+ * The library computes o^0 and S_end^0 by the chunked forward on the [B * n_seg, T / n_seg, H] view
+ * of the inputs, M(i) and the per-token read-outs by the same forward with v = 0 from the identity
+ * state, then the carry (n_seg steps per head) and the correction on warp MMAs (tf32 operands,
+ * fp32 accumulation). The result equals gdr_chunk_fwd's up to rounding.
+ *
+ * Arguments as gdr_chunk_fwd, plus n_seg >= 2. Supported: the tensor-core shapes (bf16 q/k/v,
+ * d_k = d_v = 128, chunk 64), any decay mode, T a multiple of n_seg * 64; otherwise
+ * GDR_ERR_UNSUPPORTED. S_T may be S0. workspace: gdr_chunk_fwd_scan_workspace_bytes(...) bytes
+ * (the forward's workspace for the view, a zero value tensor, the per-token read-outs in fp32 and
+ * four states per segment; plus an fp32 copy of o when o is bf16).
+ */
+int gdr_chunk_fwd_scan(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                       const float* S0, void* o, float* S_T, int B, int T, int H, int d_k, int d_v,
+                       int chunk, int mode, int dtype, int o_dtype, int n_seg, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* Workspace of gdr_chunk_fwd_scan (0 for arguments it would reject). Host-only. */
+size_t gdr_chunk_fwd_scan_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, int mode,
+                                          int dtype, int o_dtype, int n_seg);
+
+/*
  * gdr_chunk_fwd_gdn2 / gdr_decode_step_gdn2 -- Gated DeltaNet-2: separate channel-wise erase and
  * write gates in place of the single write strength beta.
  *
