@@ -80,6 +80,11 @@ def kernel_bytes(w, plan, c1):
         nc = -(-w.T // w.chunk)
         pre = inputs * c1 // nc
         return [("chunk_prep", pre), ("chunk_fused", inputs - pre + outputs)]
+    if plan == "scan":
+        # prep reads the inputs; the state kernel's o^0 and read-outs are intermediate; the carry
+        # writes S_T and the correction writes o
+        st = w.B * w.H * w.dv * w.dk * 4
+        return [("chunk_prep", inputs), ("chunk_state", 0), ("scan_carry", st), ("scan_correct", outputs - st)]
     return [("chunk_fused" if plan == "fused" else "chunk_simt", inputs + outputs)]
 
 

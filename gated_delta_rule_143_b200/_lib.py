@@ -21,7 +21,7 @@ STATUS_NAMES = {
 }
 DECAY_MODES = {"none": 0, "scalar": 1, "channel": 2}
 DTYPE_F32, DTYPE_BF16 = 0, 1
-PLANS = {0: "invalid", 1: "cuda_core", 2: "two_pass", 3: "fused", 4: "prep_fused"}
+PLANS = {0: "invalid", 1: "cuda_core", 2: "two_pass", 3: "fused", 4: "prep_fused", 5: "scan"}
 PRO_L2NORM_QK, PRO_BETA_SIGMOID, PRO_GATE_SOFTPLUS = 1, 2, 4  # gdr_prologue flags
 
 # Every symbol the header declares: name -> (restype, argtypes).

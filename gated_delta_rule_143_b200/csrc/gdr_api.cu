@@ -123,13 +123,26 @@ int prologue_check(int prologue, int mode) {
     return GDR_OK;
 }
 
-// The chunked forward behind gdr_chunk_fwd_ex (n_seg = 0) and gdr_chunk_fwd_scan (n_seg >= 2).
+// Segments gdr_chunk_fwd gives a problem on its own: few heads and long sequences, where one serial
+// chain per head leaves most SMs idle (measured on the 16-head, 65536-token workload: 4 segments run
+// in 0.73 of the time of the fused plan). 0: no segment scan.
+int auto_segments(int B, int T, int H, int dk, int dv, int chunk, int dtype, int o_dtype) {
+    constexpr int kSeg = 4;
+    const int NC = (T + chunk - 1) / chunk;
+    if ((size_t)B * H > 16 || NC < 512) return 0;
+    return scan_supported(B, T, H, dk, dv, chunk, dtype, o_dtype, kSeg) ? kSeg : 0;
+}
+
+// The chunked forward behind gdr_chunk_fwd_ex and gdr_chunk_fwd_scan. n_seg: 0 = the plan chosen from
+// the shape (auto_segments), -1 = no segment scan, >= 2 = that many segments.
 int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g, const float* beta, const float* S0,
                    void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk, int mode, int dtype,
                    int o_dtype, int prologue, const float* gate_scale, int n_seg, void* workspace,
                    size_t workspace_bytes, void* stream) {
     ProfileScope prof_scope;
     if (int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype)) return rc;
+    if (n_seg == 0) n_seg = auto_segments(B, T, H, dk, dv, chunk, dtype, o_dtype);
+    if (n_seg < 0) n_seg = 0;
     if (n_seg != 0 && !scan_supported(B, T, H, dk, dv, chunk, dtype, o_dtype, n_seg))
         return fail(GDR_ERR_UNSUPPORTED,
                     "segment scan: bf16 q/k/v, d_k = d_v = 128, chunk 64, n_seg >= 2 and T a multiple of "
@@ -216,6 +229,7 @@ size_t gdr_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int ch
     const int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype);
     memcpy(g_last_error, saved, sizeof(saved));
     if (rc != GDR_OK) return 0;
+    if (const int ns = auto_segments(B, T, H, dk, dv, chunk, dtype, o_dtype)) return scan_workspace_bytes(B, T, H, mode, ns, o_dtype);
     if (chunk_tc_supported(dk, dv, chunk, dtype, o_dtype)) return chunk_tc_workspace_bytes(B, T, H, dk, dv, chunk, mode);
     return 0;
 }
@@ -229,6 +243,10 @@ int gdr_chunk_fwd_plan(int B, int T, int H, int dk, int dv, int chunk, int mode,
     if (precomputed_chunks != nullptr) *precomputed_chunks = 0;
     if (rc != GDR_OK) return GDR_PLAN_INVALID;
     if (!chunk_tc_supported(dk, dv, chunk, dtype, o_dtype)) return GDR_PLAN_CUDA_CORE;
+    if (const int ns = auto_segments(B, T, H, dk, dv, chunk, dtype, o_dtype)) {
+        if (precomputed_chunks != nullptr) *precomputed_chunks = ns;
+        return GDR_PLAN_SCAN;
+    }
     return chunk_tc_plan(B, T, H, dk, dv, chunk, mode, precomputed_chunks);
 }
 
@@ -238,6 +256,7 @@ int gdr_chunk_fwd_launches(int B, int T, int H, int dk, int dv, int chunk, int m
     const int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype);
     memcpy(g_last_error, saved, sizeof(saved));
     if (rc != GDR_OK) return 0;
+    if (auto_segments(B, T, H, dk, dv, chunk, dtype, o_dtype)) return 4;  // prep, state, carry, correction
     return chunk_tc_supported(dk, dv, chunk, dtype, o_dtype) ? chunk_tc_launches(B, T, H, dk, dv, chunk, mode) : 1;
 }
 
@@ -547,8 +566,8 @@ extern "C" int gdr_chunk_fwd_noalloc(const void* q, const void* k, const void* v
                     need, (size_t)GDR_NOALLOC_SCRATCH_BYTES);
     void* ws = nullptr;
     if (int rc = noalloc_scratch(&ws)) return rc;
-    return gdr_chunk_fwd(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, ws,
-                         (size_t)GDR_NOALLOC_SCRATCH_BYTES, stream);
+    return chunk_fwd_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, GDR_PRO_NONE,
+                          nullptr, -1, ws, (size_t)GDR_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 // ------------------------------------------------------------ host-buffer entry point --

@@ -768,6 +768,10 @@ struct StateArgs {
     int T, H, NC;
     float scale;
     int* status;
+    // Segment scan: CTAs bh >= n_data run the transition chain of head bh - n_data over the same
+    // hand-off blocks (identity initial state, U taken as zero), writing their state to S_T2.
+    int n_data;
+    float* S_T2;
 };
 
 // Where the state pass finds hand-off block c of its head, when that block is complete, and how it
@@ -807,7 +811,7 @@ struct RingSource {       // fused kernel: chunks c < c1 were written to `pre` b
 // Walks the chunks in order, reading hand-off block c through `src`.
 template <typename Tout, typename Src>
 __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, const Src& src, uint8_t* sm,
-                           uint32_t tbase, volatile int* abort) {
+                           uint32_t tbase, volatile int* abort, bool tr = false) {
     auto stageA = [sm](int i) { return sm + kSStageA0 + i * (kSStageA1 - kSStageA0); };  // part A stage i
     auto sUT = [sm](int i) { return sm + kSUT0 + i * (kSUT1 - kSUT0); };  // U^T stage i
     auto sO = [sm](int i) { return sm + kSO0 + i * (kSO1 - kSO0); };  // output staging buffer i
@@ -1009,7 +1013,7 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
         bool ok;
         {
             float x[32];
-            const float* s0 = A.S0 ? A.S0 + ((size_t)bh * kD + j) * kD + 32 * cg : nullptr;
+            const float* s0 = (A.S0 && !tr) ? A.S0 + ((size_t)bh * kD + j) * kD + 32 * cg : nullptr;
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
                 const float4 t = s0 ? *reinterpret_cast<const float4*>(s0 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1017,6 +1021,10 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
                 x[e + 1] = t.y;
                 x[e + 2] = t.z;
                 x[e + 3] = t.w;
+            }
+            if (tr) {  // transition chain: the identity
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[e] = (j == 32 * cg + e) ? 1.f : 0.f;
             }
             hand_over(x);
             ok = decay(x, 0);
@@ -1030,8 +1038,13 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
             {
                 float x[16], u[16];
                 tmem_ld16(tD1 + lane_off + 16 * cg, x);
-                unpack8h(ld16(sUT(sb) + kmajor_off(j, 16 * cg, 128)), u);
-                unpack8h(ld16(sUT(sb) + kmajor_off(j, 16 * cg + 8, 128)), u + 8);
+                if (tr) {  // transition chain: no write (v = 0 gives U = 0)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) u[e] = 0.f;
+                } else {
+                    unpack8h(ld16(sUT(sb) + kmajor_off(j, 16 * cg, 128)), u);
+                    unpack8h(ld16(sUT(sb) + kmajor_off(j, 16 * cg + 8, 128)), u + 8);
+                }
                 tmem_ld_wait();
                 uint32_t w[8];
 #pragma unroll
@@ -1050,8 +1063,8 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
             tmem_ld_wait();
             if (c + 1 < NC) {
                 hand_over(x);
-            } else if (A.S_T != nullptr) {
-                float* dst = A.S_T + ((size_t)bh * kD + j) * kD + 32 * cg;
+            } else if ((tr ? A.S_T2 : A.S_T) != nullptr) {
+                float* dst = (tr ? A.S_T2 : A.S_T) + ((size_t)bh * kD + j) * kD + 32 * cg;
 #pragma unroll
                 for (int e = 0; e < 32; e += 4)
                     *reinterpret_cast<float4*>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
@@ -1081,10 +1094,12 @@ __device__ void state_body(const CUtensorMap* mo, const StateArgs& A, int bh, co
     }
 }
 
-// Two-pass state kernel: one CTA per (b, h), hand-off blocks from the workspace.
+// Two-pass state kernel: one CTA per (b, h), hand-off blocks from the workspace. For the segment
+// scan, CTAs n_data .. 2 n_data - 1 run the transition chains of the same heads (output map mo2).
 template <typename Tout>
 __global__ void __launch_bounds__(kStateThreads, 1)
-chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const uint8_t* __restrict__ ws) {
+chunk_state_kernel(const __grid_constant__ CUtensorMap mo, const __grid_constant__ CUtensorMap mo2, StateArgs A,
+                   const uint8_t* __restrict__ ws) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
@@ -1097,9 +1112,10 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mo, StateArgs A, const ui
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const int bh = blockIdx.x;
+    const bool tr = (int)blockIdx.x >= A.n_data;
+    const int bh = tr ? (int)blockIdx.x - A.n_data : (int)blockIdx.x;
     const WorkspaceSource src{ws + (size_t)bh * A.NC * kHandoffStride, kHandoffStride};
-    state_body<Tout>(&mo, A, bh, src, align1024(smem_raw), tmem_base, &abort_flag);
+    state_body<Tout>(tr ? &mo2 : &mo, A, bh, src, align1024(smem_raw), tmem_base, &abort_flag, tr);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1273,8 +1289,8 @@ cudaError_t launch_state(const ChunkProblem& p, const CUtensorMap& mo, int NC, c
     auto kern = chunk_state_kernel<Tout>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem);
     if (err != cudaSuccess) return err;
-    StateArgs A{p.S0, p.S_T, p.T, p.H, NC, p.scale, p.status};
-    kern<<<p.B * p.H, kStateThreads, kStateSmem, stream>>>(mo, A, static_cast<const uint8_t*>(p.workspace));
+    StateArgs A{p.S0, p.S_T, p.T, p.H, NC, p.scale, p.status, p.B * p.H, nullptr};
+    kern<<<p.B * p.H, kStateThreads, kStateSmem, stream>>>(mo, mo, A, static_cast<const uint8_t*>(p.workspace));
     profile_after_launch(stream);
     return cudaGetLastError();
 }
@@ -1336,7 +1352,7 @@ cudaError_t launch_fused(const ChunkProblem& p, const CUtensorMap& mq, const CUt
     if ((err = cudaMemsetAsync(flags, 0, flag_bytes(BH, NC), stream)) != cudaSuccess) return err;
     if (c1 > 0 && (err = launch_prep<MODE, PRO>(p, mq, mk, mv, NC, c1, ws, stream)) != cudaSuccess) return err;
     PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status, p.prologue, p.gate_scale};
-    StateArgs A{p.S0, p.S_T, p.T, p.H, NC, p.scale, p.status};
+    StateArgs A{p.S0, p.S_T, p.T, p.H, NC, p.scale, p.status, p.B * p.H, nullptr};
     CUtensorMap aq = mq, ak = mk, av = mv, ao = mo;
     void* args[] = {&aq, &ak, &av, &ao, &P, &A, &R};
     err = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(kStateThreads), args,
@@ -1413,6 +1429,37 @@ cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     if (p.o_dtype == GDR_BF16) return launch_state<__nv_bfloat16>(p, mo, NC, stream);
     return launch_state<float>(p, mo, NC, stream);
+}
+
+size_t chunk_tc_pair_workspace_bytes(int B, int T, int H) {
+    return (size_t)B * H * ((T + kC - 1) / kC) * kHandoffStride;
+}
+
+// Segment scan: the prep pass over every chunk, then one state-kernel launch whose first B * H CTAs
+// run the data chains (o -> p.o, S_T -> p.S_T) and whose other B * H CTAs run the transition chains
+// over the same hand-off blocks (identity state, no write: per-token read-outs -> o2, S_T -> S_T2).
+// p.o and o2 are fp32.
+cudaError_t launch_chunk_tc_pair(const ChunkProblem& p, void* o2, float* S_T2, cudaStream_t stream) {
+    const int NC = (p.T + kC - 1) / kC;
+    CUtensorMap mq, mk, mv, mo, mo2;
+    cudaError_t err;
+    if ((err = make_map(&mq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, 64)) != cudaSuccess) return err;
+    if ((err = make_map(&mk, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, 64)) != cudaSuccess) return err;
+    if ((err = make_map(&mv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, 64)) != cudaSuccess) return err;
+    if ((err = make_map(&mo, p.o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.B, p.T, p.H, 32)) != cudaSuccess) return err;
+    if ((err = make_map(&mo2, o2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.B, p.T, p.H, 32)) != cudaSuccess) return err;
+    uint8_t* ws = static_cast<uint8_t*>(p.workspace);
+    err = p.prologue ? launch_prep_mode<true>(p, mq, mk, mv, NC, ws, stream)
+                     : launch_prep_mode<false>(p, mq, mk, mv, NC, ws, stream);
+    if (err != cudaSuccess) return err;
+    auto kern = chunk_state_kernel<float>;
+    if ((err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem)) != cudaSuccess)
+        return err;
+    const int BH = p.B * p.H;
+    StateArgs A{p.S0, p.S_T, p.T, p.H, NC, p.scale, p.status, BH, S_T2};
+    kern<<<2 * BH, kStateThreads, kStateSmem, stream>>>(mo, mo2, A, ws);
+    profile_after_launch(stream);
+    return cudaGetLastError();
 }
 
 }  // namespace gdr

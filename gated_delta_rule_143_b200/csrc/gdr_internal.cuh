@@ -118,6 +118,11 @@ cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream);
 int chunk_tc_launches(int B, int T, int H, int dk, int dv, int chunk, int mode);
 int chunk_tc_plan(int B, int T, int H, int dk, int dv, int chunk, int mode, int* precomputed_chunks);
 
+// The prep pass and a state kernel running both the data chains and, over the same blocks, the
+// transition chains (identity state, no write) of every head; outputs fp32 (segment scan).
+size_t chunk_tc_pair_workspace_bytes(int B, int T, int H);
+cudaError_t launch_chunk_tc_pair(const ChunkProblem& p, void* o2, float* S_T2, cudaStream_t stream);
+
 // Segment scan (sequence-parallel forward) on the tensor-core path: the chunked forward on the
 // [B * n_seg, T / n_seg, H] view twice (data from a zero state; identity state with v = 0), a carry
 // of the incoming states across the segments and a tensor-core correction of the outputs.

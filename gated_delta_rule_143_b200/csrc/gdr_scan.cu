@@ -9,14 +9,16 @@
 //   S_end(i)  = S_in(i) M(i) + S_end^0(i),   M(i) = prod of the A_t of segment i,
 //   o_t       = o_t^0 + S_in(i) (scale * prod_{u <= t in segment i} A_u q_t)      (t in segment i)
 //
-// where ^0 marks the segment run from a zero state. Both parts come from the chunked forward run on
-// the [B*s, T/s, H] view of the same tensors, so every segment is an independent "sequence":
-//   run A: the inputs, S0 = 0             -> o^0 and S_end^0(i);
-//   run B: v = 0, S0 = I (d_v = d_k)      -> O_I = scale * prod A q_t per token, and S_T = M(i);
-//   carry: S_in(0) = S0, S_in(i+1) = S_in(i) M(i) + S_end^0(i) (s steps per head, rows in parallel);
-//   correction: o = o^0 + O_I S_in(i)^T on warp MMAs (tf32 operands, fp32 accumulation).
-// The chains of runs A and B are s times shorter than the sequence's and s times as many run at
-// once; the price is the second run and the correction's traffic.
+// where ^0 marks the segment run from a zero state. Both parts come from the chunked forward on the
+// [B*s, T/s, H] view of the same tensors, so every segment is an independent "sequence": one prep pass
+// writes the hand-off blocks of every chunk, and one state-kernel launch runs over them
+//   the data chains:       S0 = 0                    -> o^0 and S_end^0(i);
+//   the transition chains: S0 = I, no write (U = 0)  -> O_I = scale * prod A q_t per token, S_T = M(i)
+// (the transition of a chunk, Diag(gamma_C) - W^T K~, needs only the blocks' S-independent factors).
+// Then the carry, S_in(0) = S0, S_in(i+1) = S_in(i) M(i) + S_end^0(i) (s steps per head, rows in
+// parallel), and the correction o = o^0 + O_I S_in(i)^T on warp MMAs (tf32 operands, fp32
+// accumulation). The chains are s times shorter than the sequence's and 2 s times as many run at once;
+// the price is the transition chains and the correction's traffic.
 #include "gdr_sm100.cuh"
 
 namespace gdr {
@@ -25,14 +27,6 @@ namespace {
 using namespace sm100;
 
 constexpr int kSD = 128;  // d_k = d_v on this path
-
-__global__ void fill_identity_kernel(float* __restrict__ S, size_t n) {
-    const size_t total = n * kSD * kSD;
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
-        const int r = (int)((i / kSD) % kSD), c = (int)(i % kSD);
-        S[i] = r == c ? 1.f : 0.f;
-    }
-}
 
 // One CTA per (8 state rows, head). Segment-head (b, i, h) has index (b * s + i) * H + h in the
 // run-A/B state arrays. Writes S_in(i) for every segment and S_in(s) = S_T.
@@ -162,17 +156,16 @@ scan_correct_kernel(const float* o0, const float* __restrict__ OI, const float* 
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct ScanLayout {
-    size_t run, vzero, ident, oi, m, send, sin, o0, total;
+    size_t run, oi, m, send, sin, o0, total;
 };
 
 ScanLayout scan_layout(int B, int T, int H, int mode, int n_seg, int o_dtype) {
+    (void)mode;
     ScanLayout L{};
     const int Ts = T / n_seg;
     const size_t nsh = (size_t)B * n_seg * H, ntok = (size_t)B * T * H;
     size_t off = 0;
-    L.run = off;   off += al256(chunk_tc_workspace_bytes(B * n_seg, Ts, H, kSD, kSD, 64, mode));
-    L.vzero = off; off += al256(ntok * kSD * 2);
-    L.ident = off; off += al256(nsh * kSD * kSD * 4);
+    L.run = off;   off += al256(chunk_tc_pair_workspace_bytes(B * n_seg, Ts, H));
     L.oi = off;    off += al256(ntok * kSD * 4);
     L.m = off;     off += al256(nsh * kSD * kSD * 4);
     L.send = off;  off += al256(nsh * kSD * kSD * 4);
@@ -203,11 +196,10 @@ cudaError_t launch_scan(const ChunkProblem& p, int n_seg, cudaStream_t stream) {
     float* M = reinterpret_cast<float*>(ws + L.m);
     float* send = reinterpret_cast<float*>(ws + L.send);
     float* sin = reinterpret_cast<float*>(ws + L.sin);
-    float* ident = reinterpret_cast<float*>(ws + L.ident);
     float* o0 = p.o_dtype == GDR_F32 ? static_cast<float*>(p.o) : reinterpret_cast<float*>(ws + L.o0);
     cudaError_t err;
 
-    // run A: every segment from a zero state
+    // every segment from a zero state, and every segment's transition, over one set of blocks
     ChunkProblem a = p;
     a.B = Bs;
     a.T = Ts;
@@ -216,19 +208,8 @@ cudaError_t launch_scan(const ChunkProblem& p, int n_seg, cudaStream_t stream) {
     a.o_dtype = GDR_F32;
     a.S_T = send;
     a.workspace = ws + L.run;
-    a.workspace_bytes = L.vzero - L.run;
-    if ((err = launch_chunk_tc(a, stream)) != cudaSuccess) return err;
-    // run B: v = 0 from the identity: the segment's transition and its read-out per token
-    if ((err = cudaMemsetAsync(ws + L.vzero, 0, (size_t)p.B * p.T * p.H * kSD * 2, stream)) != cudaSuccess) return err;
-    fill_identity_kernel<<<296, 256, 0, stream>>>(ident, nsh);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    profile_after_launch(stream);
-    ChunkProblem bq = a;
-    bq.v = ws + L.vzero;
-    bq.S0 = ident;
-    bq.o = oi;
-    bq.S_T = M;
-    if ((err = launch_chunk_tc(bq, stream)) != cudaSuccess) return err;
+    a.workspace_bytes = L.oi - L.run;
+    if ((err = launch_chunk_tc_pair(a, oi, M, stream)) != cudaSuccess) return err;
     // carry the true incoming state across the segments
     const size_t carry_smem = (size_t)(kSD * kSD + kCarryRows * kSD) * sizeof(float);
     if ((err = cudaFuncSetAttribute(scan_carry_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)carry_smem)) !=

@@ -106,7 +106,8 @@ typedef enum {
  * Launches (tensor-core path): DeltaNet and the scalar gate with B * H <= 100 run as one
  * cooperative kernel with one CTA per SM, in which the per-chunk factor pipelines hand their
  * blocks to the per-head state passes through a ring in the workspace: eight blocks per head
- * (0.6 MB per head) up to 56 heads. Above 56 heads a prep kernel on every SM first writes the
+ * (0.6 MB per head) up to 56 heads (but few heads with long sequences run the segment scan of
+ * gdr_chunk_fwd_scan with 4 segments; see gdr_chunk_fwd_plan). Above 56 heads a prep kernel on every SM first writes the
  * blocks of the leading chunks of each head to the workspace, and the ring has a slot for every
  * later chunk. The workspace then holds one block (73 KB) per chunk of every head. The channel
  * gate and more heads use two kernels that exchange every block through the workspace.
@@ -293,16 +294,21 @@ typedef enum {
     GDR_PLAN_CUDA_CORE = 1,    /* one fp32 CUDA-core kernel */
     GDR_PLAN_TWO_PASS = 2,     /* tensor cores: prep kernel (all chunks), then state kernel */
     GDR_PLAN_FUSED = 3,        /* tensor cores: one cooperative kernel (prep and state passes) */
-    GDR_PLAN_PREP_FUSED = 4    /* tensor cores: prep kernel for the first chunks of every head, then
+    GDR_PLAN_PREP_FUSED = 4,   /* tensor cores: prep kernel for the first chunks of every head, then
                                   the cooperative kernel for the rest */
+    GDR_PLAN_SCAN = 5          /* tensor cores: segment scan (see gdr_chunk_fwd_scan): prep kernel, one
+                                  state kernel for the segments' data and transition chains, carry,
+                                  output correction */
 } gdr_plan;
 
 /* The plan gdr_chunk_fwd uses for this problem (a gdr_plan value). For GDR_PLAN_PREP_FUSED,
  * *precomputed_chunks (if not NULL) receives the number of leading chunks per head the first
- * kernel prepares; 0 otherwise. Chosen from the shape alone: B * H <= 56 heads run fused (the
- * chains are the bound), 57-100 heads prepare the first chunks on every SM so that the fused
- * kernel's remaining prep CTAs keep up with the chains, more than 100 heads or the channel gate
- * run two passes. */
+ * kernel prepares; for GDR_PLAN_SCAN, the number of segments; 0 otherwise. Chosen from the shape
+ * alone: at most 16 heads with at least 512 chunks each (T a multiple of 256) run the segment scan
+ * with 4 segments; otherwise B * H <= 56 heads run fused (the chains are the bound), 57-100 heads
+ * prepare the first chunks on every SM so that the fused kernel's remaining prep CTAs keep up with
+ * the chains, more than 100 heads or the channel gate run two passes. gdr_chunk_fwd_noalloc never
+ * uses the segment scan. */
 int gdr_chunk_fwd_plan(int B, int T, int H, int d_k, int d_v, int chunk, int mode, int dtype,
                        int o_dtype, int* precomputed_chunks);
 

@@ -114,6 +114,14 @@ def test_plan_query_is_host_only():
     assert gdr.chunk_fwd_plan(13, 4096, 8, 128, 128, 64, "scalar", bf) == ("two_pass", 0)
     assert gdr.chunk_fwd_plan(1, 4096, 8, 128, 128, 64, "channel", bf) == ("two_pass", 0)
     assert gdr.chunk_fwd_plan(1, 100, 2, 64, 64, 64, "scalar", torch.float32) == ("cuda_core", 0)
+    # few heads, long sequences: the segment scan with 4 segments (4 launches)
+    assert gdr.chunk_fwd_plan(1, 65536, 16, 128, 128, 64, "scalar", bf) == ("scan", 4)
+    assert gdr.chunk_fwd_plan(1, 32768, 2, 128, 128, 64, "channel", bf) == ("scan", 4)
+    assert gdr.chunk_fwd_plan(1, 32704, 2, 128, 128, 64, "scalar", bf) == ("fused", 0)  # T not a multiple of 256
+    assert gdr.chunk_fwd_plan(2, 32768, 16, 128, 128, 64, "scalar", bf)[0] == "fused"  # 32 heads
+    assert gdr.launches_per_chunk_fwd(1, 65536, 16, 128, 128, 64, "scalar", bf) == 4
+    assert gdr.workspace_bytes(1, 65536, 16, 128, 128, 64, "scalar", bf) == \
+        _lib.lib().gdr_chunk_fwd_scan_workspace_bytes(1, 65536, 16, 128, 128, 64, 1, 1, 0, 4)
     assert gdr.chunk_fwd_plan(0, 100, 2, 64, 64, 64, "scalar", torch.float32) == ("invalid", 0)
     # launches and workspace follow the plan
     assert gdr.launches_per_chunk_fwd(1, 4096, 8, 128, 128, 64, "scalar", bf) == 1

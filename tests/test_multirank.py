@@ -87,9 +87,10 @@ def test_kernel_code_digest_ignores_comments_only():
     assert bench.kernel_code_digest(a) != bench.kernel_code_digest(c)
 
 
-@pytest.mark.parametrize("plan", ["fused", "prep_fused", "two_pass", "cuda_core"])
+@pytest.mark.parametrize("plan", ["fused", "prep_fused", "two_pass", "cuda_core", "scan"])
 def test_kernel_bytes_split_the_step_bytes(plan):
-    """The roofline's per-kernel algorithmic bytes add up to the whole step's, on every plan."""
+    """The roofline's per-kernel algorithmic bytes add up to the whole step's, on every plan (the
+    segment scan's state kernel writes only intermediates, so it carries none)."""
     import bench
     from gated_delta_rule_143_b200.inputs import CHUNK_WORKLOADS
     for w in CHUNK_WORKLOADS.values():
@@ -97,4 +98,4 @@ def test_kernel_bytes_split_the_step_bytes(plan):
         c1 = (nc + 1) // 2 if plan == "prep_fused" else 0  # some chunks pre-computed, some not
         parts = bench.kernel_bytes(w, plan, c1)
         assert sum(b for _, b in parts) == bench.chunk_bytes(w)
-        assert all(b > 0 for _, b in parts)
+        assert all(b > 0 for name, b in parts if not (plan == "scan" and name == "chunk_state"))

@@ -54,3 +54,24 @@ def test_noalloc_matches_workspace_entry_point_twice():
             gdr.sync_status()
             assert torch.equal(o, o_ref), f"{mode}: o differs from the workspace entry point (call {call})"
             assert torch.equal(st, s_ref), f"{mode}: S_T differs from the workspace entry point (call {call})"
+
+
+@pytest.mark.gpu
+def test_noalloc_long_few_heads_keeps_the_ring():
+    """A shape gdr_chunk_fwd runs as a segment scan (2 heads, 512 chunks) still fits the built-in area
+    through the fused kernel's 8-slot ring: the allocation-free entry point never takes the scan.
+    Whole output against the oracle."""
+    import oracle
+    from gpu_util import TOL, rel_err
+    B, T, H = 1, 32768, 2
+    x = make_chunk_inputs(B, T, H, 128, 128, "scalar", "bf16", 74, s0_std=0.05)
+    d = {n: (None if t is None else t.cuda()) for n, t in x.items()}
+    o = torch.full((B, T, H, 128), float("nan"), device="cuda")
+    st = torch.full((B, H, 128, 128), float("nan"), device="cuda")
+    rc = _noalloc(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], o, st, B, T, H, "scalar",
+                  torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    gdr.sync_status()
+    o_ref, s_ref = oracle.recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], "scalar", S0=x["S0"])
+    assert rel_err(o.double().cpu().numpy(), o_ref)[0] <= TOL["bf16"]
+    assert rel_err(st.double().cpu().numpy(), s_ref)[0] <= TOL["bf16"]
