@@ -732,17 +732,17 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)  # about 0.25 s timed: a dozen clock samples
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--only", choices=("all", "fwd", "decode"), default="all",
+    ap.add_argument("--only", choices=("all", "fwd", "decode", "bwd"), default="all",
                     help="fwd: time the forward only (no e2e, decode or CPU baseline); decode: the decode step "
-                         "only; both for profiling runs")
+                         "only; bwd: the backward only; all three for profiling runs")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size (profiling runs)")
     ap.add_argument("--seq", type=int, default=0, help="override the workload's sequence length (profiling runs)")
     ap.add_argument("--workload", choices=sorted(CHUNK_WORKLOADS), default=WORKLOAD,
                     help="chunked-forward workload (default: the headline one; others for --only fwd runs)")
     args = ap.parse_args()
     if args.workload != WORKLOAD:
-        if args.only != "fwd" or args.impl != "ours":
-            ap.error("other workloads are timed with --only fwd (the full line describes the headline one)")
+        if args.only not in ("fwd", "bwd") or args.impl != "ours":
+            ap.error("other workloads are timed with --only fwd or bwd (the full line describes the headline one)")
         WORKLOAD = args.workload
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -753,6 +753,19 @@ def main():
         torch.cuda.set_device(dev)
         peaks, _ = load_peaks()
         print(json.dumps({"metric": "decode step", "decode": bench_decode(args, dev, peaks, 1)}))
+    elif args.only == "bwd":
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        peaks, _ = load_peaks()
+        w = CHUNK_WORKLOADS[WORKLOAD]
+        if args.batch:
+            w = dataclasses.replace(w, B=args.batch)
+        if args.seq:
+            w = dataclasses.replace(w, T=args.seq)
+        x = {k: (None if t is None else t.to(dev)) for k, t in workload_inputs(w).items()}
+        bwd = bench_backward(args, w, x, dev, peaks, torch.cuda.current_stream(dev), 1)
+        print(json.dumps({"metric": "backward", "config": {"workload": WORKLOAD, "B": w.B, "T": w.T},
+                          "backward": bwd}))
     else:
         run_ours(args)
 
