@@ -557,12 +557,25 @@ def bench_backward(args, w, x, dev, peaks, stream, world):
     ws_n = gdr._lib.lib().gdr_chunk_bwd_workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, gdr._mode(w.mode), 1)
     ws_b = torch.empty(ws_n, dtype=torch.uint8, device=dev)
 
+    n = max(3, min(args.steps, 10))
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+    for e in ev0 + [e for row in evk for e in row]:
+        e.record(stream)
+    calls = [0]
+
     def step(i=0):
+        j = calls[0] - min(args.warmup, 3)  # timed calls record per-kernel events
+        calls[0] += 1
+        if 0 <= j < n:
+            ev0[j].record(stream)
+            gdr.profile_next_call(evk[j])
         gdr.chunk_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], dO, S0=x["S0"], mode=w.mode, workspace=ws_b)
 
-    n = max(3, min(args.steps, 10))
     ms = max_over_ranks(time_device(step, n, min(args.warmup, 3), world, stream), world) / n
     gdr.sync_status()
+    k_ms = [statistics.mean((ev0[j] if c == 0 else evk[j][0]).elapsed_time(evk[j][c]) for j in range(n))
+            for c in range(2)]
     ntok = w.B * w.T * w.H
     hist = w.B * w.H * w.T * w.dv * w.dk * 4
     gbytes = w.dk * 4 if w.mode == "channel" else (4 if w.mode == "scalar" else 0)
@@ -573,8 +586,9 @@ def bench_backward(args, w, x, dev, peaks, stream, world):
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"ms_per_call": round(ms, 4), "tokens_per_s": round(job_throughput(w.B * w.T, ms, world), 1),
             "calls": n, "gpu_launches_per_call": 2, "bytes_per_call": nbytes,
+            "kernels_ms": {"bwd_history": round(k_ms[0], 4), "bwd_reverse": round(k_ms[1], 4)},
             "achieved_gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
-            "note": "fp32 CUDA-core backward: state-history kernel + reverse kernel, one CTA per head"}
+            "note": "fp32 CUDA-core backward: state-history kernel + reverse kernel, d_v / 32 CTAs per head"}
 
 
 def gdr_kernels_per_step(w):

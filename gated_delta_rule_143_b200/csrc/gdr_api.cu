@@ -425,6 +425,7 @@ int gdr_chunk_bwd(const void* q, const void* k, const void* v, const float* g, c
                   const void* dO, const float* dS_T, float* dq, float* dk_out, float* dv_out, float* dg,
                   float* dbeta, float* dS0, int B, int T, int H, int dk, int dv, int mode, int dtype,
                   void* workspace, size_t workspace_bytes, void* stream) {
+    ProfileScope prof_scope;
     if (mode != GDR_DECAY_NONE && mode != GDR_DECAY_SCALAR && mode != GDR_DECAY_CHANNEL)
         return fail(GDR_ERR_INVALID_ARG, "unknown decay mode %d", mode);
     if (dtype != GDR_F32 && dtype != GDR_BF16) return fail(GDR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
@@ -472,7 +473,7 @@ int gdr_chunk_bwd(const void* q, const void* k, const void* v, const float* g, c
     if (int rc = device_setup(&status, &major)) return rc;
     if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
     BwdProblem p{q, k, v, g, beta, S0, dO, dS_T, dq, dk_out, dv_out, dg, dbeta, dS0, workspace,
-                 B, T, H, dk, dv, mode, dtype, (float)(1.0 / sqrt((double)dk))};
+                 B, T, H, dk, dv, mode, dtype, (float)(1.0 / sqrt((double)dk)), status};
     const cudaError_t err = launch_bwd(p, static_cast<cudaStream_t>(stream));
     if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "backward launch: %s", cudaGetErrorString(err));
     return ok();

@@ -68,6 +68,7 @@ struct BwdProblem {
     void* workspace;
     int B, T, H, dk_dim, dv_dim, mode, dtype;
     float scale;
+    int* status;  // device status word (a bounded wait that expired)
 };
 
 // The prologue's elementwise steps (gdr_prologue), in fp32 with CUDA's math functions.

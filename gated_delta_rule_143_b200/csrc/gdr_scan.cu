@@ -73,20 +73,24 @@ scan_carry_kernel(const float* S0, const float* __restrict__ M, const float* __r
     }
 }
 
-// o[b, t, h, :] = o0[b, t, h, :] + O_I[b, t, h, :] S_in(b, i, h)^T for the tokens of segment i. One
-// CTA per (kCorrTiles x 64 tokens, segment-head); 8 warps, warp w computes rows 16 (w & 3) .. +16 and
-// columns 64 (w >> 2) .. +64 of each 64-token tile on m16n8k8 tf32 warp MMAs.
-constexpr int kCorrTiles = 4;
-constexpr int kLdS = kSD + 4;  // padded row stride (conflict-free fragment reads)
+// o[b, t, h, :] = o0[b, t, h, :] + O_I[b, t, h, :] S_in(b, i, h)^T for the tokens of segment i, on
+// m16n8k8 tf32 warp MMAs. S_in sits in shared memory as tf32 (once per CTA); each warp takes 16-token
+// tiles (all 128 output columns, 64 accumulators per thread) and reads its A fragments straight from
+// global memory. The sum over k is order-free, so both operands use one permutation of each 8-wide k
+// step: logical k = t and t + 4 of thread (g, t) are physical columns 2t and 2t + 1. A thread's two A
+// values per row and its two B values are then adjacent (8-byte loads; a warp reads whole 32-byte
+// sectors of O_I), and with a row stride of 136 words the B reads hit 32 distinct banks per half-warp.
+constexpr int kLdB = kSD + 8;
+constexpr int kCorrWarps = 8;
+constexpr int kCorrTilesPerWarp = 4;  // 16-token tiles per warp
+constexpr int kCorrRowsPerCta = kCorrWarps * kCorrTilesPerWarp * 16;  // 512 tokens
 
 template <typename Tout>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kCorrWarps * 32, 2)
 scan_correct_kernel(const float* o0, const float* __restrict__ OI, const float* __restrict__ Sin, Tout* o, int H,
                     int s, int Ts, bool has_s0) {
     // o0 may be o itself (fp32 output): each element is read, then written, by the same thread
-    extern __shared__ float scan_smem[];
-    float* sB = scan_smem;              // S_in, [j][c] with stride kLdS
-    float* sA = scan_smem + kSD * kLdS;  // O_I tile, [r][c] with stride kLdS
+    extern __shared__ uint32_t sBt[];  // S_in as tf32, [j][c] with row stride kLdB
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t4 = lane & 3;
     const int sh = blockIdx.y;  // (b * s + i) * H + h
@@ -95,53 +99,66 @@ scan_correct_kernel(const float* o0, const float* __restrict__ OI, const float* 
     if (!correct && static_cast<const void*>(o0) == static_cast<const void*>(o)) return;  // nothing to add
     if (correct) {
         const float4* src = reinterpret_cast<const float4*>(Sin + (size_t)sh * kSD * kSD);
-        for (int e = tid; e < kSD * kSD / 4; e += 256) {
+        for (int e = tid; e < kSD * kSD / 4; e += kCorrWarps * 32) {
             const int j = e / (kSD / 4), c4 = e % (kSD / 4);
-            *reinterpret_cast<float4*>(sB + j * kLdS + 4 * c4) = src[e];
+            const float4 v = src[e];
+            *reinterpret_cast<uint4*>(sBt + j * kLdB + 4 * c4) = make_uint4(to_tf32(v.x), to_tf32(v.y), to_tf32(v.z),
+                                                                             to_tf32(v.w));
         }
+        __syncthreads();
     }
-    const int rb = warp & 3, cb = warp >> 2;
-    for (int tile = 0; tile < kCorrTiles; ++tile) {
-        const int t0 = (blockIdx.x * kCorrTiles + tile) * 64;
+    for (int u = 0; u < kCorrTilesPerWarp; ++u) {
+        const int t0 = blockIdx.x * kCorrRowsPerCta + (warp * kCorrTilesPerWarp + u) * 16;
         if (t0 >= Ts) break;
-        const size_t row0 = ((size_t)bs * Ts + t0) * H + h;  // token row index of tile row 0 (times H)
-        float acc[8][4];
+        const size_t rg = ((size_t)bs * Ts + t0 + g) * H + h;  // token row of fragment row g
+        const size_t rg8 = rg + (size_t)8 * H;                  // and of row g + 8
+        float acc[16][4];
 #pragma unroll
-        for (int n = 0; n < 8; ++n)
+        for (int n = 0; n < 16; ++n)
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
         if (correct) {
-            __syncthreads();  // sB is written; the previous tile's readers of sA are done
-            for (int e = tid; e < 64 * kSD / 4; e += 256) {
-                const int r = e / (kSD / 4), c4 = e % (kSD / 4);
-                *reinterpret_cast<float4*>(sA + r * kLdS + 4 * c4) =
-                    *reinterpret_cast<const float4*>(OI + (row0 + (size_t)r * H) * kSD + 4 * c4);
-            }
-            __syncthreads();
-            const float* A = sA + (16 * rb) * kLdS;
-            const float* Bm = sB + (64 * cb) * kLdS;
-#pragma unroll 4
-            for (int k0 = 0; k0 < kSD; k0 += 8) {
-                const uint32_t a[4] = {to_tf32(A[g * kLdS + k0 + t4]), to_tf32(A[(g + 8) * kLdS + k0 + t4]),
-                                       to_tf32(A[g * kLdS + k0 + t4 + 4]), to_tf32(A[(g + 8) * kLdS + k0 + t4 + 4])};
 #pragma unroll
-                for (int n = 0; n < 8; ++n) {
-                    // B[c][j] = S_in[j][c]: column j = 64 cb + 8 n + g
-                    const uint32_t bb[2] = {to_tf32(Bm[(8 * n + g) * kLdS + k0 + t4]),
-                                            to_tf32(Bm[(8 * n + g) * kLdS + k0 + t4 + 4])};
-                    mma_tf32_16x8x8(acc[n], a, bb);
+            for (int kh = 0; kh < 2; ++kh) {  // two halves of k: 8 k-steps of A in registers at a time
+                float2 alo[8], ahi[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int col = 8 * (8 * kh + j) + 2 * t4;
+                    alo[j] = __ldg(reinterpret_cast<const float2*>(OI + rg * kSD + col));
+                    ahi[j] = __ldg(reinterpret_cast<const float2*>(OI + rg8 * kSD + col));
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int col = 8 * (8 * kh + j) + 2 * t4;
+                    const uint32_t a[4] = {to_tf32(alo[j].x), to_tf32(ahi[j].x), to_tf32(alo[j].y), to_tf32(ahi[j].y)};
+#pragma unroll
+                    for (int n = 0; n < 16; ++n) {
+                        const uint2 bv = *reinterpret_cast<const uint2*>(sBt + (8 * n + g) * kLdB + col);
+                        const uint32_t bb[2] = {bv.x, bv.y};
+                        mma_tf32_16x8x8(acc[n], a, bb);
+                    }
                 }
             }
         }
-        // epilogue: rows 16 rb + g (+ 8), columns 64 cb + 8 n + 2 t4 (+ 1)
+        // epilogue: rows g and g + 8, columns 8 n + 2 t4 (+ 1). Every o0 load is issued before any
+        // store (o0 may be o: with stores in between, each load would wait for the one before)
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-            const size_t row = row0 + (size_t)(16 * rb + g + 8 * half) * H;
+            const size_t row = half ? rg8 : rg;
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                const int col = 64 * cb + 8 * n + 2 * t4;
-                const float2 base = *reinterpret_cast<const float2*>(o0 + row * kSD + col);
-                const float v0 = base.x + acc[n][2 * half], v1 = base.y + acc[n][2 * half + 1];
+            for (int n = 0; n < 16; ++n) {
+                const float2 base = *reinterpret_cast<const float2*>(o0 + row * kSD + 8 * n + 2 * t4);
+                acc[n][2 * half] += base.x;
+                acc[n][2 * half + 1] += base.y;
+            }
+        }
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const size_t row = half ? rg8 : rg;
+#pragma unroll
+            for (int n = 0; n < 16; ++n) {
+                const int col = 8 * n + 2 * t4;
+                const float v0 = acc[n][2 * half], v1 = acc[n][2 * half + 1];
                 if (sizeof(Tout) == 4) {
                     *reinterpret_cast<float2*>(reinterpret_cast<float*>(o) + row * kSD + col) = make_float2(v0, v1);
                 } else {
@@ -220,8 +237,8 @@ cudaError_t launch_scan(const ChunkProblem& p, int n_seg, cudaStream_t stream) {
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     profile_after_launch(stream);
     // o = o^0 + O_I S_in^T
-    const size_t smem = (size_t)(kSD + 64) * kLdS * sizeof(float);
-    const dim3 grid((Ts / 64 + kCorrTiles - 1) / kCorrTiles, (unsigned)nsh);
+    const size_t smem = (size_t)kSD * kLdB * sizeof(uint32_t);
+    const dim3 grid((Ts + kCorrRowsPerCta - 1) / kCorrRowsPerCta, (unsigned)nsh);
     if (p.o_dtype == GDR_BF16) {
         auto kern = scan_correct_kernel<__nv_bfloat16>;
         if ((err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)

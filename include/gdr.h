@@ -312,8 +312,9 @@ typedef enum {
 int gdr_chunk_fwd_plan(int B, int T, int H, int d_k, int d_v, int chunk, int mode, int dtype,
                        int o_dtype, int* precomputed_chunks);
 
-/* Diagnostics (no counterpart in the method): per-kernel timing of the next chunked forward.
- * The next gdr_chunk_fwd or gdr_chunk_fwd_noalloc call made on the calling host thread records
+/* Diagnostics (no counterpart in the method): per-kernel timing of the next chunked forward or
+ * backward. The next gdr_chunk_fwd(_ex, _scan), gdr_chunk_fwd_noalloc or gdr_chunk_bwd call made on
+ * the calling host thread records
  * events[i] on its stream right after it enqueues its i-th kernel, for i < min(n_events,
  * launches), then forgets the events; a call that fails validation forgets them too.
  *   events    n_events cudaEvent_t handles created by the caller (owned by the caller; timing
