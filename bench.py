@@ -471,6 +471,7 @@ def run_ours(args):
     dec = bench_decode(args, dev, peaks, world)
     others = bench_workloads(args, dev, peaks) if world == 1 else None
     pro = bench_prologue(args, w, dev, ws, o, st, stream, world, rank, ms_step)
+    gdn2 = bench_gdn2(dev, peaks, stream) if world == 1 else None
     bwd = bench_backward(args, w, sets[0], dev, peaks, stream, world)
 
     line = {
@@ -492,7 +493,7 @@ def run_ours(args):
         "backward": bwd,
     }
     if others is not None:
-        line["extra"] = {"workloads": others}
+        line["extra"] = {"workloads": others, "gated_deltanet2": gdn2}
     if rank == 0 and world == 1:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
@@ -544,6 +545,32 @@ def bench_prologue(args, w, dev, ws, o, st, stream, world, rank, ms_plain):
             "steps": n, "fused_gpu_launches_per_step": gdr_kernels_per_step(w),
             "note": "raw q/k (unnormalised, bf16), beta logits, gate logits and A [H]; fused = "
                     "l2norm_qk + beta_sigmoid + gate_softplus in the library's kernels"}
+
+
+def bench_gdn2(dev, peaks, stream):
+    """Gated DeltaNet-2 (gdr_chunk_fwd_gdn2) at the Kimi Delta Attention workload's shape: the same
+    inputs plus fp32 erase [B,T,H,d_k] and write [B,T,H,d_v] gates in place of beta. Bytes as that
+    workload's, with the two gates in place of beta (2 * 512 B more per token-head)."""
+    import gated_delta_rule_143_b200 as gdr
+    from gated_delta_rule_143_b200.inputs import make_gdn2_gates
+    w = CHUNK_WORKLOADS["kda_bf16_b4_h16_t8192_d128"]
+    x = {k: (None if t is None else t.to(dev)) for k, t in workload_inputs(w).items()}
+    gates = {k: t.to(dev) for k, t in make_gdn2_gates(w.B, w.T, w.H, w.dk, w.dv, 77).items()}
+    o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=dev)
+    st = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
+
+    def step(i=0):
+        gdr.chunk_fwd_gdn2(x["q"], x["k"], x["v"], x["g"], gates["erase"], gates["write"], None, mode=w.mode, out=o,
+                           state_out=st)
+
+    n = 10
+    ms = time_device(step, n, 3, 1, stream) / n
+    gdr.sync_status()
+    nbytes = chunk_bytes(w) + w.B * w.T * w.H * 4 * (w.dk + w.dv - 1)
+    return {"workload": "gdn2 at " + w.name, "ms_per_step": round(ms, 5),
+            "tokens_per_s": round(w.B * w.T / (ms * 1e-3), 1), "steps": n, "algorithmic_bytes": nbytes,
+            "roofline_frac": round(nbytes / (peaks["hbm_gbs"] * 1e9) / (ms * 1e-3), 4),
+            "path": "channel gate's tensor-core passes with the erase / write gates"}
 
 
 def bench_backward(args, w, x, dev, peaks, stream, world):
@@ -660,8 +687,12 @@ def bench_workloads(args, dev, peaks):
     import gated_delta_rule_143_b200 as gdr
     stream = torch.cuda.current_stream(dev)
     out = {}
-    for name, w in CHUNK_WORKLOADS.items():
-        x = {k: (None if t is None else t.to(dev)) for k, t in workload_inputs(w).items()}
+    # the small fp32 workload's T = 256 runs the token recurrence; the same shape at T = 320 (five
+    # chunks) keeps the fp32 chunk form measured
+    extra = dataclasses.replace(CHUNK_WORKLOADS["gdn_f32_b1_h2_t256_d64"], name="gdn_f32_b1_h2_t320_d64_chunk_form",
+                                T=320)
+    for name, w in list(CHUNK_WORKLOADS.items()) + [(extra.name, extra)]:
+        x = {k: (None if t is None else t.to(dev)) for k, t in workload_inputs(w, seed=WORKLOAD_SEEDS.get(name, 1)).items()}
         dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
         o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=dev)
         st = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)

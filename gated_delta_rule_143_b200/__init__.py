@@ -236,6 +236,7 @@ def chunk_fwd_gdn2(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optiona
                    erase: torch.Tensor, write: torch.Tensor, S0: Optional[torch.Tensor] = None, *, mode="channel",
                    chunk: int = 64, return_state: bool = True, out: Optional[torch.Tensor] = None,
                    out_dtype: torch.dtype = torch.float32, state_out: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None,
                    stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Gated DeltaNet-2 forward (gdr_chunk_fwd_gdn2): ``erase`` fp32 [B,T,H,dk] and ``write`` fp32
     [B,T,H,dv] gates in place of beta; other arguments as ``chunk_fwd``."""
@@ -245,9 +246,13 @@ def chunk_fwd_gdn2(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: Optiona
         out = torch.empty((B, T, H, dv), dtype=out_dtype, device=q.device)
     if return_state and state_out is None:
         state_out = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device)
+    m, dt, odt = _mode(mode), _dtype(q), _dtype(out)
+    if workspace is None:
+        workspace = _workspace(lib().gdr_chunk_fwd_gdn2_workspace_bytes(B, T, H, dk, dv, chunk, m, dt, odt), q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = lib().gdr_chunk_fwd_gdn2(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(erase), _ptr(write), _ptr(S0), _ptr(out),
-                                  _ptr(state_out) if return_state else None, B, T, H, dk, dv, chunk, _mode(mode),
-                                  _dtype(q), _dtype(out), _stream_handle(stream))
+                                  _ptr(state_out) if return_state else None, B, T, H, dk, dv, chunk, m, dt, odt,
+                                  _ptr(workspace), ws_bytes, _stream_handle(stream))
     check(rc)
     return out, (state_out if return_state else None)
 

@@ -34,7 +34,8 @@ SIGNATURES = {
     "gdr_chunk_fwd_ex": (_i, [_vp] * 8 + [_i] * 10 + [_vp, _vp, _sz, _vp]),
     "gdr_decode_step": (_i, [_vp] * 7 + [_i] * 7 + [_vp]),
     "gdr_chunk_bwd": (_i, [_vp] * 14 + [_i] * 7 + [_vp, _sz, _vp]),
-    "gdr_chunk_fwd_gdn2": (_i, [_vp] * 9 + [_i] * 9 + [_vp]),
+    "gdr_chunk_fwd_gdn2": (_i, [_vp] * 9 + [_i] * 9 + [_vp, _sz, _vp]),
+    "gdr_chunk_fwd_gdn2_workspace_bytes": (_sz, [_i] * 9),
     "gdr_chunk_fwd_scan": (_i, [_vp] * 8 + [_i] * 10 + [_vp, _sz, _vp]),
     "gdr_chunk_fwd_scan_workspace_bytes": (_sz, [_i] * 10),
     "gdr_decode_step_gdn2": (_i, [_vp] * 8 + [_i] * 7 + [_vp]),

@@ -339,22 +339,45 @@ int gdr_decode_step(const void* q, const void* k, const void* v, const float* g,
                               stream);
 }
 
+// Gated DeltaNet-2 runs on the tensor cores for the channel decay at the tensor-core shapes (the
+// channel gate's two passes), on the CUDA cores otherwise.
+bool gdn2_on_tc(int dk, int dv, int chunk, int mode, int dtype, int o_dtype) {
+    return mode == GDR_DECAY_CHANNEL && chunk_tc_supported(dk, dv, chunk, dtype, o_dtype);
+}
+
+size_t gdr_chunk_fwd_gdn2_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int mode, int dtype,
+                                          int o_dtype) {
+    char saved[sizeof(g_last_error)];
+    memcpy(saved, g_last_error, sizeof(saved));
+    const int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype);
+    memcpy(g_last_error, saved, sizeof(saved));
+    if (rc != GDR_OK || !gdn2_on_tc(dk, dv, chunk, mode, dtype, o_dtype)) return 0;
+    return chunk_tc_workspace_bytes(B, T, H, dk, dv, chunk, mode);
+}
+
 int gdr_chunk_fwd_gdn2(const void* q, const void* k, const void* v, const float* g, const float* erase,
                        const float* write, const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv,
-                       int chunk, int mode, int dtype, int o_dtype, void* stream) {
+                       int chunk, int mode, int dtype, int o_dtype, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+    ProfileScope prof_scope;
     if (int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype)) return rc;
-    if (!chunk_simt_supported(dk, dv, chunk))
+    const bool on_tc = gdn2_on_tc(dk, dv, chunk, mode, dtype, o_dtype);
+    if (!on_tc && !chunk_simt_supported(dk, dv, chunk))
         return fail(GDR_ERR_UNSUPPORTED, "Gated DeltaNet-2: d_k, d_v in {32, 64, 128} and chunk 64 (got %d, %d, %d)", dk,
                     dv, chunk);
     if (!q || !k || !v || !erase || !write || !o)
         return fail(GDR_ERR_INVALID_ARG, "q, k, v, erase, write and o must be non-null");
     if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
     if (mode == GDR_DECAY_NONE) g = nullptr;
-    const void* ptrs[] = {q, k, v, g, erase, write, S0, o, S_T};
+    const void* ptrs[] = {q, k, v, g, erase, write, S0, o, S_T, workspace};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return fail(GDR_ERR_MISALIGNED, "pointer %p is not 16-byte aligned", p);
     const size_t ntok = (size_t)B * T * H, eb = elem_bytes(dtype);
     const size_t bo = ntok * dv * elem_bytes(o_dtype), bs = (size_t)B * H * dv * dk * sizeof(float);
+    const size_t need = on_tc ? chunk_tc_workspace_bytes(B, T, H, dk, dv, chunk, mode) : 0;
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
+        return fail(GDR_ERR_WORKSPACE, "workspace of %zu bytes required (got %zu at %p)", need, workspace_bytes,
+                    workspace);
     struct Span { const void* p; size_t n; const char* name; };
     const Span ins[] = {{q, ntok * dk * eb, "q"}, {k, ntok * dk * eb, "k"}, {v, ntok * dv * eb, "v"},
                         {g, mode == GDR_DECAY_CHANNEL ? ntok * dk * 4 : ntok * 4, "g"}, {erase, ntok * dk * 4, "erase"},
@@ -363,15 +386,20 @@ int gdr_chunk_fwd_gdn2(const void* q, const void* k, const void* v, const float*
         if (overlap(o, bo, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "o overlaps input %s", s.name);
         if (S_T != S0 && overlap(S_T, bs, s.p, s.n))
             return fail(GDR_ERR_INVALID_ARG, "S_T overlaps input %s (only S_T == S0 is allowed)", s.name);
+        if (need > 0 && overlap(workspace, need, s.p, s.n))
+            return fail(GDR_ERR_INVALID_ARG, "workspace overlaps %s", s.name);
     }
     if (overlap(o, bo, S_T, bs)) return fail(GDR_ERR_INVALID_ARG, "o overlaps S_T");
+    if (need > 0 && (overlap(workspace, need, o, bo) || overlap(workspace, need, S_T, bs)))
+        return fail(GDR_ERR_INVALID_ARG, "workspace overlaps an output");
     int* status = nullptr;
     int major = 0;
     if (int rc = device_setup(&status, &major)) return rc;
     if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
-    ChunkProblem p{q, k, v, g, nullptr, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, nullptr, 0, status,
-                   (float)(1.0 / sqrt((double)dk)), GDR_PRO_NONE, nullptr, erase, write};
-    const cudaError_t err = launch_chunk_simt(p, static_cast<cudaStream_t>(stream));
+    ChunkProblem p{q, k, v, g, nullptr, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, workspace,
+                   workspace_bytes, status, (float)(1.0 / sqrt((double)dk)), GDR_PRO_NONE, nullptr, erase, write};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t err = on_tc ? launch_chunk_tc(p, s) : launch_chunk_simt(p, s);
     if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "Gated DeltaNet-2 launch: %s", cudaGetErrorString(err));
     return ok();
 }

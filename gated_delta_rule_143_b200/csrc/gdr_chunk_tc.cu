@@ -102,6 +102,8 @@ struct PrepArgs {
     int* status;
     int pro;                  // gdr_prologue flags
     const float* gate_scale;  // [H] or NULL
+    const float* erase;       // Gated DeltaNet-2 (EW): [B,T,H,d_k] erase gate
+    const float* write;       // Gated DeltaNet-2 (EW): [B,T,H,d_v] write gate
 };
 
 // Inverse L2 norms of the 128 rows of the [K; Q] tile (prologue GDR_PRO_L2NORM_QK), fp32 [128]:
@@ -149,6 +151,19 @@ __device__ __forceinline__ void unpack8h(uint4 u, float* f) {
     }
 }
 __device__ __forceinline__ void st16(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
+// Eight fp32 gate values of chunk row r, columns col0 .. col0 + 7 (rows past the tail give 0).
+__device__ __forceinline__ void load_gate8(const float* gate, size_t tok0, int r, int H, int n, int col0, int ld,
+                                           float (&x)[8]) {
+    if (r < n) {
+        const float4* p = reinterpret_cast<const float4*>(gate + (tok0 + (size_t)r * H) * ld + col0);
+        const float4 a = p[0], b = p[1];
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = 0.f;
+    }
+}
 __device__ __forceinline__ uint4 ld16(const void* p) { return *reinterpret_cast<const uint4*>(p); }
 
 // 16 x 16 output tile of C = A (16 x K) * B (K x 16) on warp MMAs (tf32, fp32 accumulate).
@@ -262,7 +277,7 @@ __device__ void prep_init(const PrepSmem& ps, int lt) {
 // Computes the hand-off block of chunk c of head (b, h) into `out` (global memory). Executed by the
 // 256 threads of one pipeline (8 warps: TMEM lane quadrant q = warp & 3, column half hf = warp >> 2);
 // `it` counts the pipeline's previous tasks (mbarrier phase parity).
-template <int MODE, bool PRO>
+template <int MODE, bool PRO, bool EW = false>
 __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv,
                            const PrepSmem& ps, int b, int h, int c, uint8_t* __restrict__ out, uint32_t it, int lt,
                            uint32_t& n_copies) {
@@ -308,7 +323,8 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
             const int r = lane + 32 * m;
-            float x = (r < n) ? P.beta[tok0 + (size_t)r * H] : 0.f;
+            // Gated DeltaNet-2: the gates replace beta (1 here), e in the erase operands, w in V
+            float x = (r < n) ? (EW ? 1.f : P.beta[tok0 + (size_t)r * H]) : 0.f;
             if (sig && r < n) x = pro_sigmoid(x);
             sBeta[r] = x;
         }
@@ -474,6 +490,12 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
                 qa[e] = qx[e] * up;
                 kb[e] = kx[e] * dn;
             }
+            if (EW) {  // the erase direction e (.) k on the left of the Gram (and in K*gamma for W)
+                float er[8];
+                load_gate8(P.erase, tok0, r, H, n, col0, kD, er);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ka[e] *= er[e];
+            }
             st16(sKQ + okr, pack8h(ka));
             st16(sKQ + oqr, pack8h(qa));
             st16(sKB + kmajor_off(r, col0, 64), pack8h(kb));
@@ -544,8 +566,9 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
 #pragma unroll 1
                 for (int kk = 0; kk < cnt; ++kk) {
                     const int dch = sStrong[128 + 32 * w4 + kk];
-                    const float a = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                                        sKQ2 + kmajor_off(row, dch, 128))) * (norm ? sNrm[row] : 1.f);
+                    float a = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                                  sKQ2 + kmajor_off(row, dch, 128))) * (norm ? sNrm[row] : 1.f);
+                    if (EW && row < kC) a *= (row < n) ? P.erase[(tok0 + (size_t)row * H) * kD + dch] : 0.f;
                     const float Gr = sGam[rr * kD + dch];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
@@ -604,6 +627,12 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
                     float kc[8];
                     unpack8bf(ld16(sm + kPKQ2 + kmajor_off(r, col0, 128)), kc);
                     const float nk = norm ? sNrm[r] : 1.f;
+                    if (EW) {
+                        float er[8];
+                        load_gate8(P.erase, tok0, r, H, n, col0, kD, er);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) kc[e] *= er[e];
+                    }
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         x[e] = fl[e] ? kc[e] * nk * fast_exp2(sGam[r * kD + col0 + e])
@@ -614,6 +643,12 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
                 }
             } else {
                 unpack8bf(ld16(p), x);
+                if (EW && isv) {  // the gated write target w (.) v
+                    float wr[8];
+                    load_gate8(P.write, tok0, r, H, n, col0, kD, wr);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] *= wr[e];
+                }
                 if (!isv && (MODE == GDR_DECAY_SCALAR || norm)) {
                     float fr = MODE == GDR_DECAY_SCALAR ? fast_exp2(sGam[r]) : 1.f;
                     if (norm) fr *= sNrm[r];
@@ -696,7 +731,7 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
 // At the start of each task the tiles of the CTA's next task are prefetched into L2. The scalar
 // and DeltaNet variants run at 96 registers per thread (no spills; measured 1-2.5 % faster than
 // the 128 two CTAs per SM would allow).
-template <int MODE, bool PRO>
+template <int MODE, bool PRO, bool EW = false>
 __global__ void __maxnreg__(MODE == GDR_DECAY_CHANNEL ? 240 : 96)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                   const __grid_constant__ CUtensorMap mv, PrepArgs P, uint8_t* __restrict__ ws, int NCp, int n_tasks) {
@@ -734,7 +769,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
             tma_prefetch_l2_4d(&mv, 64, hn, cn * kC, bn);
         }
         uint8_t* out = ws + (size_t)t * kHandoffStride;
-        prep_chunk<MODE, PRO>(P, &mq, &mk, &mv, ps, b, h, c, out, it, lt, n_copies);
+        prep_chunk<MODE, PRO, EW>(P, &mq, &mk, &mv, ps, b, h, c, out, it, lt, n_copies);
     }
     if (lt == 0) bulk_wait<0>();
     tc_fence_before();
@@ -1260,17 +1295,17 @@ cudaError_t make_map(CUtensorMap* map, const void* base, CUtensorMapDataType typ
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int MODE, bool PRO>
+template <int MODE, bool PRO, bool EW = false>
 cudaError_t launch_prep(const ChunkProblem& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                         int NC, int NCp, uint8_t* blocks, cudaStream_t stream) {
-    auto kern = chunk_prep_kernel<MODE, PRO>;
+    auto kern = chunk_prep_kernel<MODE, PRO, EW>;
     const uint32_t smem = (MODE == GDR_DECAY_CHANNEL ? kPrepBytesChannel : kPrepBytesScalar) + 1024;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     // the whole unified L1 / shared array as shared memory, so that two pipelines fit per SM
     err = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (err != cudaSuccess) return err;
-    PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status, p.prologue, p.gate_scale};
+    PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status, p.prologue, p.gate_scale, p.erase, p.write};
     int dev = 0, sms = 0;
     if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
     if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
@@ -1351,7 +1386,7 @@ cudaError_t launch_fused(const ChunkProblem& p, const CUtensorMap& mq, const CUt
     RingArgs R{ring, flags, flags + (size_t)BH * depth, flags + (size_t)BH * (depth + 1), ws, BH, c1, depth};
     if ((err = cudaMemsetAsync(flags, 0, flag_bytes(BH, NC), stream)) != cudaSuccess) return err;
     if (c1 > 0 && (err = launch_prep<MODE, PRO>(p, mq, mk, mv, NC, c1, ws, stream)) != cudaSuccess) return err;
-    PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status, p.prologue, p.gate_scale};
+    PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status, p.prologue, p.gate_scale, p.erase, p.write};
     StateArgs A{p.S0, p.S_T, p.T, p.H, NC, p.scale, p.status, p.B * p.H, nullptr};
     CUtensorMap aq = mq, ak = mk, av = mv, ao = mo;
     void* args[] = {&aq, &ak, &av, &ao, &P, &A, &R};
@@ -1424,8 +1459,13 @@ cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream) {
         return p.prologue ? launch_fused_mode<true>(p, mq, mk, mv, mo, NC, stream)
                           : launch_fused_mode<false>(p, mq, mk, mv, mo, NC, stream);
     uint8_t* ws = static_cast<uint8_t*>(p.workspace);
-    err = p.prologue ? launch_prep_mode<true>(p, mq, mk, mv, NC, ws, stream)
-                     : launch_prep_mode<false>(p, mq, mk, mv, NC, ws, stream);
+    if (p.erase != nullptr) {  // Gated DeltaNet-2: the channel gate's prep with the erase / write gates
+        if (p.mode != GDR_DECAY_CHANNEL || p.prologue) return cudaErrorInvalidValue;
+        err = launch_prep<GDR_DECAY_CHANNEL, false, true>(p, mq, mk, mv, NC, NC, ws, stream);
+    } else {
+        err = p.prologue ? launch_prep_mode<true>(p, mq, mk, mv, NC, ws, stream)
+                         : launch_prep_mode<false>(p, mq, mk, mv, NC, ws, stream);
+    }
     if (err != cudaSuccess) return err;
     if (p.o_dtype == GDR_BF16) return launch_state<__nv_bfloat16>(p, mo, NC, stream);
     return launch_state<float>(p, mo, NC, stream);

@@ -236,14 +236,22 @@ size_t gdr_chunk_fwd_scan_workspace_bytes(int B, int T, int H, int d_k, int d_v,
  *   erase   [B, T, H, d_k] fp32 (decode: [B, H, d_k]); usually in [0, 1]
  *   write   [B, T, H, d_v] fp32 (decode: [B, H, d_v]); usually in [0, 1]
  *   the other arguments as gdr_chunk_fwd / gdr_decode_step (no beta; any decay mode).
- * Runs on the fp32 CUDA-core kernels (the chunk form of gdr_chunk_fwd's CUDA-core path with
- * A_ri = sum_c e_rc k_rc k_ic exp(Gamma_rc - Gamma_ic) and R = w (.) V - ((e (.) K) * gamma) S^T);
- * needs no workspace. Chunked: d_k, d_v in {32, 64, 128}, chunk 64; decode: as gdr_decode_step.
- * Errors as gdr_chunk_fwd / gdr_decode_step.
+ * In the chunk form the erase direction E = e (.) K takes the place of diag(beta) K on the left of the
+ * Gram matrix and in W, and w (.) V that of diag(beta) V in U:
+ * A_ri = sum_c E_rc k_ic exp(Gamma_rc - Gamma_ic) (i < r), W = T (E * gamma), U = T (w (.) V).
+ * With the channel decay at the tensor-core shapes (bf16, d_k = d_v = 128, chunk 64) it runs on the
+ * channel gate's two tensor-core passes and needs gdr_chunk_fwd_gdn2_workspace_bytes(...) of
+ * workspace; otherwise on the fp32 CUDA-core kernels with no workspace (d_k, d_v in {32, 64, 128},
+ * chunk 64). Decode: as gdr_decode_step. Errors as gdr_chunk_fwd / gdr_decode_step.
  */
 int gdr_chunk_fwd_gdn2(const void* q, const void* k, const void* v, const float* g, const float* erase,
                        const float* write, const float* S0, void* o, float* S_T, int B, int T, int H,
-                       int d_k, int d_v, int chunk, int mode, int dtype, int o_dtype, void* stream);
+                       int d_k, int d_v, int chunk, int mode, int dtype, int o_dtype, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* Workspace of gdr_chunk_fwd_gdn2 (0 when it runs on the CUDA cores or would be rejected). */
+size_t gdr_chunk_fwd_gdn2_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk, int mode,
+                                          int dtype, int o_dtype);
 
 int gdr_decode_step_gdn2(const void* q, const void* k, const void* v, const float* g, const float* erase,
                          const float* write, float* S, void* o, int B, int H, int d_k, int d_v, int mode,

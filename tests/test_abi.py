@@ -213,5 +213,17 @@ def test_chunk_fwd_gdn2_rejects_bad_arguments_on_host(kw, code):
     a = dict(q=1 * M, k=2 * M, v=3 * M, g=6 * M, erase=4 * M, write=5 * M, o=7 * M, dk=64, chunk=64)
     a.update(kw)
     rc = _lib.lib().gdr_chunk_fwd_gdn2(a["q"], a["k"], a["v"], a["g"], a["erase"], a["write"], None, a["o"], None, 1,
-                                       16, 1, a["dk"], 64, a["chunk"], 2, 0, 0, None)
+                                       16, 1, a["dk"], 64, a["chunk"], 2, 0, 0, None, 0, None)
     assert rc == code
+
+
+def test_chunk_fwd_gdn2_workspace_query():
+    lib = _lib.lib()
+    # the channel decay at the tensor-core shapes runs the channel gate's two passes: one block per chunk
+    assert lib.gdr_chunk_fwd_gdn2_workspace_bytes(1, 128, 2, 128, 128, 64, 2, 1, 0) == 2 * 2 * 74752
+    assert lib.gdr_chunk_fwd_gdn2_workspace_bytes(1, 128, 2, 128, 128, 64, 1, 1, 0) == 0  # scalar: CUDA cores
+    assert lib.gdr_chunk_fwd_gdn2_workspace_bytes(1, 128, 2, 64, 64, 64, 2, 0, 0) == 0    # fp32: CUDA cores
+    M = 1 << 24  # missing workspace on the tensor-core route: rejected on the host
+    rc = lib.gdr_chunk_fwd_gdn2(1 * M, 2 * M, 3 * M, 4 * M, 5 * M, 6 * M, None, 7 * M, None, 1, 128, 2, 128, 128, 64,
+                                2, 1, 0, None, 0, None)
+    assert rc == -4

@@ -90,3 +90,20 @@ def test_gdn2_decode_steps(mode, dtype, dk, dv):
         o_ref, S_ref = oracle.recurrent_gdn2(x["q"], x["k"], x["v"], x["g"], gw["erase"], gw["write"], mode, S0=S_ref)
         assert rel_err(o.double().cpu().numpy(), o_ref[:, 0])[0] <= TOL[dtype], step
     assert rel_err(Sd.double().cpu().numpy(), S_ref)[0] <= TOL[dtype]
+
+
+def test_gdn2_tensor_core_kda_workload_shape():
+    """The channel decay at the tensor-core shapes runs the channel gate's tensor-core passes: the
+    Kimi Delta Attention workload's shape (B = 4, H = 16, d = 128) at T = 2048, with 16 channels
+    decaying strongly (their terms on the CUDA cores), whole output against the oracle."""
+    x = make_chunk_inputs(4, 2048, 16, 128, 128, "channel", "bf16", 11950, s0_std=0.05)
+    x["g"][..., :16] *= 400.0  # spread far past the factored range on channels 0-15
+    gw = make_gdn2_gates(4, 2048, 16, 128, 128, 11951)
+    assert gdr._lib.lib().gdr_chunk_fwd_gdn2_workspace_bytes(4, 2048, 16, 128, 128, 64, 2, 1, 0) > 0
+    o, st = run_gdn2(x, gw["erase"], gw["write"], "channel")
+    o_ref, s_ref = oracle.recurrent_gdn2(x["q"], x["k"], x["v"], x["g"], gw["erase"], gw["write"], "channel",
+                                         S0=x["S0"])
+    eo, _ = rel_err(o, o_ref)
+    es, _ = rel_err(st, s_ref)
+    print(f"gdn2 tensor cores: o {eo:.3e}, S_T {es:.3e}")
+    assert eo <= TOL["bf16"] and es <= TOL["bf16"]
