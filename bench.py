@@ -662,7 +662,8 @@ def bench_decode(args, dev, peaks, world):
     for s in range(2):
         x = make_decode_step(w, WORKLOAD_SEEDS[DECODE], s)
         toks.append({k: (None if t is None else t.to(dev)) for k, t in x.items()})
-    o = torch.empty((w.B, w.H, w.dv), dtype=torch.float32, device=dev)
+    o = torch.empty((w.B, w.H, w.dv), dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32,
+                    device=dev)  # o in the input dtype, as decode_bytes counts it
     stream = torch.cuda.current_stream(dev)
 
     def step(i=0):

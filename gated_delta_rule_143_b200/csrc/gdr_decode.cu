@@ -66,6 +66,23 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
     const int sub = threadIdx.x & (kLanesPerRow - 1);
     const int row0 = threadIdx.x / kLanesPerRow;
     const int c0 = sub * EPL;
+    float* Sh = S + bh * (size_t)dv * DK;
+    // Loop bounds are uniform across a warp (its 4 rows share `jb`), so every lane reaches the
+    // full-mask shuffles; rows past d_v are masked.
+    const int warp_row0 = (threadIdx.x >> 5) * (32 / kLanesPerRow);
+    const int lane_row = row0 - warp_row0;
+    // the two state rows of pass jb (rows jb + lane_row and that + kRowsPerPass), zero past d_v
+    auto load_pass = [&](int jb, float (&a)[EPL], float (&b)[EPL]) {
+        const int j = jb + lane_row, j2 = j + kRowsPerPass;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) { a[i] = 0.f; b[i] = 0.f; }
+        if (j < dv) load_row(Sh + (size_t)j * DK + c0, a);
+        if (j2 < dv) load_row(Sh + (size_t)j2 * DK + c0, b);
+    };
+    // the state is nearly all of the traffic: the first pass's rows are requested before the token's
+    // inputs, so that their latency overlaps the prologue
+    float s1[EPL], s2[EPL];
+    load_pass(warp_row0, s1, s2);
 
     float kr[EPL], qr[EPL], al[EPL];
     load_vec(k + bh * DK + c0, kr);
@@ -110,22 +127,12 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
     } else {
         bt = (pro & GDR_PRO_BETA_SIGMOID) ? pro_sigmoid(beta[bh]) : beta[bh];
     }
-    float* Sh = S + bh * (size_t)dv * DK;
-
-    // Loop bounds are uniform across a warp (its 4 rows share `jb`), so every lane reaches the
-    // full-mask shuffles; rows past d_v are masked.
-    const int warp_row0 = (threadIdx.x >> 5) * (32 / kLanesPerRow);
-    const int lane_row = row0 - warp_row0;
     for (int jb = warp_row0; jb < dv; jb += 2 * kRowsPerPass) {
         const int j = jb + lane_row;
         const int j2 = j + kRowsPerPass;
         const bool ok1 = j < dv;
         const bool ok2 = j2 < dv;
-        float s1[EPL], s2[EPL];
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) { s1[i] = 0.f; s2[i] = 0.f; }
-        if (ok1) load_row(Sh + (size_t)j * DK + c0, s1);
-        if (ok2) load_row(Sh + (size_t)j2 * DK + c0, s2);
+        if (jb != warp_row0) load_pass(jb, s1, s2);
         float v1 = ok1 ? load_f32(v + bh * dv + j) : 0.f;
         float v2 = ok2 ? load_f32(v + bh * dv + j2) : 0.f;
         if (EW) {  // the gated write target

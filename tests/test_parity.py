@@ -218,6 +218,21 @@ def test_bf16_output(mode):
     assert rel_err(st, s_ref)[0] <= TOL["bf16"]
 
 
+def test_bf16_output_full_headline_workload():
+    """The headline workload (Gated DeltaNet bf16, B = 8, H = 8, T = 4096) with o in the input dtype,
+    as the bench times it: every element within the bar plus its own bf16 rounding."""
+    name = "gdn_bf16_b8_h8_t4096_d128"
+    w = CHUNK_WORKLOADS[name]
+    x = workload_inputs(w)
+    o, st = run_chunk(x, w.mode, out_dtype=torch.bfloat16)
+    o_ref, s_ref = oracle.recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], w.mode, S0=x["S0"])
+    rms = np.sqrt(np.mean(o_ref ** 2))
+    excess = np.abs(o - o_ref) - (TOL["bf16"] * rms + BF16_HALF_ULP * np.abs(o_ref))
+    assert excess.max() <= 0, excess.max()
+    assert rel_err(st, s_ref)[0] <= TOL["bf16"]
+    print(f"{name} bf16 o: max|do|/rms = {rel_err(o, o_ref)[0]:.3e}")
+
+
 def test_no_state_output():
     x = make_chunk_inputs(1, 70, 1, 128, 128, "none", "bf16", 95)
     o, st = run_chunk(x, "none", want_state=False)
