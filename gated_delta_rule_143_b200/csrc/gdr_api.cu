@@ -124,13 +124,18 @@ int prologue_check(int prologue, int mode) {
 }
 
 // Segments gdr_chunk_fwd gives a problem on its own: few heads and long sequences, where one serial
-// chain per head leaves most SMs idle (measured on the 16-head, 65536-token workload: 4 segments run
-// in 0.73 of the time of the fused plan). 0: no segment scan.
+// chain per head leaves most SMs idle. The data and transition chains of B * H * s segment-heads
+// should about fill the GPU (2 B H s <= 128) while the carry's s sequential steps stay short (s <= 16)
+// and every segment keeps at least 16 chunks. Measured at T = 65536 (fused plan: about 2.3 ms):
+// 2 heads 362 us with 16 segments, 4 heads 480 us (16), 8 heads 751 us (8), 16 heads 1.32 ms (4);
+// 16 heads at T = 16384: 411 us with 4 segments against 606 us fused. 0: no segment scan.
 int auto_segments(int B, int T, int H, int dk, int dv, int chunk, int dtype, int o_dtype) {
-    constexpr int kSeg = 4;
+    const size_t BH = (size_t)B * H;
     const int NC = (T + chunk - 1) / chunk;
-    if ((size_t)B * H > 16 || NC < 512) return 0;
-    return scan_supported(B, T, H, dk, dv, chunk, dtype, o_dtype, kSeg) ? kSeg : 0;
+    if (BH > 16 || NC < 256) return 0;
+    int s = 16;
+    while (s > 2 && (BH * s > 64 || NC / s < 16 || T % (s * chunk) != 0)) s >>= 1;
+    return scan_supported(B, T, H, dk, dv, chunk, dtype, o_dtype, s) ? s : 0;
 }
 
 // The chunked forward behind gdr_chunk_fwd_ex and gdr_chunk_fwd_scan. n_seg: 0 = the plan chosen from

@@ -107,7 +107,7 @@ typedef enum {
  * cooperative kernel with one CTA per SM, in which the per-chunk factor pipelines hand their
  * blocks to the per-head state passes through a ring in the workspace: eight blocks per head
  * (0.6 MB per head) up to 56 heads (but few heads with long sequences run the segment scan of
- * gdr_chunk_fwd_scan with 4 segments; see gdr_chunk_fwd_plan). Above 56 heads a prep kernel on every SM first writes the
+ * gdr_chunk_fwd_scan; see gdr_chunk_fwd_plan). Above 56 heads a prep kernel on every SM first writes the
  * blocks of the leading chunks of each head to the workspace, and the ring has a slot for every
  * later chunk. The workspace then holds one block (73 KB) per chunk of every head. The channel
  * gate and more heads use two kernels that exchange every block through the workspace.
@@ -312,8 +312,10 @@ typedef enum {
 /* The plan gdr_chunk_fwd uses for this problem (a gdr_plan value). For GDR_PLAN_PREP_FUSED,
  * *precomputed_chunks (if not NULL) receives the number of leading chunks per head the first
  * kernel prepares; for GDR_PLAN_SCAN, the number of segments; 0 otherwise. Chosen from the shape
- * alone: at most 16 heads with at least 512 chunks each (T a multiple of 256) run the segment scan
- * with 4 segments; otherwise B * H <= 56 heads run fused (the chains are the bound), 57-100 heads
+ * alone: at most 16 heads with at least 256 chunks each run the segment scan, with s segments, the
+ * largest power of two in 2 .. 16 with B * H * s <= 64, at least 16 chunks per segment and T a
+ * multiple of 64 s (4 segments for 16 heads, 16 for 1-4 heads); otherwise B * H <= 56 heads run
+ * fused (the chains are the bound), 57-100 heads
  * prepare the first chunks on every SM so that the fused kernel's remaining prep CTAs keep up with
  * the chains, more than 100 heads or the channel gate run two passes. gdr_chunk_fwd_noalloc never
  * uses the segment scan. */

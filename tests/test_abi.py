@@ -116,8 +116,12 @@ def test_plan_query_is_host_only():
     assert gdr.chunk_fwd_plan(1, 100, 2, 64, 64, 64, "scalar", torch.float32) == ("cuda_core", 0)
     # few heads, long sequences: the segment scan with 4 segments (4 launches)
     assert gdr.chunk_fwd_plan(1, 65536, 16, 128, 128, 64, "scalar", bf) == ("scan", 4)
-    assert gdr.chunk_fwd_plan(1, 32768, 2, 128, 128, 64, "channel", bf) == ("scan", 4)
-    assert gdr.chunk_fwd_plan(1, 32704, 2, 128, 128, 64, "scalar", bf) == ("fused", 0)  # T not a multiple of 256
+    assert gdr.chunk_fwd_plan(1, 32768, 2, 128, 128, 64, "channel", bf) == ("scan", 16)
+    assert gdr.chunk_fwd_plan(1, 65536, 8, 128, 128, 64, "scalar", bf) == ("scan", 8)
+    assert gdr.chunk_fwd_plan(1, 16384, 16, 128, 128, 64, "none", bf) == ("scan", 4)
+    assert gdr.chunk_fwd_plan(1, 16384 + 4096, 2, 128, 128, 64, "scalar", bf) == ("scan", 16)
+    assert gdr.chunk_fwd_plan(1, 16384 + 64, 2, 128, 128, 64, "scalar", bf) == ("fused", 0)  # no T % 128 == 0
+    assert gdr.chunk_fwd_plan(1, 8192, 2, 128, 128, 64, "scalar", bf) == ("fused", 0)  # 128 chunks: too short
     assert gdr.chunk_fwd_plan(2, 32768, 16, 128, 128, 64, "scalar", bf)[0] == "fused"  # 32 heads
     assert gdr.launches_per_chunk_fwd(1, 65536, 16, 128, 128, 64, "scalar", bf) == 4
     assert gdr.workspace_bytes(1, 65536, 16, 128, 128, 64, "scalar", bf) == \

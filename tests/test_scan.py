@@ -84,3 +84,25 @@ def test_scan_rejects_unsupported():
     with pytest.raises(gdr.GdrError) as e:
         gdr.chunk_fwd_scan(d["q"], d["k"], d["v"], d["g"], d["beta"], n_seg=1, mode="scalar")
     assert e.value.status == "GDR_ERR_INVALID_ARG"
+
+
+@pytest.mark.parametrize("mode", ["scalar", "channel"])
+def test_scan_chosen_by_chunk_fwd_with_prologue(mode):
+    """gdr_chunk_fwd picks the segment scan by itself for 2 heads of 32768 tokens (16 segments of 32
+    chunks); with S0 and the fused prologue (raw q/k, beta and gate logits) against the oracle's
+    prologue and recurrence."""
+    from gated_delta_rule_143_b200.inputs import make_raw_chunk_inputs
+    B, T, H = 1, 32768, 2
+    assert gdr.chunk_fwd_plan(B, T, H, 128, 128, 64, mode, torch.bfloat16) == ("scan", 16)
+    x = make_raw_chunk_inputs(B, T, H, 128, 128, mode, "bf16", 12300 + len(mode), s0_std=0.05)
+    d = {k: (None if t is None else t.cuda()) for k, t in x.items()}
+    flags = dict(l2norm_qk=True, beta_sigmoid=True, gate_softplus=True)
+    o, st = gdr.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], mode=mode, gate_scale=d["gate_scale"],
+                          **flags)
+    gdr.sync_status()
+    q, k, b, g = oracle.prologue(x["q"], x["k"], x["beta"], x["g"], mode, gate_scale=x["gate_scale"], **flags)
+    o_ref, s_ref = oracle.recurrent(q, k, x["v"].double(), g, b, mode, S0=x["S0"], f64_inputs=True)
+    eo, _ = rel_err(o.double().cpu().numpy(), o_ref)
+    es, _ = rel_err(st.double().cpu().numpy(), s_ref)
+    print(f"auto scan + prologue {mode}: o {eo:.3e}, S_T {es:.3e}")
+    assert eo <= TOL["bf16"] and es <= TOL["bf16"]
