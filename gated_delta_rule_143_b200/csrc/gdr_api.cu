@@ -138,14 +138,30 @@ int auto_segments(int B, int T, int H, int dk, int dv, int chunk, int dtype, int
     return scan_supported(B, T, H, dk, dv, chunk, dtype, o_dtype, s) ? s : 0;
 }
 
-// The chunked forward behind gdr_chunk_fwd_ex and gdr_chunk_fwd_scan. n_seg: 0 = the plan chosen from
-// the shape (auto_segments), -1 = no segment scan, >= 2 = that many segments.
+// Gated DeltaNet-2 runs on the tensor cores for the channel decay at the tensor-core shapes (the
+// channel gate's two passes), on the CUDA cores otherwise.
+bool gdn2_on_tc(int dk, int dv, int chunk, int mode, int dtype, int o_dtype) {
+    return mode == GDR_DECAY_CHANNEL && chunk_tc_supported(dk, dv, chunk, dtype, o_dtype);
+}
+
+// The chunked forward behind gdr_chunk_fwd(_ex, _scan, _noalloc) and gdr_chunk_fwd_gdn2. n_seg: 0 = the
+// plan chosen from the shape (auto_segments), -1 = no segment scan, >= 2 = that many segments. With
+// erase / write (Gated DeltaNet-2) beta is unused, and there is no prologue or segment scan.
 int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g, const float* beta, const float* S0,
                    void* o, float* S_T, int B, int T, int H, int dk, int dv, int chunk, int mode, int dtype,
-                   int o_dtype, int prologue, const float* gate_scale, int n_seg, void* workspace,
-                   size_t workspace_bytes, void* stream) {
+                   int o_dtype, int prologue, const float* gate_scale, int n_seg, const float* erase,
+                   const float* write, void* workspace, size_t workspace_bytes, void* stream) {
     ProfileScope prof_scope;
     if (int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype)) return rc;
+    const bool ew = erase != nullptr || write != nullptr;
+    if (ew) {
+        n_seg = -1;
+        beta = nullptr;
+        if (!erase || !write) return fail(GDR_ERR_INVALID_ARG, "erase and write must both be non-null");
+        if (!gdn2_on_tc(dk, dv, chunk, mode, dtype, o_dtype) && !chunk_simt_supported(dk, dv, chunk))
+            return fail(GDR_ERR_UNSUPPORTED,
+                        "Gated DeltaNet-2: d_k, d_v in {32, 64, 128} and chunk 64 (got %d, %d, %d)", dk, dv, chunk);
+    }
     if (n_seg == 0) n_seg = auto_segments(B, T, H, dk, dv, chunk, dtype, o_dtype);
     if (n_seg < 0) n_seg = 0;
     if (n_seg != 0 && !scan_supported(B, T, H, dk, dv, chunk, dtype, o_dtype, n_seg))
@@ -154,9 +170,11 @@ int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g, 
                     "n_seg * chunk (got T=%d, n_seg=%d)", T, n_seg);
     if (int rc = prologue_check(prologue, mode)) return rc;
     if (!(prologue & GDR_PRO_GATE_SOFTPLUS)) gate_scale = nullptr;
-    if (!q || !k || !v || !beta || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, beta and o must be non-null");
+    if (!q || !k || !v || (!beta && !ew) || !o)
+        return fail(GDR_ERR_INVALID_ARG, "q, k, v, beta and o must be non-null");
     if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
-    const void* ptrs[] = {q, k, v, g, beta, S0, o, S_T, workspace, gate_scale};
+    if (mode == GDR_DECAY_NONE) g = nullptr;
+    const void* ptrs[] = {q, k, v, g, beta, S0, o, S_T, workspace, gate_scale, erase, write};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return fail(GDR_ERR_MISALIGNED, "pointer %p is not 16-byte aligned", p);
     const size_t ntok = (size_t)B * T * H;
@@ -166,15 +184,17 @@ int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g, 
     const size_t bg = mode == GDR_DECAY_NONE ? 0 : (mode == GDR_DECAY_SCALAR ? bb : ntok * dk * sizeof(float));
     const size_t bs = (size_t)B * H * dv * dk * sizeof(float);
     struct Span { const void* p; size_t n; const char* name; };
-    const Span ins[] = {{q, bq, "q"}, {k, bq, "k"}, {v, bv, "v"}, {mode == GDR_DECAY_NONE ? nullptr : g, bg, "g"},
-                        {beta, bb, "beta"}, {S0, bs, "S0"}, {gate_scale, H * sizeof(float), "gate_scale"}};
+    const Span ins[] = {{q, bq, "q"}, {k, bq, "k"}, {v, bv, "v"}, {g, bg, "g"}, {beta, bb, "beta"}, {S0, bs, "S0"},
+                        {gate_scale, H * sizeof(float), "gate_scale"}, {erase, ntok * dk * sizeof(float), "erase"},
+                        {write, ntok * dv * sizeof(float), "write"}};
     for (const Span& s : ins) {
         if (overlap(o, bo, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "o overlaps input %s", s.name);
         if (S_T != S0 && overlap(S_T, bs, s.p, s.n))
             return fail(GDR_ERR_INVALID_ARG, "S_T overlaps input %s (only S_T == S0 is allowed)", s.name);
     }
     if (overlap(o, bo, S_T, bs)) return fail(GDR_ERR_INVALID_ARG, "o overlaps S_T");
-    const bool use_tc = chunk_tc_supported(dk, dv, chunk, dtype, o_dtype);
+    const bool use_tc = ew ? gdn2_on_tc(dk, dv, chunk, mode, dtype, o_dtype)
+                           : chunk_tc_supported(dk, dv, chunk, dtype, o_dtype);
     const size_t need = n_seg != 0 ? scan_workspace_bytes(B, T, H, mode, n_seg, o_dtype)
                                    : (use_tc ? chunk_tc_workspace_bytes(B, T, H, dk, dv, chunk, mode) : 0);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need))
@@ -191,9 +211,8 @@ int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g, 
     if (int rc = device_setup(&status, &major)) return rc;
     if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
 
-    ChunkProblem p{q, k, v, mode == GDR_DECAY_NONE ? nullptr : g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode,
-                   dtype, o_dtype, workspace, workspace_bytes, status, (float)(1.0 / sqrt((double)dk)), prologue,
-                   gate_scale};
+    ChunkProblem p{q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, workspace,
+                   workspace_bytes, status, (float)(1.0 / sqrt((double)dk)), prologue, gate_scale, erase, write};
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const cudaError_t err = n_seg != 0 ? launch_scan(p, n_seg, s) : (use_tc ? launch_chunk_tc(p, s) : launch_chunk_simt(p, s));
     if (err != cudaSuccess)
@@ -202,6 +221,53 @@ int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g, 
     return ok();
 }
 
+
+// The decode step behind gdr_decode_step(_ex) and gdr_decode_step_gdn2 (erase / write in place of beta,
+// no prologue).
+int decode_impl(const void* q, const void* k, const void* v, const float* g, const float* beta, float* S, void* o,
+                int B, int H, int dk, int dv, int mode, int dtype, int o_dtype, int prologue, const float* gate_scale,
+                const float* erase, const float* write, void* stream) {
+    if (int rc = check_enums(mode, dtype, o_dtype)) return rc;
+    const bool ew = erase != nullptr || write != nullptr;
+    if (ew && (!erase || !write)) return fail(GDR_ERR_INVALID_ARG, "erase and write must both be non-null");
+    if (ew) beta = nullptr, prologue = GDR_PRO_NONE;
+    if (int rc = prologue_check(prologue, mode)) return rc;
+    if (!(prologue & GDR_PRO_GATE_SOFTPLUS)) gate_scale = nullptr;
+    if (B <= 0 || H <= 0 || dk <= 0 || dv <= 0)
+        return fail(GDR_ERR_INVALID_ARG, "sizes must be positive (B=%d H=%d d_k=%d d_v=%d)", B, H, dk, dv);
+    if ((size_t)B * H > 0x7fffffffu) return fail(GDR_ERR_UNSUPPORTED, "B*H too large");
+    if (!decode_supported(dk, dv))
+        return fail(GDR_ERR_UNSUPPORTED, "unsupported d_k=%d (supported: 32, 64, 128, 256)", dk);
+    if (!q || !k || !v || (!beta && !ew) || !S || !o)
+        return fail(GDR_ERR_INVALID_ARG, "q, k, v, beta, S and o must be non-null");
+    if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
+    if (mode == GDR_DECAY_NONE) g = nullptr;
+    const void* ptrs[] = {q, k, v, g, beta, S, o, gate_scale, erase, write};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return fail(GDR_ERR_MISALIGNED, "pointer %p is not 16-byte aligned", p);
+    const size_t nh = (size_t)B * H, eb = elem_bytes(dtype);
+    const size_t bs = nh * dv * dk * sizeof(float), bo = nh * dv * elem_bytes(o_dtype);
+    struct Span { const void* p; size_t n; const char* name; };
+    const Span ins[] = {{q, nh * dk * eb, "q"}, {k, nh * dk * eb, "k"}, {v, nh * dv * eb, "v"},
+                        {mode == GDR_DECAY_NONE ? nullptr : g,
+                         mode == GDR_DECAY_CHANNEL ? nh * dk * sizeof(float) : nh * sizeof(float), "g"},
+                        {beta, nh * sizeof(float), "beta"}, {gate_scale, H * sizeof(float), "gate_scale"},
+                        {erase, nh * dk * sizeof(float), "erase"}, {write, nh * dv * sizeof(float), "write"}};
+    for (const Span& s : ins) {
+        if (overlap(S, bs, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "S overlaps input %s", s.name);
+        if (overlap(o, bo, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "o overlaps input %s", s.name);
+    }
+    if (overlap(o, bo, S, bs)) return fail(GDR_ERR_INVALID_ARG, "o overlaps S");
+    int* status = nullptr;
+    int major = 0;
+    if (int rc = device_setup(&status, &major)) return rc;
+    if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
+    DecodeProblem p{q, k, v, mode == GDR_DECAY_NONE ? nullptr : g, beta, S, o, B, H, dk, dv, mode, dtype, o_dtype,
+                    status, (float)(1.0 / sqrt((double)dk)), prologue, gate_scale, erase, write};
+    const cudaError_t err = launch_decode(p, static_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
+    return ok();
+}
 
 }  // namespace
 
@@ -270,7 +336,7 @@ int gdr_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* g
                      int mode, int dtype, int o_dtype, int prologue, const float* gate_scale, void* workspace,
                      size_t workspace_bytes, void* stream) {
     return chunk_fwd_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, prologue,
-                          gate_scale, 0, workspace, workspace_bytes, stream);
+                          gate_scale, 0, nullptr, nullptr, workspace, workspace_bytes, stream);
 }
 
 int gdr_chunk_fwd_scan(const void* q, const void* k, const void* v, const float* g, const float* beta,
@@ -279,7 +345,7 @@ int gdr_chunk_fwd_scan(const void* q, const void* k, const void* v, const float*
                        void* stream) {
     if (n_seg < 2) return fail(GDR_ERR_INVALID_ARG, "n_seg = %d (at least 2)", n_seg);
     return chunk_fwd_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, GDR_PRO_NONE,
-                          nullptr, n_seg, workspace, workspace_bytes, stream);
+                          nullptr, n_seg, nullptr, nullptr, workspace, workspace_bytes, stream);
 }
 
 size_t gdr_chunk_fwd_scan_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int mode, int dtype,
@@ -302,52 +368,14 @@ int gdr_chunk_fwd(const void* q, const void* k, const void* v, const float* g, c
 int gdr_decode_step_ex(const void* q, const void* k, const void* v, const float* g, const float* beta, float* S,
                        void* o, int B, int H, int dk, int dv, int mode, int dtype, int o_dtype, int prologue,
                        const float* gate_scale, void* stream) {
-    if (int rc = check_enums(mode, dtype, o_dtype)) return rc;
-    if (int rc = prologue_check(prologue, mode)) return rc;
-    if (!(prologue & GDR_PRO_GATE_SOFTPLUS)) gate_scale = nullptr;
-    if (B <= 0 || H <= 0 || dk <= 0 || dv <= 0)
-        return fail(GDR_ERR_INVALID_ARG, "sizes must be positive (B=%d H=%d d_k=%d d_v=%d)", B, H, dk, dv);
-    if ((size_t)B * H > 0x7fffffffu) return fail(GDR_ERR_UNSUPPORTED, "B*H too large");
-    if (!decode_supported(dk, dv))
-        return fail(GDR_ERR_UNSUPPORTED, "unsupported d_k=%d (supported: 32, 64, 128, 256)", dk);
-    if (!q || !k || !v || !beta || !S || !o) return fail(GDR_ERR_INVALID_ARG, "q, k, v, beta, S and o must be non-null");
-    if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
-    const void* ptrs[] = {q, k, v, g, beta, S, o, gate_scale};
-    for (const void* p : ptrs)
-        if (p && !aligned16(p)) return fail(GDR_ERR_MISALIGNED, "pointer %p is not 16-byte aligned", p);
-    const size_t nh = (size_t)B * H, eb = elem_bytes(dtype);
-    const size_t bs = nh * dv * dk * sizeof(float), bo = nh * dv * elem_bytes(o_dtype);
-    struct Span { const void* p; size_t n; const char* name; };
-    const Span ins[] = {{q, nh * dk * eb, "q"}, {k, nh * dk * eb, "k"}, {v, nh * dv * eb, "v"},
-                        {mode == GDR_DECAY_NONE ? nullptr : g,
-                         mode == GDR_DECAY_CHANNEL ? nh * dk * sizeof(float) : nh * sizeof(float), "g"},
-                        {beta, nh * sizeof(float), "beta"}, {gate_scale, H * sizeof(float), "gate_scale"}};
-    for (const Span& s : ins) {
-        if (overlap(S, bs, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "S overlaps input %s", s.name);
-        if (overlap(o, bo, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "o overlaps input %s", s.name);
-    }
-    if (overlap(o, bo, S, bs)) return fail(GDR_ERR_INVALID_ARG, "o overlaps S");
-    int* status = nullptr;
-    int major = 0;
-    if (int rc = device_setup(&status, &major)) return rc;
-    if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
-    DecodeProblem p{q, k, v, mode == GDR_DECAY_NONE ? nullptr : g, beta, S, o, B, H, dk, dv, mode, dtype, o_dtype,
-                    status, (float)(1.0 / sqrt((double)dk)), prologue, gate_scale};
-    const cudaError_t err = launch_decode(p, static_cast<cudaStream_t>(stream));
-    if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
-    return ok();
+    return decode_impl(q, k, v, g, beta, S, o, B, H, dk, dv, mode, dtype, o_dtype, prologue, gate_scale, nullptr,
+                       nullptr, stream);
 }
 
 int gdr_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta, float* S,
                     void* o, int B, int H, int dk, int dv, int mode, int dtype, int o_dtype, void* stream) {
     return gdr_decode_step_ex(q, k, v, g, beta, S, o, B, H, dk, dv, mode, dtype, o_dtype, GDR_PRO_NONE, nullptr,
                               stream);
-}
-
-// Gated DeltaNet-2 runs on the tensor cores for the channel decay at the tensor-core shapes (the
-// channel gate's two passes), on the CUDA cores otherwise.
-bool gdn2_on_tc(int dk, int dv, int chunk, int mode, int dtype, int o_dtype) {
-    return mode == GDR_DECAY_CHANNEL && chunk_tc_supported(dk, dv, chunk, dtype, o_dtype);
 }
 
 size_t gdr_chunk_fwd_gdn2_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int mode, int dtype,
@@ -364,87 +392,17 @@ int gdr_chunk_fwd_gdn2(const void* q, const void* k, const void* v, const float*
                        const float* write, const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv,
                        int chunk, int mode, int dtype, int o_dtype, void* workspace, size_t workspace_bytes,
                        void* stream) {
-    ProfileScope prof_scope;
-    if (int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype)) return rc;
-    const bool on_tc = gdn2_on_tc(dk, dv, chunk, mode, dtype, o_dtype);
-    if (!on_tc && !chunk_simt_supported(dk, dv, chunk))
-        return fail(GDR_ERR_UNSUPPORTED, "Gated DeltaNet-2: d_k, d_v in {32, 64, 128} and chunk 64 (got %d, %d, %d)", dk,
-                    dv, chunk);
-    if (!q || !k || !v || !erase || !write || !o)
-        return fail(GDR_ERR_INVALID_ARG, "q, k, v, erase, write and o must be non-null");
-    if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
-    if (mode == GDR_DECAY_NONE) g = nullptr;
-    const void* ptrs[] = {q, k, v, g, erase, write, S0, o, S_T, workspace};
-    for (const void* p : ptrs)
-        if (p && !aligned16(p)) return fail(GDR_ERR_MISALIGNED, "pointer %p is not 16-byte aligned", p);
-    const size_t ntok = (size_t)B * T * H, eb = elem_bytes(dtype);
-    const size_t bo = ntok * dv * elem_bytes(o_dtype), bs = (size_t)B * H * dv * dk * sizeof(float);
-    const size_t need = on_tc ? chunk_tc_workspace_bytes(B, T, H, dk, dv, chunk, mode) : 0;
-    if (need > 0 && (workspace == nullptr || workspace_bytes < need))
-        return fail(GDR_ERR_WORKSPACE, "workspace of %zu bytes required (got %zu at %p)", need, workspace_bytes,
-                    workspace);
-    struct Span { const void* p; size_t n; const char* name; };
-    const Span ins[] = {{q, ntok * dk * eb, "q"}, {k, ntok * dk * eb, "k"}, {v, ntok * dv * eb, "v"},
-                        {g, mode == GDR_DECAY_CHANNEL ? ntok * dk * 4 : ntok * 4, "g"}, {erase, ntok * dk * 4, "erase"},
-                        {write, ntok * dv * 4, "write"}, {S0, bs, "S0"}};
-    for (const Span& s : ins) {
-        if (overlap(o, bo, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "o overlaps input %s", s.name);
-        if (S_T != S0 && overlap(S_T, bs, s.p, s.n))
-            return fail(GDR_ERR_INVALID_ARG, "S_T overlaps input %s (only S_T == S0 is allowed)", s.name);
-        if (need > 0 && overlap(workspace, need, s.p, s.n))
-            return fail(GDR_ERR_INVALID_ARG, "workspace overlaps %s", s.name);
-    }
-    if (overlap(o, bo, S_T, bs)) return fail(GDR_ERR_INVALID_ARG, "o overlaps S_T");
-    if (need > 0 && (overlap(workspace, need, o, bo) || overlap(workspace, need, S_T, bs)))
-        return fail(GDR_ERR_INVALID_ARG, "workspace overlaps an output");
-    int* status = nullptr;
-    int major = 0;
-    if (int rc = device_setup(&status, &major)) return rc;
-    if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
-    ChunkProblem p{q, k, v, g, nullptr, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, workspace,
-                   workspace_bytes, status, (float)(1.0 / sqrt((double)dk)), GDR_PRO_NONE, nullptr, erase, write};
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const cudaError_t err = on_tc ? launch_chunk_tc(p, s) : launch_chunk_simt(p, s);
-    if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "Gated DeltaNet-2 launch: %s", cudaGetErrorString(err));
-    return ok();
+    if (!erase || !write) return fail(GDR_ERR_INVALID_ARG, "erase and write must both be non-null");
+    return chunk_fwd_impl(q, k, v, g, nullptr, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, GDR_PRO_NONE,
+                          nullptr, -1, erase, write, workspace, workspace_bytes, stream);
 }
 
 int gdr_decode_step_gdn2(const void* q, const void* k, const void* v, const float* g, const float* erase,
                          const float* write, float* S, void* o, int B, int H, int dk, int dv, int mode, int dtype,
                          int o_dtype, void* stream) {
-    if (int rc = check_enums(mode, dtype, o_dtype)) return rc;
-    if (B <= 0 || H <= 0 || dk <= 0 || dv <= 0)
-        return fail(GDR_ERR_INVALID_ARG, "sizes must be positive (B=%d H=%d d_k=%d d_v=%d)", B, H, dk, dv);
-    if ((size_t)B * H > 0x7fffffffu) return fail(GDR_ERR_UNSUPPORTED, "B*H too large");
-    if (!decode_supported(dk, dv))
-        return fail(GDR_ERR_UNSUPPORTED, "unsupported d_k=%d (supported: 32, 64, 128, 256)", dk);
-    if (!q || !k || !v || !erase || !write || !S || !o)
-        return fail(GDR_ERR_INVALID_ARG, "q, k, v, erase, write, S and o must be non-null");
-    if (mode != GDR_DECAY_NONE && !g) return fail(GDR_ERR_INVALID_ARG, "g must be non-null for a gated decay mode");
-    if (mode == GDR_DECAY_NONE) g = nullptr;
-    const void* ptrs[] = {q, k, v, g, erase, write, S, o};
-    for (const void* p : ptrs)
-        if (p && !aligned16(p)) return fail(GDR_ERR_MISALIGNED, "pointer %p is not 16-byte aligned", p);
-    const size_t nh = (size_t)B * H, eb = elem_bytes(dtype);
-    const size_t bs = nh * dv * dk * sizeof(float), bo = nh * dv * elem_bytes(o_dtype);
-    struct Span { const void* p; size_t n; const char* name; };
-    const Span ins[] = {{q, nh * dk * eb, "q"}, {k, nh * dk * eb, "k"}, {v, nh * dv * eb, "v"},
-                        {g, mode == GDR_DECAY_CHANNEL ? nh * dk * 4 : nh * 4, "g"}, {erase, nh * dk * 4, "erase"},
-                        {write, nh * dv * 4, "write"}};
-    for (const Span& s : ins) {
-        if (overlap(S, bs, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "S overlaps input %s", s.name);
-        if (overlap(o, bo, s.p, s.n)) return fail(GDR_ERR_INVALID_ARG, "o overlaps input %s", s.name);
-    }
-    if (overlap(o, bo, S, bs)) return fail(GDR_ERR_INVALID_ARG, "o overlaps S");
-    int* status = nullptr;
-    int major = 0;
-    if (int rc = device_setup(&status, &major)) return rc;
-    if (major != 10) return fail(GDR_ERR_DEVICE, "compute capability %d.x: this library is built for sm_100a", major);
-    DecodeProblem p{q, k, v, g, nullptr, S, o, B, H, dk, dv, mode, dtype, o_dtype, status,
-                    (float)(1.0 / sqrt((double)dk)), GDR_PRO_NONE, nullptr, erase, write};
-    const cudaError_t err = launch_decode(p, static_cast<cudaStream_t>(stream));
-    if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
-    return ok();
+    if (!erase || !write) return fail(GDR_ERR_INVALID_ARG, "erase and write must both be non-null");
+    return decode_impl(q, k, v, g, nullptr, S, o, B, H, dk, dv, mode, dtype, o_dtype, GDR_PRO_NONE, nullptr, erase,
+                       write, stream);
 }
 
 size_t gdr_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, int mode, int dtype) {
@@ -601,7 +559,7 @@ extern "C" int gdr_chunk_fwd_noalloc(const void* q, const void* k, const void* v
     void* ws = nullptr;
     if (int rc = noalloc_scratch(&ws)) return rc;
     return chunk_fwd_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, mode, dtype, o_dtype, GDR_PRO_NONE,
-                          nullptr, -1, ws, (size_t)GDR_NOALLOC_SCRATCH_BYTES, stream);
+                          nullptr, -1, nullptr, nullptr, ws, (size_t)GDR_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 // ------------------------------------------------------------ host-buffer entry point --

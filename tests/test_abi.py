@@ -231,3 +231,16 @@ def test_chunk_fwd_gdn2_workspace_query():
     rc = lib.gdr_chunk_fwd_gdn2(1 * M, 2 * M, 3 * M, 4 * M, 5 * M, 6 * M, None, 7 * M, None, 1, 128, 2, 128, 128, 64,
                                 2, 1, 0, None, 0, None)
     assert rc == -4
+
+
+def test_library_exports_only_declared_c_symbols():
+    """Every unmangled symbol libgdr.so defines is an entry point of include/gdr.h (nothing internal
+    leaks out with C linkage)."""
+    import shutil
+    import subprocess
+    if shutil.which("nm") is None:
+        pytest.skip("nm not available")
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True, check=True)
+    names = {line.split()[-1] for line in out.stdout.splitlines() if line.strip()}
+    c_names = {n for n in names if not n.startswith("_")}
+    assert c_names == set(declared_functions()), sorted(c_names ^ set(declared_functions()))
