@@ -86,7 +86,18 @@ constexpr uint32_t kPBeta = kPX + 32 * kLdX * 4;     // beta [64]
 constexpr uint32_t kPGam = kPBeta + 256;             // Gamma * log2(e): [64] or [64][128] (channel)
 constexpr uint32_t kPInvE = kPGam + 256;             // scalar gate: 2^-Gamma [64], then a "factorable" flag
 constexpr uint32_t kPKB = (kPGam + 32768 + 1023) & ~1023u;  // channel: K'' fp16 K-major 64 x 128
-constexpr uint32_t kPrepBytesScalar = (kPInvE + 512 + 1023) & ~1023u;
+// DeltaNet and the scalar gate: two regions take turns as the [K; Q] tile (32 KiB) and as A^T and T
+// (2 x 17 KiB), so that the next task's tile loads while this task finishes; the solve's scratch
+// sits in the tile's Q rows, free once the Gram product is done
+constexpr uint32_t kFRegion = 2 * 64 * kLdA * 4;
+static_assert(kLdA == kLdT && kFRegion >= 32768 && kFRegion % 1024 == 0, "a region holds A^T and T, or the tile");
+static_assert(32 * kLdX * 4 <= 8192, "the solve's scratch fits in one 8 KiB box of Q rows");
+constexpr uint32_t kFV = 2 * kFRegion;                // V bf16 (TMA) K-major 64 x 128
+constexpr uint32_t kFTBZ = kFV + 16384;               // [T diag(beta); Z]
+constexpr uint32_t kFBeta = kFTBZ + 16384;            // beta [64]
+constexpr uint32_t kFGam = kFBeta + 256;              // Gamma * log2(e) [64]
+constexpr uint32_t kFInvE = kFGam + 256;              // 2^-Gamma [64], then a "factorable" flag
+constexpr uint32_t kPrepBytesScalar = (kFInvE + 512 + 512 + 1023) & ~1023u;
 constexpr uint32_t kPKQ2 = kPKB + 16384;  // channel: second copy of the bf16 [K; Q] tile (TMA), 32 KiB
 constexpr uint32_t kPStrong = kPKQ2 + 32768;  // channel: int flags [128], then per-warp lists [4][32] + counts [4]
 constexpr uint32_t kPrepBytesChannel = kPStrong + 1024 + 1024;
@@ -109,14 +120,15 @@ struct PrepArgs {
 // Inverse L2 norms of the 128 rows of the [K; Q] tile (prologue GDR_PRO_L2NORM_QK), fp32 [128]:
 // in the slack after the scalar gate's 2^-Gamma table, or after the channel gate's strong lists.
 __host__ __device__ constexpr uint32_t nrm_off(int mode) {
-    return mode == GDR_DECAY_CHANNEL ? kPStrong + 1280 : kPInvE + 512;
+    return mode == GDR_DECAY_CHANNEL ? kPStrong + 1280 : kFInvE + 512;
 }
-static_assert(kPInvE + 512 + 512 <= kPrepBytesScalar, "norm table fits the scalar layout");
+static_assert(kFInvE + 512 + 512 <= kPrepBytesScalar, "norm table fits the scalar layout");
 static_assert(kPStrong + 1280 + 512 <= kPrepBytesChannel, "norm table fits the channel layout");
 
 struct PrepSmem {
     uint8_t* base;
-    uint64_t* bars;  // [4]: TMA, Gram, W/U, TMA of the channel gate's tile copy
+    uint64_t* bars;  // [4]: TMA ([K; Q], and V for the channel gate), Gram, W/U, TMA of V (the
+                     // channel gate: of its tile copy)
     uint32_t tmem;
     int bar_id;      // named barrier of this pipeline's 128 threads
 };
@@ -265,39 +277,47 @@ __device__ void unit_lower_inverse64(const float* __restrict__ sAt, float* __res
 }
 
 // One-time set-up of a prep pipeline's shared memory: the zero block under T diag(beta) (rows
-// 64-127 of the M = 128 operand of the W product) and the strictly upper part of T (never
-// written by the solve).
+// 64-127 of the M = 128 operand of the W product) and, for the channel gate, the strictly upper
+// part of T (never written by the solve; the other modes clear it in each task, as T moves).
+template <int MODE>
 __device__ void prep_init(const PrepSmem& ps, int lt) {
-    uint8_t* z = ps.base + kPTBZ + 8192;
+    uint8_t* z = ps.base + (MODE == GDR_DECAY_CHANNEL ? kPTBZ : kFTBZ) + 8192;
     for (int i = lt; i < 512; i += kPrepThreads) reinterpret_cast<uint4*>(z)[i] = make_uint4(0, 0, 0, 0);  // 8 KiB
-    float* sT = reinterpret_cast<float*>(ps.base + kPT);
-    for (int i = lt; i < 64 * kLdT; i += kPrepThreads) sT[i] = 0.f;
+    if (MODE == GDR_DECAY_CHANNEL) {
+        float* sT = reinterpret_cast<float*>(ps.base + kPT);
+        for (int i = lt; i < 64 * kLdT; i += kPrepThreads) sT[i] = 0.f;
+    }
 }
 
 // Computes the hand-off block of chunk c of head (b, h) into `out` (global memory). Executed by the
 // 256 threads of one pipeline (8 warps: TMEM lane quadrant q = warp & 3, column half hf = warp >> 2);
-// `it` counts the pipeline's previous tasks (mbarrier phase parity).
+// `it` counts the pipeline's previous tasks (mbarrier phase parity). DeltaNet and the scalar gate
+// load the [K; Q] tile of the pipeline's next task (chunk nc of head (nb, nh); nc < 0: none) once
+// this task's T diag(beta) is built; `pre` says that the previous task did so for this one.
 template <int MODE, bool PRO, bool EW = false>
 __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv,
                            const PrepSmem& ps, int b, int h, int c, uint8_t* __restrict__ out, uint32_t it, int lt,
-                           uint32_t& n_copies) {
+                           uint32_t& n_copies, int nb, int nh, int nc, bool pre) {
+    constexpr bool PF = MODE != GDR_DECAY_CHANNEL;  // alternating regions, tile of the next task ahead
     const int lw = lt >> 5, lane = lt & 31;
     const int q = lw & 3, hf = lw >> 2;
     const uint32_t par = it & 1u;
     uint8_t* sm = ps.base;
-    uint8_t* sKQ = sm + kPKQ;
-    uint8_t* sV = sm + kPV;
-    uint8_t* sTB = sm + kPTBZ;
-    float* sAt = reinterpret_cast<float*>(sm + kPA);
-    float* sT = reinterpret_cast<float*>(sm + kPT);
-    float* sX = reinterpret_cast<float*>(sm + kPX);
-    float* sBeta = reinterpret_cast<float*>(sm + kPBeta);
-    float* sGam = reinterpret_cast<float*>(sm + kPGam);
-    float* sInvE = reinterpret_cast<float*>(sm + kPInvE);
+    uint8_t* sKQ = sm + (PF ? par * kFRegion : kPKQ);
+    uint8_t* sAT = sm + (PF ? (par ^ 1u) * kFRegion : kPA);  // A^T, then T: the other region
+    uint8_t* sV = sm + (PF ? kFV : kPV);
+    uint8_t* sTB = sm + (PF ? kFTBZ : kPTBZ);
+    float* sAt = reinterpret_cast<float*>(sAT);
+    float* sT = reinterpret_cast<float*>(PF ? sAT + 64 * kLdA * 4 : sm + kPT);
+    float* sX = reinterpret_cast<float*>(PF ? sKQ + 8192 : sm + kPX);  // PF: the first box of Q rows
+    float* sBeta = reinterpret_cast<float*>(sm + (PF ? kFBeta : kPBeta));
+    float* sGam = reinterpret_cast<float*>(sm + (PF ? kFGam : kPGam));
+    float* sInvE = reinterpret_cast<float*>(sm + (PF ? kFInvE : kPInvE));
     uint8_t* sKB = sm + kPKB;
     uint64_t* barT = ps.bars;
     uint64_t* barG = ps.bars + 1;
     uint64_t* barW = ps.bars + 2;
+    uint64_t* barV = ps.bars + 3;  // PF only (the channel gate's tile copy uses it otherwise)
     const int T = P.T, H = P.H;
     const int c0 = c * kC;
     const int n = min(kC, T - c0);
@@ -310,13 +330,17 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
     //         cumulative log-decay (log2 units; rows past the tail repeat Gamma_{n-1}) meanwhile
     if (lt == 0) {
         bulk_wait_read<0>();  // the previous task's W / U^T bulk stores have read the K / V tiles
-        mbar_arrive_expect_tx(barT, 6 * 8192);
-        tma_load_4d(sKQ, mk, 0, h, c0, b, barT);
-        tma_load_4d(sKQ + 16384, mk, 64, h, c0, b, barT);
-        tma_load_4d(sKQ + 8192, mq, 0, h, c0, b, barT);
-        tma_load_4d(sKQ + 24576, mq, 64, h, c0, b, barT);
-        tma_load_4d(sV, mv, 0, h, c0, b, barT);
-        tma_load_4d(sV + 8192, mv, 64, h, c0, b, barT);
+        uint64_t* bv = PF ? barV : barT;
+        if (!(PF && pre)) {
+            mbar_arrive_expect_tx(barT, (PF ? 4 : 6) * 8192);
+            tma_load_4d(sKQ, mk, 0, h, c0, b, barT);
+            tma_load_4d(sKQ + 16384, mk, 64, h, c0, b, barT);
+            tma_load_4d(sKQ + 8192, mq, 0, h, c0, b, barT);
+            tma_load_4d(sKQ + 24576, mq, 64, h, c0, b, barT);
+        }
+        if (PF) mbar_arrive_expect_tx(barV, 2 * 8192);
+        tma_load_4d(sV, mv, 0, h, c0, b, bv);
+        tma_load_4d(sV + 8192, mv, 64, h, c0, b, bv);
     }
     if (lw == 7) {
         const bool sig = PRO && (P.pro & GDR_PRO_BETA_SIGMOID) != 0;
@@ -405,6 +429,19 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
     }
     mbar_wait(barT, par, P.status);
     const uint32_t tG = ps.tmem + kTG, tW = ps.tmem + kTW, tU = ps.tmem + kTU;
+    // Gram products for the scalar gate / DeltaNet straight from the bf16 tiles (a prologue's norms
+    // rescale them in the epilogue). Issued here rather than before the barrier above: measured
+    // slower there, as the other warps then wait for the issue.
+    if (PF && lt == 0) {
+        tc_fence_after();
+        const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t d = sdesc(smem_u32(sKQ) + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+            mma_f16(tG, d, d, id, ks > 0);  // B = the K rows (first 64 rows) of the same tile
+        }
+        mma_commit(barG);
+    }
     if (norm) {
         // inverse L2 norms of the 128 tile rows (K rows 0-63, Q rows 64-127; rows past the tail are
         // zero and get 0), two threads per row; the Gram products below run on the raw tiles and
@@ -421,17 +458,6 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
         ss += __shfl_xor_sync(0xffffffffu, ss, 1);
         if (half == 0) sNrm[row] = pro_inv_norm(ss);
         named_bar(ps.bar_id, kPrepThreads);
-    }
-    // Gram products for the scalar gate / DeltaNet straight from the bf16 tiles
-    if (MODE != GDR_DECAY_CHANNEL && lt == 0) {
-        tc_fence_after();
-        const uint32_t id = idesc_bf16(128, 64, false, false);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t d = sdesc(smem_u32(sKQ) + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-            mma_f16(tG, d, d, id, ks > 0);  // B = the K rows (first 64 rows) of the same tile
-        }
-        mma_commit(barG);
     }
 
     // ---- 2. Q*gamma and K*gamma_C/gamma hand-off images; channel gate: decay-factored Gram operands
@@ -602,6 +628,17 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
             for (int ci = 0; ci < 4; ++ci) st16(out + kOffP + kmajor_off(rr, 32 * hf + ci * 8, 64), pack8h(p + ci * 8));
         }
     }
+    if (PF) {
+        // the strictly upper blocks of T that the solve never writes (T_01, T_23 and the upper-right
+        // 32 x 32) but reads or scales: this region held a tile
+#pragma unroll
+        for (int j = 0; j < 6; ++j) {
+            const int i = lt + kPrepThreads * j;
+            const int r = i < 256 ? i >> 4 : i < 512 ? 32 + ((i - 256) >> 4) : (i - 512) >> 5;
+            const int col = i < 256 ? 16 + (i & 15) : i < 512 ? 48 + (i & 15) : 32 + (i & 31);
+            sT[r * kLdT + col] = 0.f;
+        }
+    }
     tc_fence_before();
     named_bar(ps.bar_id, kPrepThreads);
 
@@ -611,6 +648,7 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
         unit_lower_inverse64(sAt, sT, sX, lt, ps.bar_id + 1);
     } else {
         const int lt4 = lt - 128;
+        if (PF) mbar_wait(barV, par, P.status);
 #pragma unroll 4
         for (int j = 0; j < 16; ++j) {
             const int task = lt4 + 128 * j;
@@ -686,6 +724,16 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
             mma_f16(tU, sdesc(smem_u32(sV) + ks * 2048, 8192, 1024), tb, idU, ks > 0);
         }
         mma_commit(barW);
+        if (PF && nc >= 0) {
+            // the next task's [K; Q] tile into the region of A^T and T, which no one reads any more
+            // (every thread's accesses were ordered before the async proxy ahead of the last barrier)
+            const int nc0 = nc * kC;
+            mbar_arrive_expect_tx(barT, 4 * 8192);
+            tma_load_4d(sAT, mk, 0, nh, nc0, nb, barT);
+            tma_load_4d(sAT + 16384, mk, 64, nh, nc0, nb, barT);
+            tma_load_4d(sAT + 8192, mq, 0, nh, nc0, nb, barT);
+            tma_load_4d(sAT + 24576, mq, 64, nh, nc0, nb, barT);
+        }
     }
     __syncwarp();
     mbar_wait(barW, par, P.status);
@@ -728,9 +776,10 @@ __device__ void prep_chunk(const PrepArgs& P, const CUtensorMap* mq, const CUten
 // Standalone prep kernel: one pipeline per CTA, persistent over the chunk tasks t = blockIdx.x,
 // blockIdx.x + gridDim.x, ... for the first NCp chunks of every head (t = (b * H + h) * NCp + c, the
 // block's index in the workspace; NCp = NC on the two-pass path, the fused kernel's c1 before it).
-// At the start of each task the tiles of the CTA's next task are prefetched into L2. The scalar
-// and DeltaNet variants run at 96 registers per thread (no spills; measured 1-2.5 % faster than
-// the 128 two CTAs per SM would allow).
+// At the start of each task the tiles of the CTA's next task are prefetched into L2; for DeltaNet
+// and the scalar gate its [K; Q] tile then comes into shared memory during this task's W / U
+// products (prep kernel 241 -> 238 us at B16 H8 T4096). The scalar and DeltaNet variants run at 96
+// registers per thread (no spills; measured 1-2.5 % faster than the 128 two CTAs per SM would allow).
 template <int MODE, bool PRO, bool EW = false>
 __global__ void __maxnreg__(MODE == GDR_DECAY_CHANNEL ? 240 : 96)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
@@ -748,7 +797,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         tmem_relinquish();
     }
     PrepSmem ps{align1024(smem_raw), bars, 0, 1};
-    prep_init(ps, lt);
+    prep_init<MODE>(ps, lt);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -769,7 +818,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
             tma_prefetch_l2_4d(&mv, 64, hn, cn * kC, bn);
         }
         uint8_t* out = ws + (size_t)t * kHandoffStride;
-        prep_chunk<MODE, PRO, EW>(P, &mq, &mk, &mv, ps, b, h, c, out, it, lt, n_copies);
+        const int cn = tn % NCp, bhn = tn / NCp;
+        prep_chunk<MODE, PRO, EW>(P, &mq, &mk, &mv, ps, b, h, c, out, it, lt, n_copies, bhn / P.H, bhn % P.H,
+                                  tn < n_tasks ? cn : -1, it > 0);
     }
     if (lt == 0) bulk_wait<0>();
     tc_fence_before();
@@ -1196,7 +1247,7 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
             for (int k = 0; k < 4; ++k) mbar_init(&pbars[i][k], 1);
         fence_mbar_init();
     }
-    if (pipe < 2) prep_init(PrepSmem{sm + pipe * kPrepPipeBytes, nullptr, 0, 0}, lt);
+    if (pipe < 2) prep_init<MODE>(PrepSmem{sm + pipe * kPrepPipeBytes, nullptr, 0, 0}, lt);
     __syncthreads();
     // a head's chain consumes a chunk about every 2 us and a pipeline prepares one in about 11 us:
     // 3 CTAs (6 pipelines) per head keep the rings full; more would only wait on ring slots
@@ -1206,7 +1257,9 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
     uint32_t it = 0, n_copies = 0;  // tasks so far; channel-gate tile copies so far (mbarrier parities)
     for (;; ++it) {
         // claim the next task in consumption order (a pipeline claims only after finishing its
-        // previous task, so claims, like the state passes' reads, go in increasing order)
+        // previous task, so claims, like the state passes' reads, go in increasing order). Claiming
+        // one task ahead, to load its tile during the one before, was measured slower: the chains
+        // wait longer for the earliest blocks.
         if (lt == 0) claimed[pipe] = R.c1 * R.BH + atomicAdd(R.next_task, 1);
         named_bar(ps.bar_id, kPrepThreads);
         const int tau = claimed[pipe];
@@ -1219,7 +1272,7 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
         named_bar(ps.bar_id, kPrepThreads);
         if (!go[pipe]) break;
         uint8_t* out = R.ring + ((size_t)bh * R.depth + slot) * kHandoffStride;
-        prep_chunk<MODE, PRO>(P, mq, mk, mv, ps, bh / P.H, bh % P.H, c, out, it, lt, n_copies);
+        prep_chunk<MODE, PRO>(P, mq, mk, mv, ps, bh / P.H, bh % P.H, c, out, it, lt, n_copies, 0, 0, -1, false);
         if (lt == 0) {  // every write of the block (generic stores before prep_chunk's last barrier, bulk stores)
             bulk_wait<0>();
             fence_proxy_async_global();
@@ -1309,8 +1362,8 @@ cudaError_t launch_prep(const ChunkProblem& p, const CUtensorMap& mq, const CUte
     int dev = 0, sms = 0;
     if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
     if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
-    // pipelines per SM: two for DeltaNet and the scalar gate (2 x (114,688 + 1,024 reserved + static)
-    // bytes fit in the SM's 228 KiB), one for the channel gate
+    // pipelines per SM: two for DeltaNet and the scalar gate (2 x (kPrepBytesScalar + 1,024 alignment
+    // + 1,024 reserved + static) bytes fit in the SM's 228 KiB), one for the channel gate
     const int per_sm = MODE == GDR_DECAY_CHANNEL ? 1 : 2;
     const int n_tasks = NCp * p.H * p.B;
     const int grid = n_tasks < sms * per_sm ? n_tasks : sms * per_sm;
