@@ -1389,16 +1389,23 @@ bool use_fused(int B, int H, int mode) { return mode != GDR_DECAY_CHANNEL && (si
 
 // Chunks per head the fused kernel takes pre-computed from a prep kernel that runs before it on
 // all SMs. In the fused kernel the kSMs - BH prep CTAs must keep up with the BH chains: a chain
-// takes kChainPerTask times as long per chunk as a prep CTA (two pipelines) per task, so they
-// produce the last NC - c1 chunks in time if (NC - c1) * BH <= NC * (kSMs - BH) * kChainPerTask;
+// takes chain_per_task(BH) times as long per chunk as a prep CTA (two pipelines) per task, so they
+// produce the last NC - c1 chunks in time if (NC - c1) * BH <= NC * (kSMs - BH) * chain_per_task;
 // the remaining chunks are prepared beforehand with every SM. (A fixed SM count keeps the result,
 // and with it the workspace size, a host-only function of the shape.)
 constexpr int kSMs = 148;
-constexpr double kChainPerTask = 0.35;  // measured: chain about 2.3 us per chunk; 0.35 beat 0.29 and 0.32 at 64 heads
-constexpr int kHybridMinHeads = 57;     // below, the fused kernel alone is faster (measured at 48 heads)
+constexpr int kHybridMinHeads = 57;  // below, the fused kernel alone is faster (measured at 48 heads)
+// Measured at T = 4096 (64 chunks), the best of 0.32 / 0.35 / 0.38 / 0.42: 0.35 at 64 heads (c1 = 35,
+// 229.9 us; 0.38 within 1 us), 0.32 at 80 heads (c1 = 47, 265.6 vs 270.8 us at 0.35) and at 96
+// heads (c1 = 53, 303.5 vs 311.6 us): the prep CTAs slow down as they get fewer and the chains
+// more. Linear in between.
+double chain_per_task(int BH) {
+    const double t = (BH - 64) / 16.0;
+    return 0.35 - 0.03 * (t < 0.0 ? 0.0 : t > 1.0 ? 1.0 : t);
+}
 int fused_precomputed_chunks(int BH, int NC) {
     if (BH < kHybridMinHeads) return 0;
-    const double f = 1.0 - kChainPerTask * (kSMs - BH) / (double)BH;
+    const double f = 1.0 - chain_per_task(BH) * (kSMs - BH) / (double)BH;
     if (f <= 0.0) return 0;
     const int c1 = (int)(f * NC + 0.999);
     return c1 < NC ? c1 : NC;
