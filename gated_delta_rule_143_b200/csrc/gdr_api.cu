@@ -138,8 +138,8 @@ int auto_segments(int B, int T, int H, int dk, int dv, int chunk, int dtype, int
     return scan_supported(B, T, H, dk, dv, chunk, dtype, o_dtype, s) ? s : 0;
 }
 
-// Gated DeltaNet-2 runs on the tensor cores for the channel decay at the tensor-core shapes (the
-// channel gate's two passes), on the CUDA cores otherwise.
+// Gated DeltaNet-2 runs on the tensor cores for the channel decay at the tensor-core shapes (always
+// the two-pass plan), on the CUDA cores otherwise.
 bool gdn2_on_tc(int dk, int dv, int chunk, int mode, int dtype, int o_dtype) {
     return mode == GDR_DECAY_CHANNEL && chunk_tc_supported(dk, dv, chunk, dtype, o_dtype);
 }
@@ -196,7 +196,7 @@ int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g, 
     const bool use_tc = ew ? gdn2_on_tc(dk, dv, chunk, mode, dtype, o_dtype)
                            : chunk_tc_supported(dk, dv, chunk, dtype, o_dtype);
     const size_t need = n_seg != 0 ? scan_workspace_bytes(B, T, H, mode, n_seg, o_dtype)
-                                   : (use_tc ? chunk_tc_workspace_bytes(B, T, H, dk, dv, chunk, mode) : 0);
+                                   : (use_tc ? chunk_tc_workspace_bytes(B, T, H, dk, dv, chunk, mode, ew) : 0);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need))
         return fail(GDR_ERR_WORKSPACE, "workspace of %zu bytes required (got %zu at %p)", need, workspace_bytes,
                     workspace);
@@ -385,7 +385,7 @@ size_t gdr_chunk_fwd_gdn2_workspace_bytes(int B, int T, int H, int dk, int dv, i
     const int rc = chunk_shape_check(B, T, H, dk, dv, chunk, mode, dtype, o_dtype);
     memcpy(g_last_error, saved, sizeof(saved));
     if (rc != GDR_OK || !gdn2_on_tc(dk, dv, chunk, mode, dtype, o_dtype)) return 0;
-    return chunk_tc_workspace_bytes(B, T, H, dk, dv, chunk, mode);
+    return chunk_tc_workspace_bytes(B, T, H, dk, dv, chunk, mode, true);
 }
 
 int gdr_chunk_fwd_gdn2(const void* q, const void* k, const void* v, const float* g, const float* erase,

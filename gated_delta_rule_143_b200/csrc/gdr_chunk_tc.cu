@@ -1222,6 +1222,7 @@ static_assert(kPrepPipeBytes % 1024 == 0, "pipeline shared memory must keep 1024
 static_assert(2 * (kPrepBytesScalar + 1024 + 1024 + 64) <= 233472, "two prep pipelines per SM");
 constexpr uint32_t kFusedSmem = (2 * kPrepPipeBytes > kStateSmem - 1024 ? 2 * kPrepPipeBytes : kStateSmem - 1024) + 1024;
 constexpr int kFusedMaxHeads = 100;  // B * H above this runs the two-pass path (too few SMs left for prep)
+static_assert(kPrepBytesChannel <= kFusedSmem - 1024, "the channel gate's prep pipeline fits a fused CTA");
 
 struct RingArgs {
     uint8_t* ring;     // [BH][depth] hand-off blocks
@@ -1239,19 +1240,21 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
     __shared__ uint64_t pbars[2][4];
     __shared__ volatile int go[2];
     __shared__ volatile int claimed[2];
+    // the channel gate's pipeline takes most of the shared memory: one per CTA (warps 0-7)
+    constexpr int kPipes = MODE == GDR_DECAY_CHANNEL ? 1 : 2;
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int pipe = warp >> 3;  // 0, 1; warps 16-17 have pipe 2 and idle
+    const int pipe = warp >> 3;  // pipelines 0 .. kPipes - 1; the other warps idle
     const int lt = tid & 255;
     if (tid == 0) {
         for (int i = 0; i < 2; ++i)
             for (int k = 0; k < 4; ++k) mbar_init(&pbars[i][k], 1);
         fence_mbar_init();
     }
-    if (pipe < 2) prep_init<MODE>(PrepSmem{sm + pipe * kPrepPipeBytes, nullptr, 0, 0}, lt);
+    if (pipe < kPipes) prep_init<MODE>(PrepSmem{sm + pipe * kPrepPipeBytes, nullptr, 0, 0}, lt);
     __syncthreads();
     // a head's chain consumes a chunk about every 2 us and a pipeline prepares one in about 11 us:
-    // 3 CTAs (6 pipelines) per head keep the rings full; more would only wait on ring slots
-    if (pipe >= 2 || (int)blockIdx.x - R.BH >= 3 * R.BH + 4) return;
+    // 6 pipelines per head keep the rings full; more would only wait on ring slots
+    if (pipe >= kPipes || (int)blockIdx.x - R.BH >= (6 / kPipes) * R.BH + 4) return;
     const PrepSmem ps{sm + pipe * kPrepPipeBytes, pbars[pipe], tbase + (uint32_t)pipe * kPrepTmemCols, 1 + 2 * pipe};
     const int n_tasks = P.NC * R.BH;
     uint32_t it = 0, n_copies = 0;  // tasks so far; channel-gate tile copies so far (mbarrier parities)
@@ -1383,9 +1386,10 @@ cudaError_t launch_state(const ChunkProblem& p, const CUtensorMap& mo, int NC, c
     return cudaGetLastError();
 }
 
-// The fused kernel serves DeltaNet and the scalar gate for up to kFusedMaxHeads heads; the channel
-// gate (two of its prep pipelines do not fit in shared memory) and larger B * H use two passes.
-bool use_fused(int B, int H, int mode) { return mode != GDR_DECAY_CHANNEL && (size_t)B * H <= kFusedMaxHeads; }
+// The fused kernel serves up to kFusedMaxHeads heads (the channel gate with one prep pipeline per
+// CTA: two do not fit in shared memory); larger B * H, and Gated DeltaNet-2 (ew: erase / write
+// gates, whose prep runs only in the standalone kernel), use two passes.
+bool use_fused(int B, int H, bool ew) { return !ew && (size_t)B * H <= kFusedMaxHeads; }
 
 // Chunks per head the fused kernel takes pre-computed from a prep kernel that runs before it on
 // all SMs. In the fused kernel the kSMs - BH prep CTAs must keep up with the BH chains: a chain
@@ -1403,24 +1407,32 @@ double chain_per_task(int BH) {
     const double t = (BH - 64) / 16.0;
     return 0.35 - 0.03 * (t < 0.0 ? 0.0 : t > 1.0 ? 1.0 : t);
 }
-int fused_precomputed_chunks(int BH, int NC) {
-    if (BH < kHybridMinHeads) return 0;
-    const double f = 1.0 - chain_per_task(BH) * (kSMs - BH) / (double)BH;
+// The channel gate: one prep pipeline per CTA, each task slower (more exponentials, and 112 registers
+// in the fused kernel against 240 alone); the chain about 2 us per chunk. Measured at T = 8192, the
+// best of 0.13 / 0.16 / 0.19 / 0.22 at 32, 64 and 96 heads: 0.13 (64 heads: c1 = 107 of 128, 813 us,
+// against 835 at 0.16 and 902 for two passes; the fused kernel then at about the chain's own time).
+constexpr double kChainPerTaskChannel = 0.13;
+int fused_precomputed_chunks(int BH, int NC, int mode) {
+    const bool ch = mode == GDR_DECAY_CHANNEL;
+    if (!ch && BH < kHybridMinHeads) return 0;
+    const double f = 1.0 - (ch ? kChainPerTaskChannel : chain_per_task(BH)) * (kSMs - BH) / (double)BH;
     if (f <= 0.0) return 0;
     const int c1 = (int)(f * NC + 0.999);
     return c1 < NC ? c1 : NC;
 }
-size_t pre_bytes(int BH, int NC) { return (size_t)BH * fused_precomputed_chunks(BH, NC) * kHandoffStride; }
+size_t pre_bytes(int BH, int NC, int mode) {
+    return (size_t)BH * fused_precomputed_chunks(BH, NC, mode) * kHandoffStride;
+}
 // Ring slots per head. With chunks pre-computed, the chains spend their first c1 chunks on those
 // while the fused kernel's prep CTAs run ahead: a slot for every later chunk keeps them from
 // stalling on a full ring in that time (the blocks then mostly live in DRAM, not L2).
-int ring_depth(int BH, int NC) {
-    const int c1 = fused_precomputed_chunks(BH, NC);
+int ring_depth(int BH, int NC, int mode) {
+    const int c1 = fused_precomputed_chunks(BH, NC, mode);
     return c1 > 0 ? NC - c1 : kRing;
 }
-size_t ring_bytes(int BH, int NC) { return (size_t)BH * ring_depth(BH, NC) * kHandoffStride; }
-size_t flag_bytes(int BH, int NC) {
-    return ((size_t)(BH * (ring_depth(BH, NC) + 1) + 1) * sizeof(int) + 255) & ~size_t(255);
+size_t ring_bytes(int BH, int NC, int mode) { return (size_t)BH * ring_depth(BH, NC, mode) * kHandoffStride; }
+size_t flag_bytes(int BH, int NC, int mode) {
+    return ((size_t)(BH * (ring_depth(BH, NC, mode) + 1) + 1) * sizeof(int) + 255) & ~size_t(255);
 }
 
 template <int MODE, typename Tout, bool PRO>
@@ -1440,11 +1452,11 @@ cudaError_t launch_fused(const ChunkProblem& p, const CUtensorMap& mq, const CUt
     if (!coop || per_sm < 1 || grid - BH < 8) return cudaErrorCooperativeLaunchTooLarge;
     // workspace: [pre-computed blocks, BH x c1][ring, BH x depth][flags]
     uint8_t* ws = static_cast<uint8_t*>(p.workspace);
-    const int c1 = fused_precomputed_chunks(BH, NC), depth = ring_depth(BH, NC);
-    uint8_t* ring = ws + pre_bytes(BH, NC);
-    int* flags = reinterpret_cast<int*>(ring + ring_bytes(BH, NC));
+    const int c1 = fused_precomputed_chunks(BH, NC, MODE), depth = ring_depth(BH, NC, MODE);
+    uint8_t* ring = ws + pre_bytes(BH, NC, MODE);
+    int* flags = reinterpret_cast<int*>(ring + ring_bytes(BH, NC, MODE));
     RingArgs R{ring, flags, flags + (size_t)BH * depth, flags + (size_t)BH * (depth + 1), ws, BH, c1, depth};
-    if ((err = cudaMemsetAsync(flags, 0, flag_bytes(BH, NC), stream)) != cudaSuccess) return err;
+    if ((err = cudaMemsetAsync(flags, 0, flag_bytes(BH, NC, MODE), stream)) != cudaSuccess) return err;
     if (c1 > 0 && (err = launch_prep<MODE, PRO>(p, mq, mk, mv, NC, c1, ws, stream)) != cudaSuccess) return err;
     PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status, p.prologue, p.gate_scale, p.erase, p.write};
     StateArgs A{p.S0, p.S_T, p.T, p.H, NC, p.scale, p.status, p.B * p.H, nullptr};
@@ -1463,6 +1475,9 @@ cudaError_t launch_fused_mode(const ChunkProblem& p, const CUtensorMap& mq, cons
     if (p.mode == GDR_DECAY_NONE)
         return bf ? launch_fused<GDR_DECAY_NONE, __nv_bfloat16, PRO>(p, mq, mk, mv, mo, NC, stream)
                   : launch_fused<GDR_DECAY_NONE, float, PRO>(p, mq, mk, mv, mo, NC, stream);
+    if (p.mode == GDR_DECAY_CHANNEL)
+        return bf ? launch_fused<GDR_DECAY_CHANNEL, __nv_bfloat16, PRO>(p, mq, mk, mv, mo, NC, stream)
+                  : launch_fused<GDR_DECAY_CHANNEL, float, PRO>(p, mq, mk, mv, mo, NC, stream);
     return bf ? launch_fused<GDR_DECAY_SCALAR, __nv_bfloat16, PRO>(p, mq, mk, mv, mo, NC, stream)
               : launch_fused<GDR_DECAY_SCALAR, float, PRO>(p, mq, mk, mv, mo, NC, stream);
 }
@@ -1484,23 +1499,23 @@ bool chunk_tc_supported(int dk, int dv, int chunk, int dtype, int o_dtype) {
     return dtype == GDR_BF16 && (o_dtype == GDR_F32 || o_dtype == GDR_BF16) && dk == kD && dv == kD && chunk == kC;
 }
 
-size_t chunk_tc_workspace_bytes(int B, int T, int H, int, int, int, int mode) {
-    const int NC = (T + kC - 1) / kC;
-    if (use_fused(B, H, mode)) return pre_bytes(B * H, NC) + ring_bytes(B * H, NC) + flag_bytes(B * H, NC);
-    return (size_t)B * H * NC * kHandoffStride;
+size_t chunk_tc_workspace_bytes(int B, int T, int H, int, int, int, int mode, bool ew) {
+    const int NC = (T + kC - 1) / kC, BH = B * H;
+    if (use_fused(B, H, ew)) return pre_bytes(BH, NC, mode) + ring_bytes(BH, NC, mode) + flag_bytes(BH, NC, mode);
+    return (size_t)BH * NC * kHandoffStride;
 }
 
 int chunk_tc_plan(int B, int T, int H, int, int, int, int mode, int* precomputed_chunks) {
     const int NC = (T + kC - 1) / kC;
-    const int c1 = use_fused(B, H, mode) ? fused_precomputed_chunks(B * H, NC) : 0;
+    const int c1 = use_fused(B, H, false) ? fused_precomputed_chunks(B * H, NC, mode) : 0;
     if (precomputed_chunks != nullptr) *precomputed_chunks = c1;
-    if (!use_fused(B, H, mode)) return GDR_PLAN_TWO_PASS;
+    if (!use_fused(B, H, false)) return GDR_PLAN_TWO_PASS;
     return c1 > 0 ? GDR_PLAN_PREP_FUSED : GDR_PLAN_FUSED;
 }
 
 int chunk_tc_launches(int B, int T, int H, int, int, int, int mode) {
-    if (!use_fused(B, H, mode)) return 2;
-    return fused_precomputed_chunks(B * H, (T + kC - 1) / kC) > 0 ? 2 : 1;
+    if (!use_fused(B, H, false)) return 2;
+    return fused_precomputed_chunks(B * H, (T + kC - 1) / kC, mode) > 0 ? 2 : 1;
 }
 
 cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream) {
@@ -1515,7 +1530,7 @@ cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream) {
     else
         err = make_map(&mo, p.o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.B, p.T, p.H, 32);
     if (err != cudaSuccess) return err;
-    if (use_fused(p.B, p.H, p.mode))
+    if (use_fused(p.B, p.H, p.erase != nullptr))
         return p.prologue ? launch_fused_mode<true>(p, mq, mk, mv, mo, NC, stream)
                           : launch_fused_mode<false>(p, mq, mk, mv, mo, NC, stream);
     uint8_t* ws = static_cast<uint8_t*>(p.workspace);

@@ -114,7 +114,8 @@ cudaError_t launch_chunk_simt(const ChunkProblem& p, cudaStream_t stream);
 
 // Tensor-core (tcgen05) chunked forward: bf16, d_k = d_v = 128, chunk = 64.
 bool chunk_tc_supported(int dk, int dv, int chunk, int dtype, int o_dtype);
-size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int mode);
+// ew: Gated DeltaNet-2 (erase / write gates: the two-pass plan)
+size_t chunk_tc_workspace_bytes(int B, int T, int H, int dk, int dv, int chunk, int mode, bool ew = false);
 cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream);
 int chunk_tc_launches(int B, int T, int H, int dk, int dv, int chunk, int mode);
 int chunk_tc_plan(int B, int T, int H, int dk, int dv, int chunk, int mode, int* precomputed_chunks);

@@ -112,7 +112,10 @@ def test_plan_query_is_host_only():
     plan, c1 = gdr.chunk_fwd_plan(8, 4096, 8, 128, 128, 64, "scalar", bf)
     assert plan == "prep_fused" and 0 < c1 < 64
     assert gdr.chunk_fwd_plan(13, 4096, 8, 128, 128, 64, "scalar", bf) == ("two_pass", 0)
-    assert gdr.chunk_fwd_plan(1, 4096, 8, 128, 128, 64, "channel", bf) == ("two_pass", 0)
+    assert gdr.chunk_fwd_plan(1, 4096, 8, 128, 128, 64, "channel", bf) == ("fused", 0)
+    plan_ch, c1_ch = gdr.chunk_fwd_plan(4, 8192, 16, 128, 128, 64, "channel", bf)
+    assert plan_ch == "prep_fused" and 64 < c1_ch < 128
+    assert gdr.chunk_fwd_plan(13, 4096, 8, 128, 128, 64, "channel", bf) == ("two_pass", 0)
     assert gdr.chunk_fwd_plan(1, 100, 2, 64, 64, 64, "scalar", torch.float32) == ("cuda_core", 0)
     # few heads, long sequences: the segment scan with 4 segments (4 launches)
     assert gdr.chunk_fwd_plan(1, 65536, 16, 128, 128, 64, "scalar", bf) == ("scan", 4)
@@ -141,6 +144,14 @@ def test_plan_query_is_host_only():
     assert gdr.workspace_bytes(8, 4096, 8, 128, 128, 64, "scalar", bf) == 64 * 64 * block + flags(64, 64 - c1)
     # a short sequence keeps eight slots even when it has fewer chunks
     assert gdr.workspace_bytes(1, 100, 8, 128, 128, 64, "scalar", bf) == 8 * 8 * block + flags(8, 8)
+    # the channel gate: the same layouts; Gated DeltaNet-2 (erase / write gates) always two passes, one
+    # block per chunk of every head
+    assert gdr.workspace_bytes(1, 4096, 8, 128, 128, 64, "channel", bf) == 8 * 8 * block + flags(8, 8)
+    _, c1c = gdr.chunk_fwd_plan(4, 8192, 16, 128, 128, 64, "channel", bf)
+    assert gdr.workspace_bytes(4, 8192, 16, 128, 128, 64, "channel", bf) == 64 * 128 * block + flags(64, 128 - c1c)
+    L = _lib.lib()
+    for B, H in ((1, 8), (4, 16)):
+        assert L.gdr_chunk_fwd_gdn2_workspace_bytes(B, 8192, H, 128, 128, 64, 2, 1, 1) == B * H * 128 * block
 
 
 def test_host_entry_point_validates_on_host():

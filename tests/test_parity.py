@@ -76,6 +76,28 @@ def test_chunk_tensor_core_paths(mode, B, H, T, plan):
     check_chunk(x, mode, "bf16", label=f"{mode}/B{B}/H{H}/T{T}/{plan}")
 
 
+@pytest.mark.parametrize("B,H,T,plan", [
+    (1, 1, 5000, "fused"),        # one head, 10 prep CTAs, 79 chunks through the 8-slot ring
+    (1, 16, 64, "fused"),         # 16 heads, one chunk
+    (1, 8, 1000, "fused"),        # 8 heads, ragged tail
+    (2, 16, 700, "prep_fused"),   # 32 heads: 6 of 11 chunks prepared before the fused kernel
+    (4, 16, 1000, "prep_fused"),  # 64 heads: 14 of 16 prepared before, 2 ring slots
+    (13, 8, 130, "two_pass"),     # 104 heads
+])
+def test_chunk_tensor_core_paths_channel_gate(B, H, T, plan):
+    """The channel gate's plans (one prep pipeline per fused CTA), with a within-chunk log2-decay
+    spread of about 30 on a quarter of the channels (the exact CUDA-core terms) and alpha = 0 on
+    four more, against the oracle."""
+    got, c1 = gdr.chunk_fwd_plan(B, T, H, 128, 128, 64, "channel", torch.bfloat16)
+    assert got == plan and (c1 > 0) == (plan == "prep_fused")
+    x = make_chunk_inputs(B, T, H, 128, 128, "channel", "bf16", 4500 + B * 100 + H + T, s0_std=0.05)
+    g = x["g"].clone()
+    g[..., 96:128] = _g_for_spread(30.0)
+    g[..., 40:44] = -1e4
+    x["g"] = g
+    check_chunk(x, "channel", "bf16", label=f"channel/B{B}/H{H}/T{T}/{plan}")
+
+
 @pytest.mark.parametrize("mode", MODES)
 def test_chunk_unequal_head_dims(mode):
     x = make_chunk_inputs(1, 130, 2, 128, 64, mode, "bf16", 77, s0_std=0.05)
@@ -191,7 +213,7 @@ def test_channel_gate_every_channel_strong(gval):
 
 def test_channel_gate_strong_decays_full_workload_shape():
     """The channel-gate workload's shape at a quarter of its length (B=4, H=16, T=2048, d=128) with
-    strong decays on a quarter of the channels: the two-pass plan at full width against the oracle."""
+    strong decays on a quarter of the channels: the prep + fused plan at full width against the oracle."""
     x = make_chunk_inputs(4, 2048, 16, 128, 128, "channel", "bf16", 203)
     g = x["g"].clone()
     g[..., 96:128] = _g_for_spread(30.0)

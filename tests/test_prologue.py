@@ -49,8 +49,8 @@ def run_and_check(x, mode, dtype, flags, label="", out_dtype=torch.float32):
 
 @pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("dtype,d,T,B,H,plan", [
-    ("bf16", 128, 200, 2, 3, None),     # tensor cores: fused (channel: two passes)
-    ("bf16", 128, 130, 8, 8, None),     # tensor cores: prep + fused (channel: two passes)
+    ("bf16", 128, 200, 2, 3, None),     # tensor cores: fused
+    ("bf16", 128, 130, 8, 8, None),     # tensor cores: prep + fused (channel: fused)
     ("bf16", 128, 70, 13, 8, "two_pass"),
     ("f32", 64, 200, 2, 3, "cuda_core"),   # token recurrence, ragged last block
     ("f32", 64, 300, 1, 2, "cuda_core"),   # CUDA-core chunk form, ragged last chunk
