@@ -317,8 +317,8 @@ typedef enum {
  * multiple of 64 s (4 segments for 16 heads, 16 for 1-4 heads); otherwise B * H <= 56 heads run
  * fused (the chains are the bound), 57-100 heads
  * prepare the first chunks on every SM so that the fused kernel's remaining prep CTAs keep up with
- * the chains, more than 100 heads or the channel gate run two passes. gdr_chunk_fwd_noalloc never
- * uses the segment scan. */
+ * the chains (the channel gate at any head count where they would not), more than 100 heads run two
+ * passes (as Gated DeltaNet-2 always does). gdr_chunk_fwd_noalloc never uses the segment scan. */
 int gdr_chunk_fwd_plan(int B, int T, int H, int d_k, int d_v, int chunk, int mode, int dtype,
                        int o_dtype, int* precomputed_chunks);
 
