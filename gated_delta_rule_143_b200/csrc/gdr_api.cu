@@ -138,8 +138,8 @@ int auto_segments(int B, int T, int H, int dk, int dv, int chunk, int dtype, int
     return scan_supported(B, T, H, dk, dv, chunk, dtype, o_dtype, s) ? s : 0;
 }
 
-// Gated DeltaNet-2 runs on the tensor cores for the channel decay at the tensor-core shapes (always
-// the two-pass plan), on the CUDA cores otherwise.
+// Gated DeltaNet-2 runs on the tensor cores for the channel decay at the tensor-core shapes (the
+// channel gate's plans), on the CUDA cores otherwise.
 bool gdn2_on_tc(int dk, int dv, int chunk, int mode, int dtype, int o_dtype) {
     return mode == GDR_DECAY_CHANNEL && chunk_tc_supported(dk, dv, chunk, dtype, o_dtype);
 }

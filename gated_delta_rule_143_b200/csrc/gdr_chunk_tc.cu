@@ -1234,7 +1234,7 @@ struct RingArgs {
     int depth;         // ring slots per head: kRing, or every chunk from c1 on when c1 > 0
 };
 
-template <int MODE, bool PRO>
+template <int MODE, bool PRO, bool EW>
 __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv, const PrepArgs& P,
                           const RingArgs& R, uint8_t* sm, uint32_t tbase, volatile int* abort) {
     __shared__ uint64_t pbars[2][4];
@@ -1275,7 +1275,7 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
         named_bar(ps.bar_id, kPrepThreads);
         if (!go[pipe]) break;
         uint8_t* out = R.ring + ((size_t)bh * R.depth + slot) * kHandoffStride;
-        prep_chunk<MODE, PRO>(P, mq, mk, mv, ps, bh / P.H, bh % P.H, c, out, it, lt, n_copies, 0, 0, -1, false);
+        prep_chunk<MODE, PRO, EW>(P, mq, mk, mv, ps, bh / P.H, bh % P.H, c, out, it, lt, n_copies, 0, 0, -1, false);
         if (lt == 0) {  // every write of the block (generic stores before prep_chunk's last barrier, bulk stores)
             bulk_wait<0>();
             fence_proxy_async_global();
@@ -1285,7 +1285,7 @@ __device__ void prep_role(const CUtensorMap* mq, const CUtensorMap* mk, const CU
     }
 }
 
-template <int MODE, typename Tout, bool PRO>
+template <int MODE, typename Tout, bool PRO, bool EW>
 __global__ void __launch_bounds__(kStateThreads, 1)
 chunk_fused_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                    const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mo, PrepArgs P,
@@ -1310,7 +1310,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
                              R.c1, R.depth};
         state_body<Tout>(&mo, A, bh, src, sm, tmem_base, &abort_flag);
     } else {
-        prep_role<MODE, PRO>(&mq, &mk, &mv, P, R, sm, tmem_base, &abort_flag);
+        prep_role<MODE, PRO, EW>(&mq, &mk, &mv, P, R, sm, tmem_base, &abort_flag);
     }
     tc_fence_before();
     __syncthreads();
@@ -1386,10 +1386,9 @@ cudaError_t launch_state(const ChunkProblem& p, const CUtensorMap& mo, int NC, c
     return cudaGetLastError();
 }
 
-// The fused kernel serves up to kFusedMaxHeads heads (the channel gate with one prep pipeline per
-// CTA: two do not fit in shared memory); larger B * H, and Gated DeltaNet-2 (ew: erase / write
-// gates, whose prep runs only in the standalone kernel), use two passes.
-bool use_fused(int B, int H, bool ew) { return !ew && (size_t)B * H <= kFusedMaxHeads; }
+// The fused kernel serves up to kFusedMaxHeads heads (the channel gate, and Gated DeltaNet-2 with it,
+// with one prep pipeline per CTA: two do not fit in shared memory); larger B * H use two passes.
+bool use_fused(int B, int H) { return (size_t)B * H <= kFusedMaxHeads; }
 
 // Chunks per head the fused kernel takes pre-computed from a prep kernel that runs before it on
 // all SMs. In the fused kernel the kSMs - BH prep CTAs must keep up with the BH chains: a chain
@@ -1412,33 +1411,40 @@ double chain_per_task(int BH) {
 // best of 0.13 / 0.16 / 0.19 / 0.22 at 32, 64 and 96 heads: 0.13 (64 heads: c1 = 107 of 128, 813 us,
 // against 835 at 0.16 and 902 for two passes; the fused kernel then at about the chain's own time).
 constexpr double kChainPerTaskChannel = 0.13;
-int fused_precomputed_chunks(int BH, int NC, int mode) {
+// Gated DeltaNet-2 (ew): the channel gate's prep with the erase / write gates, about 1.6 times as long
+// per task. Measured at the KDA workload's shape (64 heads, 128 chunks): 0.08 (c1 = 115) 1193 us,
+// against 1224 us at 0.06, 1227 us at 0.10 and 1291 us for two passes.
+constexpr double kChainPerTaskGdn2 = 0.08;
+int fused_precomputed_chunks(int BH, int NC, int mode, bool ew = false) {
     const bool ch = mode == GDR_DECAY_CHANNEL;
     if (!ch && BH < kHybridMinHeads) return 0;
-    const double f = 1.0 - (ch ? kChainPerTaskChannel : chain_per_task(BH)) * (kSMs - BH) / (double)BH;
+    const double k = ch ? (ew ? kChainPerTaskGdn2 : kChainPerTaskChannel) : chain_per_task(BH);
+    const double f = 1.0 - k * (kSMs - BH) / (double)BH;
     if (f <= 0.0) return 0;
     const int c1 = (int)(f * NC + 0.999);
     return c1 < NC ? c1 : NC;
 }
-size_t pre_bytes(int BH, int NC, int mode) {
-    return (size_t)BH * fused_precomputed_chunks(BH, NC, mode) * kHandoffStride;
+size_t pre_bytes(int BH, int NC, int mode, bool ew) {
+    return (size_t)BH * fused_precomputed_chunks(BH, NC, mode, ew) * kHandoffStride;
 }
 // Ring slots per head. With chunks pre-computed, the chains spend their first c1 chunks on those
 // while the fused kernel's prep CTAs run ahead: a slot for every later chunk keeps them from
 // stalling on a full ring in that time (the blocks then mostly live in DRAM, not L2).
-int ring_depth(int BH, int NC, int mode) {
-    const int c1 = fused_precomputed_chunks(BH, NC, mode);
+int ring_depth(int BH, int NC, int mode, bool ew) {
+    const int c1 = fused_precomputed_chunks(BH, NC, mode, ew);
     return c1 > 0 ? NC - c1 : kRing;
 }
-size_t ring_bytes(int BH, int NC, int mode) { return (size_t)BH * ring_depth(BH, NC, mode) * kHandoffStride; }
-size_t flag_bytes(int BH, int NC, int mode) {
-    return ((size_t)(BH * (ring_depth(BH, NC, mode) + 1) + 1) * sizeof(int) + 255) & ~size_t(255);
+size_t ring_bytes(int BH, int NC, int mode, bool ew) {
+    return (size_t)BH * ring_depth(BH, NC, mode, ew) * kHandoffStride;
+}
+size_t flag_bytes(int BH, int NC, int mode, bool ew) {
+    return ((size_t)(BH * (ring_depth(BH, NC, mode, ew) + 1) + 1) * sizeof(int) + 255) & ~size_t(255);
 }
 
-template <int MODE, typename Tout, bool PRO>
+template <int MODE, typename Tout, bool PRO, bool EW = false>
 cudaError_t launch_fused(const ChunkProblem& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const CUtensorMap& mo, int NC, cudaStream_t stream) {
-    auto kern = chunk_fused_kernel<MODE, Tout, PRO>;
+    auto kern = chunk_fused_kernel<MODE, Tout, PRO, EW>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFusedSmem);
     if (err != cudaSuccess) return err;
     int dev = 0, sms = 0, coop = 0, per_sm = 0;
@@ -1452,12 +1458,12 @@ cudaError_t launch_fused(const ChunkProblem& p, const CUtensorMap& mq, const CUt
     if (!coop || per_sm < 1 || grid - BH < 8) return cudaErrorCooperativeLaunchTooLarge;
     // workspace: [pre-computed blocks, BH x c1][ring, BH x depth][flags]
     uint8_t* ws = static_cast<uint8_t*>(p.workspace);
-    const int c1 = fused_precomputed_chunks(BH, NC, MODE), depth = ring_depth(BH, NC, MODE);
-    uint8_t* ring = ws + pre_bytes(BH, NC, MODE);
-    int* flags = reinterpret_cast<int*>(ring + ring_bytes(BH, NC, MODE));
+    const int c1 = fused_precomputed_chunks(BH, NC, MODE, EW), depth = ring_depth(BH, NC, MODE, EW);
+    uint8_t* ring = ws + pre_bytes(BH, NC, MODE, EW);
+    int* flags = reinterpret_cast<int*>(ring + ring_bytes(BH, NC, MODE, EW));
     RingArgs R{ring, flags, flags + (size_t)BH * depth, flags + (size_t)BH * (depth + 1), ws, BH, c1, depth};
-    if ((err = cudaMemsetAsync(flags, 0, flag_bytes(BH, NC, MODE), stream)) != cudaSuccess) return err;
-    if (c1 > 0 && (err = launch_prep<MODE, PRO>(p, mq, mk, mv, NC, c1, ws, stream)) != cudaSuccess) return err;
+    if ((err = cudaMemsetAsync(flags, 0, flag_bytes(BH, NC, MODE, EW), stream)) != cudaSuccess) return err;
+    if (c1 > 0 && (err = launch_prep<MODE, PRO, EW>(p, mq, mk, mv, NC, c1, ws, stream)) != cudaSuccess) return err;
     PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status, p.prologue, p.gate_scale, p.erase, p.write};
     StateArgs A{p.S0, p.S_T, p.T, p.H, NC, p.scale, p.status, p.B * p.H, nullptr};
     CUtensorMap aq = mq, ak = mk, av = mv, ao = mo;
@@ -1501,20 +1507,21 @@ bool chunk_tc_supported(int dk, int dv, int chunk, int dtype, int o_dtype) {
 
 size_t chunk_tc_workspace_bytes(int B, int T, int H, int, int, int, int mode, bool ew) {
     const int NC = (T + kC - 1) / kC, BH = B * H;
-    if (use_fused(B, H, ew)) return pre_bytes(BH, NC, mode) + ring_bytes(BH, NC, mode) + flag_bytes(BH, NC, mode);
+    if (use_fused(B, H))
+        return pre_bytes(BH, NC, mode, ew) + ring_bytes(BH, NC, mode, ew) + flag_bytes(BH, NC, mode, ew);
     return (size_t)BH * NC * kHandoffStride;
 }
 
 int chunk_tc_plan(int B, int T, int H, int, int, int, int mode, int* precomputed_chunks) {
     const int NC = (T + kC - 1) / kC;
-    const int c1 = use_fused(B, H, false) ? fused_precomputed_chunks(B * H, NC, mode) : 0;
+    const int c1 = use_fused(B, H) ? fused_precomputed_chunks(B * H, NC, mode) : 0;
     if (precomputed_chunks != nullptr) *precomputed_chunks = c1;
-    if (!use_fused(B, H, false)) return GDR_PLAN_TWO_PASS;
+    if (!use_fused(B, H)) return GDR_PLAN_TWO_PASS;
     return c1 > 0 ? GDR_PLAN_PREP_FUSED : GDR_PLAN_FUSED;
 }
 
 int chunk_tc_launches(int B, int T, int H, int, int, int, int mode) {
-    if (!use_fused(B, H, false)) return 2;
+    if (!use_fused(B, H)) return 2;
     return fused_precomputed_chunks(B * H, (T + kC - 1) / kC, mode) > 0 ? 2 : 1;
 }
 
@@ -1530,12 +1537,19 @@ cudaError_t launch_chunk_tc(const ChunkProblem& p, cudaStream_t stream) {
     else
         err = make_map(&mo, p.o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.B, p.T, p.H, 32);
     if (err != cudaSuccess) return err;
-    if (use_fused(p.B, p.H, p.erase != nullptr))
+    // Gated DeltaNet-2: the channel gate's prep with the erase / write gates
+    const bool ew = p.erase != nullptr;
+    if (ew && (p.mode != GDR_DECAY_CHANNEL || p.prologue)) return cudaErrorInvalidValue;
+    if (use_fused(p.B, p.H)) {
+        if (ew)
+            return p.o_dtype == GDR_BF16
+                       ? launch_fused<GDR_DECAY_CHANNEL, __nv_bfloat16, false, true>(p, mq, mk, mv, mo, NC, stream)
+                       : launch_fused<GDR_DECAY_CHANNEL, float, false, true>(p, mq, mk, mv, mo, NC, stream);
         return p.prologue ? launch_fused_mode<true>(p, mq, mk, mv, mo, NC, stream)
                           : launch_fused_mode<false>(p, mq, mk, mv, mo, NC, stream);
+    }
     uint8_t* ws = static_cast<uint8_t*>(p.workspace);
-    if (p.erase != nullptr) {  // Gated DeltaNet-2: the channel gate's prep with the erase / write gates
-        if (p.mode != GDR_DECAY_CHANNEL || p.prologue) return cudaErrorInvalidValue;
+    if (ew) {
         err = launch_prep<GDR_DECAY_CHANNEL, false, true>(p, mq, mk, mv, NC, NC, ws, stream);
     } else {
         err = p.prologue ? launch_prep_mode<true>(p, mq, mk, mv, NC, ws, stream)

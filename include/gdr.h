@@ -240,7 +240,7 @@ size_t gdr_chunk_fwd_scan_workspace_bytes(int B, int T, int H, int d_k, int d_v,
  * Gram matrix and in W, and w (.) V that of diag(beta) V in U:
  * A_ri = sum_c E_rc k_ic exp(Gamma_rc - Gamma_ic) (i < r), W = T (E * gamma), U = T (w (.) V).
  * With the channel decay at the tensor-core shapes (bf16, d_k = d_v = 128, chunk 64) it runs on the
- * channel gate's two tensor-core passes and needs gdr_chunk_fwd_gdn2_workspace_bytes(...) of
+ * channel gate's tensor-core plans and needs gdr_chunk_fwd_gdn2_workspace_bytes(...) of
  * workspace; otherwise on the fp32 CUDA-core kernels with no workspace (d_k, d_v in {32, 64, 128},
  * chunk 64). Decode: as gdr_decode_step. Errors as gdr_chunk_fwd / gdr_decode_step.
  */
@@ -318,7 +318,7 @@ typedef enum {
  * fused (the chains are the bound), 57-100 heads
  * prepare the first chunks on every SM so that the fused kernel's remaining prep CTAs keep up with
  * the chains (the channel gate at any head count where they would not), more than 100 heads run two
- * passes (as Gated DeltaNet-2 always does). gdr_chunk_fwd_noalloc never uses the segment scan. */
+ * passes. gdr_chunk_fwd_noalloc never uses the segment scan. */
 int gdr_chunk_fwd_plan(int B, int T, int H, int d_k, int d_v, int chunk, int mode, int dtype,
                        int o_dtype, int* precomputed_chunks);
 

@@ -144,14 +144,16 @@ def test_plan_query_is_host_only():
     assert gdr.workspace_bytes(8, 4096, 8, 128, 128, 64, "scalar", bf) == 64 * 64 * block + flags(64, 64 - c1)
     # a short sequence keeps eight slots even when it has fewer chunks
     assert gdr.workspace_bytes(1, 100, 8, 128, 128, 64, "scalar", bf) == 8 * 8 * block + flags(8, 8)
-    # the channel gate: the same layouts; Gated DeltaNet-2 (erase / write gates) always two passes, one
-    # block per chunk of every head
+    # the channel gate: the same layouts; Gated DeltaNet-2 (erase / write gates) too, with its own
+    # share of pre-computed chunks; two passes (one block per chunk of every head) above 100 heads
     assert gdr.workspace_bytes(1, 4096, 8, 128, 128, 64, "channel", bf) == 8 * 8 * block + flags(8, 8)
     _, c1c = gdr.chunk_fwd_plan(4, 8192, 16, 128, 128, 64, "channel", bf)
     assert gdr.workspace_bytes(4, 8192, 16, 128, 128, 64, "channel", bf) == 64 * 128 * block + flags(64, 128 - c1c)
     L = _lib.lib()
-    for B, H in ((1, 8), (4, 16)):
-        assert L.gdr_chunk_fwd_gdn2_workspace_bytes(B, 8192, H, 128, 128, 64, 2, 1, 1) == B * H * 128 * block
+    assert L.gdr_chunk_fwd_gdn2_workspace_bytes(1, 8192, 8, 128, 128, 64, 2, 1, 1) == 8 * 8 * block + flags(8, 8)
+    ws2 = L.gdr_chunk_fwd_gdn2_workspace_bytes(4, 8192, 16, 128, 128, 64, 2, 1, 1)
+    assert any(ws2 == 64 * 128 * block + flags(64, d) for d in range(1, 128 - c1c))  # more chunks pre-computed
+    assert L.gdr_chunk_fwd_gdn2_workspace_bytes(13, 8192, 8, 128, 128, 64, 2, 1, 1) == 104 * 128 * block
 
 
 def test_host_entry_point_validates_on_host():
@@ -234,8 +236,10 @@ def test_chunk_fwd_gdn2_rejects_bad_arguments_on_host(kw, code):
 
 def test_chunk_fwd_gdn2_workspace_query():
     lib = _lib.lib()
-    # the channel decay at the tensor-core shapes runs the channel gate's two passes: one block per chunk
-    assert lib.gdr_chunk_fwd_gdn2_workspace_bytes(1, 128, 2, 128, 128, 64, 2, 1, 0) == 2 * 2 * 74752
+    # the channel decay at the tensor-core shapes runs the channel gate's plans: two heads run fused, a
+    # ring of eight blocks per head and the ring's flags
+    assert lib.gdr_chunk_fwd_gdn2_workspace_bytes(1, 128, 2, 128, 128, 64, 2, 1, 0) == \
+        2 * 8 * 74752 + ((2 * 9 + 1) * 4 + 255 & ~255)
     assert lib.gdr_chunk_fwd_gdn2_workspace_bytes(1, 128, 2, 128, 128, 64, 1, 1, 0) == 0  # scalar: CUDA cores
     assert lib.gdr_chunk_fwd_gdn2_workspace_bytes(1, 128, 2, 64, 64, 64, 2, 0, 0) == 0    # fp32: CUDA cores
     M = 1 << 24  # missing workspace on the tensor-core route: rejected on the host

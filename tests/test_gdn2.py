@@ -107,3 +107,17 @@ def test_gdn2_tensor_core_kda_workload_shape():
     es, _ = rel_err(st, s_ref)
     print(f"gdn2 tensor cores: o {eo:.3e}, S_T {es:.3e}")
     assert eo <= TOL["bf16"] and es <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("B,H,T", [(13, 8, 130), (1, 8, 700)])
+def test_gdn2_tensor_core_plans(B, H, T):
+    """Gated DeltaNet-2 on the channel gate's tensor-core plans: 104 heads (two passes) and 8 heads
+    (fused, 11 chunks through the ring, ragged tail), with S0, whole output against the oracle."""
+    x = make_chunk_inputs(B, T, H, 128, 128, "channel", "bf16", 12000 + B * H + T, s0_std=0.05)
+    gw = make_gdn2_gates(B, T, H, 128, 128, 12001 + B * H + T)
+    o, st = run_gdn2(x, gw["erase"], gw["write"], "channel")
+    o_ref, s_ref = oracle.recurrent_gdn2(x["q"], x["k"], x["v"], x["g"], gw["erase"], gw["write"], "channel",
+                                         S0=x["S0"])
+    eo, _ = rel_err(o, o_ref)
+    es, _ = rel_err(st, s_ref)
+    assert eo <= TOL["bf16"] and es <= TOL["bf16"], (eo, es)
