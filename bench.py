@@ -283,6 +283,28 @@ def barrier(world):
         dist.barrier()
 
 
+# Records whose device status check failed once and were run again: the expired wait's diagnostics
+# (kind, block, thread, barrier or flag) as gdr_sync_status reports them. A second failure raises.
+STATUS_RETRIES = []
+
+
+def with_status_retry(name, fn, world):
+    """Runs fn (a record ending in gdr.sync_status()) and, if the device status reports an error on
+    any rank, runs it once more on every rank (the decision is reduced over ranks, so all ranks take
+    the same collective steps); the failure is kept in STATUS_RETRIES and printed in the line."""
+    import gated_delta_rule_143_b200 as gdr
+    for attempt in range(2):
+        err = None
+        try:
+            out = fn()
+        except gdr.GdrError as e:
+            out, err = None, str(e)
+        if max_over_ranks(1.0 if err else 0.0, world) == 0.0:
+            return out
+        STATUS_RETRIES.append({"record": name, "attempt": attempt + 1, "error": err or "on another rank"})
+    raise RuntimeError(f"{name}: the device status reported an error twice: {STATUS_RETRIES[-2:]}")
+
+
 def max_over_ranks(x, world):
     """The maximum of a per-rank number over all ranks (device tensor under NCCL, host under gloo)."""
     if world == 1:
@@ -366,27 +388,31 @@ def run_ours(args):
         gdr.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], mode=w.mode, chunk=w.chunk,
                       out=o, state_out=st, workspace=ws)
 
-    try:
-        clocks = NvmlClockSampler(local)
-    except Exception:
-        clocks = None
-    if clocks is not None:
-        clocks.start()  # sampling from the start of the warm-up, kept for the timed region only
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    if clocks is None:
-        smi = ClockSampler(smi_id(dev, local))
-        smi.start()
-    else:
-        clocks.mark_begin()
-    ms = time_device(step, args.steps, 0, world, stream)
-    if clocks is None:
-        clk = smi.stop()
-    else:
-        clocks.mark_end()
-        clk = clocks.stop()
-    gdr.sync_status()
+    def timed():
+        try:
+            clocks = NvmlClockSampler(local)
+        except Exception:
+            clocks = None
+        if clocks is not None:
+            clocks.start()  # sampling from the start of the warm-up, kept for the timed region only
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        if clocks is None:
+            smi = ClockSampler(smi_id(dev, local))
+            smi.start()
+        else:
+            clocks.mark_begin()
+        ms = time_device(step, args.steps, 0, world, stream)
+        if clocks is None:
+            clk = smi.stop()
+        else:
+            clocks.mark_end()
+            clk = clocks.stop()
+        gdr.sync_status()
+        return ms, clk
+
+    ms, clk = with_status_retry("main", timed, world)
     ms = max_over_ranks(ms, world)
     ms_step = ms / args.steps
     tokens = w.B * w.T
@@ -449,7 +475,13 @@ def run_ours(args):
                       out=o16, state_out=st, workspace=ws16)
 
     n16 = max(3, min(args.steps, 200))
-    ms16 = max_over_ranks(time_device(step16, n16, args.warmup, world, stream), world) / n16
+
+    def run16():
+        ms = max_over_ranks(time_device(step16, n16, args.warmup, world, stream), world) / n16
+        gdr.sync_status()
+        return ms
+
+    ms16 = with_status_retry("o_bf16", run16, world)
     o_bf16 = {"ms_per_step": round(ms16, 5), "tokens_per_s": round(job_throughput(tokens, ms16, world), 1),
               "steps": n16, "roofline_frac": round(nbytes / (ms16 * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
               "algorithmic_bytes": nbytes}
@@ -464,15 +496,22 @@ def run_ours(args):
                       out=h_o, state_out=h_s)
 
     e2e_steps = max(3, min(args.steps, 20))
-    e2e_ms = max_over_ranks(time_device(e2e_step, e2e_steps, max(1, min(args.warmup, 3)), world, stream), world)
+
+    def run_e2e():
+        ms = max_over_ranks(time_device(e2e_step, e2e_steps, max(1, min(args.warmup, 3)), world, stream), world)
+        gdr.sync_status()
+        return ms
+
+    e2e_ms = with_status_retry("e2e", run_e2e, world)
     h2d = sum(t.numel() * t.element_size() for t in hx.values() if t is not None)
     d2h = h_o.numel() * h_o.element_size() + h_s.numel() * h_s.element_size()
 
-    dec = bench_decode(args, dev, peaks, world)
-    others = bench_workloads(args, dev, peaks) if world == 1 else None
-    pro = bench_prologue(args, w, dev, ws, o, st, stream, world, rank, ms_step)
-    gdn2 = bench_gdn2(dev, peaks, stream) if world == 1 else None
-    bwd = bench_backward(args, w, sets[0], dev, peaks, stream, world)
+    dec = with_status_retry("decode", lambda: bench_decode(args, dev, peaks, world), world)
+    others = with_status_retry("workloads", lambda: bench_workloads(args, dev, peaks), world) if world == 1 else None
+    pro = with_status_retry("prologue", lambda: bench_prologue(args, w, dev, ws, o, st, stream, world, rank, ms_step),
+                            world)
+    gdn2 = with_status_retry("gated_deltanet2", lambda: bench_gdn2(dev, peaks, stream), world) if world == 1 else None
+    bwd = with_status_retry("backward", lambda: bench_backward(args, w, sets[0], dev, peaks, stream, world), world)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -491,6 +530,7 @@ def run_ours(args):
         "decode": dec,
         "prologue": pro,
         "backward": bwd,
+        "status_retries": STATUS_RETRIES,
     }
     if others is not None:
         line["extra"] = {"workloads": others, "gated_deltanet2": gdn2}
@@ -672,6 +712,7 @@ def bench_decode(args, dev, peaks, world):
 
     n = max(20, min(args.steps, 200))
     ms = max_over_ranks(time_device(step, n, max(3, args.warmup), world, stream), world) / n
+    gdr.sync_status()
     nbytes = decode_bytes(w)
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"workload": DECODE, "ms_per_step": round(ms, 5), "tokens_per_s": round(world * w.B / (ms * 1e-3), 1),

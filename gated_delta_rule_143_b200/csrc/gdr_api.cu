@@ -50,10 +50,11 @@ struct ProfileScope {
     }
 };
 
-// Device status word: kernels record the first device-side error here (a bounded wait that
-// expired). A statically sized __device__ variable, so it needs no allocation; each device
-// that loads the library has its own copy. Host code reaches it through its address.
-__device__ int g_status_word = 0;
+// Device status record: kernels record the first device-side error here (a bounded wait that
+// expired, with where it happened). A statically sized __device__ array, so it needs no
+// allocation; each device that loads the library has its own copy. Host code reaches it through
+// its address.
+__device__ int g_status_word[kStatusWords] = {};
 
 constexpr int kMaxDevices = 64;
 std::mutex g_dev_mutex;
@@ -477,12 +478,17 @@ int gdr_sync_status(void* stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t err = cudaStreamSynchronize(s);
     if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "stream error: %s", cudaGetErrorString(err));
-    int h = 0;
-    err = cudaMemcpyAsync(&h, status, sizeof(int), cudaMemcpyDeviceToHost, s);
-    if (err == cudaSuccess) err = cudaMemsetAsync(status, 0, sizeof(int), s);
+    int rec[kStatusWords] = {};
+    err = cudaMemcpyAsync(rec, status, sizeof(rec), cudaMemcpyDeviceToHost, s);
+    if (err == cudaSuccess) err = cudaMemsetAsync(status, 0, sizeof(rec), s);
     if (err == cudaSuccess) err = cudaStreamSynchronize(s);
     if (err != cudaSuccess) return fail(GDR_ERR_CUDA, "reading the status word: %s", cudaGetErrorString(err));
-    if (h == GDR_ERR_TIMEOUT) return fail(GDR_ERR_TIMEOUT, "a kernel's bounded wait expired; its outputs are invalid");
+    const int h = rec[0];
+    if (h == GDR_ERR_TIMEOUT)
+        return fail(GDR_ERR_TIMEOUT,
+                    "a kernel's bounded wait expired; its outputs are invalid (wait kind %d, block %d, thread %d, "
+                    "detail 0x%08x)",
+                    rec[1], rec[2], rec[3], (unsigned)rec[4]);
     if (h == GDR_ERR_RANGE)
         return fail(GDR_ERR_RANGE, "a value left the range a kernel supports");
     if (h != 0) return fail(h, "device reported status %d", h);

@@ -85,6 +85,20 @@ __device__ __forceinline__ void report_status(int* status, int code) {
     if (status != nullptr) atomicCAS(status, 0, code);
 }
 
+// The status record: [0] the code; for the first expired wait also [1] which wait (1: mbarrier,
+// 2: mbarrier with abort, 3: global flag), [2] blockIdx.x, [3] threadIdx.x, [4] the barrier's shared
+// address and parity (addr | parity << 31) or the flag's target. gdr_sync_status reports and clears it.
+constexpr int kStatusWords = 8;
+__device__ __forceinline__ void report_timeout(int* status, int site, int detail) {
+    if (status != nullptr && atomicCAS(status, 0, kStatusTimeout) == 0) {
+        status[1] = site;
+        status[2] = (int)blockIdx.x;
+        status[3] = (int)threadIdx.x;
+        status[4] = detail;
+        __threadfence();
+    }
+}
+
 template <typename T>
 __device__ __forceinline__ float load_f32(const T* p);
 template <>

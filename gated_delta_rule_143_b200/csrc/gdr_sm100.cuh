@@ -65,7 +65,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (globaltimer_ns() - t0 > limit_ns) {
-            report_status(status, kStatusTimeout);
+            report_timeout(status, 1, (int)(smem_u32(bar) | (parity << 31)));
             return false;
         }
     }
@@ -82,7 +82,7 @@ __device__ __forceinline__ bool mbar_wait_abort(uint64_t* bar, uint32_t parity, 
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
         if (globaltimer_ns() - t0 > limit_ns) {
-            report_status(status, kStatusTimeout);
+            report_timeout(status, 2, (int)(smem_u32(bar) | (parity << 31)));
             *abort = 1;
             return false;
         }
@@ -113,7 +113,7 @@ __device__ __forceinline__ bool flag_wait_geq(const int* flag, int target, int* 
         if (ld_acquire_gpu(flag) >= target) return true;
         if (*abort) return false;
         if (globaltimer_ns() - t0 > limit_ns) {
-            report_status(status, kStatusTimeout);
+            report_timeout(status, 3, target);
             *abort = 1;
             return false;
         }

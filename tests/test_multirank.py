@@ -99,3 +99,55 @@ def test_kernel_bytes_split_the_step_bytes(plan):
         parts = bench.kernel_bytes(w, plan, c1)
         assert sum(b for _, b in parts) == bench.chunk_bytes(w)
         assert all(b > 0 for name, b in parts if not (plan == "scan" and name == "chunk_state"))
+
+
+def _retry_rank_main(rank, world, port, out_dir):
+    import datetime
+
+    import bench
+    from gated_delta_rule_143_b200._lib import GdrError
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        calls = []
+
+        def record():  # rank 0's device status fails on the first run only
+            calls.append(1)
+            bench.barrier(world)
+            if rank == 0 and len(calls) == 1:
+                raise GdrError(-6, "a kernel's bounded wait expired (wait kind 2, block 3, thread 0, detail 0x0)")
+            return 7
+
+        out = bench.with_status_retry("rec", record, world)
+        with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+            json.dump({"out": out, "calls": len(calls), "retries": bench.STATUS_RETRIES}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_status_retry_is_taken_by_every_rank(tmp_path):
+    """A record whose device status fails on one rank runs again on every rank (same collectives),
+    and the failure is kept for the bench line."""
+    world = 2
+    port = _free_port()
+    mp.start_processes(_retry_rank_main, args=(world, port, str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
+    assert [r["out"] for r in res] == [7, 7] and [r["calls"] for r in res] == [2, 2]
+    assert res[0]["retries"][0]["record"] == "rec" and "bounded wait" in res[0]["retries"][0]["error"]
+    assert res[1]["retries"][0]["error"] == "on another rank"
+
+
+def test_status_retry_gives_up_after_a_second_failure():
+    import bench
+    from gated_delta_rule_143_b200._lib import GdrError
+
+    def record():
+        raise GdrError(-6, "expired")
+
+    before = len(bench.STATUS_RETRIES)
+    with pytest.raises(RuntimeError):
+        bench.with_status_retry("rec2", record, 1)
+    assert len(bench.STATUS_RETRIES) == before + 2
+    assert bench.with_status_retry("rec3", lambda: 5, 1) == 5
