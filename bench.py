@@ -655,7 +655,7 @@ def bench_backward(args, w, x, dev, peaks, stream, world):
             "calls": n, "gpu_launches_per_call": 2, "bytes_per_call": nbytes,
             "kernels_ms": {"bwd_history": round(k_ms[0], 4), "bwd_reverse": round(k_ms[1], 4)},
             "achieved_gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
-            "note": "fp32 CUDA-core backward: state-history kernel + reverse kernel, d_v / 32 CTAs per head"}
+            "note": "fp32 CUDA-core backward: state-history kernel + reverse kernel, d_v / 8 CTAs per head"}
 
 
 def gdr_kernels_per_step(w):
