@@ -38,8 +38,6 @@ using namespace sm100;
 
 constexpr int kBwdWarps = 4;  // small CTAs: 20 % faster reverse sweep than 16 warps (more CTAs per SM)
 constexpr int kBwdThreads = kBwdWarps * 32;
-// the cross-warp reduction takes one thread per float4 group of dq | dk | dg (d_k <= 128) plus two
-static_assert(3 * 128 / 4 + 2 <= kBwdThreads, "the reduction's threads fit the CTA");
 
 __device__ __forceinline__ float bwd_warp_sum(float x) {
 #pragma unroll
@@ -267,31 +265,34 @@ bwd_reverse_kernel(BwdArgs A) {
         }
         if (lane == 0) redb[buf][warp][0] = gb;
         __syncthreads();
-        const int tid = threadIdx.x;
         const int nvec = (MODE == GDR_DECAY_CHANNEL ? 3 : 2) * DK / 4;  // float4 groups of dq | dk | dg
-        if (tid < nvec) {
-            const int which = tid / (DK / 4), c = 4 * (tid % (DK / 4));
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        // one item per float4 group, then dbeta and the scalar gate's dg, strided over the threads
+        for (int e = threadIdx.x; e < nvec + 2; e += kBwdThreads) {
+            if (e < nvec) {
+                const int which = e / (DK / 4), c = 4 * (e % (DK / 4));
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int w = 0; w < kBwdWarps; ++w) {
-                const float4 y = *reinterpret_cast<const float4*>(&red[buf][w][which][c]);
-                x.x += y.x;
-                x.y += y.y;
-                x.z += y.z;
-                x.w += y.w;
-            }
-            float4* dst = reinterpret_cast<float4*>((which == 0 ? A.dq : (which == 1 ? A.dk : A.dg)) + tok * DK + c);
-            if (whole_head) *dst = x;
-            else atomicAdd(dst, x);
-        } else if (tid == nvec || tid == nvec + 1) {
-            const int which = tid - nvec;  // 0: dbeta, 1: scalar-gate dg
-            if (which == 0 || MODE == GDR_DECAY_SCALAR) {
-                float x = 0.f;
-#pragma unroll
-                for (int w = 0; w < kBwdWarps; ++w) x += redb[buf][w][which];
-                float* dst = which == 0 ? A.dbeta + tok : A.dg + tok;
+                for (int w = 0; w < kBwdWarps; ++w) {
+                    const float4 y = *reinterpret_cast<const float4*>(&red[buf][w][which][c]);
+                    x.x += y.x;
+                    x.y += y.y;
+                    x.z += y.z;
+                    x.w += y.w;
+                }
+                float4* dst =
+                    reinterpret_cast<float4*>((which == 0 ? A.dq : (which == 1 ? A.dk : A.dg)) + tok * DK + c);
                 if (whole_head) *dst = x;
                 else atomicAdd(dst, x);
+            } else {
+                const int which = e - nvec;  // 0: dbeta, 1: scalar-gate dg
+                if (which == 0 || MODE == GDR_DECAY_SCALAR) {
+                    float x = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kBwdWarps; ++w) x += redb[buf][w][which];
+                    float* dst = which == 0 ? A.dbeta + tok : A.dg + tok;
+                    if (whole_head) *dst = x;
+                    else atomicAdd(dst, x);
+                }
             }
         }
         // every thread has read stage st (the barrier above): it takes the token kBwdStages later
