@@ -18,7 +18,8 @@
 //
 // dq, dk, dbeta and dg sum over the d_v rows (and over the key channels for the scalar gate).
 //
-// Two kernels, d_v / 8 CTAs per (b, h), 4 warps with two state rows each (the rows in registers;
+// Two kernels, 4 warps per CTA, d_v / 8 CTAs per (b, h) with two state rows a warp (the history
+// kernel: d_v / 4 CTAs, one row a warp) (the rows in registers;
 // lane l holds key channels l + 32 i), each token's inputs loaded one token ahead of their use:
 //  1. history: runs the recurrence forward and stores the state before every token in the workspace
 //     (T x d_v x d_k fp32 per head), so that the reverse sweep needs no recomputation;
@@ -86,6 +87,10 @@ constexpr int kBwdRowsPerWarp = 2;
 constexpr int kBwdRowsPerCta = kBwdWarps * kBwdRowsPerWarp;  // 8
 
 constexpr int kBwdStages = 3;  // reverse sweep: stored state rows in flight, one CTA-slice per token
+// The history kernel's warps take one row each: twice the warps (and stores) in flight of two rows a
+// warp, for a sweep that waits on memory.
+constexpr int kHistRowsPerWarp = 1;
+constexpr int kHistRowsPerCta = kBwdWarps * kHistRowsPerWarp;
 
 // The inputs of one token that a warp needs, loaded one token ahead of their use.
 template <int NL>
@@ -97,12 +102,12 @@ struct BwdToken {
 template <typename Tin, int MODE, int DK>
 __global__ void __launch_bounds__(kBwdThreads)
 bwd_history_kernel(BwdArgs A) {
-    constexpr int NL = DK / 32, R = kBwdRowsPerWarp;
+    constexpr int NL = DK / 32, R = kHistRowsPerWarp;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t bh = blockIdx.y;
     const int h = (int)(bh % A.H), b = (int)(bh / A.H);
     const int dv = A.dv_, T = A.T;
-    const int j0 = blockIdx.x * kBwdRowsPerCta + warp * R;  // this warp's first state row
+    const int j0 = blockIdx.x * kHistRowsPerCta + warp * R;  // this warp's first state row
     const Tin* k = static_cast<const Tin*>(A.k);
     const Tin* v = static_cast<const Tin*>(A.v);
     auto load = [&](int t, BwdToken<NL>& x) {
@@ -327,7 +332,7 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, int BH, size_t ntok, int mode, cu
                 cudaSuccess)
             return err;
     }
-    bwd_history_kernel<Tin, MODE, DK><<<grid, kBwdThreads, 0, stream>>>(a);
+    bwd_history_kernel<Tin, MODE, DK><<<dim3(a.dv_ / kHistRowsPerCta, BH), kBwdThreads, 0, stream>>>(a);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     profile_after_launch(stream);
     auto kern = bwd_reverse_kernel<Tin, MODE, DK>;
