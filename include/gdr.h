@@ -103,15 +103,14 @@ typedef enum {
  *             NULL when that is 0). Contents on entry do not matter; the library does not
  *             keep it after the enqueued work completes. Two calls in flight at the same time
  *             must not share one workspace.
- * Launches (tensor-core path): DeltaNet and the scalar gate with B * H <= 100 run as one
- * cooperative kernel with one CTA per SM, in which the per-chunk factor pipelines hand their
- * blocks to the per-head state passes through a ring in the workspace: eight blocks per head
- * (0.6 MB per head) up to 56 heads (but few heads with long sequences run the segment scan of
- * gdr_chunk_fwd_scan; see gdr_chunk_fwd_plan). Above 56 heads a prep kernel on every SM first writes the
- * blocks of the leading chunks of each head to the workspace, and the ring has a slot for every
- * later chunk. The workspace then holds one block (73 KB) per chunk of every head. The channel
- * gate and more heads use two kernels that exchange every block through the workspace.
- * gdr_chunk_fwd_plan reports which.
+ * Launches (tensor-core path): B * H <= 100 run as one cooperative kernel with one CTA per SM, in
+ * which the per-chunk factor pipelines hand their blocks to the per-head state passes through a
+ * ring in the workspace: eight blocks per head (0.6 MB per head) up to 56 heads, 17 for the channel
+ * gate (but few heads with long sequences run the segment scan of gdr_chunk_fwd_scan; see
+ * gdr_chunk_fwd_plan). Above that a prep kernel on every SM first writes the blocks of the leading
+ * chunks of each head to the workspace, and the ring has a slot for every later chunk. The
+ * workspace then holds one block (73 KB) per chunk of every head. More than 100 heads use two
+ * kernels that exchange every block through the workspace. gdr_chunk_fwd_plan reports which.
  */
 int gdr_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                   const float* S0, void* o, float* S_T, int B, int T, int H, int d_k, int d_v,
@@ -378,10 +377,10 @@ size_t gdr_chunk_fwd_host_staging_bytes(int B, int T, int H, int d_k, int d_v, i
  * (which may synchronise the device) is not allowed; a program that must not grow its device
  * footprint after start-up. This entry point takes the same arguments as gdr_chunk_fwd minus the
  * workspace and uses a fixed scratch area compiled into the library instead
- * (GDR_NOALLOC_SCRATCH_BYTES). DeltaNet and the scalar gate with B * H <= 56 need a ring of eight
- * hand-off blocks per head, which fits at any T. Larger problems need one block per chunk of every
- * head and are accepted while the total fits (see gdr_chunk_fwd_workspace_bytes). It allocates
- * nothing on any call.
+ * (GDR_NOALLOC_SCRATCH_BYTES). DeltaNet and the scalar gate with B * H <= 56 (the channel gate:
+ * <= 17) need a ring of eight hand-off blocks per head, which fits at any T. Larger problems need
+ * one block per chunk of every head and are accepted while the total fits (see
+ * gdr_chunk_fwd_workspace_bytes). It allocates nothing on any call.
  *
  *  - Shapes: only those that need scratch (bf16 q/k/v, d_k = d_v = 128, chunk = 64); other
  *    shapes need none and are rejected with GDR_ERR_UNSUPPORTED (call gdr_chunk_fwd with a null
