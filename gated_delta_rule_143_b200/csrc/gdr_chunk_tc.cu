@@ -1415,30 +1415,40 @@ constexpr double kChainPerTaskChannel = 0.13;
 // per task. Measured at the KDA workload's shape (64 heads, 128 chunks): 0.08 (c1 = 115) 1193 us,
 // against 1224 us at 0.06, 1227 us at 0.10 and 1291 us for two passes.
 constexpr double kChainPerTaskGdn2 = 0.08;
-int fused_precomputed_chunks(int BH, int NC, int mode, bool ew = false) {
-    const bool ch = mode == GDR_DECAY_CHANNEL;
-    if (!ch && BH < kHybridMinHeads) return 0;
-    const double k = ch ? (ew ? kChainPerTaskGdn2 : kChainPerTaskChannel) : chain_per_task(BH);
+// With the mixer prologue (pro) each prep task does more, so where chunks are pre-computed at all,
+// more of them are (the ratio scaled by kProChainScale). A larger c1 keeps the call inside the plain
+// call's workspace: pre-computed and ring blocks total one per chunk either way, and the flags shrink.
+constexpr double kProChainScale = 0.75;
+int precomputed_for(double k, int BH, int NC) {
     const double f = 1.0 - k * (kSMs - BH) / (double)BH;
     if (f <= 0.0) return 0;
     const int c1 = (int)(f * NC + 0.999);
     return c1 < NC ? c1 : NC;
 }
-size_t pre_bytes(int BH, int NC, int mode, bool ew) {
-    return (size_t)BH * fused_precomputed_chunks(BH, NC, mode, ew) * kHandoffStride;
+int fused_precomputed_chunks(int BH, int NC, int mode, bool ew = false, bool pro = false) {
+    const bool ch = mode == GDR_DECAY_CHANNEL;
+    if (!ch && BH < kHybridMinHeads) return 0;
+    const double k = ch ? (ew ? kChainPerTaskGdn2 : kChainPerTaskChannel) : chain_per_task(BH);
+    const int c1 = precomputed_for(k, BH, NC);
+    if (c1 == 0 || !pro) return c1;
+    const int c1p = precomputed_for(k * kProChainScale, BH, NC);
+    return c1p > c1 ? c1p : c1;
+}
+size_t pre_bytes(int BH, int NC, int mode, bool ew, bool pro = false) {
+    return (size_t)BH * fused_precomputed_chunks(BH, NC, mode, ew, pro) * kHandoffStride;
 }
 // Ring slots per head. With chunks pre-computed, the chains spend their first c1 chunks on those
 // while the fused kernel's prep CTAs run ahead: a slot for every later chunk keeps them from
 // stalling on a full ring in that time (the blocks then mostly live in DRAM, not L2).
-int ring_depth(int BH, int NC, int mode, bool ew) {
-    const int c1 = fused_precomputed_chunks(BH, NC, mode, ew);
+int ring_depth(int BH, int NC, int mode, bool ew, bool pro = false) {
+    const int c1 = fused_precomputed_chunks(BH, NC, mode, ew, pro);
     return c1 > 0 ? NC - c1 : kRing;
 }
-size_t ring_bytes(int BH, int NC, int mode, bool ew) {
-    return (size_t)BH * ring_depth(BH, NC, mode, ew) * kHandoffStride;
+size_t ring_bytes(int BH, int NC, int mode, bool ew, bool pro = false) {
+    return (size_t)BH * ring_depth(BH, NC, mode, ew, pro) * kHandoffStride;
 }
-size_t flag_bytes(int BH, int NC, int mode, bool ew) {
-    return ((size_t)(BH * (ring_depth(BH, NC, mode, ew) + 1) + 1) * sizeof(int) + 255) & ~size_t(255);
+size_t flag_bytes(int BH, int NC, int mode, bool ew, bool pro = false) {
+    return ((size_t)(BH * (ring_depth(BH, NC, mode, ew, pro) + 1) + 1) * sizeof(int) + 255) & ~size_t(255);
 }
 
 template <int MODE, typename Tout, bool PRO, bool EW = false>
@@ -1458,11 +1468,11 @@ cudaError_t launch_fused(const ChunkProblem& p, const CUtensorMap& mq, const CUt
     if (!coop || per_sm < 1 || grid - BH < 8) return cudaErrorCooperativeLaunchTooLarge;
     // workspace: [pre-computed blocks, BH x c1][ring, BH x depth][flags]
     uint8_t* ws = static_cast<uint8_t*>(p.workspace);
-    const int c1 = fused_precomputed_chunks(BH, NC, MODE, EW), depth = ring_depth(BH, NC, MODE, EW);
-    uint8_t* ring = ws + pre_bytes(BH, NC, MODE, EW);
-    int* flags = reinterpret_cast<int*>(ring + ring_bytes(BH, NC, MODE, EW));
+    const int c1 = fused_precomputed_chunks(BH, NC, MODE, EW, PRO), depth = ring_depth(BH, NC, MODE, EW, PRO);
+    uint8_t* ring = ws + pre_bytes(BH, NC, MODE, EW, PRO);
+    int* flags = reinterpret_cast<int*>(ring + ring_bytes(BH, NC, MODE, EW, PRO));
     RingArgs R{ring, flags, flags + (size_t)BH * depth, flags + (size_t)BH * (depth + 1), ws, BH, c1, depth};
-    if ((err = cudaMemsetAsync(flags, 0, flag_bytes(BH, NC, MODE, EW), stream)) != cudaSuccess) return err;
+    if ((err = cudaMemsetAsync(flags, 0, flag_bytes(BH, NC, MODE, EW, PRO), stream)) != cudaSuccess) return err;
     if (c1 > 0 && (err = launch_prep<MODE, PRO, EW>(p, mq, mk, mv, NC, c1, ws, stream)) != cudaSuccess) return err;
     PrepArgs P{p.g, p.beta, p.T, p.H, NC, p.status, p.prologue, p.gate_scale, p.erase, p.write};
     StateArgs A{p.S0, p.S_T, p.T, p.H, NC, p.scale, p.status, p.B * p.H, nullptr};

@@ -310,7 +310,8 @@ typedef enum {
 
 /* The plan gdr_chunk_fwd uses for this problem (a gdr_plan value). For GDR_PLAN_PREP_FUSED,
  * *precomputed_chunks (if not NULL) receives the number of leading chunks per head the first
- * kernel prepares; for GDR_PLAN_SCAN, the number of segments; 0 otherwise. Chosen from the shape
+ * kernel prepares (gdr_chunk_fwd_ex with prologue flags prepares a few more, its prep tasks being
+ * longer, inside the same workspace); for GDR_PLAN_SCAN, the number of segments; 0 otherwise. Chosen from the shape
  * alone: at most 16 heads with at least 256 chunks each run the segment scan, with s segments, the
  * largest power of two in 2 .. 16 with B * H * s <= 64, at least 16 chunks per segment and T a
  * multiple of 64 s (4 segments for 16 heads, 16 for 1-4 heads); otherwise B * H <= 56 heads run

@@ -159,3 +159,15 @@ def test_prologue_decode_steps(mode, dtype, dk, dv):
         assert eo <= TOL[dtype], f"step {step}: o err {eo:.3e}"
     es, _ = rel_err(Sd.double().cpu().numpy(), S_ref)
     assert es <= TOL[dtype], f"final state err {es:.3e}"
+
+
+@pytest.mark.parametrize("mode,T", [("scalar", 1024), ("channel", 2048)])
+def test_prologue_prep_fused_more_precomputed_chunks(mode, T):
+    """64 heads: with the prologue the fused plan pre-computes more leading chunks than the plain call
+    (scalar gate, 16 chunks: 11 against 9; channel gate, 32 chunks: 28 against 27) inside the plain
+    call's workspace; every step against the oracle."""
+    NC = T // 64
+    plan, c1 = gdr.chunk_fwd_plan(8, T, 8, 128, 128, 64, mode, torch.bfloat16)
+    assert plan == "prep_fused" and 0 < c1 < NC
+    x = make_raw_chunk_inputs(8, T, 8, 128, 128, mode, "bf16", 7900 + MODES.index(mode), s0_std=0.05)
+    run_and_check(x, mode, "bf16", _flags(mode), label=f"{mode} 64 heads T={T}")
